@@ -1,0 +1,379 @@
+"""Pins for the CPU oracle (no GPU).
+
+Each test fixes part of the oracle to something other than the oracle itself:
+hand-worked values from the pages (``tests/golden``), closed forms,
+invariants the pages state, special cases that reduce to a library routine,
+exact rational arithmetic, or brute force on tiny inputs.  The last test
+plants mistakes in a copy of the oracle and checks that the pins catch them.
+"""
+import json
+import math
+import os
+import random
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+from oracle import dsa_oracle as O
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- P1 hand case
+def test_hand_index_scores_and_topk():
+    g = _golden("hand_index_topk.json")
+    q = np.array(g["q"])
+    keys = np.array(g["keys"])
+    w = np.array(g["w"])
+    sc = O.index_scores_row(q, keys, w, g["idx_scale"])
+    assert sc.tolist() == g["scores_pos3"]
+    for case in g["cases"]:
+        cand = O.visible_keys(case["q_pos"], 0, len(keys))
+        s = O.index_scores_row(q, keys[cand], w, g["idx_scale"])
+        got = O.topk_row(cand, s, case["k"])
+        assert got.tolist() == case["expect"], case
+
+
+def test_visibility_rules():
+    # causal inclusive, padding, and kv_len bound
+    assert O.visible_keys(5, 0, 10).tolist() == [0, 1, 2, 3, 4, 5]
+    assert O.visible_keys(5, 3, 10).tolist() == [3, 4, 5]
+    assert O.visible_keys(2, 3, 10).tolist() == []          # padded query row
+    assert O.visible_keys(12, 0, 8).tolist() == list(range(8))
+    # pools: only complete, causally visible pools
+    assert O.visible_pools(6, 0, 10, 4).tolist() == [0]
+    assert O.visible_pools(7, 0, 10, 4).tolist() == [0, 1]
+    assert O.visible_pools(7, 0, 1, 4).tolist() == [0]
+    assert O.visible_pools(2, 3, 10, 4).tolist() == []
+
+
+# ------------------------------------------------------- P2 dense reduction
+@pytest.mark.parametrize("Hk", [1, 4])
+def test_topk_covering_all_keys_equals_dense_attention(Hk):
+    """top_k >= visible keys turns the sparse layer into dense causal attention
+    (ik_llama.cpp #2045: PPL byte-identical to dense when top_k >= n_tokens)."""
+    rng = np.random.default_rng(7)
+    B, T, HI, DI, H, kd, vd = 2, 13, 3, 8, 4, 10, 6
+    q_idx = rng.standard_normal((B, T, HI, DI))
+    k_idx = rng.standard_normal((B, T, DI))
+    w = rng.standard_normal((B, T, HI))
+    q = rng.standard_normal((B, T, H, kd))
+    k = rng.standard_normal((B, T, Hk, kd))
+    v = rng.standard_normal((B, T, Hk, vd))
+    q_pos = np.tile(np.arange(T), (B, 1))
+    kv_start = np.array([0, 4])
+    kv_len = np.array([T, T - 2])
+    wl = dict(q_idx=q_idx, k_idx=k_idx, w=w, q_pos=q_pos, kv_start=kv_start, kv_len=kv_len)
+    dense = O.dense_causal_attend(q, k, v, 0.3, q_pos, kv_start, kv_len)
+    for b in range(B):
+        for t in range(T):
+            sel, out, lse, _ = O.layer_row(b, t, wl, T, 0.25, 0.3, q, k, v)
+            np.testing.assert_allclose(out, dense[b, t], rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------- P3 hand attend
+def test_hand_attend_sets():
+    g = _golden("hand_attend.json")
+    q = np.array([g["q"]])                   # one head
+    K = np.array(g["keys"])[:, None, :]
+    V = np.array(g["values"])[:, None, :]
+    lse_map = {"0.5+ln2": 0.5 + math.log(2.0), "0.5": 0.5, "-inf": -math.inf}
+    for case in g["cases"]:
+        out, lse = O.sparse_attend_row(q, K, V, np.array(case["idx"]), g["scale"])
+        assert out[0].tolist() == pytest.approx(case["out"], abs=1e-15)
+        want = lse_map[case["lse"]]
+        if math.isinf(want):
+            assert math.isinf(lse[0]) and lse[0] < 0
+        else:
+            assert lse[0] == pytest.approx(want, abs=1e-15)
+
+
+def test_softmax_two_key_closed_form():
+    # weights e^a / (e^a + e^b) for logits a, b
+    q = np.array([1.0, 2.0])
+    K = np.array([[0.3, -0.1], [1.0, 0.25]])
+    V = np.array([[1.0, 0.0, 5.0], [0.0, 1.0, -5.0]])
+    a, b = 0.7 * (0.3 - 0.2), 0.7 * (1.0 + 0.5)
+    pa = math.exp(a) / (math.exp(a) + math.exp(b))
+    out, lse = O.attend_row(q, K, V, 0.7)
+    np.testing.assert_allclose(out, [pa, 1 - pa, 5 * pa - 5 * (1 - pa)], atol=1e-15)
+    assert lse == pytest.approx(math.log(math.exp(a) + math.exp(b)), abs=1e-14)
+
+
+def test_dense_selection_matches_torch_sdpa():
+    """With every visible key selected, the sparse attend is torch's masked SDPA."""
+    rng = np.random.default_rng(3)
+    T, H, kd, vd = 9, 3, 7, 5
+    q = rng.standard_normal((1, T, H, kd))
+    k = rng.standard_normal((1, T, H, kd))
+    v = rng.standard_normal((1, T, H, vd))
+    idx = np.array([[list(range(t + 1)) + [-1] * (T - t - 1) for t in range(T)]])
+    out, _ = O.sparse_attend(q, k, v, idx, 0.45)
+    tq = torch.tensor(q[0]).permute(1, 0, 2)
+    tk = torch.tensor(k[0]).permute(1, 0, 2)
+    tv = torch.tensor(v[0]).permute(1, 0, 2)
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True, scale=0.45)
+    np.testing.assert_allclose(out[0], ref.permute(1, 0, 2).numpy(), atol=1e-12)
+
+
+# ------------------------------------------------------- P4 WHT invariance
+def test_walsh_hadamard_rotation_leaves_scores_unchanged():
+    """(Hq).(Hk) = D q.k for the unnormalised Sylvester matrix, so scale/D gives
+    bit-identical f64 scores (ik_llama.cpp #2045: the orthonormal rotation
+    leaves q.k unchanged)."""
+    rng = np.random.default_rng(11)
+    D, HI, n = 32, 4, 40
+    Hm = scipy.linalg.hadamard(D).astype(np.float64)
+    q = rng.integers(-4, 5, (HI, D)).astype(np.float64)
+    k = rng.integers(-4, 5, (n, D)).astype(np.float64)
+    w = rng.choice([0.5, 1.0, 2.0, 4.0], HI)
+    base = O.index_scores_row(q, k, w, 1.0 / 8.0)
+    rot = O.index_scores_row(q @ Hm.T, k @ Hm.T, w, 1.0 / 8.0 / D)
+    assert np.array_equal(base, rot)
+    assert np.any(base > 0)
+
+
+# ------------------------------------------------------ P5 brute-force top-k
+def _brute_topk(cand, scores, k):
+    """Repeatedly take the best remaining candidate: highest score, then smallest index."""
+    remaining = list(zip(cand.tolist(), scores.tolist()))
+    out = []
+    while remaining and len(out) < k:
+        best = None
+        for i, s in remaining:
+            if best is None or s > best[1] or (s == best[1] and i < best[0]):
+                best = (i, s)
+        out.append(best[0])
+        remaining.remove(best)
+    return out + [O.INVALID] * (k - len(out))
+
+
+def test_topk_matches_brute_force_with_ties():
+    rnd = random.Random(5)
+    for trial in range(300):
+        n = rnd.randint(0, 40)
+        k = rnd.randint(1, 45)
+        cand = np.array(sorted(rnd.sample(range(100), n)), dtype=np.int64)
+        scores = np.array([rnd.choice([-1.0, -0.0, 0.0, 0.5, 1.0, 2.0]) for _ in range(n)])
+        got = O.topk_row(cand, scores, k).tolist()
+        assert got == _brute_topk(cand, scores + 0.0, k), (cand, scores, k)
+
+
+# -------------------------------------------------- P6 exact integer scores
+def test_tiny_workload_scores_are_exact_rationals():
+    wl = workloads.make("tiny")
+    q, k, w = wl["q_idx"][0], wl["k_idx"][0], wl["w"][0]
+    for t in (0, 17, 40, 63):
+        cand = O.visible_keys(t, 0, 64)
+        got = O.index_scores_row(q[t], k[cand], w[t], wl.idx_scale)
+        for j, s in enumerate(cand.tolist()):
+            exact = Fraction(0)
+            for h in range(wl.idx_heads):
+                dot = sum(int(q[t, h, d]) * int(k[s, d]) for d in range(wl.idx_dim))
+                exact += Fraction(w[t, h].item()) * max(Fraction(0), Fraction(dot, 8))
+            assert Fraction(got[j]) == exact
+            assert (exact * 16).denominator == 1          # multiples of 1/16
+            assert abs(exact) <= 1024
+
+
+# -------------------------------------------------------- P7 pooling cases
+def test_pooling_starts_at_first_valid_token_and_drops_partial_pool():
+    g = _golden("hand_kpool.json")
+    kp = g["kpool"]
+    rng = np.random.default_rng(2)
+    for case in g["pooling"]:
+        n = case["kv_len"]
+        k = rng.standard_normal((n, 6))
+        gate = np.zeros((n, 6))                     # constant gate: slot mean
+        assert O.n_pools_of(case["kv_start"], n, kp) == case["n_pools"]
+        assert O.kept_pools(case["kv_start"], n, kp).tolist() == list(range(case["n_pools"]))
+        pooled = O.pool_states(k, gate, case["kv_start"], n, kp, None, None, 1e-6)
+        toks = case["pool0_tokens"]
+        want = O.layer_norm(k[toks], None, None, 1e-6).mean(axis=0)
+        np.testing.assert_allclose(pooled[0], want, atol=1e-14)
+
+
+def test_pool_gate_softmax_is_per_channel_over_slots():
+    rng = np.random.default_rng(4)
+    k = rng.standard_normal((8, 3))
+    gate = np.zeros((8, 3))
+    gate[5, 0] = 60.0       # slot 1 of pool 1 dominates channel 0 only
+    gate[6, 2] = 60.0       # slot 2 of pool 1 dominates channel 2 only
+    pooled = O.pool_states(k, gate, 0, 8, 4, None, None, 1e-6)
+    kn = O.layer_norm(k, None, None, 1e-6)
+    assert pooled[1, 0] == pytest.approx(kn[5, 0], abs=1e-20 + 1e-12)
+    assert pooled[1, 2] == pytest.approx(kn[6, 2], abs=1e-12)
+    assert pooled[1, 1] == pytest.approx(kn[4:8, 1].mean(), abs=1e-14)
+
+
+# -------------------------------------------------------- P8 expand cases
+def test_expand_selection_examples():
+    g = _golden("hand_kpool.json")
+    kp = g["kpool"]
+    for case in g["expand"]:
+        npools = O.n_pools_of(case["kv_start"], case["kv_len"], kp)
+        got = O.expand_selection(case["pools"], case["q_pos"], case["kv_start"], case["kv_len"],
+                                 kp, npools, case["out_width"])
+        assert got.tolist() == case["expect"], case["worked"]
+
+
+def test_expand_selection_tail_length_and_validity():
+    kp, f, L, selk = 4, 3, 40, 5
+    width = selk * kp + kp - 1
+    npools = O.n_pools_of(f, L, kp)
+    for t in range(0, L):
+        vis = O.visible_pools(t, f, npools, kp)
+        pools = list(vis[::-1][:selk]) + [O.INVALID] * max(0, selk - len(vis))
+        out = O.expand_selection(pools, t, f, L, kp, npools, width)
+        assert out.shape == (width,)
+        toks = out[out != O.INVALID]
+        if t < f:
+            assert toks.size == 0
+            continue
+        r = t - f
+        tail = [s for s in toks.tolist() if s >= f + len(vis) * kp]
+        assert len(tail) == (min(t, L - 1) - f + 1) - len(vis) * kp
+        if (r + 1) // kp <= npools:
+            assert len(tail) == (r + 1) % kp
+        assert len(set(toks.tolist())) == toks.size                 # no duplicates
+        assert all(f <= s <= t for s in toks.tolist())              # all visible
+        assert np.all(out[toks.size:] == O.INVALID)                 # INVALID only at the end
+
+
+# ------------------------------------------------ P9 absorption identity
+def test_absorbed_mla_equals_literal_expand_kv():
+    rng = np.random.default_rng(9)
+    H, d, L, n = 3, 5, 12, 17
+    q = rng.standard_normal((H, d))
+    lat = rng.standard_normal((n, L))
+    uk = rng.standard_normal((H, d, L)) / math.sqrt(L)
+    uv = rng.standard_normal((H, d + 1, L)) / math.sqrt(L)
+    row = np.array([3, 3, 16, -1, 0, 9, 40, 5])
+    lit, lse1 = O.mla_masked_attention_row(q, lat, uk, uv, row, 0.4)
+    ab, lse2 = O.mla_absorbed_row(q, lat, uk, uv, row, 0.4)
+    np.testing.assert_allclose(lit, ab, atol=1e-10)
+    np.testing.assert_allclose(lse1, lse2, atol=1e-10)
+    # the batched absorb helpers agree with the per-head routine
+    ql = O.absorb_q(q[None], uk)[0]
+    np.testing.assert_allclose(ql[1], uk[1].T @ q[1], atol=1e-13)
+    ol = O.absorb_out(np.ones((1, H, L)), uv)[0]
+    np.testing.assert_allclose(ol[2], uv[2].sum(axis=1), atol=1e-13)
+
+
+# ------------------------------------------------------ P10 invariances
+def test_index_row_permutation_invariance():
+    rng = np.random.default_rng(1)
+    H, kd, vd, n = 4, 9, 7, 30
+    q = rng.standard_normal((H, kd))
+    K = rng.standard_normal((n, 1, kd))
+    V = rng.standard_normal((n, 1, vd))
+    row = rng.choice(n, 20, replace=False)
+    a, la = O.sparse_attend_row(q, K, V, row, 0.5)
+    b, lb = O.sparse_attend_row(q, K, V, rng.permutation(row), 0.5)
+    np.testing.assert_allclose(a, b, atol=1e-12)
+    np.testing.assert_allclose(la, lb, atol=1e-12)
+
+
+def test_multi_sequence_batch_equals_sequences_alone():
+    """ik_llama.cpp #2063 UPDATE 5: n_seq=4 equals n_seq=1 chunk for chunk."""
+    rng = np.random.default_rng(8)
+    B, T, HI, DI, H, kd, vd = 3, 11, 2, 6, 2, 5, 4
+    ts = dict(q_idx=rng.standard_normal((B, T, HI, DI)), k_idx=rng.standard_normal((B, T, DI)),
+              w=rng.standard_normal((B, T, HI)), q_pos=np.tile(np.arange(T), (B, 1)),
+              kv_start=np.array([0, 2, 5]), kv_len=np.array([T, T, 9]))
+    q = rng.standard_normal((B, T, H, kd))
+    k = rng.standard_normal((B, T, 1, kd))
+    v = rng.standard_normal((B, T, 1, vd))
+    for b in range(B):
+        alone = {key: (val[b:b + 1]) for key, val in ts.items()}
+        for t in range(T):
+            s1, o1, _, _ = O.layer_row(b, t, ts, 4, 0.3, 0.6, q, k, v)
+            s2, o2, _, _ = O.layer_row(0, t, alone, 4, 0.3, 0.6, q[b:b + 1], k[b:b + 1], v[b:b + 1])
+            assert s1.tolist() == s2.tolist()
+            np.testing.assert_array_equal(o1, o2)
+
+
+# ---------------------------------------------------------- P11 LayerNorm
+def test_layer_norm_matches_torch_and_moments():
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((5, 128)) * 3 + 1
+    w = 1 + 0.1 * rng.standard_normal(128)
+    b = 0.1 * rng.standard_normal(128)
+    got = O.layer_norm(x, w, b, 1e-6)
+    ref = torch.nn.functional.layer_norm(torch.tensor(x), (128,), torch.tensor(w), torch.tensor(b), 1e-6)
+    np.testing.assert_allclose(got, ref.numpy(), atol=1e-12)
+    plain = O.layer_norm(x, None, None, 1e-6)
+    np.testing.assert_allclose(plain.mean(axis=1), 0, atol=1e-13)
+    np.testing.assert_allclose(plain.var(axis=1), 1, atol=1e-5)
+    with pytest.raises(ValueError):
+        O.layer_norm(x, w, b, 0.0)
+
+
+# ------------------------------------------- planted mistakes are caught
+def _run_pins():
+    failures = 0
+    for fn in (test_hand_index_scores_and_topk, test_hand_attend_sets, test_softmax_two_key_closed_form,
+               test_topk_matches_brute_force_with_ties, test_walsh_hadamard_rotation_leaves_scores_unchanged,
+               test_expand_selection_examples, test_pooling_starts_at_first_valid_token_and_drops_partial_pool,
+               lambda: test_topk_covering_all_keys_equals_dense_attention(1),
+               test_absorbed_mla_equals_literal_expand_kv):
+        try:
+            fn()
+        except (AssertionError, ValueError, IndexError):
+            failures += 1
+    return failures
+
+
+@pytest.mark.parametrize("mutant", ["scale_outside_relu_negated", "drop_weight", "tie_largest_index",
+                                    "no_dedupe", "softmax_no_max_shift_sign", "pool_from_zero",
+                                    "tail_off_by_one", "absorb_transposed"])
+def test_pins_catch_planted_mistakes(monkeypatch, mutant):
+    """Plant a plausible mistake in the oracle (on the CPU) and check a pin fails."""
+    assert _run_pins() == 0
+    if mutant == "scale_outside_relu_negated":
+        orig = O.index_scores_row
+        monkeypatch.setattr(O, "index_scores_row",
+                            lambda q, k, w, s: orig(q, k, w, -s) * -1.0)
+    elif mutant == "drop_weight":
+        monkeypatch.setattr(O, "index_scores_row",
+                            lambda q, k, w, s: np.maximum(0, s * (O.f64(q) @ O.f64(k).T)).sum(0))
+    elif mutant == "tie_largest_index":
+        def bad(cand, sc, k):
+            cand = np.asarray(cand); sc = np.asarray(sc, float)
+            order = np.lexsort((-cand, -sc))
+            out = np.full(k, -1); n = min(k, cand.size); out[:n] = cand[order[:n]]
+            return out
+        monkeypatch.setattr(O, "topk_row", bad)
+    elif mutant == "no_dedupe":
+        monkeypatch.setattr(O, "index_set",
+                            lambda row, n: np.array([i for i in O.i64(row).tolist() if 0 <= i < n], dtype=np.int64))
+    elif mutant == "softmax_no_max_shift_sign":
+        def bad_attend(q, k, v, scale):
+            k = O.f64(k); v = O.f64(v)
+            z = -scale * (k @ O.f64(q)); p = np.exp(z - z.max())
+            return (p @ v) / p.sum(), float(z.max() + math.log(p.sum()))
+        monkeypatch.setattr(O, "attend_row", bad_attend)
+    elif mutant == "pool_from_zero":
+        orig = O.pool_states
+        monkeypatch.setattr(O, "pool_states", lambda k, g, f, L, kp, w, b, e: orig(k, g, 0, L - f, kp, w, b, e))
+    elif mutant == "tail_off_by_one":
+        orig = O.expand_selection
+        def bad(pools, t, f, L, kp, npools, width):
+            return orig(pools, t - 1, f, L, kp, npools, width) if t > f else orig(pools, t, f, L, kp, npools, width)
+        monkeypatch.setattr(O, "expand_selection", bad)
+    elif mutant == "absorb_transposed":
+        orig = O.mla_absorbed_row
+        def bad2(q, lat, uk, uv, row, scale):
+            out, lse = orig(q, lat, uk, uv, row, scale)
+            return out[::-1].copy(), lse[::-1].copy()
+        monkeypatch.setattr(O, "mla_absorbed_row", bad2)
+    assert _run_pins() > 0, f"mutant {mutant} survived every pin"
