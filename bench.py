@@ -1,0 +1,460 @@
+"""Benchmark of the DSA layer on B200: query tokens / second and roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload prefill|decode|chunked|kpool] [--no-extras]
+
+A step is one pass of the whole hot path over one batch: dsa_layer_forward
+(indexer scores -> top-k -> sparse MLA attend) on the workload's synthetic
+inputs, already resident in HBM.  L2 is flushed (a 256 MiB write) before each
+timed step and each step is timed alone with CUDA events on the launching
+stream.  Under torchrun every rank runs its own replica of the workload
+(weak scaling, no data-path collective); the step time is the max over ranks.
+
+``--impl reference`` times the CPU oracle (the reference arm for this build)
+on a bounded sample of the same workload and prints the same JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "DSA layer query-tokens/sec (prefill & decode, top_k=2048); % of roofline"
+UNIT = "query-tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+# --------------------------------------------------------------------- peaks
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ------------------------------------------------------------ algorithmic work
+def visible_counts(wl):
+    qp = wl["q_pos"].long()
+    ks = wl["kv_start"].long().view(-1, 1)
+    kl = wl["kv_len"].long().view(-1, 1)
+    hi = torch.minimum(qp, kl - 1)
+    return (hi - ks + 1).clamp(min=0)
+
+
+def work(wl):
+    """Algorithmic FLOPs / bytes of each stage for one step of a token-mode workload."""
+    nvis = visible_counts(wl)
+    pairs_idx = int(nvis.sum())
+    pairs_att = int(nvis.clamp(max=wl.top_k).sum())
+    esz = 2 if wl.dtype == "bf16" else 4
+    rows = wl.batch * wl.n_q
+    return {
+        "index_flop": 2.0 * pairs_idx * wl.idx_heads * wl.idx_dim,
+        # k_I read once per sequence, q_I and w read, visible fp32 scores written
+        "index_bytes": wl.batch * wl.n_kv * wl.idx_dim * esz + rows * wl.idx_heads * (wl.idx_dim * esz + 4)
+        + 4.0 * pairs_idx,
+        "topk_bytes": 4.0 * pairs_idx + 4.0 * rows * wl.top_k,
+        "attend_flop": 2.0 * pairs_att * wl.heads * (wl.kd + wl.vd),
+        # one gathered latent row per (query, selected key), q read, out written
+        "attend_bytes": float(pairs_att) * wl.kd * esz + rows * wl.heads * (wl.kd + wl.vd) * esz,
+        "rows": rows,
+    }
+
+
+# -------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms in a thread."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- distributed
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=timedelta(seconds=120))
+        return dist.get_rank(), world, int(os.environ.get("LOCAL_RANK", "0"))
+    return 0, 1, 0
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------ the CUDA path
+def device_inputs(wl):
+    return {k: v.cuda(non_blocking=False) for k, v in wl.tensors.items()}
+
+
+def layer_args(wl, t):
+    from sparse_attention_sum_b200 import runner
+    lat = t["latent"]
+    dims = runner.layer_dims(t["q_idx"], t["k_idx"], t["q"], lat, wl.vd, wl.top_k)
+    args = dict(q_idx=t["q_idx"], k_idx=t["k_idx"], w=t["w"], idx_scale=wl.idx_scale, q_pos=t["q_pos"],
+                kv_start=t["kv_start"], kv_len=t["kv_len"], q=t["q"], k=lat, v=lat,
+                attn_scale=wl.attn_scale, k_row_stride=wl.kd, v_row_stride=wl.kd)
+    return dims, args
+
+
+def time_steps(step_fn, steps, warmup, flush, stream):
+    """Each step timed alone on `stream` with CUDA events; L2 flushed in between."""
+    for _ in range(warmup):
+        step_fn()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(steps):
+        flush.fill_(1)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step_fn()
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1) / 1e3)
+    return times
+
+
+def stage_times(wl, t, dims, args, bufs, steps, flush, stream):
+    """Per-stage device times (s) of the three C-ABI calls of the layer."""
+    import sparse_attention_sum_b200 as dsa
+    B, T, S = wl.batch, wl.n_q, wl.n_kv
+    scores = bufs.ws[: B * T * S * 4].view(torch.float32)
+    idx = bufs.idx
+    calls = {
+        "index": lambda: dsa.index_scores(dims, args["q_idx"], args["k_idx"], args["w"], args["idx_scale"],
+                                          args["q_pos"], args["kv_start"], args["kv_len"], scores),
+        "topk": lambda: dsa.topk(dims, scores, args["q_pos"], args["kv_start"], args["kv_len"], wl.top_k,
+                                 idx),
+        "attend": lambda: dsa.sparse_attend(dims, args["q"], args["k"], args["k_row_stride"], args["v"],
+                                            args["v_row_stride"], idx, wl.top_k, args["attn_scale"],
+                                            bufs.out),
+    }
+    res = {}
+    for name, fn in calls.items():
+        ts = time_steps(fn, max(3, steps), 2, flush, stream)
+        res[name] = statistics.median(ts)
+    return res
+
+
+def roofline_entry(kind, amount, seconds, peaks, traffic=None):
+    if kind == "tensor":
+        achieved = amount / seconds / 1e12
+        peak = peaks["bf16_tflops"]
+        return {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "peak_source": peaks["source"] + " (burst)"}
+    achieved = amount / seconds / 1e9
+    peak = peaks["hbm_gbs"]
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peaks["source"]}
+
+
+def profiled_traffic():
+    """Per-launch DRAM traffic of the dominant kernel from the committed ncu summary, if any."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            return json.load(f)
+    except Exception:
+        return {}
+
+
+def run_ours(a):
+    import sparse_attention_sum_b200 as dsa
+    from sparse_attention_sum_b200 import runner
+
+    rank, world, local = dist_setup(a.gpus)
+    torch.cuda.set_device(local)
+    dsa.lib()
+    peaks = measured_peaks()
+    wl = workloads.make(a.workload, seed=None if rank == 0 else 1000 + rank)
+    t = device_inputs(wl)
+    dims, args = layer_args(wl, t)
+    bufs = runner.LayerBuffers(dims, "cuda", torch.bfloat16, with_idx=True)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    step = lambda: runner.dsa_layer(dims, **args, bufs=bufs)
+
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        times = time_steps(step, a.steps, a.warmup, flush, stream)
+    barrier(world)
+    torch.cuda.synchronize()
+    total = max_over_ranks(sum(times), world)
+    assert dsa.get_device_status() == 0, "device reported a bounded-wait timeout"
+    rows = wl.batch * wl.n_q
+    value = world * rows * a.steps / total
+    wk = work(wl)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": round(1e3 * total / a.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded CPU generator, bf16)",
+        "config": {"workload": f"{wl.name}: B={wl.batch} T={wl.n_q} S={wl.n_kv} top_k={wl.top_k} "
+                               f"indexer {wl.idx_heads}x{wl.idx_dim}, MLA H={wl.heads} kd={wl.kd} vd={wl.vd}",
+                   "l2": "flushed (256 MiB write) before every timed step",
+                   "parallelism": f"replicas x{world} (one independent problem per GPU)"},
+        "gpu_launches": 3 * a.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and not a.no_extras:
+        st = stage_times(wl, t, dims, args, bufs, 5, flush, stream)
+        step_med = statistics.median(times)
+        line["stages_us"] = {k: round(v * 1e6, 1) for k, v in st.items()}
+        line["stages_qtok_s"] = {k: round(rows / v, 1) for k, v in st.items()}
+        line["fused_tensor_frac"] = round((wk["index_flop"] + wk["attend_flop"]) / step_med / 1e12
+                                          / peaks["bf16_tflops"], 4)
+        traffic = profiled_traffic().get(f"attend:{wl.name}")
+        line["roofline"] = roofline_entry("tensor", wk["attend_flop"], st["attend"], peaks, traffic)
+        line["roofline"]["kernel"] = "sparse attend (dsa_sparse_attend)"
+        line["roofline_stages"] = {
+            "index": roofline_entry("tensor", wk["index_flop"], st["index"], peaks),
+            "topk": roofline_entry("hbm", wk["topk_bytes"], st["topk"], peaks),
+            "attend": roofline_entry("tensor", wk["attend_flop"], st["attend"], peaks),
+        }
+        line["e2e"] = e2e_measure(wl, a.steps, stream)
+        if a.workload == "prefill":
+            line["decode"] = decode_extra(peaks, flush, stream)
+        line["cpu_baseline"] = cpu_baseline(wl, budget_s=a.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del t, bufs
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def e2e_measure(wl, steps, stream):
+    """Same metric through the public API with host buffers: pinned H2D copies of
+    the step's inputs, the layer call, and the D2H read of the output, all timed."""
+    from sparse_attention_sum_b200 import runner
+    host = {k: v.pin_memory() for k, v in wl.tensors.items()}
+    dev_t = {k: torch.empty_like(v, device="cuda") for k, v in host.items()}
+    dims, args = layer_args(wl, dev_t)
+    bufs = runner.LayerBuffers(dims, "cuda", torch.bfloat16, with_idx=True)
+    out_host = torch.empty(bufs.out.shape, dtype=bufs.out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def step():
+        for k in host:
+            dev_t[k].copy_(host[k], non_blocking=True)
+        runner.dsa_layer(dims, **args, bufs=bufs)
+        out_host.copy_(bufs.out, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    n = max(3, min(steps, 10))
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    e1.synchronize()
+    sec = e0.elapsed_time(e1) / 1e3 / n
+    return {"value": round(wl.batch * wl.n_q / sec, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(sec * 1e3, 3)}
+
+
+def decode_extra(peaks, flush, stream):
+    """The decode workload (64 sequences x 1 query vs 32768 cached keys) and its stages."""
+    from sparse_attention_sum_b200 import runner
+    wl = workloads.make("decode")
+    t = device_inputs(wl)
+    dims, args = layer_args(wl, t)
+    bufs = runner.LayerBuffers(dims, "cuda", torch.bfloat16, with_idx=True)
+    times = time_steps(lambda: runner.dsa_layer(dims, **args, bufs=bufs), 10, 3, flush, stream)
+    st = stage_times(wl, t, dims, args, bufs, 10, flush, stream)
+    wk = work(wl)
+    rows = wl.batch * wl.n_q
+    step = statistics.median(times)
+    res = {"workload": f"decode: B={wl.batch} T=1 S={wl.n_kv} top_k={wl.top_k}",
+           "value": round(rows / step, 1), "unit": UNIT, "ms_per_step": round(step * 1e3, 4),
+           "stages_us": {k: round(v * 1e6, 1) for k, v in st.items()},
+           "roofline_attend": roofline_entry("hbm", wk["attend_bytes"], st["attend"], peaks),
+           "roofline_index": roofline_entry("hbm", wk["index_bytes"], st["index"], peaks),
+           "fused_hbm_frac": round((wk["index_bytes"] + wk["topk_bytes"] + wk["attend_bytes"]) / step / 1e9
+                                   / peaks["hbm_gbs"], 4)}
+    del t, bufs
+    torch.cuda.empty_cache()
+    return res
+
+
+# ------------------------------------------------------------ the CPU oracle
+def oracle_rows(wl, rows):
+    from oracle import dsa_oracle as O
+    lat = wl["latent"]
+    K, V = lat.unsqueeze(2), lat[..., :wl.vd].unsqueeze(2)
+    ts = wl.tensors
+    for b, t in rows:
+        O.layer_row(b, t, ts, wl.top_k, wl.idx_scale, wl.attn_scale, wl["q"], K, V)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline(wl, budget_s=15.0):
+    """Oracle query rows per second on this host, on a bounded stratified sample."""
+    import random
+    T = wl.n_q
+    rnd = random.Random(0)
+    order = [(b, t) for b in range(wl.batch) for t in (0, T - 1, min(T - 1, wl.top_k))]
+    t0 = time.perf_counter()
+    done = 0
+    while time.perf_counter() - t0 < budget_s and done < 4096:
+        batch = order if done == 0 else [(rnd.randrange(wl.batch), rnd.randrange(T)) for _ in range(4)]
+        oracle_rows(wl, batch)
+        done += len(batch)
+    el = time.perf_counter() - t0
+    return {"value": round(done / el, 3), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{done} query rows of {wl.name} (first, last, top-k boundary, then random), "
+                      f"{el:.1f} s, f64 numpy oracle, extrapolated per query row"}
+
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = workloads.make(a.workload)
+    rows_per_step = 4
+    import random
+    rnd = random.Random(1)
+    for _ in range(a.warmup):
+        oracle_rows(wl, [(0, rnd.randrange(wl.n_q))])
+    times = []
+    for _ in range(a.steps):
+        rows = [(rnd.randrange(wl.batch), rnd.randrange(wl.n_q)) for _ in range(rows_per_step)]
+        t0 = time.perf_counter()
+        oracle_rows(wl, rows)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = rows_per_step * a.steps / total
+    cores = blas_threads()
+    line = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": 1, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": round(1e3 * total / a.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded CPU generator, bf16)",
+            "config": {"workload": f"{wl.name}: B={wl.batch} T={wl.n_q} S={wl.n_kv} top_k={wl.top_k}",
+                       "sample": f"{rows_per_step} random query rows per step"},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{rows_per_step} random query rows of {wl.name} per step"},
+            "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["prefill", "decode", "chunked"], default="prefill")
+    ap.add_argument("--no-extras", action="store_true", help="skip stages, decode, e2e and CPU baseline")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    a = ap.parse_args(argv)
+    a.warmup = max(3, a.warmup)  # at least three untimed warm-up steps
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)
+
+
+if __name__ == "__main__":
+    main()

@@ -408,7 +408,7 @@ def expand_selection(pool_row, q_pos: int, kv_start: int, kv_len: int, kpool: in
         return out
     pos = 0
     for p in i64(pool_row).tolist():
-        if p == INVALID:
+        if p < 0 or p >= int(n_pools):         # INVALID and out-of-range ids hold no pool
             continue
         for j in range(kpool):
             out[pos] = f + p * kpool + j

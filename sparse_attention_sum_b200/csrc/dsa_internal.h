@@ -1,0 +1,66 @@
+// Host-side launchers of the DSA kernels (internal to libdsa; not part of the C ABI).
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "dsa.h"
+
+namespace dsa {
+
+// Device address of the status word on the current device (bounded waits
+// record DSA_ERR_TIMEOUT there).
+int* device_status_ptr();
+
+// Number of SMs of the current device.
+int sm_count();
+
+// S2 on the CUDA cores (any D_I <= 256, H_I*D_I <= 16384), fp32 or bf16 inputs.
+cudaError_t launch_index_scores_simt(const dsa_dims& d, const void* q_idx, const void* k_idx,
+                                     const float* w, float scale, const int32_t* q_pos,
+                                     const int32_t* kv_start, const int32_t* kv_len, float* scores,
+                                     cudaStream_t st);
+// S2 on the tensor cores (tcgen05, bf16, D_I == 128, H_I in {16,32,64,128}).
+bool index_scores_tc_supported(const dsa_dims& d);
+cudaError_t launch_index_scores_tc(const dsa_dims& d, const void* q_idx, const void* k_idx,
+                                   const float* w, float scale, const int32_t* q_pos,
+                                   const int32_t* kv_start, const int32_t* kv_len, float* scores,
+                                   cudaStream_t st);
+
+// S3 radix select + rank sort.
+cudaError_t launch_topk(const dsa_dims& d, const float* scores, const int32_t* q_pos,
+                        const int32_t* kv_start, const int32_t* kv_len, int k, int32_t* idx,
+                        float* vals, cudaStream_t st);
+
+// S4 on the CUDA cores (generic shapes).
+bool attend_simt_supported(const dsa_dims& d, int width);
+cudaError_t launch_attend_simt(const dsa_dims& d, const void* q, const void* k, int64_t k_stride,
+                               const void* v, int64_t v_stride, const int32_t* idx, int width,
+                               float scale, void* out, float* lse, cudaStream_t st);
+// S4 on the tensor cores (tcgen05, bf16 shared latent).
+bool attend_tc_supported(const dsa_dims& d, int64_t k_stride, const void* k, const void* v,
+                         int64_t v_stride, int width);
+cudaError_t launch_attend_tc(const dsa_dims& d, const void* q, const void* k, int64_t k_stride,
+                             const int32_t* idx, int width, float scale, void* out, float* lse,
+                             cudaStream_t st);
+
+// S6 / S7.
+cudaError_t launch_pool_states(const dsa_dims& d, const void* k, const void* gate,
+                               const float* ln_w, const float* ln_b, float eps,
+                               const int32_t* kv_start, const int32_t* kv_len, void* pooled,
+                               int32_t* n_pools, cudaStream_t st);
+cudaError_t launch_expand_selection(const dsa_dims& d, const int32_t* pool_idx,
+                                    const int32_t* q_pos, const int32_t* kv_start,
+                                    const int32_t* kv_len, const int32_t* n_pools,
+                                    int32_t* tok_idx, cudaStream_t st);
+
+// S8: batched per-head GEMM C[n,h,:] = A[n,h,:] x B[h] (bf16 in, fp32 accumulate, bf16 out).
+//   b_kn = true:  B[h] is [K, N] (N contiguous)    (absorb_q: w_uk[h] is [d, L])
+//   b_kn = false: B[h] is [N, K] (K contiguous)    (absorb_out: w_uv[h] is [e, L])
+cudaError_t launch_head_gemm(int n_rows, int heads, int K, int N, const void* A, const void* Bm,
+                             bool b_kn, void* C, cudaStream_t st);
+
+// Bounded-wait self test.
+cudaError_t launch_wait_selftest(long long timeout_ns, cudaStream_t st);
+
+}  // namespace dsa

@@ -1,0 +1,252 @@
+// S3 deterministic top-k: radix select in shared memory, then a rank sort.
+//
+// Per query row: the min(k, n_visible) visible keys with the highest score,
+// ordered by higher score and then smaller key index (metrale
+// glm5next_dsa_ref topk_pools; ik_llama.cpp #2045 ggml_top_k(min(top_k,
+// n_tokens))).
+//
+// One block per row.  Scores become order-preserving uint32 keys (signed
+// zeros merged) and are cached in shared memory when the visible range fits.
+// Four 8-bit MSB-first histogram passes (shared-memory atomics aggregated per
+// warp with match_any, a warp-wide scan of the 256 bins) find the exact k-th
+// largest key tau and how many keys equal to tau are still needed.  Each warp
+// then walks a contiguous segment of the row 32 keys at a time; ballots and a
+// block-wide prefix sum place every key > tau and the lowest-index keys == tau,
+// which keeps the tie rule exact.  Finally the k (key, index) pairs are put in
+// rank order by a bitonic sort of 64-bit composites (~key << 32 | index).
+#include "dsa_common.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+
+constexpr int kTopkMaxK = 4096;
+constexpr int kTopkCacheMax = 40960;  // keys cached in shared memory (160 KB)
+
+// Block-wide exclusive scan of one int per thread; returns the block total.
+template <int BLOCK>
+__device__ __forceinline__ int block_exclusive_scan(int v, int* scratch /*>= BLOCK/32 + 1*/, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scratch[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int s = lane < BLOCK / 32 ? scratch[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    if (lane < BLOCK / 32) scratch[lane] = s;  // inclusive warp totals
+  }
+  __syncthreads();
+  int warp_base = warp > 0 ? scratch[warp - 1] : 0;
+  total = scratch[BLOCK / 32 - 1];
+  __syncthreads();
+  return warp_base + x - v;
+}
+
+template <int BLOCK>
+__device__ void bitonic_sort_u64(uint64_t* a, int n /* power of two */) {
+  for (int size = 2; size <= n; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < (n >> 1); i += BLOCK) {
+        int lo = 2 * i - (i & (stride - 1));
+        int hi = lo + stride;
+        bool up = (lo & size) == 0;
+        uint64_t x = a[lo], y = a[hi];
+        if ((x > y) == up) {
+          a[lo] = y;
+          a[hi] = x;
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+template <int BLOCK>
+__global__ void __launch_bounds__(BLOCK)
+topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restrict__ q_pos,
+            const int32_t* __restrict__ kv_start, const int32_t* __restrict__ kv_len, int k,
+            int kpow2, int cache_cap, int32_t* __restrict__ idx_out, float* __restrict__ vals_out) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  uint64_t* sel = reinterpret_cast<uint64_t*>(smem_raw);            // [kpow2]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(sel + kpow2);         // [256]
+  int* scan = reinterpret_cast<int*>(hist + 256);                    // [64]
+  uint32_t* cache = reinterpret_cast<uint32_t*>(scan + 64);          // [cache_cap]
+  __shared__ uint32_t s_prefix, s_krem;
+
+  const int b = blockIdx.y, t = blockIdx.x;
+  const size_t row = (size_t)b * d.n_q + t;
+  const float* srow = scores + row * d.n_kv;
+  int32_t* orow = idx_out + row * k;
+  float* vrow = vals_out ? vals_out + row * k : nullptr;
+
+  KeyRange r = visible_range(q_pos[row], kv_start[b], kv_len[b], d.n_kv, d.kpool);
+  const int n = r.count();
+  const bool cached = n <= cache_cap;
+
+  if (n <= k) {
+    // every visible key is selected: just rank them
+    for (int i = threadIdx.x; i < kpow2; i += BLOCK) {
+      uint64_t c = ~0ull;
+      if (i < n) c = ((uint64_t)(~score_key(srow[r.lo + i])) << 32) | (uint32_t)(r.lo + i);
+      sel[i] = c;
+    }
+    __syncthreads();
+    bitonic_sort_u64<BLOCK>(sel, kpow2);
+    for (int i = threadIdx.x; i < k; i += BLOCK) {
+      if (i < n) {
+        uint64_t c = sel[i];
+        orow[i] = (int32_t)(uint32_t)c;
+        if (vrow) vrow[i] = key_score(~(uint32_t)(c >> 32));
+      } else {
+        orow[i] = DSA_INVALID;
+        if (vrow) vrow[i] = -INFINITY;
+      }
+    }
+    return;
+  }
+
+  if (cached)
+    for (int i = threadIdx.x; i < n; i += BLOCK) cache[i] = score_key(srow[r.lo + i]);
+  if (threadIdx.x == 0) {
+    s_prefix = 0u;
+    s_krem = (uint32_t)k;
+  }
+  __syncthreads();
+
+  // ---- radix select: find tau (the k-th largest key) digit by digit
+  uint32_t prefix = 0u, mask = 0u;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += BLOCK) hist[i] = 0u;
+    __syncthreads();
+    for (int base = (threadIdx.x & ~31); base < n; base += BLOCK) {
+      const int i = base + (threadIdx.x & 31);
+      int bin = -1;
+      if (i < n) {
+        uint32_t key = cached ? cache[i] : score_key(srow[r.lo + i]);
+        if ((key & mask) == prefix) bin = (int)((key >> shift) & 255u);
+      }
+      // lanes that hit the same bin add once (scores often share their top bits)
+      uint32_t peers = __match_any_sync(0xffffffffu, bin);
+      if (bin >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      // lane L owns digits 255-8L .. 248-8L (descending)
+      const int lane = threadIdx.x;
+      uint32_t cnt[8];
+      uint32_t lsum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        cnt[j] = hist[255 - 8 * lane - j];
+        lsum += cnt[j];
+      }
+      uint32_t incl = lsum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      uint32_t excl = incl - lsum;
+      uint32_t krem = s_krem;
+      if (excl < krem && incl >= krem) {  // the crossing digit lies in this lane's 8 bins
+        uint32_t c = excl;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (c + cnt[j] >= krem) {
+            s_prefix = prefix | ((uint32_t)(255 - 8 * lane - j) << shift);
+            s_krem = krem - c;
+            break;
+          }
+          c += cnt[j];
+        }
+      }
+    }
+    __syncthreads();
+    prefix = s_prefix;
+    mask |= 255u << shift;
+    __syncthreads();
+  }
+  const uint32_t tau = prefix;
+  const int need_eq = (int)s_krem;  // keys equal to tau still to take (lowest indices first)
+  const int n_gt = k - need_eq;
+
+  // ---- gather: each warp owns a contiguous segment, walked 32 keys at a time,
+  // so the output order of equal keys is their index order.
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int NW = BLOCK / 32;
+  const int wseg = ((n + NW - 1) / NW + 31) & ~31;
+  const int w0 = warp * wseg;
+  const int w1 = min(n, w0 + wseg);
+  int c_gt = 0, c_eq = 0;
+  for (int i = w0 + lane; i < w1; i += 32) {
+    uint32_t key = cached ? cache[i] : score_key(srow[r.lo + i]);
+    c_gt += key > tau;
+    c_eq += key == tau;
+  }
+  c_gt = __reduce_add_sync(0xffffffffu, c_gt);
+  c_eq = __reduce_add_sync(0xffffffffu, c_eq);
+  int tot;
+  int gt_base = block_exclusive_scan<BLOCK>(lane == 0 ? c_gt : 0, scan, tot);
+  int eq_base = block_exclusive_scan<BLOCK>(lane == 0 ? c_eq : 0, scan, tot);
+  gt_base = __shfl_sync(0xffffffffu, gt_base, 0);
+  eq_base = __shfl_sync(0xffffffffu, eq_base, 0);
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int b0 = w0; b0 < w1; b0 += 32) {
+    const int i = b0 + lane;
+    uint32_t key = 0u;
+    if (i < w1) key = cached ? cache[i] : score_key(srow[r.lo + i]);
+    const bool is_gt = i < w1 && key > tau;
+    const bool is_eq = i < w1 && key == tau;
+    const uint32_t m_gt = __ballot_sync(0xffffffffu, is_gt);
+    const uint32_t m_eq = __ballot_sync(0xffffffffu, is_eq);
+    const uint64_t c = ((uint64_t)(~key) << 32) | (uint32_t)(r.lo + i);
+    if (is_gt) sel[gt_base + __popc(m_gt & lt_mask)] = c;
+    if (is_eq) {
+      int rank = eq_base + __popc(m_eq & lt_mask);
+      if (rank < need_eq) sel[n_gt + rank] = c;
+    }
+    gt_base += __popc(m_gt);
+    eq_base += __popc(m_eq);
+  }
+  for (int i = k + threadIdx.x; i < kpow2; i += BLOCK) sel[i] = ~0ull;
+  __syncthreads();
+  bitonic_sort_u64<BLOCK>(sel, kpow2);
+  for (int i = threadIdx.x; i < k; i += BLOCK) {
+    uint64_t c = sel[i];
+    orow[i] = (int32_t)(uint32_t)c;
+    if (vrow) vrow[i] = key_score(~(uint32_t)(c >> 32));
+  }
+}
+
+cudaError_t launch_topk(const dsa_dims& d, const float* scores, const int32_t* q_pos,
+                        const int32_t* kv_start, const int32_t* kv_len, int k, int32_t* idx,
+                        float* vals, cudaStream_t st) {
+  int kpow2 = 1;
+  while (kpow2 < k) kpow2 <<= 1;
+  int cache_cap = d.n_kv < kTopkCacheMax ? d.n_kv : kTopkCacheMax;
+  size_t smem = (size_t)kpow2 * 8 + 256 * 4 + 64 * 4 + (size_t)cache_cap * 4;
+  dim3 grid(d.n_q, d.batch);
+  cudaError_t e;
+  if (d.n_kv > 8192) {
+    auto kern = topk_kernel<1024>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, 1024, smem, st>>>(d, scores, q_pos, kv_start, kv_len, k, kpow2, cache_cap, idx, vals);
+  } else {
+    auto kern = topk_kernel<512>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, 512, smem, st>>>(d, scores, q_pos, kv_start, kv_len, k, kpow2, cache_cap, idx, vals);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace dsa

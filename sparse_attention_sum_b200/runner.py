@@ -1,0 +1,116 @@
+"""Convenience layer over the C ABI: allocates outputs and workspaces with torch
+and chains the libdsa entry points.  No arithmetic happens here; every step
+is one libdsa call.
+
+* :func:`dsa_layer`   -- S1-S5: indexer scores, top-k, sparse MLA attend
+  (``dsa_layer_forward``).
+* :func:`kpool_layer` -- S6-S8 with S2-S4 over pools: LayerNorm + pooling,
+  pool scores, pool top-k, expand_selection, absorbed NoPE MLA attend.
+"""
+from __future__ import annotations
+
+from typing import Dict, Optional
+
+import torch
+
+from . import (BF16, F32, OP_LAYER_FORWARD, Dims, absorb_out, absorb_q, expand_selection,
+               index_scores, layer_forward, pool_states, sparse_attend, topk, workspace_size)
+
+
+def _code(dtype: torch.dtype) -> int:
+    if dtype == torch.float32:
+        return F32
+    if dtype == torch.bfloat16:
+        return BF16
+    raise ValueError(f"unsupported dtype {dtype}")
+
+
+def layer_dims(q_idx, k_idx, q, k, vd: int, top_k: int) -> Dims:
+    """Dims of a token-mode layer call from tensor shapes.
+
+    q_idx [B,T,H_I,D_I], k_idx [B,S,D_I], q [B,T,H,kd], k [B,S,Hk,kd] or a
+    shared latent [B,S,kd] (Hk = 1).
+    """
+    B, T, HI, DI = q_idx.shape
+    S = k_idx.shape[1]
+    H, kd = q.shape[2], q.shape[3]
+    Hk = 1 if k.dim() == 3 else k.shape[2]
+    return Dims(batch=B, n_q=T, n_kv=S, idx_heads=HI, idx_dim=DI, top_k=top_k, heads=H,
+                kv_heads=Hk, kd=kd, vd=vd, kpool=0, out_width=top_k, dtype=_code(q.dtype))
+
+
+class LayerBuffers:
+    """Outputs and workspace of :func:`dsa_layer`, reusable across calls."""
+
+    def __init__(self, dims: Dims, device, out_dtype, with_idx: bool = True, with_lse: bool = False):
+        rows = dims.batch * dims.n_q
+        self.out = torch.empty(dims.batch, dims.n_q, dims.heads, dims.vd, dtype=out_dtype, device=device)
+        self.idx = torch.empty(dims.batch, dims.n_q, dims.top_k, dtype=torch.int32, device=device) \
+            if with_idx else None
+        self.lse = torch.empty(dims.batch, dims.n_q, dims.heads, dtype=torch.float32, device=device) \
+            if with_lse else None
+        nbytes = workspace_size(dims, OP_LAYER_FORWARD)
+        self.ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+        self.rows = rows
+
+
+def dsa_layer(dims: Dims, q_idx, k_idx, w, idx_scale, q_pos, kv_start, kv_len, q, k, v,
+              attn_scale, k_row_stride: int, v_row_stride: int, bufs: Optional[LayerBuffers] = None,
+              idx_in=None, stream=None) -> LayerBuffers:
+    """One call of ``dsa_layer_forward``; returns the buffers holding out/idx/lse."""
+    if bufs is None:
+        bufs = LayerBuffers(dims, q.device, q.dtype)
+    layer_forward(dims, q_idx, k_idx, w, idx_scale, q_pos, kv_start, kv_len, q, k, k_row_stride, v,
+                  v_row_stride, attn_scale, bufs.out, lse=bufs.lse, idx_in=idx_in, idx_out=bufs.idx,
+                  ws=bufs.ws, stream=stream)
+    return bufs
+
+
+class KpoolBuffers:
+    """Intermediates and outputs of :func:`kpool_layer`."""
+
+    def __init__(self, B, T, S, HI, DI, kpool, select_k, out_width, H, dqk, L, dv, device,
+                 dtype=torch.bfloat16):
+        P = S // kpool
+        self.pooled = torch.empty(B, P, DI, dtype=dtype, device=device)
+        self.n_pools = torch.empty(B, dtype=torch.int32, device=device)
+        self.pool_scores = torch.empty(B, T, P, dtype=torch.float32, device=device)
+        self.pool_idx = torch.empty(B, T, select_k, dtype=torch.int32, device=device)
+        self.tok_idx = torch.empty(B, T, out_width, dtype=torch.int32, device=device)
+        self.q_lat = torch.empty(B, T, H, L, dtype=dtype, device=device)
+        self.o_lat = torch.empty(B, T, H, L, dtype=dtype, device=device)
+        self.out = torch.empty(B, T, H, dv, dtype=dtype, device=device)
+
+
+def kpool_dims(B, T, S, HI, DI, kpool, select_k, out_width, H, L, dtype=torch.bfloat16) -> Dict[str, Dims]:
+    """Dims of each call of the kpool pipeline."""
+    code = _code(dtype)
+    P = S // kpool
+    return {
+        "pool": Dims(batch=B, n_q=T, n_kv=S, idx_heads=HI, idx_dim=DI, top_k=select_k, heads=H,
+                     kv_heads=1, kd=L, vd=L, kpool=kpool, out_width=out_width, dtype=code),
+        "index": Dims(batch=B, n_q=T, n_kv=P, idx_heads=HI, idx_dim=DI, top_k=select_k, heads=H,
+                      kv_heads=1, kd=L, vd=L, kpool=kpool, out_width=out_width, dtype=code),
+        "attend": Dims(batch=B, n_q=T, n_kv=S, idx_heads=HI, idx_dim=DI, top_k=out_width, heads=H,
+                       kv_heads=1, kd=L, vd=L, kpool=0, out_width=out_width, dtype=code),
+    }
+
+
+def kpool_layer(dims: Dict[str, Dims], q_idx, k_raw, gate, ln_w, ln_b, ln_eps, w, idx_scale, q_pos,
+                kv_start, kv_len, q_nope, latent, w_uk, w_uv, attn_scale,
+                bufs: KpoolBuffers, stream=None) -> KpoolBuffers:
+    """The kpool NoPE DSA layer as a chain of libdsa calls."""
+    dp, di, da = dims["pool"], dims["index"], dims["attend"]
+    pool_states(dp, k_raw, gate, ln_w, ln_b, ln_eps, kv_start, kv_len, bufs.pooled, bufs.n_pools,
+                stream=stream)
+    index_scores(di, q_idx, bufs.pooled, w, idx_scale, q_pos, kv_start, kv_len, bufs.pool_scores,
+                 stream=stream)
+    topk(di, bufs.pool_scores, q_pos, kv_start, kv_len, di.top_k, bufs.pool_idx, stream=stream)
+    expand_selection(dp, bufs.pool_idx, q_pos, kv_start, kv_len, bufs.n_pools, bufs.tok_idx,
+                     stream=stream)
+    L = da.kd
+    absorb_q(da, q_nope, q_nope.shape[-1], w_uk, L, bufs.q_lat, stream=stream)
+    sparse_attend(da, bufs.q_lat, latent, L, latent, L, bufs.tok_idx, da.out_width, attn_scale,
+                  bufs.o_lat, stream=stream)
+    absorb_out(da, bufs.o_lat, L, w_uv, w_uv.shape[1], bufs.out, stream=stream)
+    return bufs

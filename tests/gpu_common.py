@@ -1,0 +1,117 @@
+"""Helpers shared by the GPU parity tests: device copies of workloads, row
+sampling, and the comparison rules (exact, tie-band, float tolerance)."""
+from __future__ import annotations
+
+import math
+import random
+
+import numpy as np
+import torch
+
+from oracle import dsa_oracle as O
+import sparse_attention_sum_b200 as dsa
+from sparse_attention_sum_b200 import runner
+
+# Float tolerances (attention outputs): max-abs 2e-2 (bf16) / 1e-4 (fp32) and
+# per-row cosine >= 0.9999.  Selection: bit-exact where scores are exact; else
+# every disagreement within 1e-5 * max(|tau|, max|I|) of the k-th score tau.
+ATOL = {torch.bfloat16: 2e-2, torch.float32: 1e-4}
+COS_MIN = 0.9999
+TIE_BAND = 1e-5
+
+
+def dev(wl, device="cuda"):
+    return {k: v.to(device) for k, v in wl.tensors.items()}
+
+
+def layer_inputs(wl, t):
+    """(dims, args) for runner.dsa_layer from a token-mode workload on device."""
+    if "latent" in t:
+        k = t["latent"]
+        v = t["latent"]
+        ks = vs = wl.kd
+        kk = k
+    else:
+        kk = t["k"]
+        v = t["v"]
+        ks = wl.kv_heads * wl.kd
+        vs = wl.kv_heads * wl.vd
+    dims = runner.layer_dims(t["q_idx"], t["k_idx"], t["q"], kk if kk.dim() == 4 else kk, wl.vd, wl.top_k)
+    dims.kv_heads = wl.kv_heads
+    return dims, dict(q_idx=t["q_idx"], k_idx=t["k_idx"], w=t["w"], idx_scale=wl.idx_scale,
+                      q_pos=t["q_pos"], kv_start=t["kv_start"], kv_len=t["kv_len"], q=t["q"], k=kk,
+                      v=v, attn_scale=wl.attn_scale, k_row_stride=ks, v_row_stride=vs)
+
+
+def kv_views(wl):
+    """Oracle-side K/V caches [B,S,Hk,kd] / [B,S,Hk,vd] (views, still bf16/fp32)."""
+    if "latent" in wl.tensors:
+        lat = wl["latent"]
+        return lat.unsqueeze(2), lat[..., :wl.vd].unsqueeze(2)
+    return wl["k"], wl["v"]
+
+
+def sample_rows(wl, n=12, seed=0, extra=()):
+    """First, last, the top-k boundary row and evenly spread rows (b, t)."""
+    B, T = wl.batch, wl.n_q
+    rows = {(0, 0), (B - 1, T - 1)}
+    qp = wl["q_pos"]
+    ks = wl["kv_start"]
+    for b in range(B):
+        # first row whose visible count exceeds top_k
+        for t in range(T):
+            if int(qp[b, t]) - int(ks[b]) + 1 > wl.top_k:
+                rows.add((b, t))
+                break
+    rnd = random.Random(seed)
+    while len(rows) < n:
+        rows.add((rnd.randrange(B), rnd.randrange(T)))
+    rows |= set(extra)
+    return sorted(rows)
+
+
+def cosine(a: np.ndarray, b: np.ndarray) -> float:
+    na, nb = np.linalg.norm(a), np.linalg.norm(b)
+    if na == 0 and nb == 0:
+        return 1.0
+    return float(np.dot(a.ravel(), b.ravel()) / (na * nb))
+
+
+def assert_attend_close(gpu_out, ref_out, dtype, what=""):
+    """gpu_out, ref_out: [..., H, vd] for one or more rows."""
+    g = np.asarray(gpu_out, dtype=np.float64)
+    r = np.asarray(ref_out, dtype=np.float64)
+    err = np.abs(g - r).max() if g.size else 0.0
+    assert err <= ATOL[dtype], f"{what}: max |diff| {err} > {ATOL[dtype]}"
+    gr = g.reshape(-1, g.shape[-2] * g.shape[-1]) if g.ndim >= 2 else g.reshape(1, -1)
+    rr = r.reshape(gr.shape)
+    for i in range(gr.shape[0]):
+        if np.linalg.norm(rr[i]) > 0:
+            c = cosine(gr[i], rr[i])
+            assert c >= COS_MIN, f"{what}: row {i} cosine {c}"
+
+
+def check_selection_in_band(gpu_sel, cand, ref_scores, k, what=""):
+    """GPU selection vs the oracle's scores: equal, or every difference inside the tie band.
+
+    Returns the number of differing keys (0 when the rows are identical).
+    """
+    ref_sel = O.topk_row(cand, ref_scores, k)
+    g = [int(x) for x in gpu_sel]
+    r = [int(x) for x in ref_sel]
+    if g == r:
+        return 0
+    n_valid = min(k, len(cand))
+    assert sum(1 for x in g if x != O.INVALID) == n_valid, f"{what}: selected count"
+    assert all(x == O.INVALID for x in g[n_valid:]), f"{what}: INVALID tail"
+    gs, rs = set(g[:n_valid]), set(r[:n_valid])
+    score_of = dict(zip(cand.tolist(), ref_scores.tolist()))
+    tau = score_of[r[n_valid - 1]]
+    scale_ = max(abs(tau), max(abs(x) for x in ref_scores.tolist()))
+    band = TIE_BAND * scale_
+    for key in gs ^ rs:
+        assert key in score_of, f"{what}: selected key {key} not visible"
+        assert abs(score_of[key] - tau) <= band, \
+            f"{what}: key {key} score {score_of[key]} outside tie band {band} of tau {tau}"
+    # the ranked order agrees up to swaps inside the band
+    return len(gs ^ rs)

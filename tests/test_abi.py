@@ -1,0 +1,117 @@
+"""The C-ABI library loads, exports every declared entry point, and rejects bad
+arguments on the host before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import sparse_attention_sum_b200 as dsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dsa.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(dsa.lib_path()):
+        from sparse_attention_sum_b200 import build
+        build.build()
+    return dsa.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 14
+    out = subprocess.run(["nm", "-D", "--defined-only", dsa.lib_path()], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (dsa_\w+)", out))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        assert getattr(lib, n) is not None
+
+
+def test_binding_covers_the_header():
+    assert set(_declared()) <= set(dsa._SIGS)
+
+
+def test_status_strings(lib):
+    for code, name in dsa.STATUS.items():
+        assert lib.dsa_status_string(code).decode() == name
+    assert b"sm_100a" in lib.dsa_version()
+
+
+def test_workspace_size(lib):
+    d = dsa.Dims(batch=2, n_q=3, n_kv=100, top_k=8)
+    n = dsa.workspace_size(d, dsa.OP_LAYER_FORWARD)
+    assert n == ((2 * 3 * 100 * 4 + 255) // 256) * 256 + ((2 * 3 * 8 * 4 + 255) // 256) * 256
+    assert dsa.workspace_size(d, dsa.OP_TOPK) == 0
+    assert dsa.workspace_size(d, 99) == 0
+    assert dsa.workspace_size(dsa.Dims(batch=0, n_q=1, n_kv=1, top_k=1), dsa.OP_LAYER_FORWARD) == 0
+
+
+def _call(fn, *args):
+    st = fn(*args)
+    return st, dsa.lib().dsa_last_error().decode()
+
+
+def test_host_validation_rejects_bad_arguments(lib):
+    nul = None
+    d = dsa.Dims(batch=1, n_q=4, n_kv=8, idx_heads=2, idx_dim=16, top_k=4, heads=2, kv_heads=1,
+                 kd=16, vd=8, kpool=0, out_width=4, dtype=dsa.BF16)
+    p = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+    st, msg = _call(lib.dsa_index_scores, None, p, p, p, 1.0, p, p, p, p, nul)
+    assert st == 1 and "dims" in msg
+    st, msg = _call(lib.dsa_index_scores, ctypes.byref(d), nul, p, p, 1.0, p, p, p, p, nul)
+    assert st == 1 and "non-NULL" in msg
+    st, msg = _call(lib.dsa_topk, ctypes.byref(d), p, p, p, p, 0, p, nul, nul, 0, nul)
+    assert st == 1 and "k must be" in msg
+    st, msg = _call(lib.dsa_topk, ctypes.byref(d), p, p, p, p, 5000, p, nul, nul, 0, nul)
+    assert st == 1
+    bad = dsa.Dims(**{**d.as_dict(), "heads": 3, "kv_heads": 2})
+    st, msg = _call(lib.dsa_sparse_attend, ctypes.byref(bad), p, p, 16, p, 16, p, 4, 1.0, p, nul, nul)
+    assert st == 1 and "divide" in msg
+    st, msg = _call(lib.dsa_sparse_attend, ctypes.byref(d), p, p, 8, p, 16, p, 4, 1.0, p, nul, nul)
+    assert st == 1 and "k_row_stride" in msg
+    bad = dsa.Dims(**{**d.as_dict(), "dtype": 7})
+    st, msg = _call(lib.dsa_sparse_attend, ctypes.byref(bad), p, p, 16, p, 16, p, 4, 1.0, p, nul, nul)
+    assert st == 1 and "dtype" in msg
+    # layer forward: workspace too small is reported as DSA_ERR_WORKSPACE
+    st, msg = _call(lib.dsa_layer_forward, ctypes.byref(d), p, p, p, 1.0, p, p, p, p, p, 16, p, 16, 1.0,
+                    nul, nul, p, nul, p, 8, nul)
+    assert st == 3 and "workspace" in msg
+    kp = dsa.Dims(**{**d.as_dict(), "kpool": 4})
+    st, msg = _call(lib.dsa_layer_forward, ctypes.byref(kp), p, p, p, 1.0, p, p, p, p, p, 16, p, 16, 1.0,
+                    nul, nul, p, nul, p, 1 << 20, nul)
+    assert st == 1 and "kpool" in msg
+    # kpool entry points
+    st, msg = _call(lib.dsa_pool_states, ctypes.byref(kp), p, p, nul, nul, 0.0, p, p, p, p, nul)
+    assert st == 1 and "ln_eps" in msg
+    narrow = dsa.Dims(**{**kp.as_dict(), "out_width": 4 * 4 + 2})
+    st, msg = _call(lib.dsa_expand_selection, ctypes.byref(narrow), p, p, p, p, p, p, nul)
+    assert st == 1 and "out_width" in msg
+    f32 = dsa.Dims(**{**d.as_dict(), "dtype": dsa.F32})
+    st, msg = _call(lib.dsa_absorb_q, ctypes.byref(f32), p, 16, p, 32, p, nul)
+    assert st == 2 and "bf16" in msg
+    st, msg = _call(lib.dsa_selftest_wait_timeout, 5, nul)
+    assert st == 1
+
+
+def test_binding_raises_typed_errors(lib):
+    with pytest.raises(dsa.DsaError) as ei:
+        dsa._check(1, "dsa_topk")
+    assert ei.value.name == "DSA_ERR_INVALID_ARGUMENT"
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(dsa, "_lib", None)
+    monkeypatch.setattr(dsa, "lib_path", lambda: str(tmp_path / "libdsa.so"))
+    with pytest.raises(dsa.DsaLibraryError):
+        dsa.lib()

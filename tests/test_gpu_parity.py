@@ -1,0 +1,392 @@
+"""GPU parity: every stage of the CUDA path against the CPU oracle (needs a B200).
+
+Small cases compare every element; full-size workloads (in the launch
+configuration bench.py times) compare sampled rows element by element and
+check structural properties on every row.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import dsa_oracle as O
+import sparse_attention_sum_b200 as dsa
+from sparse_attention_sum_b200 import runner
+import workloads
+from tests.gpu_common import (ATOL, assert_attend_close, check_selection_in_band, cosine, dev,
+                              kv_views, layer_inputs, sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    dsa.lib()  # fail loudly if the library is missing
+    dsa.set_kernel_policy(0)
+    yield
+    assert dsa.get_device_status() == 0
+
+
+def _np(t):
+    return t.detach().to(torch.float64).cpu().numpy()
+
+
+def _run_stages(wl, t):
+    """Index scores, top-k and attend as three separate C-ABI calls."""
+    dims, a = layer_inputs(wl, t)
+    B, T, S = wl.batch, wl.n_q, wl.n_kv
+    scores = torch.empty(B, T, S, dtype=torch.float32, device="cuda")
+    dsa.index_scores(dims, a["q_idx"], a["k_idx"], a["w"], a["idx_scale"], a["q_pos"], a["kv_start"],
+                     a["kv_len"], scores)
+    idx = torch.empty(B, T, wl.top_k, dtype=torch.int32, device="cuda")
+    vals = torch.empty(B, T, wl.top_k, dtype=torch.float32, device="cuda")
+    dsa.topk(dims, scores, a["q_pos"], a["kv_start"], a["kv_len"], wl.top_k, idx, vals)
+    out = torch.empty(B, T, wl.heads, wl.vd, dtype=t["q"].dtype, device="cuda")
+    lse = torch.empty(B, T, wl.heads, dtype=torch.float32, device="cuda")
+    dsa.sparse_attend(dims, a["q"], a["k"], a["k_row_stride"], a["v"], a["v_row_stride"], idx, wl.top_k,
+                      a["attn_scale"], out, lse)
+    torch.cuda.synchronize()
+    return dims, a, scores, idx, vals, out, lse
+
+
+# ------------------------------------------------------------- tiny (fp32)
+def test_tiny_layer_is_exact_against_oracle():
+    wl = workloads.make("tiny")
+    t = dev(wl)
+    dims, a, scores, idx, vals, out, lse = _run_stages(wl, t)
+    ref_scores = O.index_scores(wl["q_idx"], wl["k_idx"], wl["w"], wl.idx_scale, wl["q_pos"],
+                                wl["kv_start"], wl["kv_len"])
+    got = _np(scores)
+    # integer inputs, power-of-two scale and weights: exact scores, bit-identical selection
+    assert np.array_equal(got, ref_scores)
+    ref_idx = O.topk(ref_scores, wl.top_k, wl["q_pos"], wl["kv_start"], wl["kv_len"])
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    gv = vals.cpu().numpy()
+    for tt in range(wl.n_q):
+        n = min(wl.top_k, tt + 1)
+        assert np.array_equal(gv[0, tt, :n], ref_scores[0, tt, ref_idx[0, tt, :n]])
+        assert np.all(np.isneginf(gv[0, tt, n:]))
+    # attention over the (identical) selection: fp32 tolerance
+    K, V = kv_views(wl)
+    ref_out, ref_lse = O.sparse_attend(wl["q"], K, V, ref_idx, wl.attn_scale)
+    assert_attend_close(_np(out), ref_out, torch.float32, "tiny attend")
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, atol=1e-4)
+    # the fused call equals the composition
+    bufs = runner.dsa_layer(dims, **a)
+    torch.cuda.synchronize()
+    assert torch.equal(bufs.idx, idx)
+    assert torch.equal(bufs.out, out)
+
+
+def test_tiny_layer_covering_all_keys_is_dense_attention():
+    wl = workloads.make("tiny")
+    wl.top_k = 64
+    t = dev(wl)
+    dims, a = layer_inputs(wl, t)
+    bufs = runner.dsa_layer(dims, **a)
+    torch.cuda.synchronize()
+    K, V = kv_views(wl)
+    dense = O.dense_causal_attend(wl["q"], K, V, wl.attn_scale, wl["q_pos"], wl["kv_start"], wl["kv_len"])
+    assert_attend_close(_np(bufs.out), dense, torch.float32, "dense reduction")
+
+
+# --------------------------------------------------------- top-k edge cases
+def _topk_case(scores_np, q_pos, kv_start, kv_len, k, kpool=0):
+    B, T, S = scores_np.shape
+    d = dsa.Dims(batch=B, n_q=T, n_kv=S, kpool=kpool, top_k=k)
+    sc = torch.tensor(scores_np, dtype=torch.float32, device="cuda")
+    qp = torch.tensor(q_pos, dtype=torch.int32, device="cuda")
+    ks = torch.tensor(kv_start, dtype=torch.int32, device="cuda")
+    kl = torch.tensor(kv_len, dtype=torch.int32, device="cuda")
+    idx = torch.full((B, T, k), 12345, dtype=torch.int32, device="cuda")
+    vals = torch.empty(B, T, k, dtype=torch.float32, device="cuda")
+    dsa.topk(d, sc, qp, ks, kl, k, idx, vals)
+    torch.cuda.synchronize()
+    got = idx.cpu().numpy()
+    for b in range(B):
+        for t in range(T):
+            if kpool:
+                npools = O.n_pools_of(kv_start[b], kv_len[b], kpool)
+                cand = O.visible_pools(q_pos[b][t], kv_start[b], min(npools, S), kpool)
+            else:
+                cand = O.visible_keys(q_pos[b][t], kv_start[b], min(kv_len[b], S))
+            want = O.topk_row(cand, scores_np[b, t, cand].astype(np.float64), k)
+            assert got[b, t].tolist() == want.tolist(), (b, t, k)
+    return got
+
+
+@pytest.mark.parametrize("S,k", [(1, 1), (7, 16), (64, 16), (300, 37), (4096, 2048), (5000, 4096),
+                                 (33000, 2048), (50000, 2048), (2049, 2048)])
+def test_topk_bit_exact_with_heavy_ties(S, k):
+    rng = np.random.default_rng(S + k)
+    T = 6
+    # integer-valued scores: many exact ties exercise the index tie-break
+    scores = rng.integers(-3, 4, size=(2, T, S)).astype(np.float32) * 0.5
+    scores[0, 0, :] = 0.0                             # an all-equal row
+    scores[1, 1, ::2] = -0.0                          # signed zeros equal +0
+    q_pos = [[S - 1, S // 2, 0, S - 1, 3, S + 5], [S - 1, S - 1, S // 3, 1, S - 2, 2 * S]]
+    kv_start = [0, min(2, S - 1)]
+    kv_len = [S, max(1, S - 3)]
+    _topk_case(scores, q_pos, kv_start, kv_len, k)
+
+
+def test_topk_distinct_and_padded_rows():
+    rng = np.random.default_rng(0)
+    S = 9000
+    scores = rng.standard_normal((3, 4, S)).astype(np.float32)
+    q_pos = [[S - 1, 100, 5, 2047], [4, 3, S - 1, 2500], [S - 1, S - 1, S - 1, S - 1]]
+    kv_start = [0, 5, 1000]      # batch 1 row 1: padded query (q_pos < kv_start)
+    kv_len = [S, S, 6000]
+    got = _topk_case(scores, q_pos, kv_start, kv_len, 2048)
+    assert np.all(got[1, 1] == O.INVALID)
+
+
+def test_topk_pool_mode_visibility():
+    rng = np.random.default_rng(1)
+    P = 300
+    scores = rng.integers(-2, 3, size=(2, 5, P)).astype(np.float32)
+    q_pos = [[2, 3, 7, 1199, 600], [16, 17, 20, 1199, 100]]
+    _topk_case(scores, q_pos, [0, 17], [1200, 1200], 64, kpool=4)
+
+
+# -------------------------------------------------------- attend edge cases
+@pytest.mark.parametrize("dtype,H,Hk,kd,vd", [(torch.float32, 4, 4, 32, 24), (torch.float32, 8, 2, 40, 40),
+                                              (torch.bfloat16, 128, 1, 576, 512),
+                                              (torch.bfloat16, 64, 1, 512, 512),
+                                              (torch.bfloat16, 3, 1, 70, 33)])
+def test_attend_set_semantics(dtype, H, Hk, kd, vd):
+    rng = np.random.default_rng(H + kd)
+    B, T, S, W = 2, 5, 300, 40
+    shared = Hk == 1 and kd >= vd
+    q = torch.tensor(rng.standard_normal((B, T, H, kd)), dtype=dtype)
+    if shared:
+        lat = torch.tensor(rng.standard_normal((B, S, kd)) * 0.5, dtype=dtype)
+        K, V = lat.unsqueeze(2), lat[..., :vd].unsqueeze(2)
+        k_dev, v_dev, ks, vs = lat.cuda(), lat.cuda(), kd, kd
+    else:
+        K = torch.tensor(rng.standard_normal((B, S, Hk, kd)), dtype=dtype)
+        V = torch.tensor(rng.standard_normal((B, S, Hk, vd)), dtype=dtype)
+        k_dev, v_dev, ks, vs = K.cuda(), V.cuda(), Hk * kd, Hk * vd
+    idx = rng.integers(-1, S, size=(B, T, W)).astype(np.int32)
+    idx[0, 0, :] = -1                     # empty row
+    idx[0, 1, :] = 7                      # one key repeated
+    idx[0, 2, ::3] = S + 11               # out of range
+    idx[1, 0, :] = np.arange(W) % 5       # duplicates of five keys
+    idx[1, 1, :] = rng.permutation(S)[:W]
+    d = dsa.Dims(batch=B, n_q=T, n_kv=S, heads=H, kv_heads=Hk, kd=kd, vd=vd, top_k=W,
+                 dtype=dsa.F32 if dtype == torch.float32 else dsa.BF16)
+    out = torch.empty(B, T, H, vd, dtype=dtype, device="cuda")
+    lse = torch.empty(B, T, H, dtype=torch.float32, device="cuda")
+    dsa.sparse_attend(d, q.cuda(), k_dev, ks, v_dev, vs, torch.tensor(idx).cuda(), W, 0.3, out, lse)
+    torch.cuda.synchronize()
+    ref, ref_lse = O.sparse_attend(q, K, V, idx, 0.3)
+    assert_attend_close(_np(out), ref, dtype, f"attend {dtype} H{H} kd{kd}")
+    g_lse = lse.cpu().numpy()
+    assert np.all(np.isneginf(g_lse[0, 0])) and np.all(_np(out)[0, 0] == 0)
+    fin = np.isfinite(ref_lse)
+    np.testing.assert_allclose(g_lse[fin], ref_lse[fin], atol=2e-3 if dtype == torch.bfloat16 else 1e-4)
+
+
+# -------------------------------------------------- bf16 MLA layer (small)
+@pytest.mark.parametrize("name,sizes", [("prefill", dict(T=333)), ("decode", dict(B=3, S=5000)),
+                                        ("chunked", dict(T=130, S=4500))])
+def test_small_bf16_layer_against_oracle(name, sizes):
+    wl = workloads.make(name, **sizes)
+    if name == "prefill":
+        wl.top_k = 128
+    t = dev(wl)
+    dims, a, scores, idx, vals, out, lse = _run_stages(wl, t)
+    g_scores = scores.cpu().numpy().astype(np.float64)
+    g_idx = idx.cpu().numpy()
+    K, V = kv_views(wl)
+    B, T = wl.batch, wl.n_q
+    rows = [(b, tt) for b in range(B) for tt in range(T)] if B * T <= 400 else sample_rows(wl, 40)
+    n_diff_rows = 0
+    for b, tt in rows:
+        p, ks, kl = int(wl["q_pos"][b, tt]), int(wl["kv_start"][b]), int(wl["kv_len"][b])
+        cand = O.visible_keys(p, ks, kl)
+        ref = O.index_scores_row(wl["q_idx"][b, tt], wl["k_idx"][b][cand], wl["w"][b, tt], wl.idx_scale)
+        gs = g_scores[b, tt, cand]
+        scale_ = max(1.0, np.abs(ref).max())
+        assert np.abs(gs - ref).max() <= 2e-5 * scale_, (b, tt, np.abs(gs - ref).max())
+        invis = np.ones(wl.n_kv, bool)
+        invis[cand] = False
+        assert np.all(np.isneginf(g_scores[b, tt, invis]))
+        # selection kernel alone: bit-exact against the oracle top-k of the GPU's own scores
+        assert g_idx[b, tt].tolist() == O.topk_row(cand, gs, wl.top_k).tolist()
+        # end to end: inside the tie band of the oracle's scores
+        n_diff_rows += check_selection_in_band(g_idx[b, tt], cand, ref, wl.top_k, f"{name} row {(b, tt)}") > 0
+        # attend over the GPU's own selection
+        ro, rl = O.sparse_attend_row(wl["q"][b, tt], K[b], V[b], g_idx[b, tt], wl.attn_scale)
+        assert_attend_close(_np(out[b, tt]), ro, torch.bfloat16, f"{name} attend {(b, tt)}")
+    assert n_diff_rows <= max(1, len(rows) // 10)
+
+
+# ------------------------------------------------------------- kpool (small)
+def _kpool_run(wl):
+    t = dev(wl)
+    B, T, S = wl.batch, wl.n_q, wl.n_kv
+    H, L = wl.heads, wl.kd
+    dims = runner.kpool_dims(B, T, S, wl.idx_heads, wl.idx_dim, wl.kpool, wl.select_k, wl.out_width, H, L)
+    bufs = runner.KpoolBuffers(B, T, S, wl.idx_heads, wl.idx_dim, wl.kpool, wl.select_k, wl.out_width,
+                               H, t["q_nope"].shape[-1], L, t["w_uv"].shape[1], "cuda")
+    runner.kpool_layer(dims, t["q_idx"], t["k_raw"], t["gate"], t["ln_w"], t["ln_b"], wl.ln_eps, t["w"],
+                       wl.idx_scale, t["q_pos"], t["kv_start"], t["kv_len"], t["q_nope"], t["latent"],
+                       t["w_uk"], t["w_uv"], wl.attn_scale, bufs)
+    torch.cuda.synchronize()
+    return bufs
+
+
+def _kpool_check(wl, bufs, rows):
+    B = wl.batch
+    kp = wl.kpool
+    npools = bufs.n_pools.cpu().tolist()
+    pooled = bufs.pooled.float().cpu().numpy()
+    pool_scores = bufs.pool_scores.cpu().numpy().astype(np.float64)
+    pool_idx = bufs.pool_idx.cpu().numpy()
+    tok_idx = bufs.tok_idx.cpu().numpy()
+    out = _np(bufs.out)
+    q_lat = _np(bufs.q_lat)
+    refpool = {}
+    for b in range(B):
+        f, L = int(wl["kv_start"][b]), int(wl["kv_len"][b])
+        assert npools[b] == O.n_pools_of(f, L, kp)
+        ref = O.pool_states(wl["k_raw"][b], wl["gate"][b], f, L, kp, wl["ln_w"], wl["ln_b"], wl.ln_eps)
+        refpool[b] = ref
+        np.testing.assert_allclose(pooled[b, :npools[b]], ref, atol=3e-2, rtol=1e-2)
+        assert np.all(pooled[b, npools[b]:] == 0)
+    for b, tt in rows:
+        f = int(wl["kv_start"][b])
+        L = int(wl["kv_len"][b])
+        p = int(wl["q_pos"][b, tt])
+        cand = O.visible_pools(p, f, npools[b], kp)
+        # index over the GPU's pooled keys (bf16 values as stored), oracle arithmetic
+        gpk = bufs.pooled[b].cpu()
+        ref_sc = O.index_scores_row(wl["q_idx"][b, tt], gpk[cand], wl["w"][b, tt], wl.idx_scale) \
+            if cand.size else np.zeros(0)
+        if cand.size:
+            assert np.abs(pool_scores[b, tt, cand] - ref_sc).max() <= 2e-5 * max(1, np.abs(ref_sc).max())
+        assert pool_idx[b, tt].tolist() == O.topk_row(cand, pool_scores[b, tt, cand], wl.select_k).tolist()
+        check_selection_in_band(pool_idx[b, tt], cand, ref_sc, wl.select_k, f"kpool pools {(b, tt)}")
+        want_tok = O.expand_selection(pool_idx[b, tt], p, f, L, kp, npools[b], wl.out_width)
+        assert tok_idx[b, tt].tolist() == want_tok.tolist()
+        # absorbed attention over the GPU's token rows vs the literal expand_kv form
+        ro, _ = O.mla_masked_attention_row(wl["q_nope"][b, tt], wl["latent"][b], wl["w_uk"], wl["w_uv"],
+                                           tok_idx[b, tt], wl.attn_scale)
+        assert_attend_close(out[b, tt], ro, torch.bfloat16, f"kpool out {(b, tt)}")
+        np.testing.assert_allclose(q_lat[b, tt], O.absorb_q(wl["q_nope"][b, tt][None], wl["w_uk"])[0],
+                                   atol=3e-2, rtol=1e-2)
+
+
+def test_kpool_small_against_oracle():
+    wl = workloads.make("kpool", T=160, pads=(0, 3, 17, 70))
+    wl.select_k = 8
+    wl.top_k = 8
+    wl.out_width = 8 * 4 + 3
+    bufs = _kpool_run(wl)
+    rows = [(b, t) for b in range(wl.batch) for t in range(0, wl.n_q, 7)] + [(3, 69), (3, 70), (2, 20)]
+    _kpool_check(wl, bufs, rows)
+
+
+# --------------------------------------------------------- full-size workloads
+def _full_layer(name):
+    wl = workloads.make(name)
+    t = dev(wl)
+    dims, a = layer_inputs(wl, t)
+    bufs = runner.LayerBuffers(dims, "cuda", t["q"].dtype, with_idx=True, with_lse=True)
+    runner.dsa_layer(dims, **a, bufs=bufs)
+    torch.cuda.synchronize()
+    return wl, t, dims, bufs
+
+
+@pytest.mark.parametrize("name", ["prefill", "decode", "chunked"])
+def test_full_size_layer_sampled_rows(name):
+    wl, t, dims, bufs = _full_layer(name)
+    B, T, S = wl.batch, wl.n_q, wl.n_kv
+    scores = bufs.ws[: B * T * S * 4].view(torch.float32).view(B, T, S)
+    g_idx = bufs.idx.cpu().numpy()
+    K, V = kv_views(wl)
+    rows = sample_rows(wl, 12)
+    diffs = 0
+    for b, tt in rows:
+        p, ks, kl = int(wl["q_pos"][b, tt]), int(wl["kv_start"][b]), int(wl["kv_len"][b])
+        cand = O.visible_keys(p, ks, kl)
+        ref = O.index_scores_row(wl["q_idx"][b, tt], wl["k_idx"][b][cand], wl["w"][b, tt], wl.idx_scale)
+        gs = scores[b, tt].cpu().numpy().astype(np.float64)[cand]
+        assert np.abs(gs - ref).max() <= 2e-5 * max(1.0, np.abs(ref).max())
+        assert g_idx[b, tt].tolist() == O.topk_row(cand, gs, wl.top_k).tolist()
+        diffs += check_selection_in_band(g_idx[b, tt], cand, ref, wl.top_k, f"{name} {(b, tt)}") > 0
+        ro, rl = O.sparse_attend_row(wl["q"][b, tt], K[b], V[b], g_idx[b, tt], wl.attn_scale)
+        assert_attend_close(_np(bufs.out[b, tt]), ro, torch.bfloat16, f"{name} out {(b, tt)}")
+        np.testing.assert_allclose(bufs.lse[b, tt].cpu().numpy(), rl, atol=2e-3)
+    assert diffs <= max(1, len(rows) // 4)
+    # every row: count, visibility, uniqueness and rank order by the GPU's scores
+    sel = bufs.idx
+    qp = t["q_pos"].view(B, T, 1).long()
+    valid = sel >= 0
+    nvis = (qp[..., 0] - t["kv_start"].view(B, 1).long() + 1).clamp(min=0).clamp(max=S)
+    assert torch.equal(valid.sum(-1), nvis.clamp(max=wl.top_k))
+    assert bool((sel[valid].long() <= qp.expand_as(sel)[valid]).all())
+    srt = torch.sort(sel.masked_fill(~valid, -1 - 10**6), dim=-1).values
+    dup = (srt[..., 1:] == srt[..., :-1]) & (srt[..., 1:] >= 0)
+    assert not bool(dup.any())
+    sv = torch.gather(scores, 2, sel.clamp(min=0).long()).masked_fill(~valid, -math.inf)
+    assert bool((sv[..., 1:][valid[..., 1:]] <= sv[..., :-1][valid[..., 1:]]).all())
+
+
+def test_full_size_kpool_sampled_rows():
+    wl = workloads.make("kpool")
+    bufs = _kpool_run(wl)
+    rows = sample_rows(wl, 8, extra=[(3, 1028), (3, 1029), (1, 20)])
+    _kpool_check(wl, bufs, rows)
+
+
+# ----------------------------------------------------------- run properties
+def test_rerun_is_bit_identical():
+    wl = workloads.make("prefill", T=1024)
+    t = dev(wl)
+    dims, a = layer_inputs(wl, t)
+    b1 = runner.dsa_layer(dims, **a)
+    o1, i1 = b1.out.clone(), b1.idx.clone()
+    b2 = runner.dsa_layer(dims, **a)
+    torch.cuda.synchronize()
+    assert torch.equal(i1, b2.idx)
+    assert torch.equal(o1, b2.out)
+
+
+def test_multi_sequence_batch_equals_sequences_alone():
+    wl = workloads.make("decode", B=4, S=3000)
+    t = dev(wl)
+    dims, a = layer_inputs(wl, t)
+    whole = runner.dsa_layer(dims, **a)
+    torch.cuda.synchronize()
+    for b in range(wl.batch):
+        one = {k: (v[b:b + 1] if isinstance(v, torch.Tensor) else v) for k, v in a.items()}
+        d1 = dsa.Dims(**{**dims.as_dict(), "batch": 1})
+        alone = runner.dsa_layer(d1, **one)
+        torch.cuda.synchronize()
+        assert torch.equal(alone.idx[0], whole.idx[b])
+        assert torch.equal(alone.out[0], whole.out[b])
+
+
+def test_index_reuse_skips_selection():
+    wl = workloads.make("prefill", T=300)
+    wl.top_k = 64
+    t = dev(wl)
+    dims, a = layer_inputs(wl, t)
+    first = runner.dsa_layer(dims, **a)
+    again = runner.dsa_layer(dims, **a, idx_in=first.idx.clone(), bufs=runner.LayerBuffers(dims, "cuda", torch.bfloat16))
+    torch.cuda.synchronize()
+    assert torch.equal(first.out, again.out)
+
+
+def test_bounded_wait_expires_and_reports_timeout():
+    assert dsa.get_device_status() == 0
+    dsa.selftest_wait_timeout(2_000_000)      # 2 ms
+    assert dsa.get_device_status() == 5       # DSA_ERR_TIMEOUT, context still usable
+    assert dsa.get_device_status() == 0       # cleared
+    x = torch.ones(4, device="cuda") * 2
+    assert x.sum().item() == 8
