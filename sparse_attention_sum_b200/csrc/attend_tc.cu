@@ -1,6 +1,540 @@
+// S4 sparse MLA attention on the 5th-generation tensor cores (tcgen05).
+//
+// out[b,t,h,:] = sum_{i in U} softmax_i(scale * q[b,t,h,:] . c_i) c_i[:vd], U = the
+// distinct valid entries of idx[b,t,:] (fak note "GLM-5.2: the DSA sparse
+// attention moves onto the pure fak kernel", "What changed": online softmax,
+// key width kd != value width vd; metrale glm5next_dsa_ref topk_to_mask and
+// mla_masked_attention).  The key is the shared latent row c_i (kd = 512 or
+// 576 columns) and the value is its first vd = 512 columns.
+//
+// Heads are the MMA M dimension (128 rows; fewer heads leave rows unused).  A
+// 128 x 512 fp32 output accumulator fills all of one SM's tensor memory, so a
+// query is processed by a cluster of two CTAs:
+//   CTA rank 0 owns latent columns [0, 256):   q.k partial over them, O[:, 0:256)
+//   CTA rank 1 owns latent columns [256, kd):  q.k partial over them, O[:, 256:512)
+// Each CTA gathers only its own columns of every selected latent row (cp.async,
+// written straight into the 128-byte-swizzled operand layout), so no byte is
+// loaded twice.  After each 32-key chunk the two fp32 partial score tiles are
+// exchanged through distributed shared memory and summed; fp32 addition is
+// commutative, so both CTAs see bit-identical scores and take identical
+// online-softmax decisions.  P (bf16) goes to shared memory and each CTA
+// accumulates P.V for its 256 value columns in TMEM.  The running maximum is
+// only moved (and O rescaled in TMEM) when it grows by more than 2^8.
+//
+// Warp roles per CTA: warps 0-3 softmax + epilogue (one head row per thread,
+// TMEM lanes 0-127), warp 4 tcgen05.mma issue, warps 5-6 index-row dedupe and
+// cp.async gathers, warp 7 TMA of the query tile.  Every mbarrier wait is bounded.
+#include <cuda.h>
+
+#include "dsa_common.cuh"
 #include "dsa_internal.h"
+#include "dsa_sm100.cuh"
+
 namespace dsa {
-bool attend_tc_supported(const dsa_dims&, int64_t, const void*, const void*, int64_t, int) { return false; }
-cudaError_t launch_attend_tc(const dsa_dims&, const void*, const void*, int64_t, const int32_t*, int,
-                             float, void*, float*, cudaStream_t) { return cudaErrorNotSupported; }
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kChunk = 32;            // keys per pipeline step (MMA N of q.k, K of P.V)
+constexpr int kStages = 3;            // gathered key/value stages
+constexpr int kSBufs = 4;             // score buffers in TMEM
+constexpr int kMaxLocalBlocks = 5;    // 64-column blocks per CTA (rank 1 with kd = 576)
+constexpr int kBlockBytes = kChunk * 128;                  // one 64-col block of a stage: 4 KB
+constexpr int kStageBytes = kMaxLocalBlocks * kBlockBytes; // 20 KB
+constexpr int kQBlockBytes = 128 * 128;                    // 128 rows x 64 cols bf16: 16 KB
+constexpr int kPBytes = 128 * kChunk * 2;                  // 8 KB
+constexpr int kXStride = kChunk + 4;                       // floats per exchange row (bank padding)
+constexpr int kXBytes = 128 * kXStride * 4;                // 18 KB
+constexpr int kBitmapKeys = 65536;
+constexpr int kOCol = kSBufs * kChunk;                     // first TMEM column of O
+constexpr int kThreads = 256;
+constexpr int kProducerThreads = 64;
+
+struct AttTcParams {
+  int B, T, S, H, kd, width;
+  long long stride;          // latent row stride in elements
+  const bf16* latent;
+  const int32_t* idx;
+  float scale_log2;          // softmax scale * log2(e)
+  bf16* out;                 // [B,T,H,512]
+  float* lse;                // [B,T,H] or null
+  int* status;
+};
+
+struct Smem {
+  uint32_t q, kv, p, x;      // shared-window addresses
+  int* list;
+  uint32_t* bitmap;
+  uint64_t *qfull, *list_ready, *kv_full, *kv_empty, *s_full, *s_empty, *p_full, *o_done, *xfull, *drain;
+  uint32_t* tmem_slot;
+  int* n_list;
+  int* dup_flag;
+  int* abort_flag;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
 }
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_peer(uint32_t addr, uint32_t peer) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(peer));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+__device__ __forceinline__ void arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ bool try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool wait_cluster(uint32_t bar, uint32_t parity, int* status, volatile int* abort_flag) {
+  if (try_wait_cluster(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (try_wait_cluster(bar, parity)) return true;
+    if ((it & 63u) == 0u) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        record_status(status, DSA_ERR_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Shared-memory descriptor of a K-major operand without swizzle: 8x16-byte core
+// matrices, `lbo` bytes between core matrices along K, `sbo` along M/N.
+__device__ __forceinline__ uint64_t desc_noswz(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+
+// Builds the row's key list: distinct in-range entries in index-row order.
+// Deterministic, so both CTAs of the cluster obtain the same list.
+__device__ void build_list(const AttTcParams& p, const Smem& sm, size_t row) {
+  const int tid = threadIdx.x - (kThreads - 3 * 32);  // 0..63 over warps 5,6
+  const int lane = threadIdx.x & 31;
+  const bool lead = tid < 32;                          // warp 5
+  const int32_t* irow = p.idx + row * p.width;
+  const int words = (p.S + 31) >> 5;
+  for (int i = tid; i < words; i += kProducerThreads) sm.bitmap[i] = 0u;
+  if (tid == 0) *sm.dup_flag = 0;
+  named_sync(1, kProducerThreads);
+  int dup = 0;
+  for (int e = tid; e < p.width; e += kProducerThreads) {
+    const int key = irow[e];
+    if (key >= 0 && key < p.S) {
+      const uint32_t bit = 1u << (key & 31);
+      dup |= (atomicOr(&sm.bitmap[key >> 5], bit) & bit) != 0u;
+    }
+  }
+  if (__any_sync(0xffffffffu, dup) && lane == 0) *sm.dup_flag = 1;
+  named_sync(1, kProducerThreads);
+  const bool has_dup = *sm.dup_flag != 0;
+  if (has_dup) {
+    for (int i = tid; i < words; i += kProducerThreads) sm.bitmap[i] = 0u;
+    named_sync(1, kProducerThreads);
+  }
+  if (lead) {
+    int n = 0;
+    for (int e0 = 0; e0 < p.width; e0 += 32) {
+      const int e = e0 + lane;
+      const int key = e < p.width ? irow[e] : -1;
+      bool keep = key >= 0 && key < p.S;
+      if (has_dup) {
+        // first occurrence only: not seen in an earlier group, lowest lane in this group
+        const uint32_t peers = __match_any_sync(0xffffffffu, keep ? key : -1);
+        if (keep) {
+          keep = (sm.bitmap[key >> 5] & (1u << (key & 31))) == 0u && lane == __ffs(peers) - 1;
+        }
+        __syncwarp();
+        if (keep) atomicOr(&sm.bitmap[key >> 5], 1u << (key & 31));
+        __syncwarp();
+      }
+      const uint32_t m = __ballot_sync(0xffffffffu, keep);
+      if (keep) sm.list[n + __popc(m & ((1u << lane) - 1u))] = key;
+      n += __popc(m);
+    }
+    if (lane == 0) {
+      *sm.n_list = n;
+      mbar_arrive(smem_u32(sm.list_ready));
+    }
+  }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, AttTcParams p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  __shared__ int s_misc[4];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* gb = smem_raw + (base - raw);
+  Smem sm;
+  sm.q = base;
+  sm.kv = sm.q + kMaxLocalBlocks * kQBlockBytes;
+  sm.p = sm.kv + kStages * kStageBytes;
+  sm.x = sm.p + 2 * kPBytes;
+  uint32_t off = sm.x + 2 * kXBytes - base;
+  sm.list = reinterpret_cast<int*>(gb + off);
+  off += ((uint32_t)p.width * 4u + 15u) & ~15u;
+  sm.bitmap = reinterpret_cast<uint32_t*>(gb + off);
+  off += kBitmapKeys / 8;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gb + off);
+  sm.qfull = bars;
+  sm.list_ready = bars + 1;
+  sm.kv_full = bars + 2;
+  sm.kv_empty = sm.kv_full + kStages;
+  sm.s_full = sm.kv_empty + kStages;
+  sm.s_empty = sm.s_full + kSBufs;
+  sm.p_full = sm.s_empty + kSBufs;
+  sm.o_done = sm.p_full + 2;
+  sm.xfull = sm.o_done + 2;
+  sm.drain = sm.xfull + 2;
+  sm.tmem_slot = reinterpret_cast<uint32_t*>(sm.drain + 1);
+  sm.n_list = &s_misc[0];
+  sm.dup_flag = &s_misc[1];
+  sm.abort_flag = &s_misc[2];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const uint32_t peer = rank ^ 1u;
+  const size_t row = blockIdx.x >> 1;            // query row b*T + t
+  const int nkb_total = p.kd / 64;
+  const int kb0 = rank ? 4 : 0;                  // first global 64-col block of this CTA
+  const int nkb = rank ? nkb_total - 4 : 4;      // blocks this CTA owns (q.k); the first 4 are its V
+
+  if (threadIdx.x == 0) {
+    *sm.abort_flag = 0;
+    mbar_init(smem_u32(sm.qfull), 1);
+    mbar_init(smem_u32(sm.list_ready), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&sm.kv_full[s]), kProducerThreads);
+      mbar_init(smem_u32(&sm.kv_empty[s]), 1);
+    }
+    for (int s = 0; s < kSBufs; ++s) {
+      mbar_init(smem_u32(&sm.s_full[s]), 1);
+      mbar_init(smem_u32(&sm.s_empty[s]), 4);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&sm.p_full[s]), 4);
+      mbar_init(smem_u32(&sm.o_done[s]), 1);
+      mbar_init(smem_u32(&sm.xfull[s]), 128);
+    }
+    mbar_init(smem_u32(sm.drain), 1);
+    fence_barrier_init();
+  }
+  if (warp == 4) tmem_alloc(smem_u32(sm.tmem_slot), 512);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the peer's barriers are initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem = *sm.tmem_slot;
+  volatile int* abort_flag = sm.abort_flag;
+
+  if (warp == 7) {
+    // ---------------------------------------------------------------- query tile (TMA)
+    if (lane == 0) {
+      tma_prefetch_desc(&map_q);
+      mbar_arrive_expect_tx(smem_u32(sm.qfull), (uint32_t)nkb * kQBlockBytes);
+      for (int kb = 0; kb < nkb; ++kb)
+        tma_load_2d(sm.q + kb * kQBlockBytes, &map_q, smem_u32(sm.qfull), (kb0 + kb) * 64, (int)(row * p.H));
+    }
+  } else if (warp == 5 || warp == 6) {
+    // ---------------------------------------------------------------- list + gathers
+    build_list(p, sm, row);
+    named_sync(1, kProducerThreads);
+    const int n = *sm.n_list;
+    const int nch = (n + kChunk - 1) / kChunk;
+    const int tid = threadIdx.x - 5 * 32;
+    const int b = (int)(row / p.T);
+    const bf16* lat = p.latent + (size_t)b * p.S * p.stride + kb0 * 64;
+    const int segs = nkb * 8;                       // 16-byte segments per key row
+    const int per_chunk = kChunk * segs;
+    for (int j = 0; j < nch; ++j) {
+      const int s = j % kStages;
+      if (!mbar_wait(smem_u32(&sm.kv_empty[s]), ((j / kStages) & 1) ^ 1, p.status, abort_flag)) break;
+      const uint32_t st = sm.kv + s * kStageBytes;
+      for (int i = tid; i < per_chunk; i += kProducerThreads) {
+        const int r = i / segs, sg = i - r * segs;      // key row in chunk, segment in row
+        const int kb = sg >> 3, c = sg & 7;
+        const int li = j * kChunk + r;
+        const bool ok = li < n;                          // rows past the list are zero-filled
+        const int key = ok ? sm.list[li] : 0;
+        const bf16* src = lat + (size_t)key * p.stride + sg * 8;
+        const uint32_t dst = st + kb * kBlockBytes + r * 128 + ((c ^ (r & 7)) << 4);
+        cp_async_16(dst, src, ok);
+      }
+      // arrives on kv_full[s] once this thread's copies have landed
+      cp_async_mbar_arrive(smem_u32(&sm.kv_full[s]));
+    }
+    cp_async_wait_all();
+  } else if (warp == 4) {
+    // ---------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      const uint32_t id_qk = idesc_bf16(128, kChunk);
+      const uint32_t id_pv = idesc_bf16(128, 256, false, true);
+      bool ok = mbar_wait(smem_u32(sm.qfull), 0, p.status, abort_flag) &&
+                mbar_wait(smem_u32(sm.list_ready), 0, p.status, abort_flag);
+      const int n = ok ? *sm.n_list : 0;
+      const int nch = (n + kChunk - 1) / kChunk;
+      auto issue_qk = [&](int j) -> bool {
+        const int s = j % kStages, sb = j % kSBufs;
+        if (!mbar_wait(smem_u32(&sm.kv_full[s]), (j / kStages) & 1, p.status, abort_flag)) return false;
+        if (!mbar_wait(smem_u32(&sm.s_empty[sb]), ((j / kSBufs) & 1) ^ 1, p.status, abort_flag)) return false;
+        fence_proxy_async_smem();
+        tc_fence_after();
+        const uint32_t st = sm.kv + s * kStageBytes;
+        for (int kb = 0; kb < nkb; ++kb) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad = desc_sw128(sm.q + kb * kQBlockBytes + k * 32);
+            const uint64_t bd = desc_sw128(st + kb * kBlockBytes + k * 32);
+            mma_bf16_ss(tmem + sb * kChunk, ad, bd, id_qk, (kb | k) ? 1u : 0u);
+          }
+        }
+        mma_commit(smem_u32(&sm.s_full[sb]));
+        return true;
+      };
+      if (nch > 0) ok = issue_qk(0);
+      for (int j = 0; ok && j < nch; ++j) {
+        if (j + 1 < nch && !(ok = issue_qk(j + 1))) break;
+        if (!(ok = mbar_wait(smem_u32(&sm.p_full[j & 1]), (j >> 1) & 1, p.status, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t pa = sm.p + (j & 1) * kPBytes;
+        const uint32_t st = sm.kv + (j % kStages) * kStageBytes;
+#pragma unroll
+        for (int k = 0; k < kChunk / 16; ++k) {
+          const uint64_t ad = desc_noswz(pa + k * 256, 128, 512);
+          const uint64_t bd = desc_sw128(st + k * 2048, 1024, kBlockBytes);
+          mma_bf16_ss(tmem + kOCol, ad, bd, id_pv, (j | k) ? 1u : 0u);
+        }
+        mma_commit(smem_u32(&sm.kv_empty[j % kStages]));
+        mma_commit(smem_u32(&sm.o_done[j & 1]));
+      }
+      mma_commit(smem_u32(sm.drain));
+      mbar_wait(smem_u32(sm.drain), 0, nullptr, nullptr);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax + epilogue
+    const int r = warp * 32 + lane;                 // head row == TMEM lane
+    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+    float m_ref = -INFINITY, l_sum = 0.f;
+    bool ok = mbar_wait(smem_u32(sm.list_ready), 0, p.status, abort_flag);
+    const int n = ok ? *sm.n_list : 0;
+    const int nch = (n + kChunk - 1) / kChunk;
+    const uint32_t x_local = sm.x + (uint32_t)r * kXStride * 4;
+    const uint32_t x_peer = map_peer(x_local, peer);
+    const uint32_t xfull_peer[2] = {map_peer(smem_u32(&sm.xfull[0]), peer), map_peer(smem_u32(&sm.xfull[1]), peer)};
+    const float* xrow = reinterpret_cast<const float*>(gb + (sm.x - base)) + r * kXStride;
+    for (int j = 0; ok && j < nch; ++j) {
+      const int sb = j % kSBufs, xb = j & 1;
+      if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), (j / kSBufs) & 1, p.status, abort_flag))) break;
+      tc_fence_after();
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk, v);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty[sb]));
+      // exchange partial scores with the peer CTA
+      const uint32_t xo = (uint32_t)xb * kXBytes;
+#pragma unroll
+      for (int c = 0; c < kChunk; c += 4)
+        st_cluster_v4(x_peer + xo + c * 4, __uint_as_float(v[c]), __uint_as_float(v[c + 1]),
+                      __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+      arrive_remote(xfull_peer[xb]);
+      if (!(ok = wait_cluster(smem_u32(&sm.xfull[xb]), (j >> 1) & 1, p.status, abort_flag))) break;
+      const float* xr = xrow + xb * (kXBytes / 4);
+      const int valid = n - j * kChunk;
+      float x[kChunk];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kChunk; ++c) {
+        const float s = __uint_as_float(v[c]) + xr[c];
+        x[c] = c < valid ? s * p.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, x[c]);
+      }
+      // move the reference maximum only when it grows by more than 2^8
+      const bool grow = mx > m_ref + 8.f;
+      const float new_ref = grow ? mx : m_ref;
+      if (__any_sync(0xffffffffu, grow && j > 0)) {
+        if (!(ok = mbar_wait(smem_u32(&sm.o_done[(j - 1) & 1]), ((j - 1) >> 1) & 1, p.status, abort_flag))) break;
+        tc_fence_after();
+        const float f = (grow && j > 0) ? exp2f(m_ref - new_ref) : 1.f;
+        for (int c = 0; c < 256; c += 16) {
+          uint32_t o[16];
+          tmem_ld_32x32b_x16(tmem + lane_addr + kOCol + c, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+          tmem_st_32x32b_x16(tmem + lane_addr + kOCol + c, o);
+        }
+        tmem_st_wait();
+        l_sum *= f;
+      }
+      m_ref = new_ref;
+      float ps[kChunk];
+#pragma unroll
+      for (int c = 0; c < kChunk; ++c) {
+        ps[c] = exp2f(x[c] - m_ref);
+        l_sum += ps[c];
+      }
+      // P buffer (j&1) is free once the P.V of chunk j-2 has completed
+      if (j >= 2 && !(ok = mbar_wait(smem_u32(&sm.o_done[j & 1]), ((j - 2) >> 1) & 1, p.status, abort_flag))) break;
+      const uint32_t prow = sm.p + xb * kPBytes + (uint32_t)(r >> 3) * 512 + (uint32_t)(r & 7) * 16;
+#pragma unroll
+      for (int kc = 0; kc < kChunk / 8; ++kc) {
+        const uint32_t a0 = pack_bf16(ps[8 * kc + 0], ps[8 * kc + 1]);
+        const uint32_t a1 = pack_bf16(ps[8 * kc + 2], ps[8 * kc + 3]);
+        const uint32_t a2 = pack_bf16(ps[8 * kc + 4], ps[8 * kc + 5]);
+        const uint32_t a3 = pack_bf16(ps[8 * kc + 6], ps[8 * kc + 7]);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + kc * 128), "r"(a0), "r"(a1),
+                     "r"(a2), "r"(a3)
+                     : "memory");
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[xb]));
+    }
+    // epilogue: O / l -> bf16
+    const bool write = r < p.H;
+    bf16* orow = p.out + (row * p.H + r) * 512 + rank * 256;
+    if (ok && nch > 0) {
+      ok = mbar_wait(smem_u32(&sm.o_done[(nch - 1) & 1]), ((nch - 1) >> 1) & 1, p.status, abort_flag);
+      tc_fence_after();
+      const float inv = 1.f / l_sum;
+      for (int c = 0; c < 256; c += 32) {
+        uint32_t o[32];
+        tmem_ld_32x32b_x32(tmem + lane_addr + kOCol + c, o);
+        tmem_ld_wait();
+        if (write && ok) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 pk;
+            pk.x = pack_bf16(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
+            pk.y = pack_bf16(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+            pk.z = pack_bf16(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
+            pk.w = pack_bf16(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + c + i) = pk;
+          }
+        }
+      }
+      if (write && ok && rank == 0 && p.lse) p.lse[row * p.H + r] = (m_ref + log2f(l_sum)) * 0.69314718055994531f;
+    } else if (ok && write) {
+      for (int c = 0; c < 256; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+      if (rank == 0 && p.lse) p.lse[row * p.H + r] = -INFINITY;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no remote access to a CTA that has exited
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+    tmem_relinquish();
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)ptr;
+  }
+  return fn;
+}
+
+size_t smem_bytes(int width) {
+  return 1024 + (size_t)kMaxLocalBlocks * kQBlockBytes + (size_t)kStages * kStageBytes + 2 * kPBytes +
+         2 * kXBytes + (((size_t)width * 4 + 15) & ~(size_t)15) + kBitmapKeys / 8 + 8 * 32 + 16;
+}
+
+}  // namespace
+
+bool attend_tc_supported(const dsa_dims& d, int64_t k_stride, const void* k, const void* v, int64_t v_stride,
+                         int width) {
+  if (d.dtype != DSA_BF16 || d.kv_heads != 1 || d.vd != 512) return false;
+  if (!(d.kd == 512 || d.kd == 576)) return false;
+  if (!(d.heads == 64 || d.heads == 128)) return false;
+  if ((long long)d.batch * d.n_q * d.heads < 128) return false;  // the query TMA box is 128 rows
+  if (k != v || k_stride != v_stride || k_stride < d.kd || (k_stride * 2) % 16 != 0) return false;
+  if (((uintptr_t)k & 15u) != 0) return false;
+  if (d.n_kv > kBitmapKeys || width > 8192) return false;
+  if (smem_bytes(width) > 227 * 1024) return false;
+  return encode_fn() != nullptr;
+}
+
+cudaError_t launch_attend_tc(const dsa_dims& d, const void* q, const void* k, int64_t k_stride,
+                             const int32_t* idx, int width, float scale, void* out, float* lse,
+                             cudaStream_t st) {
+  AttTcParams p{};
+  p.B = d.batch;
+  p.T = d.n_q;
+  p.S = d.n_kv;
+  p.H = d.heads;
+  p.kd = d.kd;
+  p.width = width;
+  p.stride = k_stride;
+  p.latent = (const bf16*)k;
+  p.idx = idx;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.out = (bf16*)out;
+  p.lse = lse;
+  p.status = device_status_ptr();
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  // q viewed as [B*T*H rows, kd cols]; box = 64 cols x 128 rows, 128-byte swizzle
+  CUtensorMap mq;
+  cuuint64_t dims[2] = {(cuuint64_t)d.kd, (cuuint64_t)d.batch * d.n_q * d.heads};
+  cuuint64_t strides[1] = {(cuuint64_t)d.kd * 2};
+  cuuint32_t box[2] = {64u, 128u};
+  cuuint32_t estr[2] = {1u, 1u};
+  if (enc(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const size_t smem = smem_bytes(width);
+  cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const long long rows = (long long)d.batch * d.n_q;
+  attend_tc_kernel<<<dim3((unsigned)(2 * rows)), kThreads, smem, st>>>(mq, p);
+  return cudaGetLastError();
+}
+
+}  // namespace dsa

@@ -225,6 +225,40 @@ def test_small_bf16_layer_against_oracle(name, sizes):
     assert n_diff_rows <= max(1, len(rows) // 10)
 
 
+# ------------------------------------------- tensor cores vs CUDA cores
+@pytest.mark.parametrize("name,sizes,top_k", [("prefill", dict(T=300), 96), ("decode", dict(B=2, S=4100), 2048)])
+def test_tensor_core_kernels_match_cuda_core_kernels(name, sizes, top_k):
+    """Same inputs through both kernel families (dsa_set_kernel_policy)."""
+    wl = workloads.make(name, **sizes)
+    wl.top_k = top_k
+    t = dev(wl)
+    try:
+        dsa.set_kernel_policy(1)
+        _, _, sc_simt, idx_simt, _, out_simt, lse_simt = _run_stages(wl, t)
+        dsa.set_kernel_policy(0)
+        _, _, sc_tc, idx_tc, _, out_tc, lse_tc = _run_stages(wl, t)
+    finally:
+        dsa.set_kernel_policy(0)
+    fin = torch.isfinite(sc_simt)
+    assert torch.equal(fin, torch.isfinite(sc_tc))
+    scale_ = sc_simt[fin].abs().max().clamp(min=1.0)
+    assert (sc_simt[fin] - sc_tc[fin]).abs().max() <= 2e-5 * scale_
+    # attend both families over the same selection
+    dims, a = layer_inputs(wl, t)
+    outs = []
+    for pol in (1, 0):
+        dsa.set_kernel_policy(pol)
+        o = torch.empty_like(out_tc)
+        l = torch.empty_like(lse_tc)
+        dsa.sparse_attend(dims, a["q"], a["k"], a["k_row_stride"], a["v"], a["v_row_stride"], idx_simt,
+                          wl.top_k, a["attn_scale"], o, l)
+        outs.append((o, l))
+    dsa.set_kernel_policy(0)
+    torch.cuda.synchronize()
+    assert_attend_close(_np(outs[1][0]), _np(outs[0][0]), torch.bfloat16, "tc vs simt attend")
+    assert (outs[1][1] - outs[0][1]).abs().max().item() <= 2e-3
+
+
 # ------------------------------------------------------------- kpool (small)
 def _kpool_run(wl):
     t = dev(wl)
