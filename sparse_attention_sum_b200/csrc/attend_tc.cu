@@ -22,8 +22,12 @@
 // only moved (and O rescaled in TMEM) when it grows by more than 2^8.
 //
 // Warp roles per CTA: warps 0-3 softmax + epilogue (one head row per thread,
-// TMEM lanes 0-127), warp 4 tcgen05.mma issue, warps 5-6 index-row dedupe and
-// cp.async gathers, warp 7 TMA of the query tile.  Every mbarrier wait is bounded.
+// TMEM lanes 0-127); warps 8-11 read the same score rows and push them to the
+// peer ahead of the softmax (buffer reuse acknowledged by the peer's softmax);
+// warp 4 issues tcgen05.mma from a polling scheduler that lets q.k run up to
+// three chunks ahead of P.V; warps 5-6 deduplicate the index row and gather
+// the selected rows with cp.async; warp 7 loads the query tile by TMA.  Every
+// mbarrier wait is bounded.
 #include <cuda.h>
 
 #include "dsa_common.cuh"
@@ -37,7 +41,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kChunk = 32;            // keys per pipeline step (MMA N of q.k, K of P.V)
-constexpr int kStages = 3;            // gathered key/value stages
+constexpr int kStages = 4;            // gathered key/value stages
 constexpr int kSBufs = 4;             // score buffers in TMEM
 constexpr int kMaxLocalBlocks = 5;    // 64-column blocks per CTA (rank 1 with kd = 576)
 constexpr int kBlockBytes = kChunk * 128;                  // one 64-col block of a stage: 4 KB
@@ -48,7 +52,7 @@ constexpr int kXStride = kChunk + 4;                       // floats per exchang
 constexpr int kXBytes = 128 * kXStride * 4;                // 18 KB
 constexpr int kBitmapKeys = 65536;
 constexpr int kOCol = kSBufs * kChunk;                     // first TMEM column of O
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr int kProducerThreads = 64;
 
 struct AttTcParams {
@@ -66,7 +70,7 @@ struct Smem {
   uint32_t q, kv, p, x;      // shared-window addresses
   int* list;
   uint32_t* bitmap;
-  uint64_t *qfull, *list_ready, *kv_full, *kv_empty, *s_full, *s_empty, *p_full, *o_done, *xfull, *drain;
+  uint64_t *qfull, *list_ready, *kv_full, *kv_empty, *s_full, *s_empty, *p_full, *o_done, *xfull, *xfree, *drain;
   uint32_t* tmem_slot;
   int* n_list;
   int* dup_flag;
@@ -141,7 +145,7 @@ __device__ __forceinline__ uint64_t desc_noswz(uint32_t saddr, uint32_t lbo, uin
 // Builds the row's key list: distinct in-range entries in index-row order.
 // Deterministic, so both CTAs of the cluster obtain the same list.
 __device__ void build_list(const AttTcParams& p, const Smem& sm, size_t row) {
-  const int tid = threadIdx.x - (kThreads - 3 * 32);  // 0..63 over warps 5,6
+  const int tid = threadIdx.x - 5 * 32;               // 0..63 over warps 5,6
   const int lane = threadIdx.x & 31;
   const bool lead = tid < 32;                          // warp 5
   const int32_t* irow = p.idx + row * p.width;
@@ -199,15 +203,15 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, AttTcParams p) {
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* gb = smem_raw + (base - raw);
   Smem sm;
-  sm.q = base;
+  sm.x = base;                                   // peer-written: same offset in both CTAs
+  sm.q = sm.x + 2 * kXBytes;
+  sm.q = (sm.q + 1023u) & ~1023u;
   sm.kv = sm.q + kMaxLocalBlocks * kQBlockBytes;
   sm.p = sm.kv + kStages * kStageBytes;
-  sm.x = sm.p + 2 * kPBytes;
-  uint32_t off = sm.x + 2 * kXBytes - base;
+  uint32_t off = sm.p + 2 * kPBytes - base;
+  sm.bitmap = reinterpret_cast<uint32_t*>(gb + (sm.p - base));  // aliases P: used before the first P
   sm.list = reinterpret_cast<int*>(gb + off);
   off += ((uint32_t)p.width * 4u + 15u) & ~15u;
-  sm.bitmap = reinterpret_cast<uint32_t*>(gb + off);
-  off += kBitmapKeys / 8;
   uint64_t* bars = reinterpret_cast<uint64_t*>(gb + off);
   sm.qfull = bars;
   sm.list_ready = bars + 1;
@@ -218,7 +222,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, AttTcParams p) {
   sm.p_full = sm.s_empty + kSBufs;
   sm.o_done = sm.p_full + 2;
   sm.xfull = sm.o_done + 2;
-  sm.drain = sm.xfull + 2;
+  sm.xfree = sm.xfull + 2;
+  sm.drain = sm.xfree + 2;
   sm.tmem_slot = reinterpret_cast<uint32_t*>(sm.drain + 1);
   sm.n_list = &s_misc[0];
   sm.dup_flag = &s_misc[1];
@@ -242,12 +247,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, AttTcParams p) {
     }
     for (int s = 0; s < kSBufs; ++s) {
       mbar_init(smem_u32(&sm.s_full[s]), 1);
-      mbar_init(smem_u32(&sm.s_empty[s]), 4);
+      mbar_init(smem_u32(&sm.s_empty[s]), 8);   // softmax and exchange warps both read S
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&sm.p_full[s]), 4);
       mbar_init(smem_u32(&sm.o_done[s]), 1);
-      mbar_init(smem_u32(&sm.xfull[s]), 128);
+      mbar_init(smem_u32(&sm.xfull[s]), 128);   // the peer's exchange threads
+      mbar_init(smem_u32(&sm.xfree[s]), 128);   // the peer's softmax threads
     }
     mbar_init(smem_u32(sm.drain), 1);
     fence_barrier_init();
@@ -306,44 +312,93 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, AttTcParams p) {
                 mbar_wait(smem_u32(sm.list_ready), 0, p.status, abort_flag);
       const int n = ok ? *sm.n_list : 0;
       const int nch = (n + kChunk - 1) / kChunk;
-      auto issue_qk = [&](int j) -> bool {
-        const int s = j % kStages, sb = j % kSBufs;
-        if (!mbar_wait(smem_u32(&sm.kv_full[s]), (j / kStages) & 1, p.status, abort_flag)) return false;
-        if (!mbar_wait(smem_u32(&sm.s_empty[sb]), ((j / kSBufs) & 1) ^ 1, p.status, abort_flag)) return false;
-        fence_proxy_async_smem();
-        tc_fence_after();
-        const uint32_t st = sm.kv + s * kStageBytes;
-        for (int kb = 0; kb < nkb; ++kb) {
+      // q.k of chunk j may run ahead of P.V of chunk pv while stages and score buffers allow
+      int qk = 0, pv = 0;
+      unsigned long long t_last = globaltimer();
+      uint32_t spins = 0;
+      while (ok && pv < nch) {
+        bool progressed = false;
+        if (qk < nch && qk - pv < kStages - 1 &&
+            mbar_try_wait(smem_u32(&sm.kv_full[qk % kStages]), (qk / kStages) & 1) &&
+            mbar_try_wait(smem_u32(&sm.s_empty[qk % kSBufs]), ((qk / kSBufs) & 1) ^ 1)) {
+          fence_proxy_async_smem();
+          tc_fence_after();
+          const uint32_t st = sm.kv + (qk % kStages) * kStageBytes;
+          const uint32_t d = tmem + (qk % kSBufs) * kChunk;
+          for (int kb = 0; kb < nkb; ++kb) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = desc_sw128(sm.q + kb * kQBlockBytes + k * 32);
-            const uint64_t bd = desc_sw128(st + kb * kBlockBytes + k * 32);
-            mma_bf16_ss(tmem + sb * kChunk, ad, bd, id_qk, (kb | k) ? 1u : 0u);
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t ad = desc_sw128(sm.q + kb * kQBlockBytes + k * 32);
+              const uint64_t bd = desc_sw128(st + kb * kBlockBytes + k * 32);
+              mma_bf16_ss(d, ad, bd, id_qk, (kb | k) ? 1u : 0u);
+            }
+          }
+          mma_commit(smem_u32(&sm.s_full[qk % kSBufs]));
+          ++qk;
+          progressed = true;
+        }
+        if (pv < qk && mbar_try_wait(smem_u32(&sm.p_full[pv & 1]), (pv >> 1) & 1)) {
+          tc_fence_after();
+          const uint32_t pa = sm.p + (pv & 1) * kPBytes;
+          const uint32_t st = sm.kv + (pv % kStages) * kStageBytes;
+#pragma unroll
+          for (int k = 0; k < kChunk / 16; ++k) {
+            const uint64_t ad = desc_noswz(pa + k * 256, 128, 512);
+            const uint64_t bd = desc_sw128(st + k * 2048, 1024, kBlockBytes);
+            mma_bf16_ss(tmem + kOCol, ad, bd, id_pv, (pv | k) ? 1u : 0u);
+          }
+          mma_commit(smem_u32(&sm.kv_empty[pv % kStages]));
+          mma_commit(smem_u32(&sm.o_done[pv & 1]));
+          ++pv;
+          progressed = true;
+        }
+        if (progressed) {
+          spins = 0;
+        } else if ((++spins & 255u) == 0u) {
+          const unsigned long long now = globaltimer();
+          if (*abort_flag) break;
+          if (spins == 256u) t_last = now;
+          else if (now - t_last > kWaitLimitNs) {
+            record_status(p.status, DSA_ERR_TIMEOUT);
+            *abort_flag = 1;
+            break;
           }
         }
-        mma_commit(smem_u32(&sm.s_full[sb]));
-        return true;
-      };
-      if (nch > 0) ok = issue_qk(0);
-      for (int j = 0; ok && j < nch; ++j) {
-        if (j + 1 < nch && !(ok = issue_qk(j + 1))) break;
-        if (!(ok = mbar_wait(smem_u32(&sm.p_full[j & 1]), (j >> 1) & 1, p.status, abort_flag))) break;
-        tc_fence_after();
-        const uint32_t pa = sm.p + (j & 1) * kPBytes;
-        const uint32_t st = sm.kv + (j % kStages) * kStageBytes;
-#pragma unroll
-        for (int k = 0; k < kChunk / 16; ++k) {
-          const uint64_t ad = desc_noswz(pa + k * 256, 128, 512);
-          const uint64_t bd = desc_sw128(st + k * 2048, 1024, kBlockBytes);
-          mma_bf16_ss(tmem + kOCol, ad, bd, id_pv, (j | k) ? 1u : 0u);
-        }
-        mma_commit(smem_u32(&sm.kv_empty[j % kStages]));
-        mma_commit(smem_u32(&sm.o_done[j & 1]));
       }
       mma_commit(smem_u32(sm.drain));
       mbar_wait(smem_u32(sm.drain), 0, nullptr, nullptr);
     }
-  } else {
+  } else if (warp >= 8) {
+    // ---------------------------------------------------------------- score exchange
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
+    bool ok = mbar_wait(smem_u32(sm.list_ready), 0, p.status, abort_flag);
+    const int n = ok ? *sm.n_list : 0;
+    const int nch = (n + kChunk - 1) / kChunk;
+    const uint32_t x_peer = map_peer(sm.x + (uint32_t)r * kXStride * 4, peer);
+    const uint32_t xfull_peer0 = map_peer(smem_u32(&sm.xfull[0]), peer);
+    const uint32_t xfull_peer1 = map_peer(smem_u32(&sm.xfull[1]), peer);
+    for (int j = 0; ok && j < nch; ++j) {
+      const int sb = j % kSBufs, xb = j & 1;
+      if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), (j / kSBufs) & 1, p.status, abort_flag))) break;
+      tc_fence_after();
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk, v);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty[sb]));
+      // the peer has finished reading its buffer xb from chunk j-2
+      if (!(ok = wait_cluster(smem_u32(&sm.xfree[xb]), ((j >> 1) & 1) ^ 1, p.status, abort_flag))) break;
+      const uint32_t dst = x_peer + (uint32_t)xb * kXBytes;
+#pragma unroll
+      for (int c = 0; c < kChunk; c += 4)
+        st_cluster_v4(dst + c * 4, __uint_as_float(v[c]), __uint_as_float(v[c + 1]), __uint_as_float(v[c + 2]),
+                      __uint_as_float(v[c + 3]));
+      arrive_remote(xb ? xfull_peer1 : xfull_peer0);
+    }
+  } else if (warp < 4) {
     // ---------------------------------------------------------------- softmax + epilogue
     const int r = warp * 32 + lane;                 // head row == TMEM lane
     const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
@@ -351,9 +406,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, AttTcParams p) {
     bool ok = mbar_wait(smem_u32(sm.list_ready), 0, p.status, abort_flag);
     const int n = ok ? *sm.n_list : 0;
     const int nch = (n + kChunk - 1) / kChunk;
-    const uint32_t x_local = sm.x + (uint32_t)r * kXStride * 4;
-    const uint32_t x_peer = map_peer(x_local, peer);
-    const uint32_t xfull_peer[2] = {map_peer(smem_u32(&sm.xfull[0]), peer), map_peer(smem_u32(&sm.xfull[1]), peer)};
+    const uint32_t xfree_peer0 = map_peer(smem_u32(&sm.xfree[0]), peer);
+    const uint32_t xfree_peer1 = map_peer(smem_u32(&sm.xfree[1]), peer);
     const float* xrow = reinterpret_cast<const float*>(gb + (sm.x - base)) + r * kXStride;
     for (int j = 0; ok && j < nch; ++j) {
       const int sb = j % kSBufs, xb = j & 1;
@@ -365,13 +419,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, AttTcParams p) {
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty[sb]));
-      // exchange partial scores with the peer CTA
-      const uint32_t xo = (uint32_t)xb * kXBytes;
-#pragma unroll
-      for (int c = 0; c < kChunk; c += 4)
-        st_cluster_v4(x_peer + xo + c * 4, __uint_as_float(v[c]), __uint_as_float(v[c + 1]),
-                      __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
-      arrive_remote(xfull_peer[xb]);
       if (!(ok = wait_cluster(smem_u32(&sm.xfull[xb]), (j >> 1) & 1, p.status, abort_flag))) break;
       const float* xr = xrow + xb * (kXBytes / 4);
       const int valid = n - j * kChunk;
@@ -379,10 +426,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, AttTcParams p) {
       float mx = -INFINITY;
 #pragma unroll
       for (int c = 0; c < kChunk; ++c) {
-        const float s = __uint_as_float(v[c]) + xr[c];
-        x[c] = c < valid ? s * p.scale_log2 : -INFINITY;
+        const float sc = __uint_as_float(v[c]) + xr[c];
+        x[c] = c < valid ? sc * p.scale_log2 : -INFINITY;
         mx = fmaxf(mx, x[c]);
       }
+      // partner buffer xb is read: the peer may refill it
+      arrive_remote(xb ? xfree_peer1 : xfree_peer0);
       // move the reference maximum only when it grows by more than 2^8
       const bool grow = mx > m_ref + 8.f;
       const float new_ref = grow ? mx : m_ref;
@@ -481,8 +530,9 @@ EncodeTiledFn encode_fn() {
 }
 
 size_t smem_bytes(int width) {
-  return 1024 + (size_t)kMaxLocalBlocks * kQBlockBytes + (size_t)kStages * kStageBytes + 2 * kPBytes +
-         2 * kXBytes + (((size_t)width * 4 + 15) & ~(size_t)15) + kBitmapKeys / 8 + 8 * 32 + 16;
+  const size_t x = (2 * kXBytes + 1023) & ~(size_t)1023;
+  return 1024 + x + (size_t)kMaxLocalBlocks * kQBlockBytes + (size_t)kStages * kStageBytes + 2 * kPBytes +
+         (((size_t)width * 4 + 15) & ~(size_t)15) + 8 * 40 + 16;
 }
 
 }  // namespace
