@@ -12,9 +12,9 @@
 // query is processed by a cluster of two CTAs:
 //   CTA rank 0 owns latent columns [0, 256):   q.k partial over them, O[:, 0:256)
 //   CTA rank 1 owns latent columns [256, kd):  q.k partial over them, O[:, 256:512)
-// Each CTA gathers only its own columns of every selected latent row (cp.async,
-// written straight into the 128-byte-swizzled operand layout), so no byte is
-// loaded twice.  After each 32-key chunk the two fp32 partial score tiles are
+// Each CTA gathers only its own columns of every selected latent row (TMA
+// tile::gather4, written straight into the 128-byte-swizzled operand layout),
+// so no byte is loaded twice.  After each 32-key chunk the two fp32 partial score tiles are
 // exchanged through distributed shared memory and summed; fp32 addition is
 // commutative, so both CTAs see bit-identical scores and take identical
 // online-softmax decisions.  P (bf16) goes to shared memory and each CTA
@@ -25,8 +25,8 @@
 // TMEM lanes 0-127); warps 8-11 read the same score rows and push them to the
 // peer ahead of the softmax (buffer reuse acknowledged by the peer's softmax);
 // warp 4 issues tcgen05.mma from a polling scheduler that lets q.k run up to
-// three chunks ahead of P.V; warps 5-6 deduplicate the index row and gather
-// the selected rows with cp.async; warp 7 loads the query tile by TMA.  Every
+// three chunks ahead of P.V; warps 5-6 deduplicate the index row, then warp 5
+// gathers the selected rows with TMA gather4; warp 7 loads the query tile by TMA.  Every
 // mbarrier wait is bounded.
 #include <cuda.h>
 
@@ -196,7 +196,8 @@ __device__ void build_list(const AttTcParams& p, const Smem& sm, size_t row) {
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, AttTcParams p) {
+attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
+                 AttTcParams p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ int s_misc[4];
   const uint32_t raw = smem_u32(smem_raw);
@@ -242,7 +243,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, AttTcParams p) {
     mbar_init(smem_u32(sm.qfull), 1);
     mbar_init(smem_u32(sm.list_ready), 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&sm.kv_full[s]), kProducerThreads);
+      mbar_init(smem_u32(&sm.kv_full[s]), 1);
       mbar_init(smem_u32(&sm.kv_empty[s]), 1);
     }
     for (int s = 0; s < kSBufs; ++s) {
@@ -278,31 +279,33 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, AttTcParams p) {
     // ---------------------------------------------------------------- list + gathers
     build_list(p, sm, row);
     named_sync(1, kProducerThreads);
-    const int n = *sm.n_list;
-    const int nch = (n + kChunk - 1) / kChunk;
-    const int tid = threadIdx.x - 5 * 32;
-    const int b = (int)(row / p.T);
-    const bf16* lat = p.latent + (size_t)b * p.S * p.stride + kb0 * 64;
-    const int segs = nkb * 8;                       // 16-byte segments per key row
-    const int per_chunk = kChunk * segs;
-    for (int j = 0; j < nch; ++j) {
-      const int s = j % kStages;
-      if (!mbar_wait(smem_u32(&sm.kv_empty[s]), ((j / kStages) & 1) ^ 1, p.status, abort_flag)) break;
-      const uint32_t st = sm.kv + s * kStageBytes;
-      for (int i = tid; i < per_chunk; i += kProducerThreads) {
-        const int r = i / segs, sg = i - r * segs;      // key row in chunk, segment in row
-        const int kb = sg >> 3, c = sg & 7;
-        const int li = j * kChunk + r;
-        const bool ok = li < n;                          // rows past the list are zero-filled
-        const int key = ok ? sm.list[li] : 0;
-        const bf16* src = lat + (size_t)key * p.stride + sg * 8;
-        const uint32_t dst = st + kb * kBlockBytes + r * 128 + ((c ^ (r & 7)) << 4);
-        cp_async_16(dst, src, ok);
+    if (warp == 5) {
+      // TMA gather4: four selected latent rows x 64 columns per instruction, written
+      // in the 128-byte swizzled operand layout; rows past the list repeat a valid
+      // row (their scores are masked to -inf, so P = 0 there).
+      const int n = *sm.n_list;
+      const int nch = (n + kChunk - 1) / kChunk;
+      const int rowbase = (int)(row / p.T) * p.S;
+      if (lane == 0) tma_prefetch_desc(&map_kv);
+      for (int j = 0; j < nch; ++j) {
+        const int s = j % kStages;
+        if (!mbar_wait(smem_u32(&sm.kv_empty[s]), ((j / kStages) & 1) ^ 1, p.status, abort_flag)) break;
+        if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sm.kv_full[s]), (uint32_t)nkb * kBlockBytes);
+        __syncwarp();
+        const uint32_t st = sm.kv + s * kStageBytes;
+        for (int t = lane; t < 8 * nkb; t += 32) {
+          const int kb = t >> 3, g = t & 7;
+          int rr[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int li = j * kChunk + 4 * g + i;
+            rr[i] = rowbase + sm.list[li < n ? li : 0];
+          }
+          tma_gather4(st + kb * kBlockBytes + g * 512, &map_kv, smem_u32(&sm.kv_full[s]), (kb0 + kb) * 64, rr[0],
+                      rr[1], rr[2], rr[3]);
+        }
       }
-      // arrives on kv_full[s] once this thread's copies have landed
-      cp_async_mbar_arrive(smem_u32(&sm.kv_full[s]));
     }
-    cp_async_wait_all();
   } else if (warp == 4) {
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
@@ -579,11 +582,20 @@ cudaError_t launch_attend_tc(const dsa_dims& d, const void* q, const void* k, in
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
+  // latent viewed as [B*S rows, kd cols] with the caller's row stride; box = 64 cols x 1 row (gather4)
+  CUtensorMap mkv;
+  cuuint64_t kdims[2] = {(cuuint64_t)d.kd, (cuuint64_t)d.batch * d.n_kv};
+  cuuint64_t kstrides[1] = {(cuuint64_t)k_stride * 2};
+  cuuint32_t kbox[2] = {64u, 1u};
+  if (enc(&mkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(k), kdims, kstrides, kbox, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   const size_t smem = smem_bytes(width);
   cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long long rows = (long long)d.batch * d.n_q;
-  attend_tc_kernel<<<dim3((unsigned)(2 * rows)), kThreads, smem, st>>>(mq, p);
+  attend_tc_kernel<<<dim3((unsigned)(2 * rows)), kThreads, smem, st>>>(mq, mkv, p);
   return cudaGetLastError();
 }
 
