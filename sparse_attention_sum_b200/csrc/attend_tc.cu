@@ -12,9 +12,9 @@
 // query is processed by a cluster of two CTAs:
 //   CTA rank 0 owns latent columns [0, 256):   q.k partial over them, O[:, 0:256)
 //   CTA rank 1 owns latent columns [256, kd):  q.k partial over them, O[:, 256:512)
-// Each CTA gathers only its own columns of every selected latent row (TMA
-// tile::gather4, written straight into the 128-byte-swizzled operand layout),
-// so no byte is loaded twice.  After each 32-key chunk the two fp32 partial score tiles are
+// Each CTA gathers only its own columns of every selected latent row (cp.async,
+// written straight into the 128-byte-swizzled operand layout), so no byte is
+// loaded twice.  After each 32-key chunk the two fp32 partial score tiles are
 // exchanged through distributed shared memory and summed; fp32 addition is
 // commutative, so both CTAs see bit-identical scores and take identical
 // online-softmax decisions.  P (bf16) goes to shared memory and each CTA
@@ -22,12 +22,13 @@
 // only moved (and O rescaled in TMEM) when it grows by more than 2^8.
 //
 // Warp roles per CTA: warps 0-3 softmax + epilogue (one head row per thread,
-// TMEM lanes 0-127); warps 8-11 read the same score rows and push them to the
+// TMEM lanes 0-127); warps 9-12 read the same score rows and push them to the
 // peer ahead of the softmax (buffer reuse acknowledged by the peer's softmax);
-// warp 4 issues tcgen05.mma from a polling scheduler that lets q.k run up to
-// three chunks ahead of P.V; warps 5-6 deduplicate the index row, then warp 5
-// gathers the selected rows with TMA gather4; warp 7 loads the query tile by TMA.  Every
-// mbarrier wait is bounded.
+// warp 4 loads the query tile by TMA and issues tcgen05.mma from a polling
+// scheduler that lets q.k run up to three chunks ahead of P.V; warps 5-8 stage
+// and deduplicate the index row, then gather the selected rows with 16-byte
+// cp.async (four threads per row).  Remote barrier arrivals are made once per
+// warp.  Every mbarrier wait is bounded.
 #include <cuda.h>
 
 #include "dsa_common.cuh"
@@ -52,8 +53,8 @@ constexpr int kXStride = kChunk + 4;                       // floats per exchang
 constexpr int kXBytes = 128 * kXStride * 4;                // 18 KB
 constexpr int kBitmapKeys = 65536;
 constexpr int kOCol = kSBufs * kChunk;                     // first TMEM column of O
-constexpr int kThreads = 384;
-constexpr int kProducerThreads = 64;
+constexpr int kThreads = 416;          // 13 warps
+constexpr int kProducerThreads = 128;  // warps 5-8
 
 struct AttTcParams {
   int B, T, S, H, kd, width;
@@ -96,6 +97,14 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, f
 }
 __device__ __forceinline__ void arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void arrive_remote_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 __device__ __forceinline__ bool try_wait_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -142,20 +151,21 @@ __device__ __forceinline__ uint64_t desc_noswz(uint32_t saddr, uint32_t lbo, uin
   return d;
 }
 
-// Builds the row's key list: distinct in-range entries in index-row order.
-// Deterministic, so both CTAs of the cluster obtain the same list.
+// Builds the row's key list in shared memory: distinct in-range entries in
+// index-row order.  Deterministic, so both CTAs of the cluster obtain the same
+// list.  Run by the 128 producer threads (warps 5-8).
 __device__ void build_list(const AttTcParams& p, const Smem& sm, size_t row) {
-  const int tid = threadIdx.x - 5 * 32;               // 0..63 over warps 5,6
+  const int tid = threadIdx.x - 5 * 32;               // 0..127
   const int lane = threadIdx.x & 31;
-  const bool lead = tid < 32;                          // warp 5
   const int32_t* irow = p.idx + row * p.width;
   const int words = (p.S + 31) >> 5;
+  for (int e = tid; e < p.width; e += kProducerThreads) sm.list[e] = irow[e];
   for (int i = tid; i < words; i += kProducerThreads) sm.bitmap[i] = 0u;
   if (tid == 0) *sm.dup_flag = 0;
   named_sync(1, kProducerThreads);
   int dup = 0;
   for (int e = tid; e < p.width; e += kProducerThreads) {
-    const int key = irow[e];
+    const int key = sm.list[e];
     if (key >= 0 && key < p.S) {
       const uint32_t bit = 1u << (key & 31);
       dup |= (atomicOr(&sm.bitmap[key >> 5], bit) & bit) != 0u;
@@ -168,31 +178,31 @@ __device__ void build_list(const AttTcParams& p, const Smem& sm, size_t row) {
     for (int i = tid; i < words; i += kProducerThreads) sm.bitmap[i] = 0u;
     named_sync(1, kProducerThreads);
   }
-  if (lead) {
+  if (tid < 32) {
+    // in-place compaction: a group is read before any of its slots are written
     int n = 0;
     for (int e0 = 0; e0 < p.width; e0 += 32) {
       const int e = e0 + lane;
-      const int key = e < p.width ? irow[e] : -1;
+      const int key = e < p.width ? sm.list[e] : -1;
       bool keep = key >= 0 && key < p.S;
       if (has_dup) {
         // first occurrence only: not seen in an earlier group, lowest lane in this group
         const uint32_t peers = __match_any_sync(0xffffffffu, keep ? key : -1);
-        if (keep) {
-          keep = (sm.bitmap[key >> 5] & (1u << (key & 31))) == 0u && lane == __ffs(peers) - 1;
-        }
+        if (keep) keep = (sm.bitmap[key >> 5] & (1u << (key & 31))) == 0u && lane == __ffs(peers) - 1;
         __syncwarp();
         if (keep) atomicOr(&sm.bitmap[key >> 5], 1u << (key & 31));
-        __syncwarp();
       }
       const uint32_t m = __ballot_sync(0xffffffffu, keep);
       if (keep) sm.list[n + __popc(m & ((1u << lane) - 1u))] = key;
       n += __popc(m);
+      __syncwarp();
     }
     if (lane == 0) {
       *sm.n_list = n;
       mbar_arrive(smem_u32(sm.list_ready));
     }
   }
+  named_sync(1, kProducerThreads);
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -243,7 +253,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     mbar_init(smem_u32(sm.qfull), 1);
     mbar_init(smem_u32(sm.list_ready), 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&sm.kv_full[s]), 1);
+      mbar_init(smem_u32(&sm.kv_full[s]), kProducerThreads);
       mbar_init(smem_u32(&sm.kv_empty[s]), 1);
     }
     for (int s = 0; s < kSBufs; ++s) {
@@ -253,8 +263,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&sm.p_full[s]), 4);
       mbar_init(smem_u32(&sm.o_done[s]), 1);
-      mbar_init(smem_u32(&sm.xfull[s]), 128);   // the peer's exchange threads
-      mbar_init(smem_u32(&sm.xfree[s]), 128);   // the peer's softmax threads
+      mbar_init(smem_u32(&sm.xfull[s]), 4);     // one arrival per peer exchange warp
+      mbar_init(smem_u32(&sm.xfree[s]), 4);     // one arrival per peer softmax warp
     }
     mbar_init(smem_u32(sm.drain), 1);
     fence_barrier_init();
@@ -267,48 +277,38 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   const uint32_t tmem = *sm.tmem_slot;
   volatile int* abort_flag = sm.abort_flag;
 
-  if (warp == 7) {
-    // ---------------------------------------------------------------- query tile (TMA)
+  if (warp >= 5 && warp <= 8) {
+    // ---------------------------------------------------------------- list + gathers
+    build_list(p, sm, row);
+    const int n = *sm.n_list;
+    const int nch = (n + kChunk - 1) / kChunk;
+    const int tid = threadIdx.x - 5 * 32;
+    const int r = tid >> 2, part = tid & 3;               // key row in chunk, quarter of its segments
+    const int spt = 2 * nkb;                              // 16-byte segments per thread
+    const bf16* lat = p.latent + (size_t)(row / p.T) * p.S * p.stride + kb0 * 64 + part * spt * 8;
+    for (int j = 0; j < nch; ++j) {
+      const int s = j % kStages;
+      if (!mbar_wait(smem_u32(&sm.kv_empty[s]), ((j / kStages) & 1) ^ 1, p.status, abort_flag)) break;
+      const uint32_t st = sm.kv + s * kStageBytes + r * 128;
+      const int li = j * kChunk + r;
+      const bool ok = li < n;                              // rows past the list are zero-filled
+      const bf16* src = lat + (size_t)(ok ? sm.list[li] : 0) * p.stride;
+#pragma unroll 2
+      for (int i = 0; i < spt; ++i) {
+        const int sg = part * spt + i, kb = sg >> 3, c = sg & 7;
+        cp_async_16(st + kb * kBlockBytes + ((c ^ (r & 7)) << 4), src + i * 8, ok);
+      }
+      // arrives on kv_full[s] once this thread's copies have landed
+      cp_async_mbar_arrive(smem_u32(&sm.kv_full[s]));
+    }
+    cp_async_wait_all();
+  } else if (warp == 4) {
+    // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
       tma_prefetch_desc(&map_q);
       mbar_arrive_expect_tx(smem_u32(sm.qfull), (uint32_t)nkb * kQBlockBytes);
       for (int kb = 0; kb < nkb; ++kb)
         tma_load_2d(sm.q + kb * kQBlockBytes, &map_q, smem_u32(sm.qfull), (kb0 + kb) * 64, (int)(row * p.H));
-    }
-  } else if (warp == 5 || warp == 6) {
-    // ---------------------------------------------------------------- list + gathers
-    build_list(p, sm, row);
-    named_sync(1, kProducerThreads);
-    if (warp == 5) {
-      // TMA gather4: four selected latent rows x 64 columns per instruction, written
-      // in the 128-byte swizzled operand layout; rows past the list repeat a valid
-      // row (their scores are masked to -inf, so P = 0 there).
-      const int n = *sm.n_list;
-      const int nch = (n + kChunk - 1) / kChunk;
-      const int rowbase = (int)(row / p.T) * p.S;
-      if (lane == 0) tma_prefetch_desc(&map_kv);
-      for (int j = 0; j < nch; ++j) {
-        const int s = j % kStages;
-        if (!mbar_wait(smem_u32(&sm.kv_empty[s]), ((j / kStages) & 1) ^ 1, p.status, abort_flag)) break;
-        if (lane == 0) mbar_arrive_expect_tx(smem_u32(&sm.kv_full[s]), (uint32_t)nkb * kBlockBytes);
-        __syncwarp();
-        const uint32_t st = sm.kv + s * kStageBytes;
-        for (int t = lane; t < 8 * nkb; t += 32) {
-          const int kb = t >> 3, g = t & 7;
-          int rr[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int li = j * kChunk + 4 * g + i;
-            rr[i] = rowbase + sm.list[li < n ? li : 0];
-          }
-          tma_gather4(st + kb * kBlockBytes + g * 512, &map_kv, smem_u32(&sm.kv_full[s]), (kb0 + kb) * 64, rr[0],
-                      rr[1], rr[2], rr[3]);
-        }
-      }
-    }
-  } else if (warp == 4) {
-    // ---------------------------------------------------------------- MMA issue
-    if (lane == 0) {
       const uint32_t id_qk = idesc_bf16(128, kChunk);
       const uint32_t id_pv = idesc_bf16(128, 256, false, true);
       bool ok = mbar_wait(smem_u32(sm.qfull), 0, p.status, abort_flag) &&
@@ -371,7 +371,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       mma_commit(smem_u32(sm.drain));
       mbar_wait(smem_u32(sm.drain), 0, nullptr, nullptr);
     }
-  } else if (warp >= 8) {
+  } else if (warp >= 9) {
     // ---------------------------------------------------------------- score exchange
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
@@ -399,7 +399,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       for (int c = 0; c < kChunk; c += 4)
         st_cluster_v4(dst + c * 4, __uint_as_float(v[c]), __uint_as_float(v[c + 1]), __uint_as_float(v[c + 2]),
                       __uint_as_float(v[c + 3]));
-      arrive_remote(xb ? xfull_peer1 : xfull_peer0);
+      __syncwarp();
+      if (lane == 0) arrive_remote(xb ? xfull_peer1 : xfull_peer0);  // release: covers the warp's stores
     }
   } else if (warp < 4) {
     // ---------------------------------------------------------------- softmax + epilogue
@@ -423,25 +424,31 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty[sb]));
       if (!(ok = wait_cluster(smem_u32(&sm.xfull[xb]), (j >> 1) & 1, p.status, abort_flag))) break;
-      const float* xr = xrow + xb * (kXBytes / 4);
+      const float4* xr = reinterpret_cast<const float4*>(xrow + xb * (kXBytes / 4));
+      float4 pv4[kChunk / 4];
+#pragma unroll
+      for (int c = 0; c < kChunk / 4; ++c) pv4[c] = xr[c];
+      // partner buffer xb is read (values are in registers): the peer may refill it
+      __syncwarp();
+      if (lane == 0) arrive_remote_relaxed(xb ? xfree_peer1 : xfree_peer0);
       const int valid = n - j * kChunk;
       float x[kChunk];
       float mx = -INFINITY;
 #pragma unroll
       for (int c = 0; c < kChunk; ++c) {
-        const float sc = __uint_as_float(v[c]) + xr[c];
+        const float4 q4 = pv4[c >> 2];
+        const float other = (c & 3) == 0 ? q4.x : (c & 3) == 1 ? q4.y : (c & 3) == 2 ? q4.z : q4.w;
+        const float sc = __uint_as_float(v[c]) + other;
         x[c] = c < valid ? sc * p.scale_log2 : -INFINITY;
         mx = fmaxf(mx, x[c]);
       }
-      // partner buffer xb is read: the peer may refill it
-      arrive_remote(xb ? xfree_peer1 : xfree_peer0);
       // move the reference maximum only when it grows by more than 2^8
       const bool grow = mx > m_ref + 8.f;
       const float new_ref = grow ? mx : m_ref;
       if (__any_sync(0xffffffffu, grow && j > 0)) {
         if (!(ok = mbar_wait(smem_u32(&sm.o_done[(j - 1) & 1]), ((j - 1) >> 1) & 1, p.status, abort_flag))) break;
         tc_fence_after();
-        const float f = (grow && j > 0) ? exp2f(m_ref - new_ref) : 1.f;
+        const float f = (grow && j > 0) ? ex2(m_ref - new_ref) : 1.f;
         for (int c = 0; c < 256; c += 16) {
           uint32_t o[16];
           tmem_ld_32x32b_x16(tmem + lane_addr + kOCol + c, o);
@@ -457,7 +464,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       float ps[kChunk];
 #pragma unroll
       for (int c = 0; c < kChunk; ++c) {
-        ps[c] = exp2f(x[c] - m_ref);
+        ps[c] = ex2(x[c] - m_ref);
         l_sum += ps[c];
       }
       // P buffer (j&1) is free once the P.V of chunk j-2 has completed
