@@ -37,6 +37,18 @@
 
 namespace dsa {
 
+#ifdef DSA_TRACE
+// Optional per-chunk timeline of the first cluster (build with -DDSA_TRACE):
+// g_attend_trace[cta rank][event][chunk] = %globaltimer.
+__device__ unsigned long long g_attend_trace[2][16][512];
+#define TRACE(ev, j)                                                                             \
+  do {                                                                                           \
+    if (blockIdx.x < 2 && (j) < 512) g_attend_trace[blockIdx.x & 1][ev][(j)] = sm100::globaltimer(); \
+  } while (0)
+#else
+#define TRACE(ev, j) ((void)0)
+#endif
+
 namespace {
 
 using namespace sm100;
@@ -198,6 +210,7 @@ __device__ void build_list(const AttTcParams& p, const Smem& sm, size_t row) {
       __syncwarp();
     }
     if (lane == 0) {
+      TRACE(8, 1);
       *sm.n_list = n;
       mbar_arrive(smem_u32(sm.list_ready));
     }
@@ -276,6 +289,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   tc_fence_after();
   const uint32_t tmem = *sm.tmem_slot;
   volatile int* abort_flag = sm.abort_flag;
+  if (threadIdx.x == 0) TRACE(8, 0);
 
   if (warp >= 5 && warp <= 8) {
     // ---------------------------------------------------------------- list + gathers
@@ -289,6 +303,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     for (int j = 0; j < nch; ++j) {
       const int s = j % kStages;
       if (!mbar_wait(smem_u32(&sm.kv_empty[s]), ((j / kStages) & 1) ^ 1, p.status, abort_flag)) break;
+      if (tid == 0) TRACE(0, j);
       const uint32_t st = sm.kv + s * kStageBytes + r * 128;
       const int li = j * kChunk + r;
       const bool ok = li < n;                              // rows past the list are zero-filled
@@ -337,6 +352,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             }
           }
           mma_commit(smem_u32(&sm.s_full[qk % kSBufs]));
+          TRACE(1, qk);
           ++qk;
           progressed = true;
         }
@@ -352,6 +368,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           }
           mma_commit(smem_u32(&sm.kv_empty[pv % kStages]));
           mma_commit(smem_u32(&sm.o_done[pv & 1]));
+          TRACE(2, pv);
           ++pv;
           progressed = true;
         }
@@ -392,6 +409,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty[sb]));
+      if (warp == 9 && lane == 0) TRACE(3, j);
       // the peer has finished reading its buffer xb from chunk j-2
       if (!(ok = wait_cluster(smem_u32(&sm.xfree[xb]), ((j >> 1) & 1) ^ 1, p.status, abort_flag))) break;
       const uint32_t dst = x_peer + (uint32_t)xb * kXBytes;
@@ -401,6 +419,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                       __uint_as_float(v[c + 3]));
       __syncwarp();
       if (lane == 0) arrive_remote(xb ? xfull_peer1 : xfull_peer0);  // release: covers the warp's stores
+      if (warp == 9 && lane == 0) TRACE(4, j);
     }
   } else if (warp < 4) {
     // ---------------------------------------------------------------- softmax + epilogue
@@ -423,7 +442,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty[sb]));
+      if (warp == 0 && lane == 0) TRACE(5, j);
       if (!(ok = wait_cluster(smem_u32(&sm.xfull[xb]), (j >> 1) & 1, p.status, abort_flag))) break;
+      if (warp == 0 && lane == 0) TRACE(6, j);
       const float4* xr = reinterpret_cast<const float4*>(xrow + xb * (kXBytes / 4));
       float4 pv4[kChunk / 4];
 #pragma unroll
@@ -442,6 +463,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         x[c] = c < valid ? sc * p.scale_log2 : -INFINITY;
         mx = fmaxf(mx, x[c]);
       }
+      if (warp == 0 && lane == 0) TRACE(9, j);
       // move the reference maximum only when it grows by more than 2^8
       const bool grow = mx > m_ref + 8.f;
       const float new_ref = grow ? mx : m_ref;
@@ -467,8 +489,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         ps[c] = ex2(x[c] - m_ref);
         l_sum += ps[c];
       }
+      if (warp == 0 && lane == 0) TRACE(10, j);
       // P buffer (j&1) is free once the P.V of chunk j-2 has completed
       if (j >= 2 && !(ok = mbar_wait(smem_u32(&sm.o_done[j & 1]), ((j - 2) >> 1) & 1, p.status, abort_flag))) break;
+      if (warp == 0 && lane == 0) TRACE(11, j);
       const uint32_t prow = sm.p + xb * kPBytes + (uint32_t)(r >> 3) * 512 + (uint32_t)(r & 7) * 16;
 #pragma unroll
       for (int kc = 0; kc < kChunk / 8; ++kc) {
@@ -483,6 +507,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[xb]));
+      if (warp == 0 && lane == 0) TRACE(7, j);
     }
     // epilogue: O / l -> bf16
     const bool write = r < p.H;
@@ -607,3 +632,13 @@ cudaError_t launch_attend_tc(const dsa_dims& d, const void* q, const void* k, in
 }
 
 }  // namespace dsa
+
+#ifdef DSA_TRACE
+extern "C" int dsa_trace_read(unsigned long long* host) {
+  return (int)cudaMemcpyFromSymbol(host, dsa::g_attend_trace, sizeof(dsa::g_attend_trace));
+}
+extern "C" int dsa_trace_clear() {
+  static unsigned long long zero[2 * 16 * 512];
+  return (int)cudaMemcpyToSymbol(dsa::g_attend_trace, zero, sizeof(zero));
+}
+#endif
