@@ -83,7 +83,8 @@ struct Smem {
   uint32_t q, kv, p, x;      // shared-window addresses
   int* list;
   uint32_t* bitmap;
-  uint64_t *qfull, *list_ready, *kv_full, *kv_empty, *s_full, *s_empty, *p_full, *o_done, *xfull, *xfree, *drain;
+  uint64_t *qfull, *list_ready, *kv_full, *kv_empty, *s_full, *s_empty, *p_full, *o_done, *xfull, *xfree, *xread,
+      *drain;
   uint32_t* tmem_slot;
   int* n_list;
   int* dup_flag;
@@ -247,7 +248,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   sm.o_done = sm.p_full + 2;
   sm.xfull = sm.o_done + 2;
   sm.xfree = sm.xfull + 2;
-  sm.drain = sm.xfree + 2;
+  sm.xread = sm.xfree + 2;
+  sm.drain = sm.xread + 2;
   sm.tmem_slot = reinterpret_cast<uint32_t*>(sm.drain + 1);
   sm.n_list = &s_misc[0];
   sm.dup_flag = &s_misc[1];
@@ -277,7 +279,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       mbar_init(smem_u32(&sm.p_full[s]), 4);
       mbar_init(smem_u32(&sm.o_done[s]), 1);
       mbar_init(smem_u32(&sm.xfull[s]), 4);     // one arrival per peer exchange warp
-      mbar_init(smem_u32(&sm.xfree[s]), 4);     // one arrival per peer softmax warp
+      mbar_init(smem_u32(&sm.xfree[s]), 4);     // one arrival per peer exchange warp
+      mbar_init(smem_u32(&sm.xread[s]), 4);     // one arrival per local softmax warp
     }
     mbar_init(smem_u32(sm.drain), 1);
     fence_barrier_init();
@@ -337,8 +340,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       while (ok && pv < nch) {
         bool progressed = false;
         if (qk < nch && qk - pv < kStages - 1 &&
-            mbar_try_wait(smem_u32(&sm.kv_full[qk % kStages]), (qk / kStages) & 1) &&
-            mbar_try_wait(smem_u32(&sm.s_empty[qk % kSBufs]), ((qk / kSBufs) & 1) ^ 1)) {
+            mbar_test_wait(smem_u32(&sm.kv_full[qk % kStages]), (qk / kStages) & 1) &&
+            mbar_test_wait(smem_u32(&sm.s_empty[qk % kSBufs]), ((qk / kSBufs) & 1) ^ 1)) {
           fence_proxy_async_smem();
           tc_fence_after();
           const uint32_t st = sm.kv + (qk % kStages) * kStageBytes;
@@ -356,7 +359,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           ++qk;
           progressed = true;
         }
-        if (pv < qk && mbar_try_wait(smem_u32(&sm.p_full[pv & 1]), (pv >> 1) & 1)) {
+        if (pv < qk && mbar_test_wait(smem_u32(&sm.p_full[pv & 1]), (pv >> 1) & 1)) {
           tc_fence_after();
           const uint32_t pa = sm.p + (pv & 1) * kPBytes;
           const uint32_t st = sm.kv + (pv % kStages) * kStageBytes;
@@ -399,6 +402,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const uint32_t x_peer = map_peer(sm.x + (uint32_t)r * kXStride * 4, peer);
     const uint32_t xfull_peer0 = map_peer(smem_u32(&sm.xfull[0]), peer);
     const uint32_t xfull_peer1 = map_peer(smem_u32(&sm.xfull[1]), peer);
+    const uint32_t xfree_peer0 = map_peer(smem_u32(&sm.xfree[0]), peer);
+    const uint32_t xfree_peer1 = map_peer(smem_u32(&sm.xfree[1]), peer);
     for (int j = 0; ok && j < nch; ++j) {
       const int sb = j % kSBufs, xb = j & 1;
       if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), (j / kSBufs) & 1, p.status, abort_flag))) break;
@@ -410,6 +415,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty[sb]));
       if (warp == 9 && lane == 0) TRACE(3, j);
+      // our softmax has read our buffer xb of chunk j-2: tell the peer it may refill it
+      if (j >= 2) {
+        if (!(ok = mbar_wait(smem_u32(&sm.xread[xb]), ((j - 2) >> 1) & 1, p.status, abort_flag))) break;
+        __syncwarp();
+        if (lane == 0) arrive_remote_relaxed(xb ? xfree_peer1 : xfree_peer0);
+      }
       // the peer has finished reading its buffer xb from chunk j-2
       if (!(ok = wait_cluster(smem_u32(&sm.xfree[xb]), ((j >> 1) & 1) ^ 1, p.status, abort_flag))) break;
       const uint32_t dst = x_peer + (uint32_t)xb * kXBytes;
@@ -429,8 +440,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     bool ok = mbar_wait(smem_u32(sm.list_ready), 0, p.status, abort_flag);
     const int n = ok ? *sm.n_list : 0;
     const int nch = (n + kChunk - 1) / kChunk;
-    const uint32_t xfree_peer0 = map_peer(smem_u32(&sm.xfree[0]), peer);
-    const uint32_t xfree_peer1 = map_peer(smem_u32(&sm.xfree[1]), peer);
     const float* xrow = reinterpret_cast<const float*>(gb + (sm.x - base)) + r * kXStride;
     for (int j = 0; ok && j < nch; ++j) {
       const int sb = j % kSBufs, xb = j & 1;
@@ -449,9 +458,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       float4 pv4[kChunk / 4];
 #pragma unroll
       for (int c = 0; c < kChunk / 4; ++c) pv4[c] = xr[c];
-      // partner buffer xb is read (values are in registers): the peer may refill it
+      // buffer xb is read (values are in registers); the exchange warps tell the peer
       __syncwarp();
-      if (lane == 0) arrive_remote_relaxed(xb ? xfree_peer1 : xfree_peer0);
+      if (lane == 0) mbar_arrive(smem_u32(&sm.xread[xb]));
       const int valid = n - j * kChunk;
       float x[kChunk];
       float mx = -INFINITY;
