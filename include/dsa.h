@@ -231,6 +231,27 @@ dsa_status dsa_absorb_q(const dsa_dims* dims, const void* q, int32_t d, const vo
 dsa_status dsa_absorb_out(const dsa_dims* dims, const void* o_lat, int32_t L, const void* w_uv,
                           int32_t e, void* out, dsa_stream_t stream);
 
+/* Allocation-free variant of dsa_layer_forward, for callers that cannot
+ * allocate device memory where they run the layer (a serving engine that plans
+ * all memory up front and forbids allocation on its decode path, code running
+ * inside an allocator callback, a runtime handed a fixed memory budget).  The
+ * DSA pages have no counterpart: this is a library convenience, not part of the
+ * method.  Same arguments and result as dsa_layer_forward without ws/ws_bytes:
+ * the score matrix and index rows live in one fixed 16 MiB array inside the
+ * library's device memory, held by every GPU that loads the library until the
+ * process exits.  Calls whose workspace need (dsa_workspace_size) exceeds
+ * 16 MiB return DSA_ERR_WORKSPACE with a message.  The first call on a device
+ * looks up the array's device address with that device current, so make it
+ * before any stream capture.  All calls share the array and it keeps the last
+ * call's contents; calls that overlap on the GPU race on it.  No part of the
+ * array needs to start at zero. */
+dsa_status dsa_layer_forward_static(const dsa_dims* dims, const void* q_idx, const void* k_idx,
+                                    const float* w, float idx_scale, const int32_t* q_pos,
+                                    const int32_t* kv_start, const int32_t* kv_len, const void* q,
+                                    const void* k, int64_t k_row_stride, const void* v,
+                                    int64_t v_row_stride, float attn_scale, const int32_t* idx_in,
+                                    int32_t* idx_out, void* out, float* lse, dsa_stream_t stream);
+
 /* Synchronize `stream`, then return and clear the device status word:
  * DSA_ERR_TIMEOUT if any bounded device-side wait expired since the last
  * call, DSA_ERR_CUDA if the stream reports an error, DSA_OK otherwise. */

@@ -15,7 +15,7 @@ from typing import Optional
 
 __all__ = [
     "DsaError", "DsaLibraryError", "Dims", "lib", "lib_path", "INVALID", "F32", "BF16",
-    "index_scores", "topk", "sparse_attend", "layer_forward", "pool_states",
+    "index_scores", "topk", "sparse_attend", "layer_forward", "layer_forward_static", "pool_states",
     "expand_selection", "absorb_q", "absorb_out", "workspace_size", "get_device_status",
     "selftest_wait_timeout", "set_kernel_policy", "OP_TOPK", "OP_LAYER_FORWARD", "STATUS",
 ]
@@ -74,6 +74,9 @@ _SIGS = {
     "dsa_layer_forward": ([ctypes.POINTER(Dims), _VP, _VP, _F32P, ctypes.c_float, _I32P, _I32P,
                            _I32P, _VP, _VP, ctypes.c_int64, _VP, ctypes.c_int64, ctypes.c_float,
                            _I32P, _I32P, _VP, _F32P, _VP, ctypes.c_size_t, _VP], ctypes.c_int),
+    "dsa_layer_forward_static": ([ctypes.POINTER(Dims), _VP, _VP, _F32P, ctypes.c_float, _I32P, _I32P,
+                                  _I32P, _VP, _VP, ctypes.c_int64, _VP, ctypes.c_int64, ctypes.c_float,
+                                  _I32P, _I32P, _VP, _F32P, _VP], ctypes.c_int),
     "dsa_pool_states": ([ctypes.POINTER(Dims), _VP, _VP, _F32P, _F32P, ctypes.c_float, _I32P,
                          _I32P, _VP, _I32P, _VP], ctypes.c_int),
     "dsa_expand_selection": ([ctypes.POINTER(Dims), _I32P, _I32P, _I32P, _I32P, _I32P, _I32P,
@@ -176,6 +179,17 @@ def layer_forward(dims: Dims, q_idx, k_idx, w, idx_scale: float, q_pos, kv_start
                                    int(k_row_stride), _ptr(v), int(v_row_stride), attn_scale,
                                    _ptr(idx_in), _ptr(idx_out), _ptr(out), _ptr(lse), _ptr(ws), wsb,
                                    _stream(stream)), "dsa_layer_forward")
+
+
+def layer_forward_static(dims: Dims, q_idx, k_idx, w, idx_scale: float, q_pos, kv_start, kv_len, q, k,
+                         k_row_stride: int, v, v_row_stride: int, attn_scale: float, out, lse=None,
+                         idx_in=None, idx_out=None, stream=None):
+    """dsa_layer_forward with the library's fixed scratch array (no workspace argument)."""
+    _check(lib().dsa_layer_forward_static(ctypes.byref(dims), _ptr(q_idx), _ptr(k_idx), _ptr(w), idx_scale,
+                                          _ptr(q_pos), _ptr(kv_start), _ptr(kv_len), _ptr(q), _ptr(k),
+                                          int(k_row_stride), _ptr(v), int(v_row_stride), attn_scale,
+                                          _ptr(idx_in), _ptr(idx_out), _ptr(out), _ptr(lse), _stream(stream)),
+           "dsa_layer_forward_static")
 
 
 def pool_states(dims: Dims, k, gate, ln_w, ln_b, ln_eps: float, kv_start, kv_len, pooled, n_pools,

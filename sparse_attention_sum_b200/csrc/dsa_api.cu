@@ -116,6 +116,8 @@ int* device_status_ptr() {
   return ptrs[dev];
 }
 
+void set_last_error(const char* msg) { g_last_error = msg; }
+
 int sm_count() {
   static int cached[128] = {};
   int dev = 0;

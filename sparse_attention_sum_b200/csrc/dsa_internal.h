@@ -15,6 +15,9 @@ int* device_status_ptr();
 // Number of SMs of the current device.
 int sm_count();
 
+// Sets the message dsa_last_error() returns on this host thread.
+void set_last_error(const char* msg);
+
 // S2 on the CUDA cores (any D_I <= 256, H_I*D_I <= 16384), fp32 or bf16 inputs.
 cudaError_t launch_index_scores_simt(const dsa_dims& d, const void* q_idx, const void* k_idx,
                                      const float* w, float scale, const int32_t* q_pos,
