@@ -150,6 +150,11 @@ def dist_setup(n_gpus):
     return 0, 1, 0
 
 
+def replica_seed(workload: str, rank: int):
+    """Seed of this rank's replica: rank 0 runs the standard workload, others their own draw."""
+    return None if rank == 0 else 1000 + rank
+
+
 def max_over_ranks(x: float, world: int) -> float:
     if world == 1:
         return x
@@ -252,7 +257,7 @@ def run_ours(a):
     torch.cuda.set_device(local)
     dsa.lib()
     peaks = measured_peaks()
-    wl = workloads.make(a.workload, seed=None if rank == 0 else 1000 + rank)
+    wl = workloads.make(a.workload, seed=replica_seed(a.workload, rank))
     t = device_inputs(wl)
     dims, args = layer_args(wl, t)
     bufs = runner.LayerBuffers(dims, "cuda", torch.bfloat16, with_idx=True)
