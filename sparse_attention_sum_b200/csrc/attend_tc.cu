@@ -54,17 +54,17 @@ namespace {
 using namespace sm100;
 
 constexpr int kChunk = 32;            // keys per pipeline step (MMA N of q.k, K of P.V)
-constexpr int kStages = 4;            // gathered key/value stages
-constexpr int kSBufs = 4;             // score buffers in TMEM
+constexpr int kStages = 8;            // gathered key/value stages
+constexpr int kSBufs = 3;             // score buffers in TMEM (columns 0-95)
 constexpr int kMaxLocalBlocks = 5;    // 64-column blocks per CTA (rank 1 with kd = 576)
 constexpr int kBlockBytes = kChunk * 128;                  // one 64-col block of a stage: 4 KB
 constexpr int kStageBytes = kMaxLocalBlocks * kBlockBytes; // 20 KB
-constexpr int kQBlockBytes = 128 * 128;                    // 128 rows x 64 cols bf16: 16 KB
 constexpr int kPBytes = 128 * kChunk * 2;                  // 8 KB
 constexpr int kXStride = kChunk + 4;                       // floats per exchange row (bank padding)
 constexpr int kXBytes = 128 * kXStride * 4;                // 18 KB
 constexpr int kBitmapKeys = 65536;
-constexpr int kOCol = kSBufs * kChunk;                     // first TMEM column of O
+constexpr int kQCol = 96;                                  // query tile in TMEM: 2 bf16 per column
+constexpr int kOCol = 256;                                 // output accumulator: columns 256-511
 constexpr int kThreads = 416;          // 13 warps
 constexpr int kProducerThreads = 128;  // warps 5-8
 
@@ -72,6 +72,7 @@ struct AttTcParams {
   int B, T, S, H, kd, width;
   long long stride;          // latent row stride in elements
   const bf16* latent;
+  const bf16* q;             // [B,T,H,kd]
   const int32_t* idx;
   float scale_log2;          // softmax scale * log2(e)
   bf16* out;                 // [B,T,H,512]
@@ -80,7 +81,7 @@ struct AttTcParams {
 };
 
 struct Smem {
-  uint32_t q, kv, p, x;      // shared-window addresses
+  uint32_t kv, p, x;         // shared-window addresses
   int* list;
   uint32_t* bitmap;
   uint64_t *qfull, *list_ready, *kv_full, *kv_empty, *s_full, *s_empty, *p_full, *o_done, *xfull, *xfree, *xread,
@@ -220,8 +221,7 @@ __device__ void build_list(const AttTcParams& p, const Smem& sm, size_t row) {
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
-                 AttTcParams p) {
+attend_tc_kernel(const __grid_constant__ CUtensorMap map_kv, AttTcParams p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ int s_misc[4];
   const uint32_t raw = smem_u32(smem_raw);
@@ -229,9 +229,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   unsigned char* gb = smem_raw + (base - raw);
   Smem sm;
   sm.x = base;                                   // peer-written: same offset in both CTAs
-  sm.q = sm.x + 2 * kXBytes;
-  sm.q = (sm.q + 1023u) & ~1023u;
-  sm.kv = sm.q + kMaxLocalBlocks * kQBlockBytes;
+  sm.kv = (sm.x + 2 * kXBytes + 1023u) & ~1023u;
   sm.p = sm.kv + kStages * kStageBytes;
   uint32_t off = sm.p + 2 * kPBytes - base;
   sm.bitmap = reinterpret_cast<uint32_t*>(gb + (sm.p - base));  // aliases P: used before the first P
@@ -265,7 +263,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
   if (threadIdx.x == 0) {
     *sm.abort_flag = 0;
-    mbar_init(smem_u32(sm.qfull), 1);
+    mbar_init(smem_u32(sm.qfull), 4);          // one arrival per softmax warp after its Q rows are in TMEM
     mbar_init(smem_u32(sm.list_ready), 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&sm.kv_full[s]), kProducerThreads);
@@ -323,10 +321,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   } else if (warp == 4) {
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
-      tma_prefetch_desc(&map_q);
-      mbar_arrive_expect_tx(smem_u32(sm.qfull), (uint32_t)nkb * kQBlockBytes);
-      for (int kb = 0; kb < nkb; ++kb)
-        tma_load_2d(sm.q + kb * kQBlockBytes, &map_q, smem_u32(sm.qfull), (kb0 + kb) * 64, (int)(row * p.H));
       const uint32_t id_qk = idesc_bf16(128, kChunk);
       const uint32_t id_pv = idesc_bf16(128, 256, false, true);
       bool ok = mbar_wait(smem_u32(sm.qfull), 0, p.status, abort_flag) &&
@@ -349,9 +343,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           for (int kb = 0; kb < nkb; ++kb) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const uint64_t ad = desc_sw128(sm.q + kb * kQBlockBytes + k * 32);
               const uint64_t bd = desc_sw128(st + kb * kBlockBytes + k * 32);
-              mma_bf16_ss(d, ad, bd, id_qk, (kb | k) ? 1u : 0u);
+              mma_bf16_ts(d, tmem + kQCol + (kb * 4 + k) * 8, bd, id_qk, (kb | k) ? 1u : 0u);
             }
           }
           mma_commit(smem_u32(&sm.s_full[qk % kSBufs]));
@@ -437,6 +430,27 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const int r = warp * 32 + lane;                 // head row == TMEM lane
     const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
     float m_ref = -INFINITY, l_sum = 0.f;
+    {
+      // this CTA's columns of query head r -> TMEM lane r, columns kQCol.. (bf16 pairs)
+      const bool real = r < p.H;
+      const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (row * p.H + (real ? r : 0)) * p.kd + kb0 * 64);
+      for (int c0 = 0; c0 < nkb * 32; c0 += 32) {  // 32 columns = 64 bf16 = 8 x 16 bytes
+        uint32_t qv[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 u = real ? qsrc[c0 / 4 + i] : make_uint4(0, 0, 0, 0);
+          qv[4 * i] = u.x;
+          qv[4 * i + 1] = u.y;
+          qv[4 * i + 2] = u.z;
+          qv[4 * i + 3] = u.w;
+        }
+        tmem_st_32x32b_x32(tmem + lane_addr + kQCol + c0, qv);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(sm.qfull));
+    }
     bool ok = mbar_wait(smem_u32(sm.list_ready), 0, p.status, abort_flag);
     const int n = ok ? *sm.n_list : 0;
     const int nch = (n + kChunk - 1) / kChunk;
@@ -575,8 +589,8 @@ EncodeTiledFn encode_fn() {
 
 size_t smem_bytes(int width) {
   const size_t x = (2 * kXBytes + 1023) & ~(size_t)1023;
-  return 1024 + x + (size_t)kMaxLocalBlocks * kQBlockBytes + (size_t)kStages * kStageBytes + 2 * kPBytes +
-         (((size_t)width * 4 + 15) & ~(size_t)15) + 8 * 40 + 16;
+  return 1024 + x + (size_t)kStages * kStageBytes + 2 * kPBytes + (((size_t)width * 4 + 15) & ~(size_t)15) +
+         8 * 48 + 16;
 }
 
 }  // namespace
@@ -606,6 +620,7 @@ cudaError_t launch_attend_tc(const dsa_dims& d, const void* q, const void* k, in
   p.width = width;
   p.stride = k_stride;
   p.latent = (const bf16*)k;
+  p.q = (const bf16*)q;
   p.idx = idx;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.out = (bf16*)out;
@@ -613,21 +628,12 @@ cudaError_t launch_attend_tc(const dsa_dims& d, const void* q, const void* k, in
   p.status = device_status_ptr();
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
-  // q viewed as [B*T*H rows, kd cols]; box = 64 cols x 128 rows, 128-byte swizzle
-  CUtensorMap mq;
-  cuuint64_t dims[2] = {(cuuint64_t)d.kd, (cuuint64_t)d.batch * d.n_q * d.heads};
-  cuuint64_t strides[1] = {(cuuint64_t)d.kd * 2};
-  cuuint32_t box[2] = {64u, 128u};
-  cuuint32_t estr[2] = {1u, 1u};
-  if (enc(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box, estr,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
   // latent viewed as [B*S rows, kd cols] with the caller's row stride; box = 64 cols x 1 row (gather4)
   CUtensorMap mkv;
   cuuint64_t kdims[2] = {(cuuint64_t)d.kd, (cuuint64_t)d.batch * d.n_kv};
   cuuint64_t kstrides[1] = {(cuuint64_t)k_stride * 2};
   cuuint32_t kbox[2] = {64u, 1u};
+  cuuint32_t estr[2] = {1u, 1u};
   if (enc(&mkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(k), kdims, kstrides, kbox, estr,
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -636,7 +642,7 @@ cudaError_t launch_attend_tc(const dsa_dims& d, const void* q, const void* k, in
   cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long long rows = (long long)d.batch * d.n_q;
-  attend_tc_kernel<<<dim3((unsigned)(2 * rows)), kThreads, smem, st>>>(mq, mkv, p);
+  attend_tc_kernel<<<dim3((unsigned)(2 * rows)), kThreads, smem, st>>>(mkv, p);
   return cudaGetLastError();
 }
 
