@@ -65,7 +65,7 @@ constexpr int kXBytes = 128 * kXStride * 4;                // 18 KB
 constexpr int kBitmapKeys = 65536;
 constexpr int kQCol = 96;                                  // query tile in TMEM: 2 bf16 per column
 constexpr int kOCol = 256;                                 // output accumulator: columns 256-511
-constexpr int kThreads = 416;          // 13 warps
+constexpr int kThreads = 544;          // 17 warps
 constexpr int kProducerThreads = 128;  // warps 5-8
 
 struct AttTcParams {
@@ -386,19 +386,19 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_kv, AttTcParams p) {
     }
   } else if (warp >= 9) {
     // ---------------------------------------------------------------- score exchange
+    // Two sets of four warps take alternate chunks; set x owns exchange buffer x.
+    const int set = (warp - 9) >> 2;
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
     bool ok = mbar_wait(smem_u32(sm.list_ready), 0, p.status, abort_flag);
     const int n = ok ? *sm.n_list : 0;
     const int nch = (n + kChunk - 1) / kChunk;
-    const uint32_t x_peer = map_peer(sm.x + (uint32_t)r * kXStride * 4, peer);
-    const uint32_t xfull_peer0 = map_peer(smem_u32(&sm.xfull[0]), peer);
-    const uint32_t xfull_peer1 = map_peer(smem_u32(&sm.xfull[1]), peer);
-    const uint32_t xfree_peer0 = map_peer(smem_u32(&sm.xfree[0]), peer);
-    const uint32_t xfree_peer1 = map_peer(smem_u32(&sm.xfree[1]), peer);
-    for (int j = 0; ok && j < nch; ++j) {
-      const int sb = j % kSBufs, xb = j & 1;
+    const uint32_t dst = map_peer(sm.x + (uint32_t)set * kXBytes + (uint32_t)r * kXStride * 4, peer);
+    const uint32_t xfull_peer = map_peer(smem_u32(&sm.xfull[set]), peer);
+    const uint32_t xfree_peer = map_peer(smem_u32(&sm.xfree[set]), peer);
+    for (int j = set; ok && j < nch; j += 2) {
+      const int sb = j % kSBufs, use = j >> 1;       // use = how many times buffer `set` was used before
       if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), (j / kSBufs) & 1, p.status, abort_flag))) break;
       tc_fence_after();
       uint32_t v[32];
@@ -407,23 +407,22 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_kv, AttTcParams p) {
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty[sb]));
-      if (warp == 9 && lane == 0) TRACE(3, j);
-      // our softmax has read our buffer xb of chunk j-2: tell the peer it may refill it
-      if (j >= 2) {
-        if (!(ok = mbar_wait(smem_u32(&sm.xread[xb]), ((j - 2) >> 1) & 1, p.status, abort_flag))) break;
-        __syncwarp();
-        if (lane == 0) arrive_remote_relaxed(xb ? xfree_peer1 : xfree_peer0);
-      }
-      // the peer has finished reading its buffer xb from chunk j-2
-      if (!(ok = wait_cluster(smem_u32(&sm.xfree[xb]), ((j >> 1) & 1) ^ 1, p.status, abort_flag))) break;
-      const uint32_t dst = x_peer + (uint32_t)xb * kXBytes;
+      if (q4 == 1 && lane == 0) TRACE(3, j);
+      // the peer has read its buffer `set` from chunk j-2
+      if (!(ok = wait_cluster(smem_u32(&sm.xfree[set]), (use & 1) ^ 1, p.status, abort_flag))) break;
 #pragma unroll
       for (int c = 0; c < kChunk; c += 4)
         st_cluster_v4(dst + c * 4, __uint_as_float(v[c]), __uint_as_float(v[c + 1]), __uint_as_float(v[c + 2]),
                       __uint_as_float(v[c + 3]));
       __syncwarp();
-      if (lane == 0) arrive_remote(xb ? xfull_peer1 : xfull_peer0);  // release: covers the warp's stores
-      if (warp == 9 && lane == 0) TRACE(4, j);
+      if (lane == 0) arrive_remote(xfull_peer);  // release: covers the warp's stores
+      if (q4 == 1 && lane == 0) TRACE(4, j);
+      // once our softmax has read our buffer `set` for chunk j, the peer may refill it (chunk j+2)
+      if (j + 2 < nch) {
+        if (!(ok = mbar_wait(smem_u32(&sm.xread[set]), use & 1, p.status, abort_flag))) break;
+        __syncwarp();
+        if (lane == 0) arrive_remote_relaxed(xfree_peer);
+      }
     }
   } else if (warp < 4) {
     // ---------------------------------------------------------------- softmax + epilogue
