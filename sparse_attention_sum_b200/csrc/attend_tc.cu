@@ -9,26 +9,33 @@
 //
 // Heads are the MMA M dimension (128 rows; fewer heads leave rows unused).  A
 // 128 x 512 fp32 output accumulator fills all of one SM's tensor memory, so a
-// query is processed by a cluster of two CTAs:
-//   CTA rank 0 owns latent columns [0, 256):   q.k partial over them, O[:, 0:256)
-//   CTA rank 1 owns latent columns [256, kd):  q.k partial over them, O[:, 256:512)
-// Each CTA gathers only its own columns of every selected latent row (cp.async,
-// written straight into the 128-byte-swizzled operand layout), so no byte is
-// loaded twice.  After each 32-key chunk the two fp32 partial score tiles are
-// exchanged through distributed shared memory and summed; fp32 addition is
-// commutative, so both CTAs see bit-identical scores and take identical
-// online-softmax decisions.  P (bf16) goes to shared memory and each CTA
-// accumulates P.V for its 256 value columns in TMEM.  The running maximum is
-// only moved (and O rescaled in TMEM) when it grows by more than 2^8.
+// query is processed by a cluster of two CTAs, each owning half of the value
+// columns and the matching half of the key columns:
+//   rank 0: latent columns [0,256) (+ the 64 rope columns [512,576) when kd = 576),
+//           O[:, 0:256)
+//   rank 1: latent columns [256,512), O[:, 256:512)
+// Each CTA gathers only its own columns of every selected latent row (cp.async
+// straight into the 128-byte-swizzled operand layout), so no byte is loaded
+// twice.  Per 64-key chunk each CTA computes the q.k partial over its columns;
+// the two fp32 partial tiles are exchanged through distributed shared memory
+// and summed (fp32 addition is commutative, so both CTAs see bit-identical
+// scores and take identical online-softmax decisions).
 //
-// Warp roles per CTA: warps 0-3 softmax + epilogue (one head row per thread,
-// TMEM lanes 0-127); warps 9-12 read the same score rows and push them to the
-// peer ahead of the softmax (buffer reuse acknowledged by the peer's softmax);
-// warp 4 loads the query tile by TMA and issues tcgen05.mma from a polling
-// scheduler that lets q.k run up to three chunks ahead of P.V; warps 5-8 stage
-// and deduplicate the index row, then gather the selected rows with 16-byte
-// cp.async (four threads per row).  Remote barrier arrivals are made once per
-// warp.  Every mbarrier wait is bounded.
+// Tensor memory (512 columns): score buffers 0-63 and 64-127, the CTA's query
+// columns 128-255 as the A operand of q.k (two bf16 per column), O 256-511.
+// The bf16 probabilities overwrite the first 32 columns of their score buffer
+// and feed P.V straight from tensor memory.  Every tcgen05.mma here costs about
+// 100 cycles whatever its N up to 128, so q.k uses N = 64 keys per instruction
+// and P.V N = 256 value columns.  The running maximum only moves (and O is
+// rescaled in TMEM) when it grows by more than 2^8.
+//
+// Warp roles per CTA: warps 0-3 load the query columns into TMEM, then run the
+// softmax and the epilogue (one head row per thread, TMEM lanes 0-127); warps
+// 9-12 read the same score rows and push them to the peer (buffer reuse is
+// acknowledged by the peer); warp 4 issues tcgen05.mma from a polling scheduler
+// (and on rank 0 loads the rope query block by TMA); warps 5-8 stage and
+// deduplicate the index row, then gather the selected rows with 16-byte
+// cp.async.  Every mbarrier wait is bounded.
 #include <cuda.h>
 
 #include "dsa_common.cuh"
@@ -53,19 +60,18 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kChunk = 32;            // keys per pipeline step (MMA N of q.k, K of P.V)
-constexpr int kStages = 8;            // gathered key/value stages
-constexpr int kSBufs = 3;             // score buffers in TMEM (columns 0-95)
-constexpr int kMaxLocalBlocks = 5;    // 64-column blocks per CTA (rank 1 with kd = 576)
-constexpr int kBlockBytes = kChunk * 128;                  // one 64-col block of a stage: 4 KB
-constexpr int kStageBytes = kMaxLocalBlocks * kBlockBytes; // 20 KB
-constexpr int kPBytes = 128 * kChunk * 2;                  // 8 KB
-constexpr int kXStride = kChunk + 4;                       // floats per exchange row (bank padding)
-constexpr int kXBytes = 128 * kXStride * 4;                // 18 KB
-constexpr int kBitmapKeys = 65536;
-constexpr int kQCol = 96;                                  // query tile in TMEM: 2 bf16 per column
-constexpr int kOCol = 256;                                 // output accumulator: columns 256-511
-constexpr int kThreads = 544;          // 17 warps
+constexpr int kChunk = 64;             // keys per pipeline step (N of q.k, K of P.V)
+constexpr int kStages = 3;             // gathered key/value stages
+constexpr int kMaxLocalBlocks = 5;     // 64-column blocks per CTA (rank 0 with the rope block)
+constexpr int kBlockBytes = kChunk * 128;                   // one 64-col block of a stage: 8 KB
+constexpr int kStageBytes = kMaxLocalBlocks * kBlockBytes;  // 40 KB
+constexpr int kQRopeBytes = 128 * 128;                      // rope query block in smem: 16 KB
+constexpr int kXStride = kChunk + 4;                        // floats per exchange row (bank padding)
+constexpr int kXBytes = 128 * kXStride * 4;                 // 34 KB
+constexpr int kBitmapKeys = 65536;                          // dedupe bitmap (8 KB, aliases stage 0)
+constexpr int kQCol = 128;                                  // query columns in TMEM
+constexpr int kOCol = 256;                                  // output accumulator
+constexpr int kThreads = 416;          // 13 warps
 constexpr int kProducerThreads = 128;  // warps 5-8
 
 struct AttTcParams {
@@ -81,11 +87,11 @@ struct AttTcParams {
 };
 
 struct Smem {
-  uint32_t kv, p, x;         // shared-window addresses
+  uint32_t kv, x, qrope;     // shared-window addresses
   int* list;
   uint32_t* bitmap;
-  uint64_t *qfull, *list_ready, *kv_full, *kv_empty, *s_full, *s_empty, *p_full, *o_done, *xfull, *xfree, *xread,
-      *drain;
+  uint64_t *qfull, *qrope_full, *list_ready, *kv_full, *kv_empty, *s_full, *s_read, *p_full, *o_done, *xfull,
+      *xfree, *xread, *drain;
   uint32_t* tmem_slot;
   int* n_list;
   int* dup_flag;
@@ -221,7 +227,8 @@ __device__ void build_list(const AttTcParams& p, const Smem& sm, size_t row) {
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-attend_tc_kernel(const __grid_constant__ CUtensorMap map_kv, AttTcParams p) {
+attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
+                 AttTcParams p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ int s_misc[4];
   const uint32_t raw = smem_u32(smem_raw);
@@ -229,20 +236,21 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_kv, AttTcParams p) {
   unsigned char* gb = smem_raw + (base - raw);
   Smem sm;
   sm.x = base;                                   // peer-written: same offset in both CTAs
-  sm.kv = (sm.x + 2 * kXBytes + 1023u) & ~1023u;
-  sm.p = sm.kv + kStages * kStageBytes;
-  uint32_t off = sm.p + 2 * kPBytes - base;
-  sm.bitmap = reinterpret_cast<uint32_t*>(gb + (sm.p - base));  // aliases P: used before the first P
+  sm.qrope = sm.x + 2 * kXBytes;
+  sm.kv = sm.qrope + kQRopeBytes;
+  uint32_t off = sm.kv + kStages * kStageBytes - base;
+  sm.bitmap = reinterpret_cast<uint32_t*>(gb + (sm.kv - base));  // stage 0 is not written before the list is built
   sm.list = reinterpret_cast<int*>(gb + off);
   off += ((uint32_t)p.width * 4u + 15u) & ~15u;
   uint64_t* bars = reinterpret_cast<uint64_t*>(gb + off);
   sm.qfull = bars;
-  sm.list_ready = bars + 1;
-  sm.kv_full = bars + 2;
+  sm.qrope_full = bars + 1;
+  sm.list_ready = bars + 2;
+  sm.kv_full = bars + 3;
   sm.kv_empty = sm.kv_full + kStages;
   sm.s_full = sm.kv_empty + kStages;
-  sm.s_empty = sm.s_full + kSBufs;
-  sm.p_full = sm.s_empty + kSBufs;
+  sm.s_read = sm.s_full + 2;
+  sm.p_full = sm.s_read + 2;
   sm.o_done = sm.p_full + 2;
   sm.xfull = sm.o_done + 2;
   sm.xfree = sm.xfull + 2;
@@ -257,28 +265,28 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_kv, AttTcParams p) {
   const uint32_t rank = cluster_rank();
   const uint32_t peer = rank ^ 1u;
   const size_t row = blockIdx.x >> 1;            // query row b*T + t
-  const int nkb_total = p.kd / 64;
-  const int kb0 = rank ? 4 : 0;                  // first global 64-col block of this CTA
-  const int nkb = rank ? nkb_total - 4 : 4;      // blocks this CTA owns (q.k); the first 4 are its V
+  const bool rope = rank == 0 && p.kd == 576;    // rank 0 also owns the rope block
+  const int nlb = rope ? 5 : 4;                  // 64-column blocks gathered and used by q.k
+  // global 64-column block of local block lb (the first four are this CTA's value columns)
+  auto gblock = [&](int lb) { return rank ? 4 + lb : (lb < 4 ? lb : 8); };
 
   if (threadIdx.x == 0) {
     *sm.abort_flag = 0;
-    mbar_init(smem_u32(sm.qfull), 4);          // one arrival per softmax warp after its Q rows are in TMEM
+    mbar_init(smem_u32(sm.qfull), 4);            // one arrival per softmax warp once its Q rows are in TMEM
+    mbar_init(smem_u32(sm.qrope_full), 1);
     mbar_init(smem_u32(sm.list_ready), 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&sm.kv_full[s]), kProducerThreads);
       mbar_init(smem_u32(&sm.kv_empty[s]), 1);
     }
-    for (int s = 0; s < kSBufs; ++s) {
-      mbar_init(smem_u32(&sm.s_full[s]), 1);
-      mbar_init(smem_u32(&sm.s_empty[s]), 8);   // softmax and exchange warps both read S
-    }
     for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&sm.s_full[s]), 1);
+      mbar_init(smem_u32(&sm.s_read[s]), 4);      // exchange warps have read the score buffer
       mbar_init(smem_u32(&sm.p_full[s]), 4);
       mbar_init(smem_u32(&sm.o_done[s]), 1);
-      mbar_init(smem_u32(&sm.xfull[s]), 4);     // one arrival per peer exchange warp
-      mbar_init(smem_u32(&sm.xfree[s]), 4);     // one arrival per peer exchange warp
-      mbar_init(smem_u32(&sm.xread[s]), 4);     // one arrival per local softmax warp
+      mbar_init(smem_u32(&sm.xfull[s]), 4);       // one arrival per peer exchange warp
+      mbar_init(smem_u32(&sm.xfree[s]), 4);       // one arrival per peer exchange warp
+      mbar_init(smem_u32(&sm.xread[s]), 4);       // one arrival per local softmax warp
     }
     mbar_init(smem_u32(sm.drain), 1);
     fence_barrier_init();
@@ -298,9 +306,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_kv, AttTcParams p) {
     const int n = *sm.n_list;
     const int nch = (n + kChunk - 1) / kChunk;
     const int tid = threadIdx.x - 5 * 32;
-    const int r = tid >> 2, part = tid & 3;               // key row in chunk, quarter of its segments
-    const int spt = 2 * nkb;                              // 16-byte segments per thread
-    const bf16* lat = p.latent + (size_t)(row / p.T) * p.S * p.stride + kb0 * 64 + part * spt * 8;
+    const int r = tid >> 1, half = tid & 1;              // key row in chunk, half of its segments
+    const int spt = nlb * 4;                             // 16-byte segments per thread
+    const bf16* lat = p.latent + (size_t)(row / p.T) * p.S * p.stride;
     for (int j = 0; j < nch; ++j) {
       const int s = j % kStages;
       if (!mbar_wait(smem_u32(&sm.kv_empty[s]), ((j / kStages) & 1) ^ 1, p.status, abort_flag)) break;
@@ -309,10 +317,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_kv, AttTcParams p) {
       const int li = j * kChunk + r;
       const bool ok = li < n;                              // rows past the list are zero-filled
       const bf16* src = lat + (size_t)(ok ? sm.list[li] : 0) * p.stride;
-#pragma unroll 2
+#pragma unroll 4
       for (int i = 0; i < spt; ++i) {
-        const int sg = part * spt + i, kb = sg >> 3, c = sg & 7;
-        cp_async_16(st + kb * kBlockBytes + ((c ^ (r & 7)) << 4), src + i * 8, ok);
+        const int sg = half * spt + i, lb = sg >> 3, c = sg & 7;
+        cp_async_16(st + lb * kBlockBytes + ((c ^ (r & 7)) << 4), src + gblock(lb) * 64 + c * 8, ok);
       }
       // arrives on kv_full[s] once this thread's copies have landed
       cp_async_mbar_arrive(smem_u32(&sm.kv_full[s]));
@@ -321,46 +329,51 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_kv, AttTcParams p) {
   } else if (warp == 4) {
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
+      if (rope) {
+        tma_prefetch_desc(&map_q);
+        mbar_arrive_expect_tx(smem_u32(sm.qrope_full), kQRopeBytes);
+        tma_load_2d(sm.qrope, &map_q, smem_u32(sm.qrope_full), 512, (int)(row * p.H));
+      }
       const uint32_t id_qk = idesc_bf16(128, kChunk);
       const uint32_t id_pv = idesc_bf16(128, 256, false, true);
       bool ok = mbar_wait(smem_u32(sm.qfull), 0, p.status, abort_flag) &&
+                (!rope || mbar_wait(smem_u32(sm.qrope_full), 0, p.status, abort_flag)) &&
                 mbar_wait(smem_u32(sm.list_ready), 0, p.status, abort_flag);
       const int n = ok ? *sm.n_list : 0;
       const int nch = (n + kChunk - 1) / kChunk;
-      // q.k of chunk j may run ahead of P.V of chunk pv while stages and score buffers allow
       int qk = 0, pv = 0;
       unsigned long long t_last = globaltimer();
       uint32_t spins = 0;
       while (ok && pv < nch) {
         bool progressed = false;
-        if (qk < nch && qk - pv < kStages - 1 &&
-            mbar_test_wait(smem_u32(&sm.kv_full[qk % kStages]), (qk / kStages) & 1) &&
-            mbar_test_wait(smem_u32(&sm.s_empty[qk % kSBufs]), ((qk / kSBufs) & 1) ^ 1)) {
+        // q.k of chunk qk: its stage is loaded and P.V of chunk qk-2 (same score buffer) is done
+        if (qk < nch && mbar_test_wait(smem_u32(&sm.kv_full[qk % kStages]), (qk / kStages) & 1) &&
+            mbar_test_wait(smem_u32(&sm.o_done[qk & 1]), ((qk >> 1) & 1) ^ 1)) {
           fence_proxy_async_smem();
           tc_fence_after();
           const uint32_t st = sm.kv + (qk % kStages) * kStageBytes;
-          const uint32_t d = tmem + (qk % kSBufs) * kChunk;
-          for (int kb = 0; kb < nkb; ++kb) {
+          const uint32_t d = tmem + (qk & 1) * kChunk;
+          for (int lb = 0; lb < nlb; ++lb) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const uint64_t bd = desc_sw128(st + kb * kBlockBytes + k * 32);
-              mma_bf16_ts(d, tmem + kQCol + (kb * 4 + k) * 8, bd, id_qk, (kb | k) ? 1u : 0u);
+              const uint64_t bd = desc_sw128(st + lb * kBlockBytes + k * 32);
+              const uint32_t acc = (lb | k) ? 1u : 0u;
+              if (lb < 4) mma_bf16_ts(d, tmem + kQCol + (lb * 4 + k) * 8, bd, id_qk, acc);
+              else mma_bf16_ss(d, desc_sw128(sm.qrope + k * 32), bd, id_qk, acc);
             }
           }
-          mma_commit(smem_u32(&sm.s_full[qk % kSBufs]));
+          mma_commit(smem_u32(&sm.s_full[qk & 1]));
           TRACE(1, qk);
           ++qk;
           progressed = true;
         }
         if (pv < qk && mbar_test_wait(smem_u32(&sm.p_full[pv & 1]), (pv >> 1) & 1)) {
           tc_fence_after();
-          const uint32_t pa = sm.p + (pv & 1) * kPBytes;
           const uint32_t st = sm.kv + (pv % kStages) * kStageBytes;
 #pragma unroll
           for (int k = 0; k < kChunk / 16; ++k) {
-            const uint64_t ad = desc_noswz(pa + k * 256, 128, 512);
             const uint64_t bd = desc_sw128(st + k * 2048, 1024, kBlockBytes);
-            mma_bf16_ss(tmem + kOCol, ad, bd, id_pv, (pv | k) ? 1u : 0u);
+            mma_bf16_ts(tmem + kOCol, tmem + (pv & 1) * kChunk + k * 8, bd, id_pv, (pv | k) ? 1u : 0u);
           }
           mma_commit(smem_u32(&sm.kv_empty[pv % kStages]));
           mma_commit(smem_u32(&sm.o_done[pv & 1]));
@@ -386,54 +399,52 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_kv, AttTcParams p) {
     }
   } else if (warp >= 9) {
     // ---------------------------------------------------------------- score exchange
-    // Two sets of four warps take alternate chunks; set x owns exchange buffer x.
-    const int set = (warp - 9) >> 2;
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
     bool ok = mbar_wait(smem_u32(sm.list_ready), 0, p.status, abort_flag);
     const int n = ok ? *sm.n_list : 0;
     const int nch = (n + kChunk - 1) / kChunk;
-    const uint32_t dst = map_peer(sm.x + (uint32_t)set * kXBytes + (uint32_t)r * kXStride * 4, peer);
-    const uint32_t xfull_peer = map_peer(smem_u32(&sm.xfull[set]), peer);
-    const uint32_t xfree_peer = map_peer(smem_u32(&sm.xfree[set]), peer);
-    for (int j = set; ok && j < nch; j += 2) {
-      const int sb = j % kSBufs, use = j >> 1;       // use = how many times buffer `set` was used before
-      if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), (j / kSBufs) & 1, p.status, abort_flag))) break;
+    const uint32_t dst0 = map_peer(sm.x + (uint32_t)r * kXStride * 4, peer);
+    for (int j = 0; ok && j < nch; ++j) {
+      const int sb = j & 1, use = j >> 1;
+      if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), use & 1, p.status, abort_flag))) break;
       tc_fence_after();
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk, v);
+      uint32_t v[kChunk];
+      tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty[sb]));
+      if (lane == 0) mbar_arrive(smem_u32(&sm.s_read[sb]));
       if (q4 == 1 && lane == 0) TRACE(3, j);
-      // the peer has read its buffer `set` from chunk j-2
-      if (!(ok = wait_cluster(smem_u32(&sm.xfree[set]), (use & 1) ^ 1, p.status, abort_flag))) break;
+      // the peer has read its buffer sb from chunk j-2
+      if (!(ok = wait_cluster(smem_u32(&sm.xfree[sb]), (use & 1) ^ 1, p.status, abort_flag))) break;
+      const uint32_t dst = dst0 + (uint32_t)sb * kXBytes;
 #pragma unroll
       for (int c = 0; c < kChunk; c += 4)
         st_cluster_v4(dst + c * 4, __uint_as_float(v[c]), __uint_as_float(v[c + 1]), __uint_as_float(v[c + 2]),
                       __uint_as_float(v[c + 3]));
       __syncwarp();
-      if (lane == 0) arrive_remote(xfull_peer);  // release: covers the warp's stores
+      if (lane == 0) arrive_remote(map_peer(smem_u32(&sm.xfull[sb]), peer));  // release: covers the warp's stores
       if (q4 == 1 && lane == 0) TRACE(4, j);
-      // once our softmax has read our buffer `set` for chunk j, the peer may refill it (chunk j+2)
+      // once our softmax has read our buffer sb for chunk j, the peer may refill it (chunk j+2)
       if (j + 2 < nch) {
-        if (!(ok = mbar_wait(smem_u32(&sm.xread[set]), use & 1, p.status, abort_flag))) break;
+        if (!(ok = mbar_wait(smem_u32(&sm.xread[sb]), use & 1, p.status, abort_flag))) break;
         __syncwarp();
-        if (lane == 0) arrive_remote_relaxed(xfree_peer);
+        if (lane == 0) arrive_remote_relaxed(map_peer(smem_u32(&sm.xfree[sb]), peer));
       }
     }
   } else if (warp < 4) {
     // ---------------------------------------------------------------- softmax + epilogue
     const int r = warp * 32 + lane;                 // head row == TMEM lane
     const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
-    float m_ref = -INFINITY, l_sum = 0.f;
     {
-      // this CTA's columns of query head r -> TMEM lane r, columns kQCol.. (bf16 pairs)
+      // value-side query columns of head r -> TMEM lane r, columns kQCol.. (bf16 pairs)
       const bool real = r < p.H;
-      const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (row * p.H + (real ? r : 0)) * p.kd + kb0 * 64);
-      for (int c0 = 0; c0 < nkb * 32; c0 += 32) {  // 32 columns = 64 bf16 = 8 x 16 bytes
+      const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (row * p.H + (real ? r : 0)) * p.kd + rank * 256);
+#pragma unroll 1
+      for (int c0 = 0; c0 < 128; c0 += 32) {       // 32 columns = 64 bf16 = 8 x 16 bytes
         uint32_t qv[32];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -450,41 +461,40 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_kv, AttTcParams p) {
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(sm.qfull));
     }
+    float m_ref = -INFINITY, l_sum = 0.f;
     bool ok = mbar_wait(smem_u32(sm.list_ready), 0, p.status, abort_flag);
     const int n = ok ? *sm.n_list : 0;
     const int nch = (n + kChunk - 1) / kChunk;
     const float* xrow = reinterpret_cast<const float*>(gb + (sm.x - base)) + r * kXStride;
     for (int j = 0; ok && j < nch; ++j) {
-      const int sb = j % kSBufs, xb = j & 1;
-      if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), (j / kSBufs) & 1, p.status, abort_flag))) break;
+      const int sb = j & 1, use = j >> 1;
+      if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), use & 1, p.status, abort_flag))) break;
       tc_fence_after();
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk, v);
+      uint32_t v[kChunk];
+      tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
       tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty[sb]));
       if (warp == 0 && lane == 0) TRACE(5, j);
-      if (!(ok = wait_cluster(smem_u32(&sm.xfull[xb]), (j >> 1) & 1, p.status, abort_flag))) break;
+      if (!(ok = wait_cluster(smem_u32(&sm.xfull[sb]), use & 1, p.status, abort_flag))) break;
       if (warp == 0 && lane == 0) TRACE(6, j);
-      const float4* xr = reinterpret_cast<const float4*>(xrow + xb * (kXBytes / 4));
-      float4 pv4[kChunk / 4];
-#pragma unroll
-      for (int c = 0; c < kChunk / 4; ++c) pv4[c] = xr[c];
-      // buffer xb is read (values are in registers); the exchange warps tell the peer
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.xread[xb]));
+      const float4* xr = reinterpret_cast<const float4*>(xrow + sb * (kXBytes / 4));
       const int valid = n - j * kChunk;
-      float x[kChunk];
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < kChunk; ++c) {
-        const float4 q4 = pv4[c >> 2];
-        const float other = (c & 3) == 0 ? q4.x : (c & 3) == 1 ? q4.y : (c & 3) == 2 ? q4.z : q4.w;
-        const float sc = __uint_as_float(v[c]) + other;
-        x[c] = c < valid ? sc * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, x[c]);
+      for (int c4 = 0; c4 < kChunk / 4; ++c4) {
+        const float4 o4 = xr[c4];
+        const float ov[4] = {o4.x, o4.y, o4.z, o4.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int c = 4 * c4 + i;
+          const float x = c < valid ? (__uint_as_float(v[c]) + ov[i]) * p.scale_log2 : -INFINITY;
+          v[c] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
       }
+      // our buffer sb is read (values are in registers); the exchange warps tell the peer
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.xread[sb]));
       if (warp == 0 && lane == 0) TRACE(9, j);
       // move the reference maximum only when it grows by more than 2^8
       const bool grow = mx > m_ref + 8.f;
@@ -505,30 +515,22 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_kv, AttTcParams p) {
         l_sum *= f;
       }
       m_ref = new_ref;
-      float ps[kChunk];
+      uint32_t pk[kChunk / 2];
 #pragma unroll
-      for (int c = 0; c < kChunk; ++c) {
-        ps[c] = ex2(x[c] - m_ref);
-        l_sum += ps[c];
+      for (int c = 0; c < kChunk; c += 2) {
+        const float p0 = ex2(__uint_as_float(v[c]) - m_ref);
+        const float p1 = ex2(__uint_as_float(v[c + 1]) - m_ref);
+        l_sum += p0 + p1;
+        pk[c / 2] = pack_bf16(p0, p1);
       }
       if (warp == 0 && lane == 0) TRACE(10, j);
-      // P buffer (j&1) is free once the P.V of chunk j-2 has completed
-      if (j >= 2 && !(ok = mbar_wait(smem_u32(&sm.o_done[j & 1]), ((j - 2) >> 1) & 1, p.status, abort_flag))) break;
-      if (warp == 0 && lane == 0) TRACE(11, j);
-      const uint32_t prow = sm.p + xb * kPBytes + (uint32_t)(r >> 3) * 512 + (uint32_t)(r & 7) * 16;
-#pragma unroll
-      for (int kc = 0; kc < kChunk / 8; ++kc) {
-        const uint32_t a0 = pack_bf16(ps[8 * kc + 0], ps[8 * kc + 1]);
-        const uint32_t a1 = pack_bf16(ps[8 * kc + 2], ps[8 * kc + 3]);
-        const uint32_t a2 = pack_bf16(ps[8 * kc + 4], ps[8 * kc + 5]);
-        const uint32_t a3 = pack_bf16(ps[8 * kc + 6], ps[8 * kc + 7]);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + kc * 128), "r"(a0), "r"(a1),
-                     "r"(a2), "r"(a3)
-                     : "memory");
-      }
-      fence_proxy_async_smem();
+      // P overwrites the first 32 columns of the score buffer once the exchange warps have read it
+      if (!(ok = mbar_wait(smem_u32(&sm.s_read[sb]), use & 1, p.status, abort_flag))) break;
+      tmem_st_32x32b_x32(tmem + lane_addr + sb * kChunk, pk);
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[xb]));
+      if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[sb]));
       if (warp == 0 && lane == 0) TRACE(7, j);
     }
     // epilogue: O / l -> bf16
@@ -545,12 +547,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_kv, AttTcParams p) {
         if (write && ok) {
 #pragma unroll
           for (int i = 0; i < 32; i += 8) {
-            uint4 pk;
-            pk.x = pack_bf16(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
-            pk.y = pack_bf16(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
-            pk.z = pack_bf16(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
-            pk.w = pack_bf16(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + c + i) = pk;
+            uint4 pkv;
+            pkv.x = pack_bf16(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
+            pkv.y = pack_bf16(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+            pkv.z = pack_bf16(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
+            pkv.w = pack_bf16(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + c + i) = pkv;
           }
         }
       }
@@ -587,9 +589,8 @@ EncodeTiledFn encode_fn() {
 }
 
 size_t smem_bytes(int width) {
-  const size_t x = (2 * kXBytes + 1023) & ~(size_t)1023;
-  return 1024 + x + (size_t)kStages * kStageBytes + 2 * kPBytes + (((size_t)width * 4 + 15) & ~(size_t)15) +
-         8 * 48 + 16;
+  return 1024 + 2 * (size_t)kXBytes + kQRopeBytes + (size_t)kStages * kStageBytes +
+         (((size_t)width * 4 + 15) & ~(size_t)15) + 8 * 32 + 16;
 }
 
 }  // namespace
@@ -627,6 +628,16 @@ cudaError_t launch_attend_tc(const dsa_dims& d, const void* q, const void* k, in
   p.status = device_status_ptr();
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
+  // q viewed as [B*T*H rows, kd cols]; box = 64 cols x 128 rows (the rope block of rank 0)
+  CUtensorMap mq;
+  cuuint64_t qdims[2] = {(cuuint64_t)d.kd, (cuuint64_t)d.batch * d.n_q * d.heads};
+  cuuint64_t qstrides[1] = {(cuuint64_t)d.kd * 2};
+  cuuint32_t qbox[2] = {64u, 128u};
+  cuuint32_t qestr[2] = {1u, 1u};
+  if (enc(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), qdims, qstrides, qbox, qestr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   // latent viewed as [B*S rows, kd cols] with the caller's row stride; box = 64 cols x 1 row (gather4)
   CUtensorMap mkv;
   cuuint64_t kdims[2] = {(cuuint64_t)d.kd, (cuuint64_t)d.batch * d.n_kv};
@@ -641,7 +652,7 @@ cudaError_t launch_attend_tc(const dsa_dims& d, const void* q, const void* k, in
   cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long long rows = (long long)d.batch * d.n_q;
-  attend_tc_kernel<<<dim3((unsigned)(2 * rows)), kThreads, smem, st>>>(mkv, p);
+  attend_tc_kernel<<<dim3((unsigned)(2 * rows)), kThreads, smem, st>>>(mq, mkv, p);
   return cudaGetLastError();
 }
 
