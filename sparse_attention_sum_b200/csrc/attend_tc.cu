@@ -66,8 +66,7 @@ constexpr int kMaxLocalBlocks = 5;     // 64-column blocks per CTA (rank 0 with 
 constexpr int kBlockBytes = kChunk * 128;                   // one 64-col block of a stage: 8 KB
 constexpr int kStageBytes = kMaxLocalBlocks * kBlockBytes;  // 40 KB
 constexpr int kQRopeBytes = 128 * 128;                      // rope query block in smem: 16 KB
-constexpr int kXStride = kChunk + 4;                        // floats per exchange row (bank padding)
-constexpr int kXBytes = 128 * kXStride * 4;                 // 34 KB
+constexpr int kXBytes = kChunk * 128 * 4;                   // exchange tile [key][head] fp32: 32 KB
 constexpr int kBitmapKeys = 65536;                          // dedupe bitmap (8 KB, aliases stage 0)
 constexpr int kQCol = 128;                                  // query columns in TMEM
 constexpr int kOCol = 256;                                  // output accumulator
@@ -114,6 +113,9 @@ __device__ __forceinline__ uint32_t map_peer(uint32_t addr, uint32_t peer) {
 __device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
   asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
+}
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float a) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(a) : "memory");
 }
 __device__ __forceinline__ void arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
@@ -405,7 +407,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     bool ok = mbar_wait(smem_u32(sm.list_ready), 0, p.status, abort_flag);
     const int n = ok ? *sm.n_list : 0;
     const int nch = (n + kChunk - 1) / kChunk;
-    const uint32_t dst0 = map_peer(sm.x + (uint32_t)r * kXStride * 4, peer);
+    const uint32_t dst0 = map_peer(sm.x + (uint32_t)r * 4, peer);   // column r of the [key][head] tile
     for (int j = 0; ok && j < nch; ++j) {
       const int sb = j & 1, use = j >> 1;
       if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), use & 1, p.status, abort_flag))) break;
@@ -421,10 +423,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       // the peer has read its buffer sb from chunk j-2
       if (!(ok = wait_cluster(smem_u32(&sm.xfree[sb]), (use & 1) ^ 1, p.status, abort_flag))) break;
       const uint32_t dst = dst0 + (uint32_t)sb * kXBytes;
+      // key-major: for each key the warp's 32 lanes write 128 contiguous bytes
 #pragma unroll
-      for (int c = 0; c < kChunk; c += 4)
-        st_cluster_v4(dst + c * 4, __uint_as_float(v[c]), __uint_as_float(v[c + 1]), __uint_as_float(v[c + 2]),
-                      __uint_as_float(v[c + 3]));
+      for (int c = 0; c < kChunk; ++c) st_cluster_f32(dst + c * 512, __uint_as_float(v[c]));
       __syncwarp();
       if (lane == 0) arrive_remote(map_peer(smem_u32(&sm.xfull[sb]), peer));  // release: covers the warp's stores
       if (q4 == 1 && lane == 0) TRACE(4, j);
@@ -465,7 +466,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     bool ok = mbar_wait(smem_u32(sm.list_ready), 0, p.status, abort_flag);
     const int n = ok ? *sm.n_list : 0;
     const int nch = (n + kChunk - 1) / kChunk;
-    const float* xrow = reinterpret_cast<const float*>(gb + (sm.x - base)) + r * kXStride;
+    const float* xcol = reinterpret_cast<const float*>(gb + (sm.x - base)) + r;   // column r of [key][head]
     for (int j = 0; ok && j < nch; ++j) {
       const int sb = j & 1, use = j >> 1;
       if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), use & 1, p.status, abort_flag))) break;
@@ -477,20 +478,14 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       if (warp == 0 && lane == 0) TRACE(5, j);
       if (!(ok = wait_cluster(smem_u32(&sm.xfull[sb]), use & 1, p.status, abort_flag))) break;
       if (warp == 0 && lane == 0) TRACE(6, j);
-      const float4* xr = reinterpret_cast<const float4*>(xrow + sb * (kXBytes / 4));
+      const float* xr = xcol + sb * (kXBytes / 4);
       const int valid = n - j * kChunk;
       float mx = -INFINITY;
 #pragma unroll
-      for (int c4 = 0; c4 < kChunk / 4; ++c4) {
-        const float4 o4 = xr[c4];
-        const float ov[4] = {o4.x, o4.y, o4.z, o4.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int c = 4 * c4 + i;
-          const float x = c < valid ? (__uint_as_float(v[c]) + ov[i]) * p.scale_log2 : -INFINITY;
-          v[c] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
+      for (int c = 0; c < kChunk; ++c) {
+        const float x = c < valid ? (__uint_as_float(v[c]) + xr[c * 128]) * p.scale_log2 : -INFINITY;
+        v[c] = __float_as_uint(x);
+        mx = fmaxf(mx, x);
       }
       // our buffer sb is read (values are in registers); the exchange warps tell the peer
       __syncwarp();
