@@ -12,8 +12,9 @@
 // largest key tau and how many keys equal to tau are still needed.  Each warp
 // then walks a contiguous segment of the row 32 keys at a time; ballots and a
 // block-wide prefix sum place every key > tau and the lowest-index keys == tau,
-// which keeps the tie rule exact.  Finally the k (key, index) pairs are put in
-// rank order by a bitonic sort of 64-bit composites (~key << 32 | index).
+// which keeps the tie rule exact.  Finally the (key, index) pairs are put in
+// rank order by a stable four-pass LSD radix sort on the key (descending), so
+// equal keys keep ascending index order.
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
 
@@ -50,22 +51,65 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch /*>= BLO
   return warp_base + x - v;
 }
 
+// Stable LSD radix sort of m (key, index) pairs by key, descending: four 8-bit
+// passes.  Each warp owns a contiguous segment and per-(digit, warp) offsets
+// keep equal keys in their input order, so ties stay in ascending index order.
+// a, b: ping-pong buffers of m uint64 (key << 32 | index); hist: NW*256 uint32.
+// The result ends in `a`.
 template <int BLOCK>
-__device__ void bitonic_sort_u64(uint64_t* a, int n /* power of two */) {
-  for (int size = 2; size <= n; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < (n >> 1); i += BLOCK) {
-        int lo = 2 * i - (i & (stride - 1));
-        int hi = lo + stride;
-        bool up = (lo & size) == 0;
-        uint64_t x = a[lo], y = a[hi];
-        if ((x > y) == up) {
-          a[lo] = y;
-          a[hi] = x;
-        }
-      }
-      __syncthreads();
+__device__ void radix_sort_desc(uint64_t* a, uint64_t* b, uint32_t* hist, int* scan, int m) {
+  constexpr int NW = BLOCK / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int seg = ((m + NW - 1) / NW + 31) & ~31;
+  const int w0 = warp * seg, w1 = min(m, w0 + seg);
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int shift = 32; shift < 64; shift += 8) {
+    for (int i = threadIdx.x; i < NW * 256; i += BLOCK) hist[i] = 0u;
+    __syncthreads();
+    uint32_t* h = hist + warp * 256;
+    for (int g = w0; g < w1; g += 32) {
+      const int i = g + lane;
+      const int d = i < w1 ? 255 - (int)((a[i] >> shift) & 255u) : -1;
+      const uint32_t peers = __match_any_sync(0xffffffffu, d);
+      if (d >= 0 && (peers & lt) == 0u) h[d] += __popc(peers);
+      __syncwarp();
     }
+    __syncthreads();
+    // offset[w][d] = sum over digits < d of all counts + counts of warps < w at digit d
+    int tot = 0;
+    if (threadIdx.x < 256) {
+      const int d = threadIdx.x;
+      for (int w = 0; w < NW; ++w) {
+        const uint32_t c = hist[w * 256 + d];
+        hist[w * 256 + d] = tot;
+        tot += c;
+      }
+    }
+    int total;
+    const int base = block_exclusive_scan<BLOCK>(threadIdx.x < 256 ? tot : 0, scan, total);
+    if (threadIdx.x < 256)
+      for (int w = 0; w < NW; ++w) hist[w * 256 + threadIdx.x] += base;
+    __syncthreads();
+    for (int g = w0; g < w1; g += 32) {
+      const int i = g + lane;
+      uint64_t e = 0;
+      int d = -1;
+      if (i < w1) {
+        e = a[i];
+        d = 255 - (int)((e >> shift) & 255u);
+      }
+      const uint32_t peers = __match_any_sync(0xffffffffu, d);
+      if (d >= 0) {
+        b[h[d] + __popc(peers & lt)] = e;
+      }
+      __syncwarp();
+      if (d >= 0 && (peers & lt) == 0u) h[d] += __popc(peers);
+      __syncwarp();
+    }
+    __syncthreads();
+    uint64_t* t = a;
+    a = b;
+    b = t;
   }
 }
 
@@ -73,10 +117,12 @@ template <int BLOCK>
 __global__ void __launch_bounds__(BLOCK)
 topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restrict__ q_pos,
             const int32_t* __restrict__ kv_start, const int32_t* __restrict__ kv_len, int k,
-            int kpow2, int cache_cap, int32_t* __restrict__ idx_out, float* __restrict__ vals_out) {
+            int cache_cap, int32_t* __restrict__ idx_out, float* __restrict__ vals_out) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  uint64_t* sel = reinterpret_cast<uint64_t*>(smem_raw);            // [kpow2]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(sel + kpow2);         // [256]
+  uint64_t* sel = reinterpret_cast<uint64_t*>(smem_raw);            // [k]   selected (key, index)
+  uint64_t* tmp = sel + k;                                           // [k]   sort ping-pong
+  uint32_t* rhist = reinterpret_cast<uint32_t*>(tmp + k);            // [BLOCK/32 * 256]
+  uint32_t* hist = rhist + (BLOCK / 32) * 256;                       // [256]
   int* scan = reinterpret_cast<int*>(hist + 256);                    // [64]
   uint32_t* cache = reinterpret_cast<uint32_t*>(scan + 64);          // [cache_cap]
   __shared__ uint32_t s_prefix, s_krem;
@@ -92,19 +138,16 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
   const bool cached = n <= cache_cap;
 
   if (n <= k) {
-    // every visible key is selected: just rank them
-    for (int i = threadIdx.x; i < kpow2; i += BLOCK) {
-      uint64_t c = ~0ull;
-      if (i < n) c = ((uint64_t)(~score_key(srow[r.lo + i])) << 32) | (uint32_t)(r.lo + i);
-      sel[i] = c;
-    }
+    // every visible key is selected: rank them (inputs in index order)
+    for (int i = threadIdx.x; i < n; i += BLOCK)
+      sel[i] = ((uint64_t)score_key(srow[r.lo + i]) << 32) | (uint32_t)(r.lo + i);
     __syncthreads();
-    bitonic_sort_u64<BLOCK>(sel, kpow2);
+    radix_sort_desc<BLOCK>(sel, tmp, rhist, scan, n);
     for (int i = threadIdx.x; i < k; i += BLOCK) {
       if (i < n) {
-        uint64_t c = sel[i];
+        const uint64_t c = sel[i];
         orow[i] = (int32_t)(uint32_t)c;
-        if (vrow) vrow[i] = key_score(~(uint32_t)(c >> 32));
+        if (vrow) vrow[i] = key_score((uint32_t)(c >> 32));
       } else {
         orow[i] = DSA_INVALID;
         if (vrow) vrow[i] = -INFINITY;
@@ -207,7 +250,7 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
     const bool is_eq = i < w1 && key == tau;
     const uint32_t m_gt = __ballot_sync(0xffffffffu, is_gt);
     const uint32_t m_eq = __ballot_sync(0xffffffffu, is_eq);
-    const uint64_t c = ((uint64_t)(~key) << 32) | (uint32_t)(r.lo + i);
+    const uint64_t c = ((uint64_t)key << 32) | (uint32_t)(r.lo + i);
     if (is_gt) sel[gt_base + __popc(m_gt & lt_mask)] = c;
     if (is_eq) {
       int rank = eq_base + __popc(m_eq & lt_mask);
@@ -216,35 +259,37 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
     gt_base += __popc(m_gt);
     eq_base += __popc(m_eq);
   }
-  for (int i = k + threadIdx.x; i < kpow2; i += BLOCK) sel[i] = ~0ull;
   __syncthreads();
-  bitonic_sort_u64<BLOCK>(sel, kpow2);
+  // gt keys came first in index order, then the taken tau keys in index order:
+  // the stable sort keeps every run of equal keys in ascending index order
+  radix_sort_desc<BLOCK>(sel, tmp, rhist, scan, k);
   for (int i = threadIdx.x; i < k; i += BLOCK) {
-    uint64_t c = sel[i];
+    const uint64_t c = sel[i];
     orow[i] = (int32_t)(uint32_t)c;
-    if (vrow) vrow[i] = key_score(~(uint32_t)(c >> 32));
+    if (vrow) vrow[i] = key_score((uint32_t)(c >> 32));
   }
 }
 
 cudaError_t launch_topk(const dsa_dims& d, const float* scores, const int32_t* q_pos,
                         const int32_t* kv_start, const int32_t* kv_len, int k, int32_t* idx,
                         float* vals, cudaStream_t st) {
-  int kpow2 = 1;
-  while (kpow2 < k) kpow2 <<= 1;
+  const int block = d.n_kv > 8192 ? 1024 : 512;
   int cache_cap = d.n_kv < kTopkCacheMax ? d.n_kv : kTopkCacheMax;
-  size_t smem = (size_t)kpow2 * 8 + 256 * 4 + 64 * 4 + (size_t)cache_cap * 4;
+  const size_t fixed = (size_t)k * 16 + (size_t)(block / 32) * 256 * 4 + 256 * 4 + 64 * 4;
+  if (fixed + (size_t)cache_cap * 4 > 220 * 1024) cache_cap = (int)((220 * 1024 - fixed) / 4);
+  size_t smem = fixed + (size_t)cache_cap * 4;
   dim3 grid(d.n_q, d.batch);
   cudaError_t e;
   if (d.n_kv > 8192) {
     auto kern = topk_kernel<1024>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, 1024, smem, st>>>(d, scores, q_pos, kv_start, kv_len, k, kpow2, cache_cap, idx, vals);
+    kern<<<grid, 1024, smem, st>>>(d, scores, q_pos, kv_start, kv_len, k, cache_cap, idx, vals);
   } else {
     auto kern = topk_kernel<512>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, 512, smem, st>>>(d, scores, q_pos, kv_start, kv_len, k, kpow2, cache_cap, idx, vals);
+    kern<<<grid, 512, smem, st>>>(d, scores, q_pos, kv_start, kv_len, k, cache_cap, idx, vals);
   }
   return cudaGetLastError();
 }
