@@ -11,18 +11,21 @@
 // 128 x 512 fp32 output accumulator fills all of one SM's tensor memory, so a
 // query is processed by a cluster of two CTAs, each owning half of the value
 // columns and the matching half of the key columns:
-//   rank 0: latent columns [0,256) (+ the 64 rope columns [512,576) when kd = 576),
-//           O[:, 0:256)
-//   rank 1: latent columns [256,512), O[:, 256:512)
+//   rank 0: latent columns [0,256)   (+ rope columns [512,544) when kd = 576), O[:, 0:256)
+//   rank 1: latent columns [256,512) (+ rope columns [544,576) when kd = 576), O[:, 256:512)
 // Each CTA gathers only its own columns of every selected latent row (cp.async
 // straight into the 128-byte-swizzled operand layout), so no byte is loaded
 // twice.  Per 64-key chunk each CTA computes the q.k partial over its columns;
 // the two fp32 partial tiles are exchanged through distributed shared memory
 // and summed (fp32 addition is commutative, so both CTAs see bit-identical
-// scores and take identical online-softmax decisions).
+// scores and take identical online-softmax decisions).  The exchange uses
+// st.async, which completes the peer's barrier by byte count, so the sender
+// never waits for a round trip.
 //
-// Tensor memory (512 columns): score buffers 0-63 and 64-127, the CTA's query
-// columns 128-255 as the A operand of q.k (two bf16 per column), O 256-511.
+// Tensor memory (512 columns): score buffers 0-63 and 64-127, the CTA's four
+// value-side query blocks 128-255 as the A operand of q.k (two bf16 per
+// column), O 256-511.  The 32 rope columns of each CTA use a 64-byte-swizzled
+// shared-memory operand.
 // The bf16 probabilities overwrite the first 32 columns of their score buffer
 // and feed P.V straight from tensor memory.  Every tcgen05.mma here costs about
 // 100 cycles whatever its N up to 128, so q.k uses N = 64 keys per instruction
@@ -33,7 +36,7 @@
 // softmax and the epilogue (one head row per thread, TMEM lanes 0-127); warps
 // 9-12 read the same score rows and push them to the peer (buffer reuse is
 // acknowledged by the peer); warp 4 issues tcgen05.mma from a polling scheduler
-// (and on rank 0 loads the rope query block by TMA); warps 5-8 stage and
+// (and loads the CTA's rope query columns by TMA); warps 5-8 stage and
 // deduplicate the index row, then gather the selected rows with 16-byte
 // cp.async.  Every mbarrier wait is bounded.
 #include <cuda.h>
@@ -61,11 +64,11 @@ namespace {
 using namespace sm100;
 
 constexpr int kChunk = 64;             // keys per pipeline step (N of q.k, K of P.V)
-constexpr int kStages = 3;             // gathered key/value stages
-constexpr int kMaxLocalBlocks = 5;     // 64-column blocks per CTA (rank 0 with the rope block)
+constexpr int kStages = 4;             // gathered key/value stages
 constexpr int kBlockBytes = kChunk * 128;                   // one 64-col block of a stage: 8 KB
-constexpr int kStageBytes = kMaxLocalBlocks * kBlockBytes;  // 40 KB
-constexpr int kQRopeBytes = 128 * 128;                      // rope query block in smem: 16 KB
+constexpr int kRopeOff = 4 * kBlockBytes;                   // 32 rope columns after the 4 value blocks
+constexpr int kStageBytes = kRopeOff + kChunk * 64;         // 36 KB
+constexpr int kQRopeBytes = 128 * 64;                       // rope query columns in smem: 8 KB
 constexpr int kXBytes = kChunk * 128 * 4;                   // exchange tile [key][head] fp32: 32 KB
 constexpr int kBitmapKeys = 65536;                          // dedupe bitmap (8 KB, aliases stage 0)
 constexpr int kQCol = 128;                                  // query columns in TMEM
@@ -114,8 +117,10 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, f
   asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
 }
-__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float a) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(a) : "memory");
+__device__ __forceinline__ void st_async_b32(uint32_t addr, uint32_t v, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(addr), "r"(v),
+               "r"(remote_bar)
+               : "memory");
 }
 __device__ __forceinline__ void arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
@@ -267,10 +272,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   const uint32_t rank = cluster_rank();
   const uint32_t peer = rank ^ 1u;
   const size_t row = blockIdx.x >> 1;            // query row b*T + t
-  const bool rope = rank == 0 && p.kd == 576;    // rank 0 also owns the rope block
-  const int nlb = rope ? 5 : 4;                  // 64-column blocks gathered and used by q.k
-  // global 64-column block of local block lb (the first four are this CTA's value columns)
-  auto gblock = [&](int lb) { return rank ? 4 + lb : (lb < 4 ? lb : 8); };
+  const bool rope = p.kd == 576;                 // each CTA owns 32 of the 64 rope columns
+  const int rope_col = 512 + 32 * (int)rank;
 
   if (threadIdx.x == 0) {
     *sm.abort_flag = 0;
@@ -286,12 +289,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       mbar_init(smem_u32(&sm.s_read[s]), 4);      // exchange warps have read the score buffer
       mbar_init(smem_u32(&sm.p_full[s]), 4);
       mbar_init(smem_u32(&sm.o_done[s]), 1);
-      mbar_init(smem_u32(&sm.xfull[s]), 4);       // one arrival per peer exchange warp
+      mbar_init(smem_u32(&sm.xfull[s]), 1);       // armed by our softmax; completed by the peer's st.async bytes
       mbar_init(smem_u32(&sm.xfree[s]), 4);       // one arrival per peer exchange warp
       mbar_init(smem_u32(&sm.xread[s]), 4);       // one arrival per local softmax warp
     }
     mbar_init(smem_u32(sm.drain), 1);
     fence_barrier_init();
+    for (int s = 0; s < 2; ++s) mbar_arrive_expect_tx(smem_u32(&sm.xfull[s]), kXBytes);  // first use of each buffer
   }
   if (warp == 4) tmem_alloc(smem_u32(sm.tmem_slot), 512);
   tc_fence_before();
@@ -309,7 +313,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const int nch = (n + kChunk - 1) / kChunk;
     const int tid = threadIdx.x - 5 * 32;
     const int r = tid >> 1, half = tid & 1;              // key row in chunk, half of its segments
-    const int spt = nlb * 4;                             // 16-byte segments per thread
+    const int spt = rope ? 18 : 16;                      // 16-byte segments per thread (36 or 32 per row)
     const bf16* lat = p.latent + (size_t)(row / p.T) * p.S * p.stride;
     for (int j = 0; j < nch; ++j) {
       const int s = j % kStages;
@@ -319,10 +323,16 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       const int li = j * kChunk + r;
       const bool ok = li < n;                              // rows past the list are zero-filled
       const bf16* src = lat + (size_t)(ok ? sm.list[li] : 0) * p.stride;
-#pragma unroll 4
+#pragma unroll 2
       for (int i = 0; i < spt; ++i) {
-        const int sg = half * spt + i, lb = sg >> 3, c = sg & 7;
-        cp_async_16(st + lb * kBlockBytes + ((c ^ (r & 7)) << 4), src + gblock(lb) * 64 + c * 8, ok);
+        const int sg = half * spt + i;
+        if (sg < 32) {   // value-side block lb, 128-byte swizzle
+          const int lb = sg >> 3, c = sg & 7;
+          cp_async_16(st + lb * kBlockBytes + ((c ^ (r & 7)) << 4), src + (4 * (int)rank + lb) * 64 + c * 8, ok);
+        } else {         // rope columns, 64-byte rows with the 64-byte swizzle
+          const int c = sg - 32;
+          cp_async_16(st - r * 128 + kRopeOff + r * 64 + ((c ^ ((r >> 1) & 3)) << 4), src + rope_col + c * 8, ok);
+        }
       }
       // arrives on kv_full[s] once this thread's copies have landed
       cp_async_mbar_arrive(smem_u32(&sm.kv_full[s]));
@@ -334,7 +344,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       if (rope) {
         tma_prefetch_desc(&map_q);
         mbar_arrive_expect_tx(smem_u32(sm.qrope_full), kQRopeBytes);
-        tma_load_2d(sm.qrope, &map_q, smem_u32(sm.qrope_full), 512, (int)(row * p.H));
+        tma_load_2d(sm.qrope, &map_q, smem_u32(sm.qrope_full), rope_col, (int)(row * p.H));
       }
       const uint32_t id_qk = idesc_bf16(128, kChunk);
       const uint32_t id_pv = idesc_bf16(128, 256, false, true);
@@ -355,14 +365,16 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           tc_fence_after();
           const uint32_t st = sm.kv + (qk % kStages) * kStageBytes;
           const uint32_t d = tmem + (qk & 1) * kChunk;
-          for (int lb = 0; lb < nlb; ++lb) {
+          for (int lb = 0; lb < 4; ++lb) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint64_t bd = desc_sw128(st + lb * kBlockBytes + k * 32);
-              const uint32_t acc = (lb | k) ? 1u : 0u;
-              if (lb < 4) mma_bf16_ts(d, tmem + kQCol + (lb * 4 + k) * 8, bd, id_qk, acc);
-              else mma_bf16_ss(d, desc_sw128(sm.qrope + k * 32), bd, id_qk, acc);
-            }
+            for (int k = 0; k < 4; ++k)
+              mma_bf16_ts(d, tmem + kQCol + (lb * 4 + k) * 8, desc_sw128(st + lb * kBlockBytes + k * 32), id_qk,
+                          (lb | k) ? 1u : 0u);
+          }
+          if (rope) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+              mma_bf16_ss(d, desc_sw64(sm.qrope + k * 32), desc_sw64(st + kRopeOff + k * 32), id_qk, 1u);
           }
           mma_commit(smem_u32(&sm.s_full[qk & 1]));
           TRACE(1, qk);
@@ -423,11 +435,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       // the peer has read its buffer sb from chunk j-2
       if (!(ok = wait_cluster(smem_u32(&sm.xfree[sb]), (use & 1) ^ 1, p.status, abort_flag))) break;
       const uint32_t dst = dst0 + (uint32_t)sb * kXBytes;
-      // key-major: for each key the warp's 32 lanes write 128 contiguous bytes
+      // key-major: for each key the warp's 32 lanes write 128 contiguous bytes; each
+      // store completes its bytes on the peer's barrier (no round trip here)
+      const uint32_t xbar = map_peer(smem_u32(&sm.xfull[sb]), peer);
 #pragma unroll
-      for (int c = 0; c < kChunk; ++c) st_cluster_f32(dst + c * 512, __uint_as_float(v[c]));
-      __syncwarp();
-      if (lane == 0) arrive_remote(map_peer(smem_u32(&sm.xfull[sb]), peer));  // release: covers the warp's stores
+      for (int c = 0; c < kChunk; ++c) st_async_b32(dst + c * 512, v[c], xbar);
       if (q4 == 1 && lane == 0) TRACE(4, j);
       // once our softmax has read our buffer sb for chunk j, the peer may refill it (chunk j+2)
       if (j + 2 < nch) {
@@ -477,7 +489,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       tmem_ld_wait();
       if (warp == 0 && lane == 0) TRACE(5, j);
       if (!(ok = wait_cluster(smem_u32(&sm.xfull[sb]), use & 1, p.status, abort_flag))) break;
-      if (warp == 0 && lane == 0) TRACE(6, j);
+      if (warp == 0 && lane == 0) {
+        TRACE(6, j);
+        if (j + 2 < nch) mbar_arrive_expect_tx(smem_u32(&sm.xfull[sb]), kXBytes);  // arm the next use
+      }
       const float* xr = xcol + sb * (kXBytes / 4);
       const int valid = n - j * kChunk;
       float mx = -INFINITY;
@@ -623,14 +638,14 @@ cudaError_t launch_attend_tc(const dsa_dims& d, const void* q, const void* k, in
   p.status = device_status_ptr();
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
-  // q viewed as [B*T*H rows, kd cols]; box = 64 cols x 128 rows (the rope block of rank 0)
+  // q viewed as [B*T*H rows, kd cols]; box = 32 cols x 128 rows, 64-byte swizzle (a CTA's rope columns)
   CUtensorMap mq;
   cuuint64_t qdims[2] = {(cuuint64_t)d.kd, (cuuint64_t)d.batch * d.n_q * d.heads};
   cuuint64_t qstrides[1] = {(cuuint64_t)d.kd * 2};
-  cuuint32_t qbox[2] = {64u, 128u};
+  cuuint32_t qbox[2] = {32u, 128u};
   cuuint32_t qestr[2] = {1u, 1u};
   if (enc(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), qdims, qstrides, qbox, qestr,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   // latent viewed as [B*S rows, kd cols] with the caller's row stride; box = 64 cols x 1 row (gather4)

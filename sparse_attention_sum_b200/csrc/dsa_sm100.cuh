@@ -231,6 +231,18 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t sbo = 10
   return d;
 }
 
+// Same for the 64-byte swizzle (layout code 4): rows of 64 bytes (32 bf16),
+// 8-row atoms of 512 bytes stacked at `sbo` bytes.
+__device__ __forceinline__ uint64_t desc_sw64(uint32_t saddr, uint32_t sbo = 512) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)4 << 61;
+  return d;
+}
+
 // Instruction descriptor of tcgen05.mma kind::f16: bf16 A and B, fp32 D,
 // M = 128 or 64, N multiple of 16 (<= 256); a_mn / b_mn select MN-major operands.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn = false, bool b_mn = false) {
