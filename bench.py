@@ -1,7 +1,7 @@
 """Benchmark of the DSA layer on B200: query tokens / second and roofline fraction.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload prefill|decode|chunked|kpool] [--no-extras]
+                    [--workload prefill|decode|chunked] [--no-extras] [--profile-once]
 
 A step is one pass of the whole hot path over one batch: dsa_layer_forward
 (indexer scores -> top-k -> sparse MLA attend) on the workload's synthetic
@@ -9,6 +9,10 @@ inputs, already resident in HBM.  L2 is flushed (a 256 MiB write) before each
 timed step and each step is timed alone with CUDA events on the launching
 stream.  Under torchrun every rank runs its own replica of the workload
 (weak scaling, no data-path collective); the step time is the max over ranks.
+
+``--profile-once`` makes one call of each stage entry point (dsa_index_scores,
+dsa_topk, dsa_sparse_attend) on the workload and exits, timing nothing: the
+command an ncu capture of the three stage kernels runs.
 
 ``--impl reference`` times the CPU oracle (the reference arm for this build)
 on a bounded sample of the same workload and prints the same JSON line.
@@ -249,6 +253,31 @@ def profiled_traffic():
         return {}
 
 
+def profile_once(a):
+    """One call of each stage entry point (three launches), for a profiler to capture."""
+    import sparse_attention_sum_b200 as dsa
+    from sparse_attention_sum_b200 import runner
+    torch.cuda.set_device(0)
+    dsa.lib()
+    wl = workloads.make(a.workload)
+    t = device_inputs(wl)
+    dims, args = layer_args(wl, t)
+    bufs = runner.LayerBuffers(dims, "cuda", torch.bfloat16, with_idx=True)
+    B, T, S = wl.batch, wl.n_q, wl.n_kv
+    scores = bufs.ws[: B * T * S * 4].view(torch.float32)
+    dsa.index_scores(dims, args["q_idx"], args["k_idx"], args["w"], args["idx_scale"], args["q_pos"],
+                     args["kv_start"], args["kv_len"], scores)
+    dsa.topk(dims, scores, args["q_pos"], args["kv_start"], args["kv_len"], wl.top_k, bufs.idx)
+    dsa.sparse_attend(dims, args["q"], args["k"], args["k_row_stride"], args["v"], args["v_row_stride"],
+                      bufs.idx, wl.top_k, args["attn_scale"], bufs.out)
+    torch.cuda.synchronize()
+    status = dsa.get_device_status()
+    print(json.dumps({"profile_once": wl.name, "device_status": status,
+                      "device_bytes": torch.cuda.max_memory_allocated()}), flush=True)
+    if status != 0:
+        sys.exit(1)
+
+
 def run_ours(a):
     import sparse_attention_sum_b200 as dsa
     from sparse_attention_sum_b200 import runner
@@ -453,10 +482,14 @@ def main(argv=None):
     ap.add_argument("--workload", choices=["prefill", "decode", "chunked"], default="prefill")
     ap.add_argument("--no-extras", action="store_true", help="skip stages, decode, e2e and CPU baseline")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--profile-once", action="store_true",
+                    help="one call of each stage entry point, no timing (for an ncu capture)")
     a = ap.parse_args(argv)
     a.warmup = max(3, a.warmup)  # at least three untimed warm-up steps
     if a.impl == "reference":
         run_reference(a)
+    elif a.profile_once:
+        profile_once(a)
     else:
         run_ours(a)
 

@@ -32,8 +32,9 @@
 // and P.V N = 256 value columns.  The running maximum only moves (and O is
 // rescaled in TMEM) when it grows by more than 2^8.
 //
-// Warp roles per CTA: warps 0-3 load the query columns into TMEM, then run the
-// softmax and the epilogue (one head row per thread, TMEM lanes 0-127); warps
+// Warp roles per CTA: warps 0-3 and 13-16 load the query columns into TMEM, then
+// run the softmax and the epilogue (one head row per thread, TMEM lanes 0-127;
+// the two groups take the two halves of every chunk's keys and of O); warps
 // 9-12 read the same score rows and push them to the peer (buffer reuse is
 // acknowledged by the peer); warp 4 issues tcgen05.mma from a polling scheduler
 // (and loads the CTA's rope query columns by TMA); warps 5-8 stage and
@@ -73,7 +74,7 @@ constexpr int kXBytes = kChunk * 128 * 4;                   // exchange tile [ke
 constexpr int kBitmapKeys = 65536;                          // dedupe bitmap (8 KB, aliases stage 0)
 constexpr int kQCol = 128;                                  // query columns in TMEM
 constexpr int kOCol = 256;                                  // output accumulator
-constexpr int kThreads = 416;          // 13 warps
+constexpr int kThreads = 544;          // 17 warps
 constexpr int kProducerThreads = 128;  // warps 5-8
 
 struct AttTcParams {
@@ -90,10 +91,12 @@ struct AttTcParams {
 
 struct Smem {
   uint32_t kv, x, qrope;     // shared-window addresses
-  int* list;
-  uint32_t* bitmap;
+  uint16_t* list;            // deduplicated key rows (n_kv <= 65536 on this path)
+  int* raw;                  // the index row as given (staged in gather stage 0)
+  uint32_t* bitmap;          // dedupe bitmap (gather stage 0, before the first gather)
+  float* mx;                 // [2 parities][2 groups][128 rows] half-row maxima, then partial sums
   uint64_t *qfull, *qrope_full, *list_ready, *kv_full, *kv_empty, *s_full, *s_read, *p_full, *o_done, *xfull,
-      *xfree, *xread, *drain;
+      *xfree, *xread, *mxready, *lready, *drain;
   uint32_t* tmem_slot;
   int* n_list;
   int* dup_flag;
@@ -186,13 +189,13 @@ __device__ void build_list(const AttTcParams& p, const Smem& sm, size_t row) {
   const int lane = threadIdx.x & 31;
   const int32_t* irow = p.idx + row * p.width;
   const int words = (p.S + 31) >> 5;
-  for (int e = tid; e < p.width; e += kProducerThreads) sm.list[e] = irow[e];
+  for (int e = tid; e < p.width; e += kProducerThreads) sm.raw[e] = irow[e];
   for (int i = tid; i < words; i += kProducerThreads) sm.bitmap[i] = 0u;
   if (tid == 0) *sm.dup_flag = 0;
   named_sync(1, kProducerThreads);
   int dup = 0;
   for (int e = tid; e < p.width; e += kProducerThreads) {
-    const int key = sm.list[e];
+    const int key = sm.raw[e];
     if (key >= 0 && key < p.S) {
       const uint32_t bit = 1u << (key & 31);
       dup |= (atomicOr(&sm.bitmap[key >> 5], bit) & bit) != 0u;
@@ -206,11 +209,11 @@ __device__ void build_list(const AttTcParams& p, const Smem& sm, size_t row) {
     named_sync(1, kProducerThreads);
   }
   if (tid < 32) {
-    // in-place compaction: a group is read before any of its slots are written
+    // order-preserving compaction into the key list
     int n = 0;
     for (int e0 = 0; e0 < p.width; e0 += 32) {
       const int e = e0 + lane;
-      const int key = e < p.width ? sm.list[e] : -1;
+      const int key = e < p.width ? sm.raw[e] : -1;
       bool keep = key >= 0 && key < p.S;
       if (has_dup) {
         // first occurrence only: not seen in an earlier group, lowest lane in this group
@@ -220,7 +223,7 @@ __device__ void build_list(const AttTcParams& p, const Smem& sm, size_t row) {
         if (keep) atomicOr(&sm.bitmap[key >> 5], 1u << (key & 31));
       }
       const uint32_t m = __ballot_sync(0xffffffffu, keep);
-      if (keep) sm.list[n + __popc(m & ((1u << lane) - 1u))] = key;
+      if (keep) sm.list[n + __popc(m & ((1u << lane) - 1u))] = (uint16_t)key;
       n += __popc(m);
       __syncwarp();
     }
@@ -236,7 +239,7 @@ __device__ void build_list(const AttTcParams& p, const Smem& sm, size_t row) {
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
                  AttTcParams p) {
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ int s_misc[4];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -246,9 +249,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   sm.qrope = sm.x + 2 * kXBytes;
   sm.kv = sm.qrope + kQRopeBytes;
   uint32_t off = sm.kv + kStages * kStageBytes - base;
-  sm.bitmap = reinterpret_cast<uint32_t*>(gb + (sm.kv - base));  // stage 0 is not written before the list is built
-  sm.list = reinterpret_cast<int*>(gb + off);
-  off += ((uint32_t)p.width * 4u + 15u) & ~15u;
+  // stage 0 is not gathered into before the list is built: bitmap (8 KB) then the raw row
+  sm.bitmap = reinterpret_cast<uint32_t*>(gb + (sm.kv - base));
+  sm.raw = reinterpret_cast<int*>(gb + (sm.kv - base) + kBitmapKeys / 8);
+  sm.list = reinterpret_cast<uint16_t*>(gb + off);
+  off += ((uint32_t)p.width * 2u + 15u) & ~15u;
+  sm.mx = reinterpret_cast<float*>(gb + off);
+  off += 2 * 2 * 128 * 4;
   uint64_t* bars = reinterpret_cast<uint64_t*>(gb + off);
   sm.qfull = bars;
   sm.qrope_full = bars + 1;
@@ -262,7 +269,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   sm.xfull = sm.o_done + 2;
   sm.xfree = sm.xfull + 2;
   sm.xread = sm.xfree + 2;
-  sm.drain = sm.xread + 2;
+  sm.mxready = sm.xread + 2;
+  sm.lready = sm.mxready + 2;
+  sm.drain = sm.lready + 1;
   sm.tmem_slot = reinterpret_cast<uint32_t*>(sm.drain + 1);
   sm.n_list = &s_misc[0];
   sm.dup_flag = &s_misc[1];
@@ -277,7 +286,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
   if (threadIdx.x == 0) {
     *sm.abort_flag = 0;
-    mbar_init(smem_u32(sm.qfull), 4);            // one arrival per softmax warp once its Q rows are in TMEM
+    mbar_init(smem_u32(sm.qfull), 8);            // one arrival per softmax warp once its Q columns are in TMEM
+    mbar_init(smem_u32(sm.lready), 8);
     mbar_init(smem_u32(sm.qrope_full), 1);
     mbar_init(smem_u32(sm.list_ready), 1);
     for (int s = 0; s < kStages; ++s) {
@@ -287,11 +297,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&sm.s_full[s]), 1);
       mbar_init(smem_u32(&sm.s_read[s]), 4);      // exchange warps have read the score buffer
-      mbar_init(smem_u32(&sm.p_full[s]), 4);
+      mbar_init(smem_u32(&sm.p_full[s]), 8);      // both softmax groups
+      mbar_init(smem_u32(&sm.mxready[s]), 8);
       mbar_init(smem_u32(&sm.o_done[s]), 1);
       mbar_init(smem_u32(&sm.xfull[s]), 1);       // armed by our softmax; completed by the peer's st.async bytes
       mbar_init(smem_u32(&sm.xfree[s]), 4);       // one arrival per peer exchange warp
-      mbar_init(smem_u32(&sm.xread[s]), 4);       // one arrival per local softmax warp
+      mbar_init(smem_u32(&sm.xread[s]), 8);       // one arrival per local softmax warp
     }
     mbar_init(smem_u32(sm.drain), 1);
     fence_barrier_init();
@@ -312,30 +323,37 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const int n = *sm.n_list;
     const int nch = (n + kChunk - 1) / kChunk;
     const int tid = threadIdx.x - 5 * 32;
-    const int r = tid >> 1, half = tid & 1;              // key row in chunk, half of its segments
-    const int spt = rope ? 18 : 16;                      // 16-byte segments per thread (36 or 32 per row)
+    const int w = warp - 5;                              // 0..3
+    const int c8 = lane & 7, sub = lane >> 3;            // value blocks: 16-byte segment, block
+    const int c4 = lane & 3, rr = lane >> 2;             // rope: 16-byte segment, row of eight
     const bf16* lat = p.latent + (size_t)(row / p.T) * p.S * p.stride;
     for (int j = 0; j < nch; ++j) {
       const int s = j % kStages;
       if (!mbar_wait(smem_u32(&sm.kv_empty[s]), ((j / kStages) & 1) ^ 1, p.status, abort_flag)) break;
       if (tid == 0) TRACE(0, j);
-      const uint32_t st = sm.kv + s * kStageBytes + r * 128;
-      const int li = j * kChunk + r;
-      const bool ok = li < n;                              // rows past the list are zero-filled
-      const bf16* src = lat + (size_t)(ok ? sm.list[li] : 0) * p.stride;
-#pragma unroll 2
-      for (int i = 0; i < spt; ++i) {
-        const int sg = half * spt + i;
-        if (sg < 32) {   // value-side block lb, 128-byte swizzle
-          const int lb = sg >> 3, c = sg & 7;
-          cp_async_16(st + lb * kBlockBytes + ((c ^ (r & 7)) << 4), src + (4 * (int)rank + lb) * 64 + c * 8, ok);
-        } else {         // rope columns, 64-byte rows with the 64-byte swizzle
-          const int c = sg - 32;
-          cp_async_16(st - r * 128 + kRopeOff + r * 64 + ((c ^ ((r >> 1) & 3)) << 4), src + rope_col + c * 8, ok);
+      const uint32_t stb = sm.kv + s * kStageBytes;
+      // each group of 8 lanes copies one 128-byte line: a warp moves 512 contiguous bytes of a row
+#pragma unroll 4
+      for (int it = 0; it < 16; ++it) {
+        const int r = it * 4 + w;
+        const int li = j * kChunk + r;
+        const bool ok = li < n;                          // rows past the list are zero-filled
+        const bf16* src = lat + (size_t)(ok ? sm.list[li] : 0) * p.stride + (4 * (int)rank + sub) * 64 + c8 * 8;
+        cp_async_16(stb + sub * kBlockBytes + r * 128 + ((c8 ^ (r & 7)) << 4), src, ok);
+      }
+      if (rope) {
+#pragma unroll
+        for (int it = 0; it < 2; ++it) {
+          const int r = (it * 4 + w) * 8 + rr;
+          const int li = j * kChunk + r;
+          const bool ok = li < n;
+          const bf16* src = lat + (size_t)(ok ? sm.list[li] : 0) * p.stride + rope_col + c4 * 8;
+          cp_async_16(stb + kRopeOff + r * 64 + ((c4 ^ ((r >> 1) & 3)) << 4), src, ok);
         }
       }
       // arrives on kv_full[s] once this thread's copies have landed
       cp_async_mbar_arrive(smem_u32(&sm.kv_full[s]));
+      if (tid == 0) TRACE(11, j);
     }
     cp_async_wait_all();
   } else if (warp == 4) {
@@ -411,7 +429,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       mma_commit(smem_u32(sm.drain));
       mbar_wait(smem_u32(sm.drain), 0, nullptr, nullptr);
     }
-  } else if (warp >= 9) {
+  } else if (warp >= 9 && warp <= 12) {
     // ---------------------------------------------------------------- score exchange
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
@@ -448,16 +466,20 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         if (lane == 0) arrive_remote_relaxed(map_peer(smem_u32(&sm.xfree[sb]), peer));
       }
     }
-  } else if (warp < 4) {
+  } else if (warp < 4 || warp >= 13) {
     // ---------------------------------------------------------------- softmax + epilogue
-    const int r = warp * 32 + lane;                 // head row == TMEM lane
-    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+    // Group g (warps 0-3 or 13-16) takes keys 32g..32g+31 of every chunk and O columns 128g..128g+127.
+    const int g = warp < 4 ? 0 : 1;
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;                   // head row == TMEM lane
+    const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
+    const bool lead = g == 0 && q4 == 0 && lane == 0;
     {
-      // value-side query columns of head r -> TMEM lane r, columns kQCol.. (bf16 pairs)
+      // value-side query columns of head r -> TMEM lane r (bf16 pairs); group g loads 64 columns
       const bool real = r < p.H;
       const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (row * p.H + (real ? r : 0)) * p.kd + rank * 256);
 #pragma unroll 1
-      for (int c0 = 0; c0 < 128; c0 += 32) {       // 32 columns = 64 bf16 = 8 x 16 bytes
+      for (int c0 = 64 * g; c0 < 64 * g + 64; c0 += 32) {   // 32 columns = 64 bf16 = 8 x 16 bytes
         uint32_t qv[32];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -483,21 +505,20 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       const int sb = j & 1, use = j >> 1;
       if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), use & 1, p.status, abort_flag))) break;
       tc_fence_after();
-      uint32_t v[kChunk];
-      tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk + 32 * g, v);
       tmem_ld_wait();
-      if (warp == 0 && lane == 0) TRACE(5, j);
+      if (lead) TRACE(5, j);
       if (!(ok = wait_cluster(smem_u32(&sm.xfull[sb]), use & 1, p.status, abort_flag))) break;
-      if (warp == 0 && lane == 0) {
+      if (lead) {
         TRACE(6, j);
         if (j + 2 < nch) mbar_arrive_expect_tx(smem_u32(&sm.xfull[sb]), kXBytes);  // arm the next use
       }
-      const float* xr = xcol + sb * (kXBytes / 4);
-      const int valid = n - j * kChunk;
+      const float* xr = xcol + sb * (kXBytes / 4) + 32 * g * 128;
+      const int valid = n - j * kChunk - 32 * g;
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < kChunk; ++c) {
+      for (int c = 0; c < 32; ++c) {
         const float x = c < valid ? (__uint_as_float(v[c]) + xr[c * 128]) * p.scale_log2 : -INFINITY;
         v[c] = __float_as_uint(x);
         mx = fmaxf(mx, x);
@@ -505,15 +526,22 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       // our buffer sb is read (values are in registers); the exchange warps tell the peer
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.xread[sb]));
-      if (warp == 0 && lane == 0) TRACE(9, j);
-      // move the reference maximum only when it grows by more than 2^8
+      // row maximum over both halves of the chunk
+      float* mxb = sm.mx + (j & 1) * 256;
+      mxb[g * 128 + r] = mx;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.mxready[j & 1]));
+      if (!(ok = mbar_wait(smem_u32(&sm.mxready[j & 1]), use & 1, p.status, abort_flag))) break;
+      mx = fmaxf(mx, mxb[(1 - g) * 128 + r]);
+      if (lead) TRACE(9, j);
+      // move the reference maximum only when it grows by more than 2^8 (both groups agree)
       const bool grow = mx > m_ref + 8.f;
       const float new_ref = grow ? mx : m_ref;
       if (__any_sync(0xffffffffu, grow && j > 0)) {
         if (!(ok = mbar_wait(smem_u32(&sm.o_done[(j - 1) & 1]), ((j - 1) >> 1) & 1, p.status, abort_flag))) break;
         tc_fence_after();
         const float f = (grow && j > 0) ? ex2(m_ref - new_ref) : 1.f;
-        for (int c = 0; c < 256; c += 16) {
+        for (int c = 128 * g; c < 128 * g + 128; c += 16) {
           uint32_t o[16];
           tmem_ld_32x32b_x16(tmem + lane_addr + kOCol + c, o);
           tmem_ld_wait();
@@ -525,34 +553,40 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         l_sum *= f;
       }
       m_ref = new_ref;
-      uint32_t pk[kChunk / 2];
+      uint32_t pk[16];
 #pragma unroll
-      for (int c = 0; c < kChunk; c += 2) {
+      for (int c = 0; c < 32; c += 2) {
         const float p0 = ex2(__uint_as_float(v[c]) - m_ref);
         const float p1 = ex2(__uint_as_float(v[c + 1]) - m_ref);
         l_sum += p0 + p1;
         pk[c / 2] = pack_bf16(p0, p1);
       }
-      if (warp == 0 && lane == 0) TRACE(10, j);
-      // P overwrites the first 32 columns of the score buffer once the exchange warps have read it
+      if (lead) TRACE(10, j);
+      // P (keys 32g..32g+31) overwrites columns 16g..16g+15 of the score buffer once the exchange warps have read it
       if (!(ok = mbar_wait(smem_u32(&sm.s_read[sb]), use & 1, p.status, abort_flag))) break;
-      tmem_st_32x32b_x32(tmem + lane_addr + sb * kChunk, pk);
+      tmem_st_32x32b_x16(tmem + lane_addr + sb * kChunk + 16 * g, pk);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[sb]));
-      if (warp == 0 && lane == 0) TRACE(7, j);
+      if (lead) TRACE(7, j);
     }
-    // epilogue: O / l -> bf16
+    // epilogue: O / (l0 + l1) -> bf16, group g writes O columns 128g..128g+127
     const bool write = r < p.H;
-    bf16* orow = p.out + (row * p.H + r) * 512 + rank * 256;
+    bf16* orow = p.out + (row * p.H + r) * 512 + rank * 256 + 128 * g;
     if (ok && nch > 0) {
-      ok = mbar_wait(smem_u32(&sm.o_done[(nch - 1) & 1]), ((nch - 1) >> 1) & 1, p.status, abort_flag);
+      float* lb = sm.mx + (nch & 1) * 256;           // not read again after chunk nch-2
+      lb[g * 128 + r] = l_sum;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(sm.lready));
+      ok = mbar_wait(smem_u32(sm.lready), 0, p.status, abort_flag) &&
+           mbar_wait(smem_u32(&sm.o_done[(nch - 1) & 1]), ((nch - 1) >> 1) & 1, p.status, abort_flag);
+      const float l_all = l_sum + lb[(1 - g) * 128 + r];
       tc_fence_after();
-      const float inv = 1.f / l_sum;
-      for (int c = 0; c < 256; c += 32) {
+      const float inv = 1.f / l_all;
+      for (int c = 0; c < 128; c += 32) {
         uint32_t o[32];
-        tmem_ld_32x32b_x32(tmem + lane_addr + kOCol + c, o);
+        tmem_ld_32x32b_x32(tmem + lane_addr + kOCol + 128 * g + c, o);
         tmem_ld_wait();
         if (write && ok) {
 #pragma unroll
@@ -566,10 +600,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           }
         }
       }
-      if (write && ok && rank == 0 && p.lse) p.lse[row * p.H + r] = (m_ref + log2f(l_sum)) * 0.69314718055994531f;
+      if (write && ok && rank == 0 && g == 0 && p.lse)
+        p.lse[row * p.H + r] = (m_ref + log2f(l_all)) * 0.69314718055994531f;
     } else if (ok && write) {
-      for (int c = 0; c < 256; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
-      if (rank == 0 && p.lse) p.lse[row * p.H + r] = -INFINITY;
+      for (int c = 0; c < 128; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+      if (rank == 0 && g == 0 && p.lse) p.lse[row * p.H + r] = -INFINITY;
     }
   }
   tc_fence_before();
@@ -600,7 +635,7 @@ EncodeTiledFn encode_fn() {
 
 size_t smem_bytes(int width) {
   return 1024 + 2 * (size_t)kXBytes + kQRopeBytes + (size_t)kStages * kStageBytes +
-         (((size_t)width * 4 + 15) & ~(size_t)15) + 8 * 32 + 16;
+         (((size_t)width * 2 + 15) & ~(size_t)15) + 2 * 2 * 128 * 4 + 8 * 32 + 16;
 }
 
 }  // namespace
@@ -613,7 +648,7 @@ bool attend_tc_supported(const dsa_dims& d, int64_t k_stride, const void* k, con
   if ((long long)d.batch * d.n_q * d.heads < 128) return false;  // the query TMA box is 128 rows
   if (k != v || k_stride != v_stride || k_stride < d.kd || (k_stride * 2) % 16 != 0) return false;
   if (((uintptr_t)k & 15u) != 0) return false;
-  if (d.n_kv > kBitmapKeys || width > 8192) return false;
+  if (d.n_kv > kBitmapKeys || width > 8192) return false;  // bitmap + raw row fit in the (idle) gather stages
   if (smem_bytes(width) > 227 * 1024) return false;
   return encode_fn() != nullptr;
 }
