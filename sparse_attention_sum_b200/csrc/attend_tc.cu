@@ -13,9 +13,9 @@
 // columns and the matching half of the key columns:
 //   rank 0: latent columns [0,256)   (+ rope columns [512,544) when kd = 576), O[:, 0:256)
 //   rank 1: latent columns [256,512) (+ rope columns [544,576) when kd = 576), O[:, 256:512)
-// Each CTA gathers only its own columns of every selected latent row (cp.async
-// straight into the 128-byte-swizzled operand layout), so no byte is loaded
-// twice.  Per 64-key chunk each CTA computes the q.k partial over its columns;
+// Each CTA gathers only its own columns of every selected latent row (TMA
+// tile::gather4, four rows per instruction, straight into the swizzled operand
+// layout), so no byte is loaded twice.  Per 64-key chunk each CTA computes the q.k partial over its columns;
 // the two fp32 partial tiles are exchanged through distributed shared memory
 // and summed (fp32 addition is commutative, so both CTAs see bit-identical
 // scores and take identical online-softmax decisions).  The exchange uses
@@ -38,8 +38,9 @@
 // 9-12 read the same score rows and push them to the peer (buffer reuse is
 // acknowledged by the peer); warp 4 issues tcgen05.mma from a polling scheduler
 // (and loads the CTA's rope query columns by TMA); warps 5-8 stage and
-// deduplicate the index row, then gather the selected rows with 16-byte
-// cp.async.  Every mbarrier wait is bounded.
+// deduplicate the index row, then each issues the gathers of one value block
+// and a quarter of the rope block (TMA runs them off the load/store pipe that
+// the softmax and exchange warps use).  Every mbarrier wait is bounded.
 #include <cuda.h>
 
 #include "dsa_common.cuh"
@@ -70,7 +71,7 @@ constexpr int kBlockBytes = kChunk * 128;                   // one 64-col block 
 constexpr int kRopeOff = 4 * kBlockBytes;                   // 32 rope columns after the 4 value blocks
 constexpr int kStageBytes = kRopeOff + kChunk * 64;         // 36 KB
 constexpr int kQRopeBytes = 128 * 64;                       // rope query columns in smem: 8 KB
-constexpr int kXBytes = kChunk * 128 * 4;                   // exchange tile [key][head] fp32: 32 KB
+constexpr int kXBytes = kChunk * 128 * 4;                   // exchange tile [key/4][head][4] fp32: 32 KB
 constexpr int kBitmapKeys = 65536;                          // dedupe bitmap (8 KB, aliases stage 0)
 constexpr int kQCol = 128;                                  // query columns in TMEM
 constexpr int kOCol = 256;                                  // output accumulator
@@ -120,9 +121,9 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, f
   asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
 }
-__device__ __forceinline__ void st_async_b32(uint32_t addr, uint32_t v, uint32_t remote_bar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(addr), "r"(v),
-               "r"(remote_bar)
+__device__ __forceinline__ void st_async_v4(uint32_t addr, const uint32_t* v, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
+               "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(remote_bar)
                : "memory");
 }
 __device__ __forceinline__ void arrive_remote(uint32_t cluster_addr) {
@@ -161,7 +162,6 @@ __device__ __forceinline__ bool wait_cluster(uint32_t bar, uint32_t parity, int*
     }
   }
 }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
@@ -238,6 +238,7 @@ __device__ void build_list(const AttTcParams& p, const Smem& sm, size_t row) {
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
+                 const __grid_constant__ CUtensorMap map_rope,
                  AttTcParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ int s_misc[4];
@@ -291,7 +292,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     mbar_init(smem_u32(sm.qrope_full), 1);
     mbar_init(smem_u32(sm.list_ready), 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&sm.kv_full[s]), kProducerThreads);
+      mbar_init(smem_u32(&sm.kv_full[s]), 1);     // one expect-tx arrival; the gathers complete the bytes
       mbar_init(smem_u32(&sm.kv_empty[s]), 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -322,40 +323,42 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     build_list(p, sm, row);
     const int n = *sm.n_list;
     const int nch = (n + kChunk - 1) / kChunk;
-    const int tid = threadIdx.x - 5 * 32;
-    const int w = warp - 5;                              // 0..3
-    const int c8 = lane & 7, sub = lane >> 3;            // value blocks: 16-byte segment, block
-    const int c4 = lane & 3, rr = lane >> 2;             // rope: 16-byte segment, row of eight
-    const bf16* lat = p.latent + (size_t)(row / p.T) * p.S * p.stride;
+    const int w = warp - 5;                              // 0..3: value block w; rope rows 16w..16w+15
+    const int rowbase = (int)(row / p.T) * p.S;          // latent row of key 0 of this query's sequence
+    const uint32_t stage_bytes = rope ? kStageBytes : 4 * kBlockBytes;
+    if (lane == 0) {
+      tma_prefetch_desc(&map_kv);
+      if (rope) tma_prefetch_desc(&map_rope);
+    }
     for (int j = 0; j < nch; ++j) {
       const int s = j % kStages;
       if (!mbar_wait(smem_u32(&sm.kv_empty[s]), ((j / kStages) & 1) ^ 1, p.status, abort_flag)) break;
-      if (tid == 0) TRACE(0, j);
+      if (w == 0 && lane == 0) {
+        TRACE(0, j);
+        mbar_arrive_expect_tx(smem_u32(&sm.kv_full[s]), stage_bytes);
+      }
       const uint32_t stb = sm.kv + s * kStageBytes;
-      // each group of 8 lanes copies one 128-byte line: a warp moves 512 contiguous bytes of a row
-#pragma unroll 4
-      for (int it = 0; it < 16; ++it) {
-        const int r = it * 4 + w;
-        const int li = j * kChunk + r;
-        const bool ok = li < n;                          // rows past the list are zero-filled
-        const bf16* src = lat + (size_t)(ok ? sm.list[li] : 0) * p.stride + (4 * (int)rank + sub) * 64 + c8 * 8;
-        cp_async_16(stb + sub * kBlockBytes + r * 128 + ((c8 ^ (r & 7)) << 4), src, ok);
-      }
-      if (rope) {
+      const uint32_t bar = smem_u32(&sm.kv_full[s]);
+      // TMA tile::gather4: four selected rows per instruction, written in the swizzled operand
+      // layout.  Rows past the list repeat the list's first key (their scores are masked, P = 0).
+      // Lanes 0-15 gather 64 value columns of keys 4*lane..4*lane+3 into block w; lanes 16-19
+      // gather the 32 rope columns of keys 4*(4w+lane-16).. into the 64-byte swizzled rope block.
+      const int g = lane < 16 ? lane : 4 * w + (lane - 16);
+      if (lane < 16 || (rope && lane < 20)) {
+        int rr[4];
 #pragma unroll
-        for (int it = 0; it < 2; ++it) {
-          const int r = (it * 4 + w) * 8 + rr;
-          const int li = j * kChunk + r;
-          const bool ok = li < n;
-          const bf16* src = lat + (size_t)(ok ? sm.list[li] : 0) * p.stride + rope_col + c4 * 8;
-          cp_async_16(stb + kRopeOff + r * 64 + ((c4 ^ ((r >> 1) & 3)) << 4), src, ok);
+        for (int i = 0; i < 4; ++i) {
+          const int li = j * kChunk + 4 * g + i;
+          rr[i] = rowbase + (int)sm.list[li < n ? li : 0];
         }
+        if (lane < 16)
+          tma_gather4(stb + w * kBlockBytes + g * 512, &map_kv, bar, (4 * (int)rank + w) * 64, rr[0], rr[1], rr[2],
+                      rr[3]);
+        else
+          tma_gather4(stb + kRopeOff + g * 256, &map_rope, bar, rope_col, rr[0], rr[1], rr[2], rr[3]);
       }
-      // arrives on kv_full[s] once this thread's copies have landed
-      cp_async_mbar_arrive(smem_u32(&sm.kv_full[s]));
-      if (tid == 0) TRACE(11, j);
+      if (w == 0 && lane == 0) TRACE(11, j);
     }
-    cp_async_wait_all();
   } else if (warp == 4) {
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
@@ -379,7 +382,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         // q.k of chunk qk: its stage is loaded and P.V of chunk qk-2 (same score buffer) is done
         if (qk < nch && mbar_test_wait(smem_u32(&sm.kv_full[qk % kStages]), (qk / kStages) & 1) &&
             mbar_test_wait(smem_u32(&sm.o_done[qk & 1]), ((qk >> 1) & 1) ^ 1)) {
-          fence_proxy_async_smem();
           tc_fence_after();
           const uint32_t st = sm.kv + (qk % kStages) * kStageBytes;
           const uint32_t d = tmem + (qk & 1) * kChunk;
@@ -415,7 +417,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         }
         if (progressed) {
           spins = 0;
-        } else if ((++spins & 255u) == 0u) {
+          continue;
+        }
+        __nanosleep(32);  // keep the shared-memory pipe free for the other warps while polling
+        if ((++spins & 255u) == 0u) {
           const unsigned long long now = globaltimer();
           if (*abort_flag) break;
           if (spins == 256u) t_last = now;
@@ -437,7 +442,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     bool ok = mbar_wait(smem_u32(sm.list_ready), 0, p.status, abort_flag);
     const int n = ok ? *sm.n_list : 0;
     const int nch = (n + kChunk - 1) / kChunk;
-    const uint32_t dst0 = map_peer(sm.x + (uint32_t)r * 4, peer);   // column r of the [key][head] tile
+    const uint32_t dst0 = map_peer(sm.x + (uint32_t)r * 16, peer);  // head r's 16 bytes of each [key/4][head][4] row
     for (int j = 0; ok && j < nch; ++j) {
       const int sb = j & 1, use = j >> 1;
       if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), use & 1, p.status, abort_flag))) break;
@@ -453,11 +458,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       // the peer has read its buffer sb from chunk j-2
       if (!(ok = wait_cluster(smem_u32(&sm.xfree[sb]), (use & 1) ^ 1, p.status, abort_flag))) break;
       const uint32_t dst = dst0 + (uint32_t)sb * kXBytes;
-      // key-major: for each key the warp's 32 lanes write 128 contiguous bytes; each
-      // store completes its bytes on the peer's barrier (no round trip here)
+      // [key/4][head][4 keys]: each store writes 4 keys of head r, the warp 512 contiguous
+      // bytes; each store completes its bytes on the peer's barrier (no round trip here)
       const uint32_t xbar = map_peer(smem_u32(&sm.xfull[sb]), peer);
 #pragma unroll
-      for (int c = 0; c < kChunk; ++c) st_async_b32(dst + c * 512, v[c], xbar);
+      for (int c = 0; c < kChunk; c += 4) st_async_v4(dst + c * 512, &v[c], xbar);
       if (q4 == 1 && lane == 0) TRACE(4, j);
       // once our softmax has read our buffer sb for chunk j, the peer may refill it (chunk j+2)
       if (j + 2 < nch) {
@@ -474,6 +479,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const int r = q4 * 32 + lane;                   // head row == TMEM lane
     const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
     const bool lead = g == 0 && q4 == 0 && lane == 0;
+    [[maybe_unused]] const bool lead1 = g == 1 && q4 == 0 && lane == 0;
     {
       // value-side query columns of head r -> TMEM lane r (bf16 pairs); group g loads 64 columns
       const bool real = r < p.H;
@@ -500,7 +506,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     bool ok = mbar_wait(smem_u32(sm.list_ready), 0, p.status, abort_flag);
     const int n = ok ? *sm.n_list : 0;
     const int nch = (n + kChunk - 1) / kChunk;
-    const float* xcol = reinterpret_cast<const float*>(gb + (sm.x - base)) + r;   // column r of [key][head]
+    const float4* xcol = reinterpret_cast<const float4*>(gb + (sm.x - base)) + r;  // head r of [key/4][head][4]
     for (int j = 0; ok && j < nch; ++j) {
       const int sb = j & 1, use = j >> 1;
       if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), use & 1, p.status, abort_flag))) break;
@@ -509,19 +515,26 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk + 32 * g, v);
       tmem_ld_wait();
       if (lead) TRACE(5, j);
+      if (lead1) TRACE(12, j);
       if (!(ok = wait_cluster(smem_u32(&sm.xfull[sb]), use & 1, p.status, abort_flag))) break;
+      if (lead1) TRACE(13, j);
       if (lead) {
         TRACE(6, j);
         if (j + 2 < nch) mbar_arrive_expect_tx(smem_u32(&sm.xfull[sb]), kXBytes);  // arm the next use
       }
-      const float* xr = xcol + sb * (kXBytes / 4) + 32 * g * 128;
+      const float4* xr = xcol + sb * (kXBytes / 16) + 8 * g * 128;
       const int valid = n - j * kChunk - 32 * g;
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float x = c < valid ? (__uint_as_float(v[c]) + xr[c * 128]) * p.scale_log2 : -INFINITY;
-        v[c] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
+      for (int c = 0; c < 32; c += 4) {
+        const float4 x4 = xr[(c / 4) * 128];
+        const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float x = c + i < valid ? (__uint_as_float(v[c + i]) + xs[i]) * p.scale_log2 : -INFINITY;
+          v[c + i] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
       }
       // our buffer sb is read (values are in registers); the exchange warps tell the peer
       __syncwarp();
@@ -534,6 +547,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       if (!(ok = mbar_wait(smem_u32(&sm.mxready[j & 1]), use & 1, p.status, abort_flag))) break;
       mx = fmaxf(mx, mxb[(1 - g) * 128 + r]);
       if (lead) TRACE(9, j);
+      if (lead1) TRACE(14, j);
       // move the reference maximum only when it grows by more than 2^8 (both groups agree)
       const bool grow = mx > m_ref + 8.f;
       const float new_ref = grow ? mx : m_ref;
@@ -570,6 +584,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[sb]));
       if (lead) TRACE(7, j);
+      if (lead1) TRACE(15, j);
     }
     // epilogue: O / (l0 + l1) -> bf16, group g writes O columns 128g..128g+127
     const bool write = r < p.H;
@@ -693,11 +708,18 @@ cudaError_t launch_attend_tc(const dsa_dims& d, const void* q, const void* k, in
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
+  // the same rows, 32 rope columns per box with the 64-byte swizzle of the rope operand
+  CUtensorMap mrope;
+  cuuint32_t rbox[2] = {32u, 1u};
+  if (enc(&mrope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(k), kdims, kstrides, rbox, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   const size_t smem = smem_bytes(width);
   cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long long rows = (long long)d.batch * d.n_q;
-  attend_tc_kernel<<<dim3((unsigned)(2 * rows)), kThreads, smem, st>>>(mq, mkv, p);
+  attend_tc_kernel<<<dim3((unsigned)(2 * rows)), kThreads, smem, st>>>(mq, mkv, mrope, p);
   return cudaGetLastError();
 }
 
