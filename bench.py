@@ -11,7 +11,7 @@ stream.  Under torchrun every rank runs its own replica of the workload
 (weak scaling, no data-path collective); the step time is the max over ranks.
 
 ``--profile-once`` makes one call of each stage entry point (dsa_index_scores,
-dsa_topk, dsa_sparse_attend) on the workload and exits, timing nothing: the
+dsa_topk_set, dsa_sparse_attend) on the workload and exits, timing nothing: the
 command an ncu capture of the three stage kernels runs.
 
 ``--impl reference`` times the CPU oracle (the reference arm for this build)
@@ -209,7 +209,7 @@ def time_steps(step_fn, steps, warmup, flush, stream):
 
 
 def stage_times(wl, t, dims, args, bufs, steps, flush, stream):
-    """Per-stage device times (s) of the three C-ABI calls of the layer."""
+    """Per-stage device times (s) of the three C-ABI calls the fused layer makes."""
     import sparse_attention_sum_b200 as dsa
     B, T, S = wl.batch, wl.n_q, wl.n_kv
     scores = bufs.ws[: B * T * S * 4].view(torch.float32)
@@ -217,8 +217,9 @@ def stage_times(wl, t, dims, args, bufs, steps, flush, stream):
     calls = {
         "index": lambda: dsa.index_scores(dims, args["q_idx"], args["k_idx"], args["w"], args["idx_scale"],
                                           args["q_pos"], args["kv_start"], args["kv_len"], scores),
-        "topk": lambda: dsa.topk(dims, scores, args["q_pos"], args["kv_start"], args["kv_len"], wl.top_k,
-                                 idx),
+        # the fused layer's form of the selection (the set in key order, no rank sort)
+        "topk": lambda: dsa.topk_set(dims, scores, args["q_pos"], args["kv_start"], args["kv_len"], wl.top_k,
+                                     idx),
         "attend": lambda: dsa.sparse_attend(dims, args["q"], args["k"], args["k_row_stride"], args["v"],
                                             args["v_row_stride"], idx, wl.top_k, args["attn_scale"],
                                             bufs.out),
@@ -267,7 +268,7 @@ def profile_once(a):
     scores = bufs.ws[: B * T * S * 4].view(torch.float32)
     dsa.index_scores(dims, args["q_idx"], args["k_idx"], args["w"], args["idx_scale"], args["q_pos"],
                      args["kv_start"], args["kv_len"], scores)
-    dsa.topk(dims, scores, args["q_pos"], args["kv_start"], args["kv_len"], wl.top_k, bufs.idx)
+    dsa.topk_set(dims, scores, args["q_pos"], args["kv_start"], args["kv_len"], wl.top_k, bufs.idx)
     dsa.sparse_attend(dims, args["q"], args["k"], args["k_row_stride"], args["v"], args["v_row_stride"],
                       bufs.idx, wl.top_k, args["attn_scale"], bufs.out)
     torch.cuda.synchronize()

@@ -145,6 +145,18 @@ dsa_status dsa_topk(const dsa_dims* dims, const float* scores, const int32_t* q_
                     const int32_t* kv_start, const int32_t* kv_len, int32_t k, int32_t* idx,
                     float* vals, void* ws, size_t ws_bytes, dsa_stream_t stream);
 
+/* S3' — the same selection as a set.
+ * Selects exactly the keys dsa_topk(k) selects (same scores, same visibility,
+ * same tie rule) and lists them in ascending key order, DSA_INVALID after
+ * them; vals (or NULL) holds each listed key's score, -inf in INVALID slots.
+ * The attention reads a selection as a set, so this is the form the fused
+ * layer uses: it needs no rank sort.  Arguments as in dsa_topk (no workspace).
+ * (The pages define the selection as a set; dsa_topk's rank order is this
+ * library's deterministic listing of it.) */
+dsa_status dsa_topk_set(const dsa_dims* dims, const float* scores, const int32_t* q_pos,
+                        const int32_t* kv_start, const int32_t* kv_len, int32_t k, int32_t* idx,
+                        float* vals, dsa_stream_t stream);
+
 /* S4 — sparse attention over the selected keys.
  * For every (b,t,h): U = the set of distinct entries i of idx[b,t,:] with
  * 0 <= i < S (duplicates collapse, DSA_INVALID and out-of-range entries are
@@ -174,7 +186,10 @@ dsa_status dsa_sparse_attend(const dsa_dims* dims, const void* q, const void* k,
  * attend reads).  idx_in != NULL skips S2/S3 and attends over the caller's
  * rows [B,T,top_k] (reuse of an earlier layer's selection); otherwise the
  * selection is written to idx_out [B,T,top_k] when idx_out != NULL, or kept in
- * the workspace.  All other arguments are as in the three calls above.
+ * the workspace.  The selection is the set dsa_topk(top_k) picks (same
+ * scores, same tie rule) listed in ascending key order, DSA_INVALID after it:
+ * the attention reads it as a set, so no rank sort is spent on it.  All other
+ * arguments are as in the three calls above.
  * Reads dims: every field of the three calls; kpool must be 0. */
 dsa_status dsa_layer_forward(const dsa_dims* dims, const void* q_idx, const void* k_idx,
                              const float* w, float idx_scale, const int32_t* q_pos,

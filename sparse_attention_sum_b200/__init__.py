@@ -15,7 +15,7 @@ from typing import Optional
 
 __all__ = [
     "DsaError", "DsaLibraryError", "Dims", "lib", "lib_path", "INVALID", "F32", "BF16",
-    "index_scores", "topk", "sparse_attend", "layer_forward", "layer_forward_static", "pool_states",
+    "index_scores", "topk", "topk_set", "sparse_attend", "layer_forward", "layer_forward_static", "pool_states",
     "expand_selection", "absorb_q", "absorb_out", "workspace_size", "get_device_status",
     "selftest_wait_timeout", "set_kernel_policy", "OP_TOPK", "OP_LAYER_FORWARD", "STATUS",
 ]
@@ -69,6 +69,8 @@ _SIGS = {
                           _I32P, _F32P, _VP], ctypes.c_int),
     "dsa_topk": ([ctypes.POINTER(Dims), _F32P, _I32P, _I32P, _I32P, ctypes.c_int32, _I32P, _F32P,
                   _VP, ctypes.c_size_t, _VP], ctypes.c_int),
+    "dsa_topk_set": ([ctypes.POINTER(Dims), _F32P, _I32P, _I32P, _I32P, ctypes.c_int32, _I32P, _F32P, _VP],
+                     ctypes.c_int),
     "dsa_sparse_attend": ([ctypes.POINTER(Dims), _VP, _VP, ctypes.c_int64, _VP, ctypes.c_int64,
                            _I32P, ctypes.c_int32, ctypes.c_float, _VP, _F32P, _VP], ctypes.c_int),
     "dsa_layer_forward": ([ctypes.POINTER(Dims), _VP, _VP, _F32P, ctypes.c_float, _I32P, _I32P,
@@ -161,6 +163,12 @@ def topk(dims: Dims, scores, q_pos, kv_start, kv_len, k: int, idx, vals=None, ws
     _check(lib().dsa_topk(ctypes.byref(dims), _ptr(scores), _ptr(q_pos), _ptr(kv_start),
                           _ptr(kv_len), int(k), _ptr(idx), _ptr(vals), _ptr(ws), wsb,
                           _stream(stream)), "dsa_topk")
+
+
+def topk_set(dims: Dims, scores, q_pos, kv_start, kv_len, k: int, idx, vals=None, stream=None):
+    """dsa_topk's selection listed in ascending key order (the fused layer's form)."""
+    _check(lib().dsa_topk_set(ctypes.byref(dims), _ptr(scores), _ptr(q_pos), _ptr(kv_start), _ptr(kv_len),
+                              int(k), _ptr(idx), _ptr(vals), _stream(stream)), "dsa_topk_set")
 
 
 def sparse_attend(dims: Dims, q, k, k_row_stride: int, v, v_row_stride: int, idx, width: int,

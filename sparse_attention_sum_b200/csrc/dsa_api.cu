@@ -212,6 +212,17 @@ dsa_status dsa_index_scores(const dsa_dims* d, const void* q_idx, const void* k_
   return ok();
 }
 
+namespace {
+dsa_status topk_checked(const dsa_dims* d, const float* scores, const int32_t* q_pos, const int32_t* kv_start,
+                        const int32_t* kv_len, int32_t k, int32_t* idx, float* vals, bool ranked,
+                        dsa_stream_t stream) {
+  if (d->batch > 65535) return fail(DSA_ERR_UNSUPPORTED, "dsa_topk: grid too large");
+  cudaError_t e = dsa::launch_topk(*d, scores, q_pos, kv_start, kv_len, k, idx, vals, ranked, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "dsa_topk launch");
+  return ok();
+}
+}  // namespace
+
 dsa_status dsa_topk(const dsa_dims* d, const float* scores, const int32_t* q_pos,
                     const int32_t* kv_start, const int32_t* kv_len, int32_t k, int32_t* idx,
                     float* vals, void* ws, size_t ws_bytes, dsa_stream_t stream) {
@@ -221,10 +232,15 @@ dsa_status dsa_topk(const dsa_dims* d, const float* scores, const int32_t* q_pos
   if ((s = check_visibility(q_pos, kv_start, kv_len))) return s;
   if (ws_bytes < dsa_workspace_size(d, DSA_OP_TOPK))
     return fail(DSA_ERR_WORKSPACE, "dsa_topk: workspace too small");
-  if (d->n_q > 2147483647 || d->batch > 65535) return fail(DSA_ERR_UNSUPPORTED, "dsa_topk: grid too large");
-  cudaError_t e = dsa::launch_topk(*d, scores, q_pos, kv_start, kv_len, k, idx, vals, (cudaStream_t)stream);
-  if (e != cudaSuccess) return cuda_fail(e, "dsa_topk launch");
-  return ok();
+  return topk_checked(d, scores, q_pos, kv_start, kv_len, k, idx, vals, true, stream);
+}
+
+dsa_status dsa_topk_set(const dsa_dims* d, const float* scores, const int32_t* q_pos, const int32_t* kv_start,
+                        const int32_t* kv_len, int32_t k, int32_t* idx, float* vals, dsa_stream_t stream) {
+  dsa_status s = check_topk(d, scores, k, idx);
+  if (s) return s;
+  if ((s = check_visibility(q_pos, kv_start, kv_len))) return s;
+  return topk_checked(d, scores, q_pos, kv_start, kv_len, k, idx, vals, false, stream);
 }
 
 dsa_status dsa_sparse_attend(const dsa_dims* d, const void* q, const void* k, int64_t k_row_stride,
@@ -272,8 +288,8 @@ dsa_status dsa_layer_forward(const dsa_dims* d, const void* q_idx, const void* k
     int32_t* idx = idx_out ? idx_out : idx_ws;
     if ((s = dsa_index_scores(d, q_idx, k_idx, w, idx_scale, q_pos, kv_start, kv_len, scores, stream)))
       return s;
-    if ((s = dsa_topk(d, scores, q_pos, kv_start, kv_len, d->top_k, idx, nullptr, nullptr, 0, stream)))
-      return s;
+    // the attention reads the selection as a set: same keys as dsa_topk, listed in key order
+    if ((s = dsa_topk_set(d, scores, q_pos, kv_start, kv_len, d->top_k, idx, nullptr, stream))) return s;
     sel = idx;
   }
   return dsa_sparse_attend(d, q, k, k_row_stride, v, v_row_stride, sel, d->top_k, attn_scale, out,

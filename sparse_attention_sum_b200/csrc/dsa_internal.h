@@ -30,10 +30,11 @@ cudaError_t launch_index_scores_tc(const dsa_dims& d, const void* q_idx, const v
                                    const int32_t* kv_start, const int32_t* kv_len, float* scores,
                                    cudaStream_t st);
 
-// S3 radix select + rank sort.
+// S3 radix select, then a rank sort (ranked) or an ascending-key-order listing of
+// the same selection (!ranked, the fused layer's set).
 cudaError_t launch_topk(const dsa_dims& d, const float* scores, const int32_t* q_pos,
                         const int32_t* kv_start, const int32_t* kv_len, int k, int32_t* idx,
-                        float* vals, cudaStream_t st);
+                        float* vals, bool ranked, cudaStream_t st);
 
 // S4 on the CUDA cores (generic shapes).
 bool attend_simt_supported(const dsa_dims& d, int width);

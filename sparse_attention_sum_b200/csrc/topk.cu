@@ -15,12 +15,16 @@
 // which keeps the tie rule exact.  Finally the (key, index) pairs are put in
 // rank order by a stable four-pass LSD radix sort on the key (descending), so
 // equal keys keep ascending index order.
+//
+// The unranked variant (the fused layer's selection, which the attention reads
+// as a set) selects the same keys under the same rule and lists them in
+// ascending key order: a row with at most k visible keys is its visible range,
+// and a longer row needs the select passes and one ordered compaction, no sort.
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
 
 namespace dsa {
 
-constexpr int kTopkMaxK = 4096;
 constexpr int kTopkCacheMax = 40960;  // keys cached in shared memory (160 KB)
 
 // Block-wide exclusive scan of one int per thread; returns the block total.
@@ -113,16 +117,17 @@ __device__ void radix_sort_desc(uint64_t* a, uint64_t* b, uint32_t* hist, int* s
   }
 }
 
-template <int BLOCK>
+template <int BLOCK, bool RANKED>
 __global__ void __launch_bounds__(BLOCK)
 topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restrict__ q_pos,
             const int32_t* __restrict__ kv_start, const int32_t* __restrict__ kv_len, int k,
             int cache_cap, int32_t* __restrict__ idx_out, float* __restrict__ vals_out) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int ksel = RANKED ? k : 0;                                   // the unranked variant keeps no pairs
   uint64_t* sel = reinterpret_cast<uint64_t*>(smem_raw);            // [k]   selected (key, index)
-  uint64_t* tmp = sel + k;                                           // [k]   sort ping-pong
-  uint32_t* rhist = reinterpret_cast<uint32_t*>(tmp + k);            // [BLOCK/32 * 256]
-  uint32_t* hist = rhist + (BLOCK / 32) * 256;                       // [256]
+  uint64_t* tmp = sel + ksel;                                        // [k]   sort ping-pong
+  uint32_t* rhist = reinterpret_cast<uint32_t*>(tmp + ksel);         // [BLOCK/32 * 256] (ranked only)
+  uint32_t* hist = rhist + (RANKED ? (BLOCK / 32) * 256 : 0);        // [256]
   int* scan = reinterpret_cast<int*>(hist + 256);                    // [64]
   uint32_t* cache = reinterpret_cast<uint32_t*>(scan + 64);          // [cache_cap]
   __shared__ uint32_t s_prefix, s_krem;
@@ -137,7 +142,15 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
   const int n = r.count();
   const bool cached = n <= cache_cap;
 
-  if (n <= k) {
+  if (!RANKED && n <= k) {
+    // every visible key is selected: the visible range, in key order
+    for (int i = threadIdx.x; i < k; i += BLOCK) {
+      orow[i] = i < n ? r.lo + i : DSA_INVALID;
+      if (vrow) vrow[i] = i < n ? key_score(score_key(srow[r.lo + i])) : -INFINITY;
+    }
+    return;
+  }
+  if (RANKED && n <= k) {
     // every visible key is selected: rank them (inputs in index order)
     for (int i = threadIdx.x; i < n; i += BLOCK)
       sel[i] = ((uint64_t)score_key(srow[r.lo + i]) << 32) | (uint32_t)(r.lo + i);
@@ -242,6 +255,28 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
   gt_base = __shfl_sync(0xffffffffu, gt_base, 0);
   eq_base = __shfl_sync(0xffffffffu, eq_base, 0);
   const uint32_t lt_mask = (1u << lane) - 1u;
+  if (!RANKED) {
+    // ascending key order: key i goes to (#gt before i) + min(#eq before i, need_eq)
+    for (int b0 = w0; b0 < w1; b0 += 32) {
+      const int i = b0 + lane;
+      uint32_t key = 0u;
+      if (i < w1) key = cached ? cache[i] : score_key(srow[r.lo + i]);
+      const bool is_gt = i < w1 && key > tau;
+      const bool is_eq = i < w1 && key == tau;
+      const uint32_t m_gt = __ballot_sync(0xffffffffu, is_gt);
+      const uint32_t m_eq = __ballot_sync(0xffffffffu, is_eq);
+      const int gt_before = gt_base + __popc(m_gt & lt_mask);
+      const int eq_before = eq_base + __popc(m_eq & lt_mask);
+      if (is_gt || (is_eq && eq_before < need_eq)) {
+        const int pos = gt_before + min(eq_before, need_eq);
+        orow[pos] = r.lo + i;
+        if (vrow) vrow[pos] = key_score(key);
+      }
+      gt_base += __popc(m_gt);
+      eq_base += __popc(m_eq);
+    }
+    return;
+  }
   for (int b0 = w0; b0 < w1; b0 += 32) {
     const int i = b0 + lane;
     uint32_t key = 0u;
@@ -270,28 +305,31 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
   }
 }
 
+namespace {
+template <int BLOCK, bool RANKED>
+cudaError_t launch_topk_t(const dsa_dims& d, const float* scores, const int32_t* q_pos, const int32_t* kv_start,
+                          const int32_t* kv_len, int k, int32_t* idx, float* vals, cudaStream_t st) {
+  int cache_cap = d.n_kv < kTopkCacheMax ? d.n_kv : kTopkCacheMax;
+  const size_t fixed =
+      (RANKED ? (size_t)k * 16 + (size_t)(BLOCK / 32) * 256 * 4 : 0) + 256 * 4 + 64 * 4;
+  if (fixed + (size_t)cache_cap * 4 > 220 * 1024) cache_cap = (int)((220 * 1024 - fixed) / 4);
+  const size_t smem = fixed + (size_t)cache_cap * 4;
+  auto kern = topk_kernel<BLOCK, RANKED>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(d.n_q, d.batch), BLOCK, smem, st>>>(d, scores, q_pos, kv_start, kv_len, k, cache_cap, idx, vals);
+  return cudaGetLastError();
+}
+}  // namespace
+
 cudaError_t launch_topk(const dsa_dims& d, const float* scores, const int32_t* q_pos,
                         const int32_t* kv_start, const int32_t* kv_len, int k, int32_t* idx,
-                        float* vals, cudaStream_t st) {
-  const int block = d.n_kv > 8192 ? 1024 : 512;
-  int cache_cap = d.n_kv < kTopkCacheMax ? d.n_kv : kTopkCacheMax;
-  const size_t fixed = (size_t)k * 16 + (size_t)(block / 32) * 256 * 4 + 256 * 4 + 64 * 4;
-  if (fixed + (size_t)cache_cap * 4 > 220 * 1024) cache_cap = (int)((220 * 1024 - fixed) / 4);
-  size_t smem = fixed + (size_t)cache_cap * 4;
-  dim3 grid(d.n_q, d.batch);
-  cudaError_t e;
-  if (d.n_kv > 8192) {
-    auto kern = topk_kernel<1024>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    kern<<<grid, 1024, smem, st>>>(d, scores, q_pos, kv_start, kv_len, k, cache_cap, idx, vals);
-  } else {
-    auto kern = topk_kernel<512>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    kern<<<grid, 512, smem, st>>>(d, scores, q_pos, kv_start, kv_len, k, cache_cap, idx, vals);
-  }
-  return cudaGetLastError();
+                        float* vals, bool ranked, cudaStream_t st) {
+  if (d.n_kv > 8192)
+    return ranked ? launch_topk_t<1024, true>(d, scores, q_pos, kv_start, kv_len, k, idx, vals, st)
+                  : launch_topk_t<1024, false>(d, scores, q_pos, kv_start, kv_len, k, idx, vals, st);
+  return ranked ? launch_topk_t<512, true>(d, scores, q_pos, kv_start, kv_len, k, idx, vals, st)
+                : launch_topk_t<512, false>(d, scores, q_pos, kv_start, kv_len, k, idx, vals, st);
 }
 
 }  // namespace dsa

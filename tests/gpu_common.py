@@ -91,6 +91,17 @@ def assert_attend_close(gpu_out, ref_out, dtype, what=""):
             assert c >= COS_MIN, f"{what}: row {i} cosine {c}"
 
 
+def key_order(sel):
+    """Selection rows [..., k] listed in ascending key order, DSA_INVALID after the keys
+    (how dsa_layer_forward lists the set that dsa_topk ranks)."""
+    if isinstance(sel, torch.Tensor):
+        big = torch.iinfo(torch.int32).max
+        s = torch.sort(sel.masked_fill(sel < 0, big), dim=-1).values
+        return s.masked_fill(s == big, O.INVALID)
+    keys = sorted(int(x) for x in sel if int(x) != O.INVALID)
+    return keys + [O.INVALID] * (len(sel) - len(keys))
+
+
 def check_selection_in_band(gpu_sel, cand, ref_scores, k, what=""):
     """GPU selection vs the oracle's scores: equal, or every difference inside the tie band.
 

@@ -4,7 +4,6 @@ Small cases compare every element; full-size workloads (in the launch
 configuration bench.py times) compare sampled rows element by element and
 check structural properties on every row.
 """
-import math
 
 import numpy as np
 import pytest
@@ -14,7 +13,7 @@ from oracle import dsa_oracle as O
 import sparse_attention_sum_b200 as dsa
 from sparse_attention_sum_b200 import runner
 import workloads
-from tests.gpu_common import (ATOL, assert_attend_close, check_selection_in_band, cosine, dev,
+from tests.gpu_common import (ATOL, assert_attend_close, check_selection_in_band, cosine, dev, key_order,
                               kv_views, layer_inputs, sample_rows)
 
 pytestmark = pytest.mark.gpu
@@ -74,11 +73,16 @@ def test_tiny_layer_is_exact_against_oracle():
     ref_out, ref_lse = O.sparse_attend(wl["q"], K, V, ref_idx, wl.attn_scale)
     assert_attend_close(_np(out), ref_out, torch.float32, "tiny attend")
     np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, atol=1e-4)
-    # the fused call equals the composition
+    # the fused call: dsa_topk's set listed in key order, attended as in the composition
     bufs = runner.dsa_layer(dims, **a)
     torch.cuda.synchronize()
-    assert torch.equal(bufs.idx, idx)
-    assert torch.equal(bufs.out, out)
+    assert torch.equal(bufs.idx, key_order(idx))
+    again = torch.empty_like(out)
+    dsa.sparse_attend(dims, a["q"], a["k"], a["k_row_stride"], a["v"], a["v_row_stride"], bufs.idx, wl.top_k,
+                      a["attn_scale"], again)
+    torch.cuda.synchronize()
+    assert torch.equal(bufs.out, again)
+    assert_attend_close(_np(bufs.out), ref_out, torch.float32, "tiny fused layer")
 
 
 def test_tiny_layer_covering_all_keys_is_dense_attention():
@@ -104,8 +108,19 @@ def _topk_case(scores_np, q_pos, kv_start, kv_len, k, kpool=0):
     idx = torch.full((B, T, k), 12345, dtype=torch.int32, device="cuda")
     vals = torch.empty(B, T, k, dtype=torch.float32, device="cuda")
     dsa.topk(d, sc, qp, ks, kl, k, idx, vals)
+    set_idx = torch.full_like(idx, 12345)
+    set_vals = torch.empty_like(vals)
+    dsa.topk_set(d, sc, qp, ks, kl, k, set_idx, set_vals)
     torch.cuda.synchronize()
     got = idx.cpu().numpy()
+    # the set form: the same keys in ascending key order, each with its score
+    assert torch.equal(set_idx, key_order(idx))
+    gv, sv = vals.cpu().numpy(), set_vals.cpu().numpy()
+    for b in range(B):
+        for t in range(T):
+            pos = {int(x): i for i, x in enumerate(got[b, t]) if x >= 0}
+            for j, x in enumerate(set_idx[b, t].tolist()):
+                assert (sv[b, t, j] == gv[b, t, pos[x]]) if x >= 0 else np.isneginf(sv[b, t, j])
     for b in range(B):
         for t in range(T):
             if kpool:
@@ -223,6 +238,29 @@ def test_small_bf16_layer_against_oracle(name, sizes):
         ro, rl = O.sparse_attend_row(wl["q"][b, tt], K[b], V[b], g_idx[b, tt], wl.attn_scale)
         assert_attend_close(_np(out[b, tt]), ro, torch.bfloat16, f"{name} attend {(b, tt)}")
     assert n_diff_rows <= max(1, len(rows) // 10)
+    # the fused layer lists the same selection in key order; its attention matches the composition
+    fused = runner.dsa_layer(dims, **a)
+    torch.cuda.synchronize()
+    assert torch.equal(fused.idx, key_order(idx))
+    assert_attend_close(_np(fused.out), _np(out), torch.bfloat16, f"{name} fused vs composition")
+
+
+@pytest.mark.parametrize("name,sizes,top_k", [("prefill", dict(T=300), 96), ("decode", dict(B=2, S=5000), 2048)])
+def test_fused_layer_all_scores_tied_takes_lowest_keys(name, sizes, top_k):
+    # indexer weights 0: every visible score is 0, so the tie rule alone decides
+    wl = workloads.make(name, **sizes)
+    wl.top_k = top_k
+    t = dev(wl)
+    t["w"].zero_()
+    dims, a = layer_inputs(wl, t)
+    bufs = runner.dsa_layer(dims, **a)
+    torch.cuda.synchronize()
+    sel = bufs.idx.cpu().numpy()
+    for b in range(wl.batch):
+        for tt in range(wl.n_q):
+            cand = O.visible_keys(int(wl["q_pos"][b, tt]), int(wl["kv_start"][b]), int(wl["kv_len"][b]))
+            want = cand[:top_k].tolist()
+            assert sel[b, tt].tolist() == want + [O.INVALID] * (top_k - len(want)), (b, tt)
 
 
 # ------------------------------------------- tensor cores vs CUDA cores
@@ -351,24 +389,24 @@ def test_full_size_layer_sampled_rows(name):
         ref = O.index_scores_row(wl["q_idx"][b, tt], wl["k_idx"][b][cand], wl["w"][b, tt], wl.idx_scale)
         gs = scores[b, tt].cpu().numpy().astype(np.float64)[cand]
         assert np.abs(gs - ref).max() <= 2e-5 * max(1.0, np.abs(ref).max())
-        assert g_idx[b, tt].tolist() == O.topk_row(cand, gs, wl.top_k).tolist()
+        assert g_idx[b, tt].tolist() == key_order(O.topk_row(cand, gs, wl.top_k).tolist())
         diffs += check_selection_in_band(g_idx[b, tt], cand, ref, wl.top_k, f"{name} {(b, tt)}") > 0
         ro, rl = O.sparse_attend_row(wl["q"][b, tt], K[b], V[b], g_idx[b, tt], wl.attn_scale)
         assert_attend_close(_np(bufs.out[b, tt]), ro, torch.bfloat16, f"{name} out {(b, tt)}")
         np.testing.assert_allclose(bufs.lse[b, tt].cpu().numpy(), rl, atol=2e-3)
     assert diffs <= max(1, len(rows) // 4)
-    # every row: count, visibility, uniqueness and rank order by the GPU's scores
+    # every row: count, visibility, ascending key order, and the same set dsa_topk ranks
     sel = bufs.idx
     qp = t["q_pos"].view(B, T, 1).long()
     valid = sel >= 0
     nvis = (qp[..., 0] - t["kv_start"].view(B, 1).long() + 1).clamp(min=0).clamp(max=S)
     assert torch.equal(valid.sum(-1), nvis.clamp(max=wl.top_k))
     assert bool((sel[valid].long() <= qp.expand_as(sel)[valid]).all())
-    srt = torch.sort(sel.masked_fill(~valid, -1 - 10**6), dim=-1).values
-    dup = (srt[..., 1:] == srt[..., :-1]) & (srt[..., 1:] >= 0)
-    assert not bool(dup.any())
-    sv = torch.gather(scores, 2, sel.clamp(min=0).long()).masked_fill(~valid, -math.inf)
-    assert bool((sv[..., 1:][valid[..., 1:]] <= sv[..., :-1][valid[..., 1:]]).all())
+    assert bool((sel[..., 1:][valid[..., 1:]] > sel[..., :-1][valid[..., 1:]]).all())
+    ranked = torch.empty_like(sel)
+    dsa.topk(dims, scores, t["q_pos"], t["kv_start"], t["kv_len"], wl.top_k, ranked)
+    torch.cuda.synchronize()
+    assert torch.equal(key_order(ranked), sel)
 
 
 def test_full_size_kpool_sampled_rows():
