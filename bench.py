@@ -245,13 +245,27 @@ def roofline_entry(kind, amount, seconds, peaks, traffic=None):
 
 
 def profiled_traffic():
-    """Per-launch DRAM traffic of the dominant kernel from the committed ncu summary, if any."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    """Per-launch DRAM traffic from the committed ncu summaries (profiles/traffic.txt), keyed by
+    kernel:workload; an entry whose kernel source changed since the capture is dropped."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    res = {}
     try:
-        with open(path) as f:
-            return json.load(f)
-    except Exception:
-        return {}
+        lines = open(path).read().splitlines()
+    except OSError:
+        return res
+    for ln in lines:
+        parts = ln.split()
+        if not parts or parts[0].startswith("#") or len(parts) < 4:
+            continue
+        key, nbytes, src, digest = parts[:4]
+        try:
+            cur = hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest()[:16]
+        except OSError:
+            continue
+        if cur == digest:
+            res[key] = int(nbytes)
+    return res
 
 
 def profile_once(a):

@@ -95,6 +95,7 @@ struct Smem {
   uint16_t* list;            // deduplicated key rows (n_kv <= 65536 on this path)
   int* raw;                  // the index row as given (staged in gather stage 0)
   uint32_t* bitmap;          // dedupe bitmap (gather stage 0, before the first gather)
+  int* bitmap_tail;          // 4 per-warp counts of the list compaction
   float* mx;                 // [2 parities][2 groups][128 rows] half-row maxima, then partial sums
   uint64_t *qfull, *qrope_full, *list_ready, *kv_full, *kv_empty, *s_full, *s_read, *p_full, *o_done, *xfull,
       *xfree, *xread, *mxready, *lready, *drain;
@@ -186,10 +187,20 @@ __device__ __forceinline__ uint64_t desc_noswz(uint32_t saddr, uint32_t lbo, uin
 // list.  Run by the 128 producer threads (warps 5-8).
 __device__ void build_list(const AttTcParams& p, const Smem& sm, size_t row) {
   const int tid = threadIdx.x - 5 * 32;               // 0..127
-  const int lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31, w = tid >> 5;
   const int32_t* irow = p.idx + row * p.width;
   const int words = (p.S + 31) >> 5;
-  for (int e = tid; e < p.width; e += kProducerThreads) sm.raw[e] = irow[e];
+  // stage the index row: independent 16-byte loads in flight together
+  if ((p.width & 3) == 0 && ((reinterpret_cast<uintptr_t>(irow) & 15u) == 0)) {
+    const int4* src = reinterpret_cast<const int4*>(irow);
+    int4* dst = reinterpret_cast<int4*>(sm.raw);
+    const int n4 = p.width >> 2;
+#pragma unroll 4
+    for (int e = tid; e < n4; e += kProducerThreads) dst[e] = __ldg(src + e);
+  } else {
+#pragma unroll 8
+    for (int e = tid; e < p.width; e += kProducerThreads) sm.raw[e] = __ldg(irow + e);
+  }
   for (int i = tid; i < words; i += kProducerThreads) sm.bitmap[i] = 0u;
   if (tid == 0) *sm.dup_flag = 0;
   named_sync(1, kProducerThreads);
@@ -204,24 +215,54 @@ __device__ void build_list(const AttTcParams& p, const Smem& sm, size_t row) {
   if (__any_sync(0xffffffffu, dup) && lane == 0) *sm.dup_flag = 1;
   named_sync(1, kProducerThreads);
   const bool has_dup = *sm.dup_flag != 0;
-  if (has_dup) {
-    for (int i = tid; i < words; i += kProducerThreads) sm.bitmap[i] = 0u;
+  if (!has_dup) {
+    // no repeated key: keep every in-range entry.  Each warp compacts a contiguous quarter of
+    // the row 32 entries at a time (ballots), after a scan of the four quarters' counts.
+    const int q = (((p.width + 3) >> 2) + 31) & ~31;
+    const int e0 = w * q, e1 = min(p.width, e0 + q);
+    int cnt = 0;
+    for (int b = e0; b < e1; b += 32) {
+      const int e = b + lane;
+      const int key = e < e1 ? sm.raw[e] : -1;
+      cnt += __popc(__ballot_sync(0xffffffffu, key >= 0 && key < p.S));
+    }
+    int* wtot = sm.bitmap_tail;                       // 4 ints past the bitmap's words
+    if (lane == 0) wtot[w] = cnt;
     named_sync(1, kProducerThreads);
+    int base = 0;
+    for (int k = 0; k < w; ++k) base += wtot[k];
+    const int total = wtot[0] + wtot[1] + wtot[2] + wtot[3];
+    for (int b = e0; b < e1; b += 32) {
+      const int e = b + lane;
+      const int key = e < e1 ? sm.raw[e] : -1;
+      const bool keep = key >= 0 && key < p.S;
+      const uint32_t m = __ballot_sync(0xffffffffu, keep);
+      if (keep) sm.list[base + __popc(m & ((1u << lane) - 1u))] = (uint16_t)key;
+      base += __popc(m);
+    }
+    named_sync(1, kProducerThreads);
+    if (tid == 0) {
+      TRACE(8, 1);
+      *sm.n_list = total;
+      mbar_arrive(smem_u32(sm.list_ready));
+    }
+    named_sync(1, kProducerThreads);
+    return;
   }
+  for (int i = tid; i < words; i += kProducerThreads) sm.bitmap[i] = 0u;
+  named_sync(1, kProducerThreads);
   if (tid < 32) {
-    // order-preserving compaction into the key list
+    // repeated keys: order-preserving compaction by one warp, first occurrence only
+    // (not seen in an earlier group of 32, lowest lane within its group)
     int n = 0;
     for (int e0 = 0; e0 < p.width; e0 += 32) {
       const int e = e0 + lane;
       const int key = e < p.width ? sm.raw[e] : -1;
       bool keep = key >= 0 && key < p.S;
-      if (has_dup) {
-        // first occurrence only: not seen in an earlier group, lowest lane in this group
-        const uint32_t peers = __match_any_sync(0xffffffffu, keep ? key : -1);
-        if (keep) keep = (sm.bitmap[key >> 5] & (1u << (key & 31))) == 0u && lane == __ffs(peers) - 1;
-        __syncwarp();
-        if (keep) atomicOr(&sm.bitmap[key >> 5], 1u << (key & 31));
-      }
+      const uint32_t peers = __match_any_sync(0xffffffffu, keep ? key : -1);
+      if (keep) keep = (sm.bitmap[key >> 5] & (1u << (key & 31))) == 0u && lane == __ffs(peers) - 1;
+      __syncwarp();
+      if (keep) atomicOr(&sm.bitmap[key >> 5], 1u << (key & 31));
       const uint32_t m = __ballot_sync(0xffffffffu, keep);
       if (keep) sm.list[n + __popc(m & ((1u << lane) - 1u))] = (uint16_t)key;
       n += __popc(m);
@@ -242,6 +283,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                  AttTcParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ int s_misc[4];
+  __shared__ int s_wcount[4];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* gb = smem_raw + (base - raw);
@@ -277,6 +319,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   sm.n_list = &s_misc[0];
   sm.dup_flag = &s_misc[1];
   sm.abort_flag = &s_misc[2];
+  sm.bitmap_tail = s_wcount;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
