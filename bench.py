@@ -87,59 +87,87 @@ def work(wl):
 
 # -------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms in a thread."""
+    """SM clock and clock-event reasons of this process's GPU, sampled every 5 ms in a thread
+    through NVML (the device is found by its PCI bus id, so CUDA_VISIBLE_DEVICES cannot confuse
+    it), else through nvidia-smi every 200 ms.  Reading only: no setting is touched."""
 
+    REASONS = (("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20), ("hw_thermal_slowdown", 0x40),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
-        self.dev = device_index
+        pr = torch.cuda.get_device_properties(device_index)
+        self.bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+        self.samples = []            # (sm_mhz, max_mhz, reason names)
+        self.stop = threading.Event()
         self.proc = None
-        self.lines = []
+        self.source = None
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.Q}",
+            import pynvml as N
+            N.nvmlInit()
+            h = N.nvmlDeviceGetHandleByPciBusId(self.bus.encode())
+            mx = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
+
+            def run():
+                while not self.stop.is_set():
+                    try:
+                        sm = N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)
+                        r = N.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((float(sm), float(mx), [n for n, b in self.REASONS if r & b]))
+                    except Exception:
+                        pass
+                    self.stop.wait(0.005)
+            self.source = "nvml"
+            self.t = threading.Thread(target=run, daemon=True)
+            self.t.start()
+            return self
+        except Exception:
+            pass
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.bus}", f"--query-gpu={self.Q}",
                                           "--format=csv,noheader,nounits", "-lms", "200"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+            self.source = "nvidia-smi"
+            self.t = threading.Thread(target=self._read_smi, daemon=True)
             self.t.start()
         except Exception:
             self.proc = None
         return self
 
-    def _read(self):
+    def _read_smi(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            parts = [p.strip() for p in line.strip().split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                self.samples.append((float(parts[1]), float(parts[2]),
+                                     [n for n, v in zip(names, parts[5:9]) if v.lower() == "active"]))
+            except ValueError:
+                continue
 
     def __exit__(self, *a):
+        self.stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        elif self.source == "nvml":
+            self.t.join(timeout=1)
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
+        reasons = sorted({n for _, _, rs in self.samples for n in rs})
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples),
+                "sm_max_mhz": max(s[1] for s in self.samples), "reasons": reasons,
+                "samples": len(self.samples), "source": self.source, "gpu": self.bus}
 
 
 # --------------------------------------------------------------- distributed
@@ -350,6 +378,8 @@ def run_ours(a):
         line["e2e"] = e2e_measure(wl, a.steps, stream)
         if a.workload == "prefill":
             line["decode"] = decode_extra(peaks, flush, stream)
+            line["chunked"] = chunked_extra(peaks, flush, stream)
+            line["kpool"] = kpool_extra(peaks, flush, stream)
         line["cpu_baseline"] = cpu_baseline(wl, budget_s=a.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -360,37 +390,61 @@ def run_ours(a):
 
 
 def e2e_measure(wl, steps, stream):
-    """Same metric through the public API with host buffers: pinned H2D copies of
-    the step's inputs, the layer call, and the D2H read of the output, all timed."""
+    """Same metric through the public API with host buffers.  Every step copies its inputs from
+    pinned host memory to the device, runs the fused layer and reads its output back to pinned
+    host memory, all inside the timed region.  Steps are pipelined the way a serving loop runs
+    them: step i+1's upload (one copy stream) overlaps step i's layer (the compute stream) and
+    step i-1's download (a second copy stream); two device buffer sets alternate."""
     from sparse_attention_sum_b200 import runner
     host = {k: v.pin_memory() for k, v in wl.tensors.items()}
-    dev_t = {k: torch.empty_like(v, device="cuda") for k, v in host.items()}
-    dims, args = layer_args(wl, dev_t)
-    bufs = runner.LayerBuffers(dims, "cuda", torch.bfloat16, with_idx=True)
-    out_host = torch.empty(bufs.out.shape, dtype=bufs.out.dtype).pin_memory()
+    sets = []
+    for _ in range(2):
+        dev_t = {k: torch.empty_like(v, device="cuda") for k, v in host.items()}
+        dims, args = layer_args(wl, dev_t)
+        bufs = runner.LayerBuffers(dims, "cuda", torch.bfloat16, with_idx=True)
+        sets.append((dev_t, dims, args, bufs))
+    out_host = torch.empty(sets[0][3].out.shape, dtype=sets[0][3].out.dtype).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = out_host.numel() * out_host.element_size()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    uploaded = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    downloaded = [torch.cuda.Event() for _ in range(2)]
+    for e in downloaded:
+        e.record(down)
 
-    def step():
-        for k in host:
-            dev_t[k].copy_(host[k], non_blocking=True)
-        runner.dsa_layer(dims, **args, bufs=bufs)
-        out_host.copy_(bufs.out, non_blocking=True)
+    def run(n):
+        for i in range(n):
+            b = i & 1
+            dev_t, dims, args, bufs = sets[b]
+            with torch.cuda.stream(up):
+                up.wait_event(computed[b]) if i >= 2 else None     # set b's inputs are free again
+                for k in host:
+                    dev_t[k].copy_(host[k], non_blocking=True)
+                uploaded[b].record(up)
+            stream.wait_event(uploaded[b])
+            stream.wait_event(downloaded[b])                        # set b's output was read back
+            runner.dsa_layer(dims, **args, bufs=bufs, stream=stream)
+            computed[b].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(computed[b])
+                out_host.copy_(bufs.out, non_blocking=True)
+                downloaded[b].record(down)
 
-    for _ in range(2):
-        step()
+    run(2)
     torch.cuda.synchronize()
+    n = max(4, min(steps, 10))
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    n = max(3, min(steps, 10))
-    e0.record(stream)
-    for _ in range(n):
-        step()
-    e1.record(stream)
+    e0.record(up)
+    run(n)
+    down.wait_event(computed[(n - 1) & 1])
+    e1.record(down)
     e1.synchronize()
     sec = e0.elapsed_time(e1) / 1e3 / n
     return {"value": round(wl.batch * wl.n_q / sec, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": round(sec * 1e3, 3)}
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(sec * 1e3, 3),
+            "pipelined": "upload of step i+1 and download of step i-1 overlap step i's layer"}
 
 
 def decode_extra(peaks, flush, stream):
@@ -412,6 +466,82 @@ def decode_extra(peaks, flush, stream):
            "roofline_index": roofline_entry("hbm", wk["index_bytes"], st["index"], peaks),
            "fused_hbm_frac": round((wk["index_bytes"] + wk["topk_bytes"] + wk["attend_bytes"]) / step / 1e9
                                    / peaks["hbm_gbs"], 4)}
+    del t, bufs
+    torch.cuda.empty_cache()
+    return res
+
+
+def chunked_extra(peaks, flush, stream):
+    """Chunked prefill: 4096 queries at positions 28672..32767 against 32768 keys (hot-spot keys)."""
+    from sparse_attention_sum_b200 import runner
+    wl = workloads.make("chunked")
+    t = device_inputs(wl)
+    dims, args = layer_args(wl, t)
+    bufs = runner.LayerBuffers(dims, "cuda", torch.bfloat16, with_idx=True)
+    times = time_steps(lambda: runner.dsa_layer(dims, **args, bufs=bufs), 5, 3, flush, stream)
+    st = stage_times(wl, t, dims, args, bufs, 5, flush, stream)
+    wk = work(wl)
+    rows = wl.batch * wl.n_q
+    step = statistics.median(times)
+    res = {"workload": f"chunked: B={wl.batch} T={wl.n_q} S={wl.n_kv} top_k={wl.top_k}",
+           "value": round(rows / step, 1), "unit": UNIT, "ms_per_step": round(step * 1e3, 4),
+           "stages_us": {k: round(v * 1e6, 1) for k, v in st.items()},
+           "roofline_index": roofline_entry("tensor", wk["index_flop"], st["index"], peaks),
+           "roofline_attend": roofline_entry("tensor", wk["attend_flop"], st["attend"], peaks),
+           "fused_tensor_frac": round((wk["index_flop"] + wk["attend_flop"]) / step / 1e12 / peaks["bf16_tflops"], 4)}
+    del t, bufs
+    torch.cuda.empty_cache()
+    return res
+
+
+def kpool_extra(peaks, flush, stream):
+    """The kpool NoPE layer (4 sequences x 8192 tokens, left padding, kpool 4, select_k 512, H=64
+    absorbed into a 512-wide latent): every call of the chain timed alone, and the whole chain."""
+    import sparse_attention_sum_b200 as dsa
+    from sparse_attention_sum_b200 import runner
+    wl = workloads.make("kpool")
+    t = device_inputs(wl)
+    B, T, S = wl.batch, wl.n_q, wl.n_kv
+    H, L = wl.heads, wl.kd
+    dq, dv = t["q_nope"].shape[-1], t["w_uv"].shape[1]
+    dims = runner.kpool_dims(B, T, S, wl.idx_heads, wl.idx_dim, wl.kpool, wl.select_k, wl.out_width, H, L)
+    bufs = runner.KpoolBuffers(B, T, S, wl.idx_heads, wl.idx_dim, wl.kpool, wl.select_k, wl.out_width,
+                               H, dq, L, dv, "cuda")
+    dp, di, da = dims["pool"], dims["index"], dims["attend"]
+    chain = lambda: runner.kpool_layer(dims, t["q_idx"], t["k_raw"], t["gate"], t["ln_w"], t["ln_b"], wl.ln_eps,
+                                       t["w"], wl.idx_scale, t["q_pos"], t["kv_start"], t["kv_len"], t["q_nope"],
+                                       t["latent"], t["w_uk"], t["w_uv"], wl.attn_scale, bufs)
+    times = time_steps(chain, 3, 3, flush, stream)
+    calls = {
+        "pool_states": lambda: dsa.pool_states(dp, t["k_raw"], t["gate"], t["ln_w"], t["ln_b"], wl.ln_eps,
+                                               t["kv_start"], t["kv_len"], bufs.pooled, bufs.n_pools),
+        "index": lambda: dsa.index_scores(di, t["q_idx"], bufs.pooled, t["w"], wl.idx_scale, t["q_pos"],
+                                          t["kv_start"], t["kv_len"], bufs.pool_scores),
+        "topk": lambda: dsa.topk(di, bufs.pool_scores, t["q_pos"], t["kv_start"], t["kv_len"], di.top_k,
+                                 bufs.pool_idx),
+        "expand": lambda: dsa.expand_selection(dp, bufs.pool_idx, t["q_pos"], t["kv_start"], t["kv_len"],
+                                               bufs.n_pools, bufs.tok_idx),
+        "absorb_q": lambda: dsa.absorb_q(da, t["q_nope"], dq, t["w_uk"], L, bufs.q_lat),
+        "attend": lambda: dsa.sparse_attend(da, bufs.q_lat, t["latent"], L, t["latent"], L, bufs.tok_idx,
+                                            da.out_width, wl.attn_scale, bufs.o_lat),
+        "absorb_out": lambda: dsa.absorb_out(da, bufs.o_lat, L, t["w_uv"], dv, bufs.out),
+    }
+    st = {k: statistics.median(time_steps(f, 3, 1, flush, stream)) for k, f in calls.items()}
+    index_pairs = int(torch.isfinite(bufs.pool_scores).sum())
+    attend_pairs = int((bufs.tok_idx >= 0).sum())
+    valid_rows = int((t["q_pos"] >= t["kv_start"].view(-1, 1)).sum())
+    flop = {"index": 2.0 * index_pairs * wl.idx_heads * wl.idx_dim,
+            "attend": 2.0 * attend_pairs * H * (L + L),
+            "absorb": 2 * (2.0 * B * T * H * dq * L)}
+    step = statistics.median(times)
+    res = {"workload": f"kpool: B={B} T=S={S} left pad {wl['kv_start'].tolist()} kpool={wl.kpool} "
+                       f"select_k={wl.select_k} width={wl.out_width}, NoPE MLA H={H} latent {L}",
+           "value": round(B * T / step, 1), "value_valid_rows": round(valid_rows / step, 1), "unit": UNIT,
+           "ms_per_step": round(step * 1e3, 3), "stages_us": {k: round(v * 1e6, 1) for k, v in st.items()},
+           "roofline_index": roofline_entry("tensor", flop["index"], st["index"], peaks),
+           "roofline_attend": roofline_entry("tensor", flop["attend"], st["attend"], peaks),
+           "roofline_absorb": roofline_entry("tensor", flop["absorb"], st["absorb_q"] + st["absorb_out"], peaks),
+           "fused_tensor_frac": round(sum(flop.values()) / step / 1e12 / peaks["bf16_tflops"], 4)}
     del t, bufs
     torch.cuda.empty_cache()
     return res

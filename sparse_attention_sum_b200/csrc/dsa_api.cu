@@ -349,8 +349,10 @@ dsa_status dsa_absorb_q(const dsa_dims* d, const void* q, int32_t dq, const void
                         void* q_lat, dsa_stream_t stream) {
   dsa_status s = check_absorb(d, q, dq, w_uk, L, q_lat);
   if (s) return s;
-  cudaError_t e = dsa::launch_head_gemm(d->batch * d->n_q, d->heads, dq, L, q, w_uk, true, q_lat,
-                                        (cudaStream_t)stream);
+  const int rows = d->batch * d->n_q;
+  cudaError_t e = g_policy == 0 && dsa::head_gemm_tc_supported(rows, d->heads, dq, L, q, w_uk, true, q_lat)
+                      ? dsa::launch_head_gemm_tc(rows, d->heads, dq, L, q, w_uk, true, q_lat, (cudaStream_t)stream)
+                      : dsa::launch_head_gemm(rows, d->heads, dq, L, q, w_uk, true, q_lat, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "dsa_absorb_q launch");
   return ok();
 }
@@ -359,8 +361,10 @@ dsa_status dsa_absorb_out(const dsa_dims* d, const void* o_lat, int32_t L, const
                           int32_t dv, void* out, dsa_stream_t stream) {
   dsa_status s = check_absorb(d, o_lat, L, w_uv, dv, out);
   if (s) return s;
-  cudaError_t e = dsa::launch_head_gemm(d->batch * d->n_q, d->heads, L, dv, o_lat, w_uv, false, out,
-                                        (cudaStream_t)stream);
+  const int rows = d->batch * d->n_q;
+  cudaError_t e = g_policy == 0 && dsa::head_gemm_tc_supported(rows, d->heads, L, dv, o_lat, w_uv, false, out)
+                      ? dsa::launch_head_gemm_tc(rows, d->heads, L, dv, o_lat, w_uv, false, out, (cudaStream_t)stream)
+                      : dsa::launch_head_gemm(rows, d->heads, L, dv, o_lat, w_uv, false, out, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "dsa_absorb_out launch");
   return ok();
 }

@@ -63,6 +63,11 @@ cudaError_t launch_expand_selection(const dsa_dims& d, const int32_t* pool_idx,
 //   b_kn = false: B[h] is [N, K] (K contiguous)    (absorb_out: w_uv[h] is [e, L])
 cudaError_t launch_head_gemm(int n_rows, int heads, int K, int N, const void* A, const void* Bm,
                              bool b_kn, void* C, cudaStream_t st);
+// The same on tcgen05 (n_rows >= 128, K % 64 == 0, K <= 512, B[h] <= 128 KB, 16-byte aligned).
+bool head_gemm_tc_supported(int n_rows, int heads, int K, int N, const void* A, const void* Bm, bool b_kn,
+                            const void* C);
+cudaError_t launch_head_gemm_tc(int n_rows, int heads, int K, int N, const void* A, const void* Bm, bool b_kn,
+                                void* C, cudaStream_t st);
 
 // Bounded-wait self test.
 cudaError_t launch_wait_selftest(long long timeout_ns, cudaStream_t st);

@@ -263,6 +263,41 @@ def test_fused_layer_all_scores_tied_takes_lowest_keys(name, sizes, top_k):
             assert sel[b, tt].tolist() == want + [O.INVALID] * (top_k - len(want)), (b, tt)
 
 
+# ------------------------------------------------ S8 absorption GEMMs
+@pytest.mark.parametrize("n_rows,H", [(128, 2), (300, 4), (1400, 16)])
+def test_absorb_gemms_match_oracle_and_cuda_core_kernel(n_rows, H):
+    # ragged row counts (several 128-row tiles and a tail); at 1400 x 16 a CTA takes 2-3 items
+    # and some ranges cross a head boundary (B reloaded, both accumulators in turn)
+    g = torch.Generator().manual_seed(n_rows + H)
+    q = (torch.randn(n_rows, H, 128, generator=g)).to(torch.bfloat16)
+    o_lat = (torch.randn(n_rows, H, 512, generator=g)).to(torch.bfloat16)
+    w_uk = (torch.randn(H, 128, 512, generator=g) / 512 ** 0.5).to(torch.bfloat16)
+    w_uv = (torch.randn(H, 128, 512, generator=g) / 512 ** 0.5).to(torch.bfloat16)
+    d = dsa.Dims(batch=1, n_q=n_rows, heads=H, dtype=dsa.BF16)
+    qd, od, ukd, uvd = (x.cuda() for x in (q, o_lat, w_uk, w_uv))
+    outs = {}
+    for policy in (0, 1):
+        prev = dsa.set_kernel_policy(policy)
+        try:
+            q_lat = torch.full((n_rows, H, 512), float("nan"), dtype=torch.bfloat16, device="cuda")
+            out = torch.full((n_rows, H, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+            dsa.absorb_q(d, qd, 128, ukd, 512, q_lat)
+            dsa.absorb_out(d, od, 512, uvd, 128, out)
+            torch.cuda.synchronize()
+            outs[policy] = (q_lat.double().cpu().numpy(), out.double().cpu().numpy())
+        finally:
+            dsa.set_kernel_policy(prev)
+    ref_q = O.absorb_q(q.float().numpy(), w_uk.float().numpy())
+    ref_o = O.absorb_out(o_lat.float().numpy(), w_uv.float().numpy())
+    for policy, (gq, go) in outs.items():
+        # fp32 accumulation of bf16 products, one bf16 rounding of the result
+        np.testing.assert_allclose(gq, ref_q, atol=2e-2, rtol=1e-2, err_msg=f"absorb_q policy {policy}")
+        np.testing.assert_allclose(go, ref_o, atol=2e-2, rtol=1e-2, err_msg=f"absorb_out policy {policy}")
+    # the two kernel families differ only in summation order
+    np.testing.assert_allclose(outs[0][0], outs[1][0], atol=1e-2, rtol=1e-2)
+    np.testing.assert_allclose(outs[0][1], outs[1][1], atol=1e-2, rtol=1e-2)
+
+
 # ------------------------------------------- tensor cores vs CUDA cores
 @pytest.mark.parametrize("name,sizes,top_k", [("prefill", dict(T=300), 96), ("decode", dict(B=2, S=4100), 2048)])
 def test_tensor_core_kernels_match_cuda_core_kernels(name, sizes, top_k):
