@@ -88,19 +88,29 @@ struct AttTcParams {
   bf16* out;                 // [B,T,H,512]
   float* lse;                // [B,T,H] or null
   int* status;
+  int list_bitmap;           // 1: the dedupe bitmap fits in the key-list buffer
+  int out_v8;                // 1: out is 32-byte aligned (256-bit stores)
 };
+
+// Key-list buffer: width uint16 entries, grown to hold the dedupe bitmap of S keys when
+// `with_bitmap` (then the bitmap needs no gather stage).
+__host__ __device__ inline size_t list_bytes(int width, int S, bool with_bitmap) {
+  size_t b = (size_t)width * 2;
+  const size_t bm = (size_t)((S + 31) / 32) * 4;
+  if (with_bitmap && bm > b) b = bm;
+  return (b + 15) & ~(size_t)15;
+}
 
 struct Smem {
   uint32_t kv, x, qrope;     // shared-window addresses
-  uint16_t* list;            // deduplicated key rows (n_kv <= 65536 on this path)
-  int* raw;                  // the index row as given (staged in gather stage 0)
-  uint32_t* bitmap;          // dedupe bitmap (gather stage 0, before the first gather)
-  int* bitmap_tail;          // 4 per-warp counts of the list compaction
-  float* mx;                 // [2 parities][2 groups][128 rows] half-row maxima, then partial sums
-  uint64_t *qfull, *qrope_full, *list_ready, *kv_full, *kv_empty, *s_full, *s_read, *p_full, *o_done, *xfull,
-      *xfree, *xread, *mxready, *lready, *drain;
+  uint16_t* list;            // deduplicated key rows of the row being gathered (n_kv <= 65536)
+  int* wcount;               // 4 per-warp counts of the list compaction
+  float* mx;                 // [2 parities][2 groups][128 rows] half-row maxima
+  float* lsum;               // [2 groups][128 rows] partial row sums for the epilogue
+  uint64_t *qfull, *qrope_full, *list_ready, *list_taken, *kv_full, *kv_empty, *s_full, *s_read, *p_full, *o_done,
+      *o_free, *xfull, *xfree, *xread, *mxready, *lready, *drain;
   uint32_t* tmem_slot;
-  int* n_list;
+  int* n_list;               // [2]: list length of the published row, by row parity
   int* dup_flag;
   int* abort_flag;
 };
@@ -125,6 +135,11 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, f
 __device__ __forceinline__ void st_async_v4(uint32_t addr, const uint32_t* v, uint32_t remote_bar) {
   asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
                "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(remote_bar)
+               : "memory");
+}
+__device__ __forceinline__ void st_global_v8(void* ptr, const uint32_t* v) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(ptr), "r"(v[0]), "r"(v[1]),
+               "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
                : "memory");
 }
 __device__ __forceinline__ void arrive_remote(uint32_t cluster_addr) {
@@ -163,6 +178,17 @@ __device__ __forceinline__ bool wait_cluster(uint32_t bar, uint32_t parity, int*
     }
   }
 }
+// Named barrier that also returns whether any participating thread passed `pred`
+// (bar.red.or): the producer warps take every early exit together.
+__device__ __forceinline__ bool named_any(int id, int n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
@@ -182,107 +208,147 @@ __device__ __forceinline__ uint64_t desc_noswz(uint32_t saddr, uint32_t lbo, uin
   return d;
 }
 
-// Builds the row's key list in shared memory: distinct in-range entries in
-// index-row order.  Deterministic, so both CTAs of the cluster obtain the same
-// list.  Run by the 128 producer threads (warps 5-8).
-__device__ void build_list(const AttTcParams& p, const Smem& sm, size_t row) {
-  const int tid = threadIdx.x - 5 * 32;               // 0..127
-  const int lane = threadIdx.x & 31, w = tid >> 5;
-  const int32_t* irow = p.idx + row * p.width;
-  const int words = (p.S + 31) >> 5;
-  // stage the index row: independent 16-byte loads in flight together
-  if ((p.width & 3) == 0 && ((reinterpret_cast<uintptr_t>(irow) & 15u) == 0)) {
-    const int4* src = reinterpret_cast<const int4*>(irow);
-    int4* dst = reinterpret_cast<int4*>(sm.raw);
-    const int n4 = p.width >> 2;
-#pragma unroll 4
-    for (int e = tid; e < n4; e += kProducerThreads) dst[e] = __ldg(src + e);
-  } else {
-#pragma unroll 8
-    for (int e = tid; e < p.width; e += kProducerThreads) sm.raw[e] = __ldg(irow + e);
-  }
-  for (int i = tid; i < words; i += kProducerThreads) sm.bitmap[i] = 0u;
-  if (tid == 0) *sm.dup_flag = 0;
-  named_sync(1, kProducerThreads);
-  int dup = 0;
-  for (int e = tid; e < p.width; e += kProducerThreads) {
-    const int key = sm.raw[e];
-    if (key >= 0 && key < p.S) {
-      const uint32_t bit = 1u << (key & 31);
-      dup |= (atomicOr(&sm.bitmap[key >> 5], bit) & bit) != 0u;
+// Row list construction, by the 128 producer threads (warps 5-8): the distinct in-range
+// entries of the index row in index-row order.  Deterministic, so both CTAs of the
+// cluster obtain the same list.  Entry e = w*q + 32*it + lane belongs to warp w; rows of
+// up to 2176 entries are read from global memory once into registers.
+constexpr int kListCache = 17;  // rows of up to 2176 entries (top_k 2048; kpool widths 2051)
+
+struct RowKeys {
+  int q, e0, e1;
+  bool cached;
+  int key[kListCache];
+};
+
+__device__ void load_row(const AttTcParams& p, const int32_t* irow, RowKeys& rk) {
+  const int tid = threadIdx.x - 5 * 32, lane = threadIdx.x & 31, w = tid >> 5;
+  rk.q = (((p.width + 3) >> 2) + 31) & ~31;
+  rk.e0 = w * rk.q;
+  rk.e1 = min(p.width, rk.e0 + rk.q);
+  rk.cached = rk.q <= 32 * kListCache;
+  if (rk.cached) {
+#pragma unroll
+    for (int it = 0; it < kListCache; ++it) {
+      const int e = rk.e0 + 32 * it + lane;
+      rk.key[it] = e < rk.e1 ? __ldg(irow + e) : -1;
     }
   }
-  if (__any_sync(0xffffffffu, dup) && lane == 0) *sm.dup_flag = 1;
+}
+
+// Marks every in-range key in `bitmap` (cleared first); returns whether any key repeats.
+__device__ bool mark_keys(const AttTcParams& p, const int32_t* irow, const RowKeys& rk, uint32_t* bitmap) {
+  const int tid = threadIdx.x - 5 * 32, lane = threadIdx.x & 31;
+  const int words = (p.S + 31) >> 5;
+  for (int i = tid; i < words; i += kProducerThreads) bitmap[i] = 0u;
   named_sync(1, kProducerThreads);
-  const bool has_dup = *sm.dup_flag != 0;
-  if (!has_dup) {
-    // no repeated key: keep every in-range entry.  Each warp compacts a contiguous quarter of
-    // the row 32 entries at a time (ballots), after a scan of the four quarters' counts.
-    const int q = (((p.width + 3) >> 2) + 31) & ~31;
-    const int e0 = w * q, e1 = min(p.width, e0 + q);
-    int cnt = 0;
-    for (int b = e0; b < e1; b += 32) {
+  bool dup = false;
+  if (rk.cached) {
+#pragma unroll
+    for (int it = 0; it < kListCache; ++it) {
+      const int key = rk.key[it];
+      if (key >= 0 && key < p.S) {
+        const uint32_t bit = 1u << (key & 31);
+        dup |= (atomicOr(&bitmap[key >> 5], bit) & bit) != 0u;
+      }
+    }
+  } else {
+    for (int b = rk.e0; b < rk.e1; b += 32) {
       const int e = b + lane;
-      const int key = e < e1 ? sm.raw[e] : -1;
+      const int key = e < rk.e1 ? __ldg(irow + e) : -1;
+      if (key >= 0 && key < p.S) {
+        const uint32_t bit = 1u << (key & 31);
+        dup |= (atomicOr(&bitmap[key >> 5], bit) & bit) != 0u;
+      }
+    }
+  }
+  return named_any(1, kProducerThreads, dup);
+}
+
+// No repeated key: keep every in-range entry.  Each warp compacts its contiguous quarter of
+// the row 32 entries at a time (ballots), after a scan of the four quarters' counts.
+__device__ int compact_unique(const AttTcParams& p, const Smem& sm, const int32_t* irow, const RowKeys& rk) {
+  const int tid = threadIdx.x - 5 * 32, lane = threadIdx.x & 31, w = tid >> 5;
+  const uint32_t below = (1u << lane) - 1u;
+  int cnt = 0;
+  if (rk.cached) {
+#pragma unroll
+    for (int it = 0; it < kListCache; ++it)
+      cnt += __popc(__ballot_sync(0xffffffffu, rk.key[it] >= 0 && rk.key[it] < p.S));
+  } else {
+    for (int b = rk.e0; b < rk.e1; b += 32) {
+      const int e = b + lane;
+      const int key = e < rk.e1 ? __ldg(irow + e) : -1;
       cnt += __popc(__ballot_sync(0xffffffffu, key >= 0 && key < p.S));
     }
-    int* wtot = sm.bitmap_tail;                       // 4 ints past the bitmap's words
-    if (lane == 0) wtot[w] = cnt;
-    named_sync(1, kProducerThreads);
-    int base = 0;
-    for (int k = 0; k < w; ++k) base += wtot[k];
-    const int total = wtot[0] + wtot[1] + wtot[2] + wtot[3];
-    for (int b = e0; b < e1; b += 32) {
-      const int e = b + lane;
-      const int key = e < e1 ? sm.raw[e] : -1;
+  }
+  if (lane == 0) sm.wcount[w] = cnt;
+  named_sync(1, kProducerThreads);   // counts visible; every thread is past the bitmap
+  int base = 0;
+  for (int k = 0; k < w; ++k) base += sm.wcount[k];
+  const int total = sm.wcount[0] + sm.wcount[1] + sm.wcount[2] + sm.wcount[3];
+  if (rk.cached) {
+#pragma unroll
+    for (int it = 0; it < kListCache; ++it) {
+      const int key = rk.key[it];
       const bool keep = key >= 0 && key < p.S;
       const uint32_t m = __ballot_sync(0xffffffffu, keep);
-      if (keep) sm.list[base + __popc(m & ((1u << lane) - 1u))] = (uint16_t)key;
+      if (keep) sm.list[base + __popc(m & below)] = (uint16_t)key;
       base += __popc(m);
     }
-    named_sync(1, kProducerThreads);
-    if (tid == 0) {
-      TRACE(8, 1);
-      *sm.n_list = total;
-      mbar_arrive(smem_u32(sm.list_ready));
+  } else {
+    for (int b = rk.e0; b < rk.e1; b += 32) {
+      const int e = b + lane;
+      const int key = e < rk.e1 ? __ldg(irow + e) : -1;
+      const bool keep = key >= 0 && key < p.S;
+      const uint32_t m = __ballot_sync(0xffffffffu, keep);
+      if (keep) sm.list[base + __popc(m & below)] = (uint16_t)key;
+      base += __popc(m);
     }
-    named_sync(1, kProducerThreads);
-    return;
   }
-  for (int i = tid; i < words; i += kProducerThreads) sm.bitmap[i] = 0u;
+  named_sync(1, kProducerThreads);   // the counts are read before the next row rewrites them
+  return total;
+}
+
+// Repeated keys: order-preserving compaction by one warp, first occurrence only (not seen in
+// an earlier group of 32, lowest lane within its group).  `bitmap` must not overlap the list.
+__device__ int compact_first(const AttTcParams& p, const Smem& sm, const int32_t* irow, uint32_t* bitmap) {
+  const int tid = threadIdx.x - 5 * 32, lane = threadIdx.x & 31;
+  const int words = (p.S + 31) >> 5;
+  for (int i = tid; i < words; i += kProducerThreads) bitmap[i] = 0u;
   named_sync(1, kProducerThreads);
   if (tid < 32) {
-    // repeated keys: order-preserving compaction by one warp, first occurrence only
-    // (not seen in an earlier group of 32, lowest lane within its group)
     int n = 0;
     for (int e0 = 0; e0 < p.width; e0 += 32) {
       const int e = e0 + lane;
-      const int key = e < p.width ? sm.raw[e] : -1;
+      const int key = e < p.width ? __ldg(irow + e) : -1;
       bool keep = key >= 0 && key < p.S;
       const uint32_t peers = __match_any_sync(0xffffffffu, keep ? key : -1);
-      if (keep) keep = (sm.bitmap[key >> 5] & (1u << (key & 31))) == 0u && lane == __ffs(peers) - 1;
+      if (keep) keep = (bitmap[key >> 5] & (1u << (key & 31))) == 0u && lane == __ffs(peers) - 1;
       __syncwarp();
-      if (keep) atomicOr(&sm.bitmap[key >> 5], 1u << (key & 31));
+      if (keep) atomicOr(&bitmap[key >> 5], 1u << (key & 31));
       const uint32_t m = __ballot_sync(0xffffffffu, keep);
       if (keep) sm.list[n + __popc(m & ((1u << lane) - 1u))] = (uint16_t)key;
       n += __popc(m);
       __syncwarp();
     }
-    if (lane == 0) {
-      TRACE(8, 1);
-      *sm.n_list = n;
-      mbar_arrive(smem_u32(sm.list_ready));
-    }
+    if (lane == 0) sm.wcount[0] = n;
   }
   named_sync(1, kProducerThreads);
+  const int total = sm.wcount[0];
+  named_sync(1, kProducerThreads);
+  return total;
 }
 
+// Persistent: cluster c (of gridDim.x / 2) processes query rows c, c + #clusters, ...
+// All per-chunk barriers run on a global chunk counter across the cluster's rows, so
+// the next row's list build, query load and first gathers overlap the current row's
+// last chunks, and a row's epilogue overlaps the next row's first q.k.
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
                  const __grid_constant__ CUtensorMap map_rope,
                  AttTcParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  __shared__ int s_misc[4];
+  __shared__ int s_misc[5];
   __shared__ int s_wcount[4];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -292,18 +358,18 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   sm.qrope = sm.x + 2 * kXBytes;
   sm.kv = sm.qrope + kQRopeBytes;
   uint32_t off = sm.kv + kStages * kStageBytes - base;
-  // stage 0 is not gathered into before the list is built: bitmap (8 KB) then the raw row
-  sm.bitmap = reinterpret_cast<uint32_t*>(gb + (sm.kv - base));
-  sm.raw = reinterpret_cast<int*>(gb + (sm.kv - base) + kBitmapKeys / 8);
   sm.list = reinterpret_cast<uint16_t*>(gb + off);
-  off += ((uint32_t)p.width * 2u + 15u) & ~15u;
+  off += (uint32_t)list_bytes(p.width, p.S, p.list_bitmap != 0);
   sm.mx = reinterpret_cast<float*>(gb + off);
   off += 2 * 2 * 128 * 4;
+  sm.lsum = reinterpret_cast<float*>(gb + off);
+  off += 2 * 128 * 4;
   uint64_t* bars = reinterpret_cast<uint64_t*>(gb + off);
   sm.qfull = bars;
   sm.qrope_full = bars + 1;
   sm.list_ready = bars + 2;
-  sm.kv_full = bars + 3;
+  sm.list_taken = bars + 3;
+  sm.kv_full = bars + 4;
   sm.kv_empty = sm.kv_full + kStages;
   sm.s_full = sm.kv_empty + kStages;
   sm.s_read = sm.s_full + 2;
@@ -313,27 +379,33 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   sm.xfree = sm.xfull + 2;
   sm.xread = sm.xfree + 2;
   sm.mxready = sm.xread + 2;
-  sm.lready = sm.mxready + 2;
+  sm.o_free = sm.mxready + 2;
+  sm.lready = sm.o_free + 1;
   sm.drain = sm.lready + 1;
   sm.tmem_slot = reinterpret_cast<uint32_t*>(sm.drain + 1);
-  sm.n_list = &s_misc[0];
-  sm.dup_flag = &s_misc[1];
-  sm.abort_flag = &s_misc[2];
-  sm.bitmap_tail = s_wcount;
+  sm.n_list = &s_misc[0];                        // [0], [1]
+  sm.dup_flag = &s_misc[2];
+  sm.abort_flag = &s_misc[3];
+  sm.wcount = s_wcount;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
   const uint32_t peer = rank ^ 1u;
-  const size_t row = blockIdx.x >> 1;            // query row b*T + t
   const bool rope = p.kd == 576;                 // each CTA owns 32 of the 64 rope columns
   const int rope_col = 512 + 32 * (int)rank;
+  const long long n_rows = (long long)p.B * p.T;
+  const int ncl = (int)(gridDim.x >> 1), cid = (int)(blockIdx.x >> 1);
+  const int my_rows = n_rows > cid ? (int)((n_rows - 1 - cid) / ncl + 1) : 0;
+  auto row_of = [&](int i) { return (size_t)cid + (size_t)i * ncl; };
 
   if (threadIdx.x == 0) {
     *sm.abort_flag = 0;
-    mbar_init(smem_u32(sm.qfull), 8);            // one arrival per softmax warp once its Q columns are in TMEM
-    mbar_init(smem_u32(sm.lready), 8);
+    mbar_init(smem_u32(sm.qfull), 4);            // per row: each exchange warp's Q rows are in TMEM
     mbar_init(smem_u32(sm.qrope_full), 1);
-    mbar_init(smem_u32(sm.list_ready), 1);
+    mbar_init(smem_u32(sm.list_ready), 1);       // per row: the producer published n_list
+    mbar_init(smem_u32(sm.list_taken), 13);      // per row: MMA + 8 softmax + 4 exchange warps read it
+    mbar_init(smem_u32(sm.o_free), 8);           // per non-empty row: the epilogue has read O
+    mbar_init(smem_u32(sm.lready), 8);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&sm.kv_full[s]), 1);     // one expect-tx arrival; the gathers complete the bytes
       mbar_init(smem_u32(&sm.kv_empty[s]), 1);
@@ -362,72 +434,135 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   if (threadIdx.x == 0) TRACE(8, 0);
 
   if (warp >= 5 && warp <= 8) {
-    // ---------------------------------------------------------------- list + gathers
-    build_list(p, sm, row);
-    const int n = *sm.n_list;
-    const int nch = (n + kChunk - 1) / kChunk;
+    // ---------------------------------------------------------------- lists + gathers
     const int w = warp - 5;                              // 0..3: value block w; rope rows 16w..16w+15
-    const int rowbase = (int)(row / p.T) * p.S;          // latent row of key 0 of this query's sequence
     const uint32_t stage_bytes = rope ? kStageBytes : 4 * kBlockBytes;
     if (lane == 0) {
       tma_prefetch_desc(&map_kv);
       if (rope) tma_prefetch_desc(&map_rope);
     }
-    for (int j = 0; j < nch; ++j) {
-      const int s = j % kStages;
-      if (!mbar_wait(smem_u32(&sm.kv_empty[s]), ((j / kStages) & 1) ^ 1, p.status, abort_flag)) break;
-      if (w == 0 && lane == 0) {
-        TRACE(0, j);
-        mbar_arrive_expect_tx(smem_u32(&sm.kv_full[s]), stage_bytes);
+    long long gc = 0;                                    // global chunk counter
+    bool ok = true;
+    for (int i = 0; i < my_rows; ++i) {
+      const size_t row = row_of(i);
+      const int32_t* irow = p.idx + row * p.width;
+      RowKeys rk;
+      load_row(p, irow, rk);                             // in flight while the waits below run
+      // every consumer has read the previous row's length before this row's is published
+      const int s0 = (int)(gc % kStages);
+      bool got = true;
+      if (w == 0 && lane == 0) got = i == 0 || mbar_wait(smem_u32(sm.list_taken), (i - 1) & 1, p.status, abort_flag);
+      if (named_any(1, kProducerThreads, !got)) {
+        ok = false;
+        break;
       }
-      const uint32_t stb = sm.kv + s * kStageBytes;
-      const uint32_t bar = smem_u32(&sm.kv_full[s]);
-      // TMA tile::gather4: four selected rows per instruction, written in the swizzled operand
-      // layout.  Rows past the list repeat the list's first key (their scores are masked, P = 0).
-      // Lanes 0-15 gather 64 value columns of keys 4*lane..4*lane+3 into block w; lanes 16-19
-      // gather the 32 rope columns of keys 4*(4w+lane-16).. into the 64-byte swizzled rope block.
-      const int g = lane < 16 ? lane : 4 * w + (lane - 16);
-      if (lane < 16 || (rope && lane < 20)) {
-        int rr[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int li = j * kChunk + 4 * g + i;
-          rr[i] = rowbase + (int)sm.list[li < n ? li : 0];
+      // the dedupe bitmap: the list buffer (free once the previous row's gathers are issued) when
+      // it fits, else the stage of this row's first chunk (free once its P.V is done)
+      uint32_t* stage_bitmap = reinterpret_cast<uint32_t*>(gb + (sm.kv + s0 * kStageBytes - base));
+      auto wait_stage = [&]() {
+        bool g2 = true;
+        if (w == 0 && lane == 0)
+          g2 = mbar_wait(smem_u32(&sm.kv_empty[s0]), (uint32_t)(((gc / kStages) & 1) ^ 1), p.status, abort_flag);
+        return !named_any(1, kProducerThreads, !g2);
+      };
+      if (!p.list_bitmap && !wait_stage()) {
+        ok = false;
+        break;
+      }
+      const bool dup = mark_keys(p, irow, rk, p.list_bitmap ? reinterpret_cast<uint32_t*>(sm.list) : stage_bitmap);
+      int n;
+      if (!dup) {
+        n = compact_unique(p, sm, irow, rk);
+      } else {
+        if (p.list_bitmap && !wait_stage()) {
+          ok = false;
+          break;
         }
-        if (lane < 16)
-          tma_gather4(stb + w * kBlockBytes + g * 512, &map_kv, bar, (4 * (int)rank + w) * 64, rr[0], rr[1], rr[2],
-                      rr[3]);
-        else
-          tma_gather4(stb + kRopeOff + g * 256, &map_rope, bar, rope_col, rr[0], rr[1], rr[2], rr[3]);
+        n = compact_first(p, sm, irow, stage_bitmap);
       }
-      if (w == 0 && lane == 0) TRACE(11, j);
+      fence_proxy_async_smem();                          // bitmap writes ordered before gathers into the stage
+      named_sync(1, kProducerThreads);
+      if (w == 0 && lane == 0) {
+        sm.n_list[i & 1] = n;
+        TRACE(8, 1);
+        mbar_arrive(smem_u32(sm.list_ready));
+      }
+      const int nch = (n + kChunk - 1) / kChunk;
+      const int rowbase = (int)(row / p.T) * p.S;        // latent row of key 0 of this query's sequence
+      for (int j = 0; j < nch; ++j, ++gc) {
+        const int s = (int)(gc % kStages);
+        if (!(ok = mbar_wait(smem_u32(&sm.kv_empty[s]), (uint32_t)(((gc / kStages) & 1) ^ 1), p.status, abort_flag)))
+          break;
+        if (w == 0 && lane == 0) {
+          TRACE(0, gc);
+          mbar_arrive_expect_tx(smem_u32(&sm.kv_full[s]), stage_bytes);
+        }
+        const uint32_t stb = sm.kv + s * kStageBytes;
+        const uint32_t bar = smem_u32(&sm.kv_full[s]);
+        // TMA tile::gather4: four selected rows per instruction, written in the swizzled operand
+        // layout.  Rows past the list repeat the list's first key (their scores are masked, P = 0).
+        // Lanes 0-15 gather 64 value columns of keys 4*lane..4*lane+3 into block w; lanes 16-19
+        // gather the 32 rope columns of keys 4*(4w+lane-16).. into the 64-byte swizzled rope block.
+        const int g = lane < 16 ? lane : 4 * w + (lane - 16);
+        if (lane < 16 || (rope && lane < 20)) {
+          int rr[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int li = j * kChunk + 4 * g + k;
+            rr[k] = rowbase + (int)sm.list[li < n ? li : 0];
+          }
+          if (lane < 16)
+            tma_gather4(stb + w * kBlockBytes + g * 512, &map_kv, bar, (4 * (int)rank + w) * 64, rr[0], rr[1],
+                        rr[2], rr[3]);
+          else
+            tma_gather4(stb + kRopeOff + g * 256, &map_rope, bar, rope_col, rr[0], rr[1], rr[2], rr[3]);
+        }
+        if (w == 0 && lane == 0) TRACE(11, gc);
+      }
+      // the list buffer is rewritten for the next row only after these gathers were issued;
+      // a failed wait in any producer warp ends the loop for all four
+      if (named_any(1, kProducerThreads, !ok)) break;
     }
   } else if (warp == 4) {
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
-      if (rope) {
-        tma_prefetch_desc(&map_q);
-        mbar_arrive_expect_tx(smem_u32(sm.qrope_full), kQRopeBytes);
-        tma_load_2d(sm.qrope, &map_q, smem_u32(sm.qrope_full), rope_col, (int)(row * p.H));
-      }
       const uint32_t id_qk = idesc_bf16(128, kChunk);
       const uint32_t id_pv = idesc_bf16(128, 256, false, true);
-      bool ok = mbar_wait(smem_u32(sm.qfull), 0, p.status, abort_flag) &&
-                (!rope || mbar_wait(smem_u32(sm.qrope_full), 0, p.status, abort_flag)) &&
-                mbar_wait(smem_u32(sm.list_ready), 0, p.status, abort_flag);
-      const int n = ok ? *sm.n_list : 0;
-      const int nch = (n + kChunk - 1) / kChunk;
-      int qk = 0, pv = 0;
+      // q.k position: row index qi (in this cluster's sequence), chunk qj of qn; pv likewise.
+      // Rows without keys are skipped; ring[] keeps the chunk counts of the last non-empty rows.
+      int qi = 0, qj = 0, qn = -1, q_ne = 0;
+      int pj = 0, p_ne = 0;
+      int ring[4] = {0, 0, 0, 0};
+      long long gq = 0, gp = 0;
+      bool ok = true;
       unsigned long long t_last = globaltimer();
       uint32_t spins = 0;
-      while (ok && pv < nch) {
+      while (ok) {
         bool progressed = false;
-        // q.k of chunk qk: its stage is loaded and P.V of chunk qk-2 (same score buffer) is done
-        if (qk < nch && mbar_test_wait(smem_u32(&sm.kv_full[qk % kStages]), (qk / kStages) & 1) &&
-            mbar_test_wait(smem_u32(&sm.o_done[qk & 1]), ((qk >> 1) & 1) ^ 1)) {
+        if (qn < 0 && qi < my_rows && mbar_test_wait(smem_u32(sm.list_ready), qi & 1)) {
+          const int n = sm.n_list[qi & 1];
+          mbar_arrive(smem_u32(sm.list_taken));
+          qn = (n + kChunk - 1) / kChunk;
+          qj = 0;
+          if (qn == 0) {
+            ++qi;
+            qn = -1;
+          } else {
+            ring[q_ne & 3] = qn;
+            ++q_ne;
+          }
+          progressed = true;
+        }
+        // q.k of chunk gq: at a row start its query is loaded; its stage is loaded; P.V of chunk
+        // gq-2 (same score buffer) is done
+        if (qn > 0 &&
+            (qj > 0 || (mbar_test_wait(smem_u32(sm.qfull), qi & 1) &&
+                        (!rope || mbar_test_wait(smem_u32(sm.qrope_full), qi & 1)))) &&
+            mbar_test_wait(smem_u32(&sm.kv_full[gq % kStages]), (uint32_t)((gq / kStages) & 1)) &&
+            mbar_test_wait(smem_u32(&sm.o_done[gq & 1]), (uint32_t)(((gq >> 1) & 1) ^ 1))) {
           tc_fence_after();
-          const uint32_t st = sm.kv + (qk % kStages) * kStageBytes;
-          const uint32_t d = tmem + (qk & 1) * kChunk;
+          const uint32_t st = sm.kv + (gq % kStages) * kStageBytes;
+          const uint32_t d = tmem + (gq & 1) * kChunk;
           for (int lb = 0; lb < 4; ++lb) {
 #pragma unroll
             for (int k = 0; k < 4; ++k)
@@ -439,25 +574,36 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             for (int k = 0; k < 2; ++k)
               mma_bf16_ss(d, desc_sw64(sm.qrope + k * 32), desc_sw64(st + kRopeOff + k * 32), id_qk, 1u);
           }
-          mma_commit(smem_u32(&sm.s_full[qk & 1]));
-          TRACE(1, qk);
-          ++qk;
+          mma_commit(smem_u32(&sm.s_full[gq & 1]));
+          TRACE(1, gq);
+          ++gq;
+          if (++qj == qn) {
+            ++qi;
+            qn = -1;
+          }
           progressed = true;
         }
-        if (pv < qk && mbar_test_wait(smem_u32(&sm.p_full[pv & 1]), (pv >> 1) & 1)) {
+        // P.V of chunk gp: its P is in TMEM; at a row start the previous row's O has been read
+        if (gp < gq && (pj > 0 || p_ne == 0 || mbar_test_wait(smem_u32(sm.o_free), (p_ne - 1) & 1)) &&
+            mbar_test_wait(smem_u32(&sm.p_full[gp & 1]), (uint32_t)((gp >> 1) & 1))) {
           tc_fence_after();
-          const uint32_t st = sm.kv + (pv % kStages) * kStageBytes;
+          const uint32_t st = sm.kv + (gp % kStages) * kStageBytes;
 #pragma unroll
           for (int k = 0; k < kChunk / 16; ++k) {
             const uint64_t bd = desc_sw128(st + k * 2048, 1024, kBlockBytes);
-            mma_bf16_ts(tmem + kOCol, tmem + (pv & 1) * kChunk + k * 8, bd, id_pv, (pv | k) ? 1u : 0u);
+            mma_bf16_ts(tmem + kOCol, tmem + (gp & 1) * kChunk + k * 8, bd, id_pv, (pj | k) ? 1u : 0u);
           }
-          mma_commit(smem_u32(&sm.kv_empty[pv % kStages]));
-          mma_commit(smem_u32(&sm.o_done[pv & 1]));
-          TRACE(2, pv);
-          ++pv;
+          mma_commit(smem_u32(&sm.kv_empty[gp % kStages]));
+          mma_commit(smem_u32(&sm.o_done[gp & 1]));
+          TRACE(2, gp);
+          ++gp;
+          if (++pj == ring[p_ne & 3]) {
+            pj = 0;
+            ++p_ne;
+          }
           progressed = true;
         }
+        if (qi >= my_rows && gp == gq) break;    // every row's lists read, every chunk's P.V issued
         if (progressed) {
           spins = 0;
           continue;
@@ -482,36 +628,89 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
-    bool ok = mbar_wait(smem_u32(sm.list_ready), 0, p.status, abort_flag);
-    const int n = ok ? *sm.n_list : 0;
-    const int nch = (n + kChunk - 1) / kChunk;
     const uint32_t dst0 = map_peer(sm.x + (uint32_t)r * 16, peer);  // head r's 16 bytes of each [key/4][head][4] row
-    for (int j = 0; ok && j < nch; ++j) {
-      const int sb = j & 1, use = j >> 1;
-      if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), use & 1, p.status, abort_flag))) break;
-      tc_fence_after();
-      uint32_t v[kChunk];
-      tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-      tmem_ld_wait();
+    const bool real = r < p.H;
+    // Query of row i into TMEM: the CTA's 256 value-side columns of head r as bf16 pairs in
+    // lane r, columns kQCol..kQCol+127, plus the rope columns by TMA.  Called only when every
+    // q.k of earlier rows is complete (these warps have read all their scores).
+    auto load_q = [&](int i) {
+      const size_t qrow = row_of(i);
+      if (warp == 9 && lane == 0 && rope) {
+        mbar_arrive_expect_tx(smem_u32(sm.qrope_full), kQRopeBytes);
+        tma_load_2d(sm.qrope, &map_q, smem_u32(sm.qrope_full), rope_col, (int)(qrow * p.H));
+      }
+      const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (qrow * p.H + (real ? r : 0)) * p.kd + rank * 256);
+#pragma unroll 1
+      for (int c0 = 0; c0 < 128; c0 += 32) {      // 32 columns = 64 bf16 = 8 x 16 bytes
+        uint32_t qv[32];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint4 u = real ? qsrc[c0 / 4 + k] : make_uint4(0, 0, 0, 0);
+          qv[4 * k] = u.x;
+          qv[4 * k + 1] = u.y;
+          qv[4 * k + 2] = u.z;
+          qv[4 * k + 3] = u.w;
+        }
+        tmem_st_32x32b_x32(tmem + lane_addr + kQCol + c0, qv);
+      }
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.s_read[sb]));
-      if (q4 == 1 && lane == 0) TRACE(3, j);
-      // the peer has read its buffer sb from chunk j-2
-      if (!(ok = wait_cluster(smem_u32(&sm.xfree[sb]), (use & 1) ^ 1, p.status, abort_flag))) break;
-      const uint32_t dst = dst0 + (uint32_t)sb * kXBytes;
-      // [key/4][head][4 keys]: each store writes 4 keys of head r, the warp 512 contiguous
-      // bytes; each store completes its bytes on the peer's barrier (no round trip here)
-      const uint32_t xbar = map_peer(smem_u32(&sm.xfull[sb]), peer);
+      if (lane == 0) mbar_arrive(smem_u32(sm.qfull));
+      // the following row's query lines are pulled into L2 meanwhile
+      if (i + 1 < my_rows && real) {
+        const bf16* nq = p.q + (row_of(i + 1) * p.H + r) * p.kd + rank * 256;
 #pragma unroll
-      for (int c = 0; c < kChunk; c += 4) st_async_v4(dst + c * 512, &v[c], xbar);
-      if (q4 == 1 && lane == 0) TRACE(4, j);
-      // once our softmax has read our buffer sb for chunk j, the peer may refill it (chunk j+2)
-      if (j + 2 < nch) {
-        if (!(ok = mbar_wait(smem_u32(&sm.xread[sb]), use & 1, p.status, abort_flag))) break;
+        for (int k = 0; k < 4; ++k) asm volatile("prefetch.global.L2 [%0];" ::"l"(nq + 64 * k) : "memory");
+      }
+    };
+    if (my_rows > 0) load_q(0);
+    long long gc = 0;
+    bool ok = true;
+    for (int i = 0; ok && i < my_rows; ++i) {
+      if (!(ok = mbar_wait(smem_u32(sm.list_ready), i & 1, p.status, abort_flag))) break;
+      const int n = sm.n_list[i & 1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(sm.list_taken));
+      const int nch = (n + kChunk - 1) / kChunk;
+      if (nch == 0 && i + 1 < my_rows) load_q(i + 1);
+      for (int j = 0; j < nch; ++j, ++gc) {
+        const int sb = (int)(gc & 1);
+        const uint32_t use = (uint32_t)((gc >> 1) & 1);
+        if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), use, p.status, abort_flag))) break;
+        tc_fence_after();
+        uint32_t v[kChunk];
+        tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.s_read[sb]));
+        if (q4 == 1 && lane == 0) TRACE(3, gc);
+        // the peer has read its buffer sb from chunk gc-2
+        if (!(ok = wait_cluster(smem_u32(&sm.xfree[sb]), use ^ 1u, p.status, abort_flag))) break;
+        const uint32_t dst = dst0 + (uint32_t)sb * kXBytes;
+        // [key/4][head][4 keys]: each store writes 4 keys of head r, the warp 512 contiguous
+        // bytes; each store completes its bytes on the peer's barrier (no round trip here)
+        const uint32_t xbar = map_peer(smem_u32(&sm.xfull[sb]), peer);
+#pragma unroll
+        for (int c = 0; c < kChunk; c += 4) st_async_v4(dst + c * 512, &v[c], xbar);
+        if (q4 == 1 && lane == 0) TRACE(4, gc);
+        if (j + 1 == nch) break;                     // the last chunk's buffer is released below
+        // once our softmax has read our buffer sb of chunk gc, the peer may refill it
+        if (!(ok = mbar_wait(smem_u32(&sm.xread[sb]), use, p.status, abort_flag))) break;
         __syncwarp();
         if (lane == 0) arrive_remote_relaxed(map_peer(smem_u32(&sm.xfree[sb]), peer));
+      }
+      if (ok && nch > 0) {
+        // the row's last q.k is complete (its scores were just read): load the next row's query,
+        // then release the last chunk's exchange buffer
+        if (i + 1 < my_rows) load_q(i + 1);
+        const int sb = (int)(gc & 1);
+        if (!(ok = mbar_wait(smem_u32(&sm.xread[sb]), (uint32_t)((gc >> 1) & 1), p.status, abort_flag))) break;
+        __syncwarp();
+        if (lane == 0) arrive_remote_relaxed(map_peer(smem_u32(&sm.xfree[sb]), peer));
+        ++gc;
       }
     }
   } else if (warp < 4 || warp >= 13) {
@@ -522,148 +721,158 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const int r = q4 * 32 + lane;                   // head row == TMEM lane
     const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
     const bool lead = g == 0 && q4 == 0 && lane == 0;
-    [[maybe_unused]] const bool lead1 = g == 1 && q4 == 0 && lane == 0;
-    {
-      // value-side query columns of head r -> TMEM lane r (bf16 pairs); group g loads 64 columns
-      const bool real = r < p.H;
-      const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (row * p.H + (real ? r : 0)) * p.kd + rank * 256);
-#pragma unroll 1
-      for (int c0 = 64 * g; c0 < 64 * g + 64; c0 += 32) {   // 32 columns = 64 bf16 = 8 x 16 bytes
-        uint32_t qv[32];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 u = real ? qsrc[c0 / 4 + i] : make_uint4(0, 0, 0, 0);
-          qv[4 * i] = u.x;
-          qv[4 * i + 1] = u.y;
-          qv[4 * i + 2] = u.z;
-          qv[4 * i + 3] = u.w;
-        }
-        tmem_st_32x32b_x32(tmem + lane_addr + kQCol + c0, qv);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(sm.qfull));
-    }
-    float m_ref = -INFINITY, l_sum = 0.f;
-    bool ok = mbar_wait(smem_u32(sm.list_ready), 0, p.status, abort_flag);
-    const int n = ok ? *sm.n_list : 0;
-    const int nch = (n + kChunk - 1) / kChunk;
+    const bool real = r < p.H;
     const float4* xcol = reinterpret_cast<const float4*>(gb + (sm.x - base)) + r;  // head r of [key/4][head][4]
-    for (int j = 0; ok && j < nch; ++j) {
-      const int sb = j & 1, use = j >> 1;
-      if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), use & 1, p.status, abort_flag))) break;
-      tc_fence_after();
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk + 32 * g, v);
-      tmem_ld_wait();
-      if (lead) TRACE(5, j);
-      if (lead1) TRACE(12, j);
-      if (!(ok = wait_cluster(smem_u32(&sm.xfull[sb]), use & 1, p.status, abort_flag))) break;
-      if (lead1) TRACE(13, j);
-      if (lead) {
-        TRACE(6, j);
-        if (j + 2 < nch) mbar_arrive_expect_tx(smem_u32(&sm.xfull[sb]), kXBytes);  // arm the next use
-      }
-      const float4* xr = xcol + sb * (kXBytes / 16) + 8 * g * 128;
-      const int valid = n - j * kChunk - 32 * g;
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 32; c += 4) {
-        const float4 x4 = xr[(c / 4) * 128];
-        const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float x = c + i < valid ? (__uint_as_float(v[c + i]) + xs[i]) * p.scale_log2 : -INFINITY;
-          v[c + i] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
-      }
-      // our buffer sb is read (values are in registers); the exchange warps tell the peer
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.xread[sb]));
-      // row maximum over both halves of the chunk
-      float* mxb = sm.mx + (j & 1) * 256;
-      mxb[g * 128 + r] = mx;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.mxready[j & 1]));
-      if (!(ok = mbar_wait(smem_u32(&sm.mxready[j & 1]), use & 1, p.status, abort_flag))) break;
-      mx = fmaxf(mx, mxb[(1 - g) * 128 + r]);
-      if (lead) TRACE(9, j);
-      if (lead1) TRACE(14, j);
-      // move the reference maximum only when it grows by more than 2^8 (both groups agree)
-      const bool grow = mx > m_ref + 8.f;
-      const float new_ref = grow ? mx : m_ref;
-      if (__any_sync(0xffffffffu, grow && j > 0)) {
-        if (!(ok = mbar_wait(smem_u32(&sm.o_done[(j - 1) & 1]), ((j - 1) >> 1) & 1, p.status, abort_flag))) break;
-        tc_fence_after();
-        const float f = (grow && j > 0) ? ex2(m_ref - new_ref) : 1.f;
-        for (int c = 128 * g; c < 128 * g + 128; c += 16) {
-          uint32_t o[16];
-          tmem_ld_32x32b_x16(tmem + lane_addr + kOCol + c, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-          tmem_st_32x32b_x16(tmem + lane_addr + kOCol + c, o);
-        }
-        tmem_st_wait();
-        l_sum *= f;
-      }
-      m_ref = new_ref;
-      uint32_t pk[16];
-#pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        const float p0 = ex2(__uint_as_float(v[c]) - m_ref);
-        const float p1 = ex2(__uint_as_float(v[c + 1]) - m_ref);
-        l_sum += p0 + p1;
-        pk[c / 2] = pack_bf16(p0, p1);
-      }
-      if (lead) TRACE(10, j);
-      // P (keys 32g..32g+31) overwrites columns 16g..16g+15 of the score buffer once the exchange warps have read it
-      if (!(ok = mbar_wait(smem_u32(&sm.s_read[sb]), use & 1, p.status, abort_flag))) break;
-      tmem_st_32x32b_x16(tmem + lane_addr + sb * kChunk + 16 * g, pk);
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[sb]));
-      if (lead) TRACE(7, j);
-      if (lead1) TRACE(15, j);
-    }
-    // epilogue: O / (l0 + l1) -> bf16, group g writes O columns 128g..128g+127
-    const bool write = r < p.H;
-    bf16* orow = p.out + (row * p.H + r) * 512 + rank * 256 + 128 * g;
-    if (ok && nch > 0) {
-      float* lb = sm.mx + (nch & 1) * 256;           // not read again after chunk nch-2
-      lb[g * 128 + r] = l_sum;
+    long long gc = 0;
+    bool ok = true;
+    // the epilogue of a row runs after the next row's query load, so it overlaps that row's first q.k
+    bool pending = false;
+    size_t p_row = 0;
+    long long p_last = 0;
+    float p_mref = 0.f, p_lsum = 0.f;
+    int n_epi = 0;
+    auto epilogue = [&]() {
+      bf16* orow = p.out + (p_row * p.H + r) * 512 + rank * 256 + 128 * g;
+      sm.lsum[g * 128 + r] = p_lsum;
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(sm.lready));
-      ok = mbar_wait(smem_u32(sm.lready), 0, p.status, abort_flag) &&
-           mbar_wait(smem_u32(&sm.o_done[(nch - 1) & 1]), ((nch - 1) >> 1) & 1, p.status, abort_flag);
-      const float l_all = l_sum + lb[(1 - g) * 128 + r];
+      ok = mbar_wait(smem_u32(sm.lready), n_epi & 1, p.status, abort_flag) &&
+           mbar_wait(smem_u32(&sm.o_done[p_last & 1]), (uint32_t)((p_last >> 1) & 1), p.status, abort_flag);
+      const float l_all = p_lsum + sm.lsum[(1 - g) * 128 + r];
       tc_fence_after();
       const float inv = 1.f / l_all;
       for (int c = 0; c < 128; c += 32) {
         uint32_t o[32];
         tmem_ld_32x32b_x32(tmem + lane_addr + kOCol + 128 * g + c, o);
         tmem_ld_wait();
-        if (write && ok) {
+        if (real && ok) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            uint4 pkv;
-            pkv.x = pack_bf16(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
-            pkv.y = pack_bf16(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
-            pkv.z = pack_bf16(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
-            pkv.w = pack_bf16(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + c + i) = pkv;
+          for (int k = 0; k < 16; ++k) pk[k] = pack_bf16(__uint_as_float(o[2 * k]) * inv, __uint_as_float(o[2 * k + 1]) * inv);
+          if (p.out_v8) {
+            // 32 contiguous bytes (one full sector) per store
+            st_global_v8(orow + c, pk);
+            st_global_v8(orow + c + 16, pk + 8);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              *reinterpret_cast<uint4*>(orow + c + 8 * k) = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
           }
         }
       }
-      if (write && ok && rank == 0 && g == 0 && p.lse)
-        p.lse[row * p.H + r] = (m_ref + log2f(l_all)) * 0.69314718055994531f;
-    } else if (ok && write) {
-      for (int c = 0; c < 128; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
-      if (rank == 0 && g == 0 && p.lse) p.lse[row * p.H + r] = -INFINITY;
+      if (real && ok && rank == 0 && g == 0 && p.lse)
+        p.lse[p_row * p.H + r] = (p_mref + log2f(l_all)) * 0.69314718055994531f;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(sm.o_free));  // P.V of the next row may overwrite O
+      ++n_epi;
+      pending = false;
+    };
+    for (int i = 0; ok && i < my_rows; ++i) {
+      const size_t row = row_of(i);
+      if (pending) {
+        epilogue();
+        if (!ok) break;
+      }
+      if (!(ok = mbar_wait(smem_u32(sm.list_ready), i & 1, p.status, abort_flag))) break;
+      const int n = sm.n_list[i & 1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(sm.list_taken));
+      const int nch = (n + kChunk - 1) / kChunk;
+      if (nch == 0) {
+        // no key selected: out = 0, lse = -inf
+        if (real) {
+          bf16* orow = p.out + (row * p.H + r) * 512 + rank * 256 + 128 * g;
+          for (int c = 0; c < 128; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+          if (rank == 0 && g == 0 && p.lse) p.lse[row * p.H + r] = -INFINITY;
+        }
+        continue;
+      }
+      float m_ref = -INFINITY, l_sum = 0.f;
+      for (int j = 0; ok && j < nch; ++j, ++gc) {
+        const int sb = (int)(gc & 1);
+        const uint32_t use = (uint32_t)((gc >> 1) & 1);
+        if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), use, p.status, abort_flag))) break;
+        tc_fence_after();
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk + 32 * g, v);
+        tmem_ld_wait();
+        if (lead) TRACE(5, gc);
+        if (!(ok = wait_cluster(smem_u32(&sm.xfull[sb]), use, p.status, abort_flag))) break;
+        if (lead) {
+          TRACE(6, gc);
+          mbar_arrive_expect_tx(smem_u32(&sm.xfull[sb]), kXBytes);  // arm the next use
+        }
+        const float4* xr = xcol + sb * (kXBytes / 16) + 8 * g * 128;
+        const int valid = n - j * kChunk - 32 * g;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          const float4 x4 = xr[(c / 4) * 128];
+          const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float x = c + k < valid ? (__uint_as_float(v[c + k]) + xs[k]) * p.scale_log2 : -INFINITY;
+            v[c + k] = __float_as_uint(x);
+            mx = fmaxf(mx, x);
+          }
+        }
+        // our buffer sb is read (values are in registers); the exchange warps tell the peer
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.xread[sb]));
+        // row maximum over both halves of the chunk
+        float* mxb = sm.mx + sb * 256;
+        mxb[g * 128 + r] = mx;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.mxready[sb]));
+        if (!(ok = mbar_wait(smem_u32(&sm.mxready[sb]), use, p.status, abort_flag))) break;
+        mx = fmaxf(mx, mxb[(1 - g) * 128 + r]);
+        if (lead) TRACE(9, gc);
+        // move the reference maximum only when it grows by more than 2^8 (both groups agree)
+        const bool grow = mx > m_ref + 8.f;
+        const float new_ref = grow ? mx : m_ref;
+        if (__any_sync(0xffffffffu, grow && j > 0)) {
+          const long long pg = gc - 1;
+          if (!(ok = mbar_wait(smem_u32(&sm.o_done[pg & 1]), (uint32_t)((pg >> 1) & 1), p.status, abort_flag))) break;
+          tc_fence_after();
+          const float f = (grow && j > 0) ? ex2(m_ref - new_ref) : 1.f;
+          for (int c = 128 * g; c < 128 * g + 128; c += 16) {
+            uint32_t o[16];
+            tmem_ld_32x32b_x16(tmem + lane_addr + kOCol + c, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
+            tmem_st_32x32b_x16(tmem + lane_addr + kOCol + c, o);
+          }
+          tmem_st_wait();
+          l_sum *= f;
+        }
+        m_ref = new_ref;
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const float p0 = ex2(__uint_as_float(v[c]) - m_ref);
+          const float p1 = ex2(__uint_as_float(v[c + 1]) - m_ref);
+          l_sum += p0 + p1;
+          pk[c / 2] = pack_bf16(p0, p1);
+        }
+        if (lead) TRACE(10, gc);
+        // P (keys 32g..32g+31) overwrites columns 16g..16g+15 of the score buffer once the exchange warps have read it
+        if (!(ok = mbar_wait(smem_u32(&sm.s_read[sb]), use, p.status, abort_flag))) break;
+        tmem_st_32x32b_x16(tmem + lane_addr + sb * kChunk + 16 * g, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[sb]));
+        if (lead) TRACE(7, gc);
+      }
+      pending = true;
+      p_row = row;
+      p_last = gc - 1;
+      p_mref = m_ref;
+      p_lsum = l_sum;
     }
+    if (ok && pending) epilogue();
   }
   tc_fence_before();
   __syncthreads();
@@ -691,10 +900,12 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-size_t smem_bytes(int width) {
-  return 1024 + 2 * (size_t)kXBytes + kQRopeBytes + (size_t)kStages * kStageBytes +
-         (((size_t)width * 2 + 15) & ~(size_t)15) + 2 * 2 * 128 * 4 + 8 * 32 + 16;
+size_t smem_bytes(int width, int S, bool with_bitmap) {
+  return 1024 + 2 * (size_t)kXBytes + kQRopeBytes + (size_t)kStages * kStageBytes + list_bytes(width, S, with_bitmap) +
+         2 * 2 * 128 * 4 + 2 * 128 * 4 + 8 * 40 + 16;
 }
+
+bool bitmap_in_list(int width, int S) { return smem_bytes(width, S, true) <= 227 * 1024; }
 
 }  // namespace
 
@@ -707,7 +918,7 @@ bool attend_tc_supported(const dsa_dims& d, int64_t k_stride, const void* k, con
   if (k != v || k_stride != v_stride || k_stride < d.kd || (k_stride * 2) % 16 != 0) return false;
   if (((uintptr_t)k & 15u) != 0) return false;
   if (d.n_kv > kBitmapKeys || width > 8192) return false;  // bitmap + raw row fit in the (idle) gather stages
-  if (smem_bytes(width) > 227 * 1024) return false;
+  if (smem_bytes(width, d.n_kv, false) > 227 * 1024) return false;
   return encode_fn() != nullptr;
 }
 
@@ -758,11 +969,18 @@ cudaError_t launch_attend_tc(const dsa_dims& d, const void* q, const void* k, in
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  const size_t smem = smem_bytes(width);
+  p.list_bitmap = bitmap_in_list(width, d.n_kv) ? 1 : 0;
+  p.out_v8 = ((uintptr_t)out & 31u) == 0 ? 1 : 0;
+  const size_t smem = smem_bytes(width, d.n_kv, p.list_bitmap != 0);
   cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  // persistent clusters: one per SM pair (or one per row when there are fewer rows)
   const long long rows = (long long)d.batch * d.n_q;
-  attend_tc_kernel<<<dim3((unsigned)(2 * rows)), kThreads, smem, st>>>(mq, mkv, mrope, p);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long clusters = rows < sms / 2 ? rows : sms / 2;
+  attend_tc_kernel<<<dim3((unsigned)(2 * clusters)), kThreads, smem, st>>>(mq, mkv, mrope, p);
   return cudaGetLastError();
 }
 
