@@ -537,6 +537,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       bool ok = true;
       unsigned long long t_last = globaltimer();
       uint32_t spins = 0;
+#ifdef DSA_TRACE
+      bool trace_q = false, trace_kv = false;
+#endif
       while (ok) {
         bool progressed = false;
         if (qn < 0 && qi < my_rows && mbar_test_wait(smem_u32(sm.list_ready), qi & 1)) {
@@ -553,6 +556,18 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           }
           progressed = true;
         }
+#ifdef DSA_TRACE
+        if (qn > 0 && qj == 0) {
+          if (mbar_test_wait(smem_u32(sm.qfull), qi & 1) && !trace_q) {
+            TRACE(12, gq);
+            trace_q = true;
+          }
+          if (mbar_test_wait(smem_u32(&sm.kv_full[gq % kStages]), (uint32_t)((gq / kStages) & 1)) && !trace_kv) {
+            TRACE(13, gq);
+            trace_kv = true;
+          }
+        }
+#endif
         // q.k of chunk gq: at a row start its query is loaded; its stage is loaded; P.V of chunk
         // gq-2 (same score buffer) is done
         if (qn > 0 &&
@@ -576,6 +591,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           }
           mma_commit(smem_u32(&sm.s_full[gq & 1]));
           TRACE(1, gq);
+#ifdef DSA_TRACE
+          trace_q = trace_kv = false;
+#endif
           ++gq;
           if (++qj == qn) {
             ++qi;

@@ -287,9 +287,22 @@ cudaError_t launch_index_scores_tc(const dsa_dims& d, const void* q_idx, const v
   p.n_qtiles = (p.T + p.NQ - 1) / p.NQ;
   p.n_ktiles = (p.S + kKeysPerTile - 1) / kKeysPerTile;
   const int sms = sm_count();
-  int splits = (sms * 2 + p.B * p.n_qtiles - 1) / (p.B * p.n_qtiles);
-  if (splits < 1) splits = 1;
-  if (splits > p.n_ktiles) splits = p.n_ktiles;
+  // Key-range splits per query tile: one CTA per SM, so the time is about (waves) x (tiles per
+  // CTA + a fixed cost of ~3 tiles for the query load and pipeline fill).  Pick the split count
+  // that minimises it; a count that leaves a nearly empty last wave loses to a finer one.
+  const long long qt = (long long)p.B * p.n_qtiles;
+  int splits = 1;
+  long long best = -1;
+  for (int s2 = 1; s2 <= p.n_ktiles && s2 <= 512; ++s2) {
+    const int tps = (p.n_ktiles + s2 - 1) / s2;
+    const int used = (p.n_ktiles + tps - 1) / tps;           // splits that get tiles
+    const long long waves = (qt * used + sms - 1) / sms;
+    const long long cost = waves * (tps + 3);
+    if (best < 0 || cost < best) {
+      best = cost;
+      splits = used;
+    }
+  }
   p.tiles_per_split = (p.n_ktiles + splits - 1) / splits;
   splits = (p.n_ktiles + p.tiles_per_split - 1) / p.tiles_per_split;
   p.epi_warps = p.NQ >= 2 ? 8 : 4;

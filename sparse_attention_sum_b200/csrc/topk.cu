@@ -26,6 +26,8 @@
 namespace dsa {
 
 constexpr int kTopkCacheMax = 40960;  // keys cached in shared memory (160 KB)
+constexpr int kHist12 = 4096;         // first-pass histogram: the top 12 bits of a key
+constexpr int kCand = 4096;           // keys of the threshold's 12-bit bin resolved on their own
 
 // Block-wide exclusive scan of one int per thread; returns the block total.
 template <int BLOCK>
@@ -53,6 +55,38 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch /*>= BLO
   total = scratch[BLOCK / 32 - 1];
   __syncthreads();
   return warp_base + x - v;
+}
+
+// In a histogram of `nbins` bins (bin = a digit, counted over the keys still in play), find
+// the digit holding the `kneed`-th largest key, scanning digits from the top: *s_bin gets
+// the digit and *s_krem how many keys of that digit are still needed.  Block-wide.
+template <int BLOCK>
+__device__ void find_crossing(const uint32_t* hist, int nbins, uint32_t kneed, int* scan, uint32_t* s_bin,
+                              uint32_t* s_krem) {
+  const int per = nbins >= BLOCK ? nbins / BLOCK : 1;    // digits per thread (<= 8)
+  const int owners = nbins / per;
+  uint32_t cnt[8];
+  uint32_t lsum = 0;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    cnt[u] = (u < per && (int)threadIdx.x < owners) ? hist[nbins - 1 - (per * (int)threadIdx.x + u)] : 0u;
+    lsum += cnt[u];
+  }
+  int total;
+  const uint32_t excl = (uint32_t)block_exclusive_scan<BLOCK>((int)lsum, scan, total);
+  if ((int)threadIdx.x < owners && excl < kneed && excl + lsum >= kneed) {
+    uint32_t c = excl;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (u < per && c + cnt[u] >= kneed) {
+        *s_bin = (uint32_t)(nbins - 1 - (per * (int)threadIdx.x + u));
+        *s_krem = kneed - c;
+        break;
+      }
+      c += cnt[u];
+    }
+  }
+  __syncthreads();
 }
 
 // Stable LSD radix sort of m (key, index) pairs by key, descending: four 8-bit
@@ -129,8 +163,11 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
   uint32_t* rhist = reinterpret_cast<uint32_t*>(tmp + ksel);         // [BLOCK/32 * 256] (ranked only)
   uint32_t* hist = rhist + (RANKED ? (BLOCK / 32) * 256 : 0);        // [256]
   int* scan = reinterpret_cast<int*>(hist + 256);                    // [64]
-  uint32_t* cache = reinterpret_cast<uint32_t*>(scan + 64);          // [cache_cap]
-  __shared__ uint32_t s_prefix, s_krem;
+  uint32_t* hist12 = reinterpret_cast<uint32_t*>(scan + 64);         // [kHist12]
+  uint32_t* cand = hist12 + kHist12;                                 // [kCand]
+  uint32_t* cache = cand + kCand;                                    // [cache_cap]
+  __shared__ uint32_t s_prefix, s_krem, s_bin;
+  __shared__ int s_ncand;
 
   const int b = blockIdx.y, t = blockIdx.x;
   const size_t row = (size_t)b * d.n_q + t;
@@ -169,66 +206,95 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
     return;
   }
 
-  if (cached)
-    for (int i = threadIdx.x; i < n; i += BLOCK) cache[i] = score_key(srow[r.lo + i]);
-  if (threadIdx.x == 0) {
-    s_prefix = 0u;
-    s_krem = (uint32_t)k;
+  // ---- threshold: tau = the k-th largest key.  One pass over the row (filling the cache)
+  // counts the top 12 bits; the keys of the bin holding the k-th largest then become a small
+  // candidate set, and the low 20 bits are resolved over it alone (12 + 8 bits).
+  const int lane0 = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kHist12; i += BLOCK) hist12[i] = 0u;
+  if (threadIdx.x == 0) s_ncand = 0;
+  __syncthreads();
+  constexpr int kU = 8;                 // independent loads in flight per thread
+  for (int base = (threadIdx.x & ~31); base < n; base += BLOCK * kU) {
+    float v[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i = base + u * BLOCK + lane0;
+      v[u] = i < n ? __ldg(srow + r.lo + i) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i = base + u * BLOCK + lane0;
+      if (i < n) {
+        const uint32_t key = score_key(v[u]);
+        if (cached) cache[i] = key;
+        atomicAdd(&hist12[key >> 20], 1u);
+      }
+    }
   }
   __syncthreads();
-
-  // ---- radix select: find tau (the k-th largest key) digit by digit
-  uint32_t prefix = 0u, mask = 0u;
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  find_crossing<BLOCK>(hist12, kHist12, (uint32_t)k, scan, &s_bin, &s_krem);
+  const uint32_t b1 = s_bin, krem1 = s_krem;
+  const uint32_t nb1 = hist12[b1];
+  uint32_t prefix = 0u;
+  if (nb1 <= (uint32_t)kCand) {
+    // collect the bin's keys (any order: only their values matter here)
+    for (int base = (threadIdx.x & ~31); base < n; base += BLOCK) {
+      const int i = base + lane0;
+      uint32_t key = 0u;
+      bool in = false;
+      if (i < n) {
+        key = cached ? cache[i] : score_key(srow[r.lo + i]);
+        in = (key >> 20) == b1;
+      }
+      const uint32_t m = __ballot_sync(0xffffffffu, in);
+      int slot = 0;
+      if (lane0 == 0 && m) slot = atomicAdd(&s_ncand, __popc(m));
+      slot = __shfl_sync(0xffffffffu, slot, 0);
+      if (in) cand[slot + __popc(m & ((1u << lane0) - 1u))] = key;
+    }
+    __syncthreads();
+    // bits 19..8 of the candidates
+    for (int i = threadIdx.x; i < kHist12; i += BLOCK) hist12[i] = 0u;
+    __syncthreads();
+    for (int c = threadIdx.x; c < (int)nb1; c += BLOCK) atomicAdd(&hist12[(cand[c] >> 8) & 4095u], 1u);
+    __syncthreads();
+    find_crossing<BLOCK>(hist12, kHist12, krem1, scan, &s_bin, &s_krem);
+    const uint32_t b2 = s_bin, krem2 = s_krem;
+    // bits 7..0 of the candidates whose bits 19..8 are b2
     for (int i = threadIdx.x; i < 256; i += BLOCK) hist[i] = 0u;
     __syncthreads();
-    for (int base = (threadIdx.x & ~31); base < n; base += BLOCK) {
-      const int i = base + (threadIdx.x & 31);
-      int bin = -1;
-      if (i < n) {
-        uint32_t key = cached ? cache[i] : score_key(srow[r.lo + i]);
-        if ((key & mask) == prefix) bin = (int)((key >> shift) & 255u);
-      }
-      // lanes that hit the same bin add once (scores often share their top bits)
-      uint32_t peers = __match_any_sync(0xffffffffu, bin);
-      if (bin >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+    for (int c = threadIdx.x; c < (int)nb1; c += BLOCK)
+      if (((cand[c] >> 8) & 4095u) == b2) atomicAdd(&hist[cand[c] & 255u], 1u);
+    __syncthreads();
+    find_crossing<BLOCK>(hist, 256, krem2, scan, &s_bin, &s_krem);
+    prefix = (b1 << 20) | (b2 << 8) | s_bin;
+  } else {
+    // a crowded bin (e.g. many equal scores): 8-bit digits over the whole row
+    if (threadIdx.x == 0) {
+      s_prefix = 0u;
+      s_krem = (uint32_t)k;
     }
     __syncthreads();
-    if (threadIdx.x < 32) {
-      // lane L owns digits 255-8L .. 248-8L (descending)
-      const int lane = threadIdx.x;
-      uint32_t cnt[8];
-      uint32_t lsum = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        cnt[j] = hist[255 - 8 * lane - j];
-        lsum += cnt[j];
-      }
-      uint32_t incl = lsum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      uint32_t excl = incl - lsum;
-      uint32_t krem = s_krem;
-      if (excl < krem && incl >= krem) {  // the crossing digit lies in this lane's 8 bins
-        uint32_t c = excl;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (c + cnt[j] >= krem) {
-            s_prefix = prefix | ((uint32_t)(255 - 8 * lane - j) << shift);
-            s_krem = krem - c;
-            break;
-          }
-          c += cnt[j];
+    uint32_t mask = 0u;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = threadIdx.x; i < 256; i += BLOCK) hist[i] = 0u;
+      __syncthreads();
+      for (int base = (threadIdx.x & ~31); base < n; base += BLOCK) {
+        const int i = base + lane0;
+        int bin = -1;
+        if (i < n) {
+          const uint32_t key = cached ? cache[i] : score_key(srow[r.lo + i]);
+          if ((key & mask) == prefix) bin = (int)((key >> shift) & 255u);
         }
+        const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+        if (bin >= 0 && lane0 == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
       }
+      __syncthreads();
+      const uint32_t krem = s_krem;
+      find_crossing<BLOCK>(hist, 256, krem, scan, &s_bin, &s_krem);
+      prefix |= s_bin << shift;
+      mask |= 255u << shift;
     }
-    __syncthreads();
-    prefix = s_prefix;
-    mask |= 255u << shift;
-    __syncthreads();
   }
   const uint32_t tau = prefix;
   const int need_eq = (int)s_krem;  // keys equal to tau still to take (lowest indices first)
@@ -310,8 +376,8 @@ template <int BLOCK, bool RANKED>
 cudaError_t launch_topk_t(const dsa_dims& d, const float* scores, const int32_t* q_pos, const int32_t* kv_start,
                           const int32_t* kv_len, int k, int32_t* idx, float* vals, cudaStream_t st) {
   int cache_cap = d.n_kv < kTopkCacheMax ? d.n_kv : kTopkCacheMax;
-  const size_t fixed =
-      (RANKED ? (size_t)k * 16 + (size_t)(BLOCK / 32) * 256 * 4 : 0) + 256 * 4 + 64 * 4;
+  const size_t fixed = (RANKED ? (size_t)k * 16 + (size_t)(BLOCK / 32) * 256 * 4 : 0) + 256 * 4 + 64 * 4 +
+                       (size_t)(kHist12 + kCand) * 4;
   if (fixed + (size_t)cache_cap * 4 > 220 * 1024) cache_cap = (int)((220 * 1024 - fixed) / 4);
   const size_t smem = fixed + (size_t)cache_cap * 4;
   auto kern = topk_kernel<BLOCK, RANKED>;
