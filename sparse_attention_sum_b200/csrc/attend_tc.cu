@@ -343,6 +343,9 @@ __device__ int compact_first(const AttTcParams& p, const Smem& sm, const int32_t
 // All per-chunk barriers run on a global chunk counter across the cluster's rows, so
 // the next row's list build, query load and first gathers overlap the current row's
 // last chunks, and a row's epilogue overlaps the next row's first q.k.
+// kHalfHeads: H = 64, so the head rows 64-127 of the M = 128 tiles are padding; the warps that own
+// them skip their softmax and exchange work (separate instantiation, so H = 128 pays nothing).
+template <bool kHalfHeads>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
                  const __grid_constant__ CUtensorMap map_rope,
@@ -422,7 +425,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     }
     mbar_init(smem_u32(sm.drain), 1);
     fence_barrier_init();
-    for (int s = 0; s < 2; ++s) mbar_arrive_expect_tx(smem_u32(&sm.xfull[s]), kXBytes);  // first use of each buffer
+    for (int s = 0; s < 2; ++s) mbar_arrive_expect_tx(smem_u32(&sm.xfull[s]), 64u * p.H * 4u);  // first use of each buffer
   }
   if (warp == 4) tmem_alloc(smem_u32(sm.tmem_slot), 512);
   tc_fence_before();
@@ -648,6 +651,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
     const uint32_t dst0 = map_peer(sm.x + (uint32_t)r * 16, peer);  // head r's 16 bytes of each [key/4][head][4] row
     const bool real = r < p.H;
+    const bool act = !kHalfHeads || q4 < 2;        // warp-uniform: this warp's head rows exist
     // Query of row i into TMEM: the CTA's 256 value-side columns of head r as bf16 pairs in
     // lane r, columns kQCol..kQCol+127, plus the rope columns by TMA.  Called only when every
     // q.k of earlier rows is complete (these warps have read all their scores).
@@ -659,7 +663,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       }
       const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (qrow * p.H + (real ? r : 0)) * p.kd + rank * 256);
 #pragma unroll 1
-      for (int c0 = 0; c0 < 128; c0 += 32) {      // 32 columns = 64 bf16 = 8 x 16 bytes
+      for (int c0 = 0; act && c0 < 128; c0 += 32) {      // 32 columns = 64 bf16 = 8 x 16 bytes
         uint32_t qv[32];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
@@ -696,23 +700,29 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         const int sb = (int)(gc & 1);
         const uint32_t use = (uint32_t)((gc >> 1) & 1);
         if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), use, p.status, abort_flag))) break;
-        tc_fence_after();
-        uint32_t v[kChunk];
-        tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&sm.s_read[sb]));
-        if (q4 == 1 && lane == 0) TRACE(3, gc);
-        // the peer has read its buffer sb from chunk gc-2
-        if (!(ok = wait_cluster(smem_u32(&sm.xfree[sb]), use ^ 1u, p.status, abort_flag))) break;
-        const uint32_t dst = dst0 + (uint32_t)sb * kXBytes;
-        // [key/4][head][4 keys]: each store writes 4 keys of head r, the warp 512 contiguous
-        // bytes; each store completes its bytes on the peer's barrier (no round trip here)
-        const uint32_t xbar = map_peer(smem_u32(&sm.xfull[sb]), peer);
+        if (act) {
+          tc_fence_after();
+          uint32_t v[kChunk];
+          tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+          tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&sm.s_read[sb]));
+          if (q4 == 1 && lane == 0) TRACE(3, gc);
+          // the peer has read its buffer sb from chunk gc-2
+          if (!(ok = wait_cluster(smem_u32(&sm.xfree[sb]), use ^ 1u, p.status, abort_flag))) break;
+          const uint32_t dst = dst0 + (uint32_t)sb * kXBytes;
+          // [key/4][head][4 keys]: each store writes 4 keys of head r, the warp 512 contiguous
+          // bytes; each store completes its bytes on the peer's barrier (no round trip here)
+          const uint32_t xbar = map_peer(smem_u32(&sm.xfull[sb]), peer);
 #pragma unroll
-        for (int c = 0; c < kChunk; c += 4) st_async_v4(dst + c * 512, &v[c], xbar);
+          for (int c = 0; c < kChunk; c += 4) st_async_v4(dst + c * 512, &v[c], xbar);
+        } else {
+          // head rows >= H: nothing to read or send
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&sm.s_read[sb]));
+        }
         if (q4 == 1 && lane == 0) TRACE(4, gc);
         if (j + 1 == nch) break;                     // the last chunk's buffer is released below
         // once our softmax has read our buffer sb of chunk gc, the peer may refill it
@@ -740,6 +750,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
     const bool lead = g == 0 && q4 == 0 && lane == 0;
     const bool real = r < p.H;
+    const bool act = !kHalfHeads || q4 < 2;         // warp-uniform: this warp's head rows exist
     const float4* xcol = reinterpret_cast<const float4*>(gb + (sm.x - base)) + r;  // head r of [key/4][head][4]
     long long gc = 0;
     bool ok = true;
@@ -759,7 +770,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       const float l_all = p_lsum + sm.lsum[(1 - g) * 128 + r];
       tc_fence_after();
       const float inv = 1.f / l_all;
-      for (int c = 0; c < 128; c += 32) {
+      for (int c = 0; act && c < 128; c += 32) {
         uint32_t o[32];
         tmem_ld_32x32b_x32(tmem + lane_addr + kOCol + 128 * g + c, o);
         tmem_ld_wait();
@@ -811,6 +822,15 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         const int sb = (int)(gc & 1);
         const uint32_t use = (uint32_t)((gc >> 1) & 1);
         if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), use, p.status, abort_flag))) break;
+        if (!act) {
+          // head rows >= H (H = 64): keep every barrier's count, compute nothing
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&sm.xread[sb]));
+          if (lane == 0) mbar_arrive(smem_u32(&sm.mxready[sb]));
+          if (!(ok = mbar_wait(smem_u32(&sm.mxready[sb]), use, p.status, abort_flag))) break;
+          if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[sb]));
+          continue;
+        }
         tc_fence_after();
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk + 32 * g, v);
@@ -819,7 +839,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         if (!(ok = wait_cluster(smem_u32(&sm.xfull[sb]), use, p.status, abort_flag))) break;
         if (lead) {
           TRACE(6, gc);
-          mbar_arrive_expect_tx(smem_u32(&sm.xfull[sb]), kXBytes);  // arm the next use
+          mbar_arrive_expect_tx(smem_u32(&sm.xfull[sb]), 64u * p.H * 4u);  // arm the next use (H rows)
         }
         const float4* xr = xcol + sb * (kXBytes / 16) + 8 * g * 128;
         const int valid = n - j * kChunk - 32 * g;
@@ -990,7 +1010,8 @@ cudaError_t launch_attend_tc(const dsa_dims& d, const void* q, const void* k, in
   p.list_bitmap = bitmap_in_list(width, d.n_kv) ? 1 : 0;
   p.out_v8 = ((uintptr_t)out & 31u) == 0 ? 1 : 0;
   const size_t smem = smem_bytes(width, d.n_kv, p.list_bitmap != 0);
-  cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = d.heads == 64 ? attend_tc_kernel<true> : attend_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   // persistent clusters: one per SM pair (or one per row when there are fewer rows)
   const long long rows = (long long)d.batch * d.n_q;
@@ -998,7 +1019,7 @@ cudaError_t launch_attend_tc(const dsa_dims& d, const void* q, const void* k, in
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long clusters = rows < sms / 2 ? rows : sms / 2;
-  attend_tc_kernel<<<dim3((unsigned)(2 * clusters)), kThreads, smem, st>>>(mq, mkv, mrope, p);
+  kern<<<dim3((unsigned)(2 * clusters)), kThreads, smem, st>>>(mq, mkv, mrope, p);
   return cudaGetLastError();
 }
 
