@@ -302,7 +302,8 @@ def profile_once(a):
     from sparse_attention_sum_b200 import runner
     torch.cuda.set_device(0)
     dsa.lib()
-    wl = workloads.make(a.workload)
+    sizes = {k: v for k, v in (("T", a.T), ("S", a.S)) if v}
+    wl = workloads.make(a.workload, **sizes)
     t = device_inputs(wl)
     dims, args = layer_args(wl, t)
     bufs = runner.LayerBuffers(dims, "cuda", torch.bfloat16, with_idx=True)
@@ -629,6 +630,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--profile-once", action="store_true",
                     help="one call of each stage entry point, no timing (for an ncu capture)")
+    ap.add_argument("--T", type=int, default=0, help="--profile-once: queries per sequence (smaller capture)")
+    ap.add_argument("--S", type=int, default=0, help="--profile-once: keys per sequence (smaller capture)")
     a = ap.parse_args(argv)
     a.warmup = max(3, a.warmup)  # at least three untimed warm-up steps
     if a.impl == "reference":
