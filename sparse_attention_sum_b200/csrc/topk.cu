@@ -7,9 +7,12 @@
 //
 // One block per row.  Scores become order-preserving uint32 keys (signed
 // zeros merged) and are cached in shared memory when the visible range fits.
-// Four 8-bit MSB-first histogram passes (shared-memory atomics aggregated per
-// warp with match_any, a warp-wide scan of the 256 bins) find the exact k-th
-// largest key tau and how many keys equal to tau are still needed.  Each warp
+// One pass counts the top 12 bits of every key (plain shared atomics); the
+// keys of the bin that holds the k-th largest become a small candidate set
+// whose low 20 bits are resolved alone (12 + 8 bits).  That gives the exact
+// k-th largest key tau and how many keys equal to tau are still needed.  A
+// crowded bin (many equal scores) falls back to four 8-bit passes over the
+// row (shared atomics aggregated per warp with ballots).  Each warp
 // then walks a contiguous segment of the row 32 keys at a time; ballots and a
 // block-wide prefix sum place every key > tau and the lowest-index keys == tau,
 // which keeps the tie rule exact.  Finally the (key, index) pairs are put in
@@ -55,6 +58,20 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch /*>= BLO
   total = scratch[BLOCK / 32 - 1];
   __syncthreads();
   return warp_base + x - v;
+}
+
+// Lanes of the warp holding the same 8-bit digit d (0..255) as this lane, from one ballot
+// per bit (the address-divergence unit behind match.any is the bottleneck otherwise).
+// Lanes with d < 0 take no part; their own result is meaningless.
+__device__ __forceinline__ uint32_t same_digit_lanes(int d) {
+  uint32_t m = __ballot_sync(0xffffffffu, d >= 0);
+#pragma unroll
+  for (int b = 0; b < 8; ++b) {
+    const bool bit = (d >> b) & 1;
+    const uint32_t bb = __ballot_sync(0xffffffffu, bit);
+    m &= bit ? bb : ~bb;
+  }
+  return m;
 }
 
 // In a histogram of `nbins` bins (bin = a digit, counted over the keys still in play), find
@@ -108,7 +125,7 @@ __device__ void radix_sort_desc(uint64_t* a, uint64_t* b, uint32_t* hist, int* s
     for (int g = w0; g < w1; g += 32) {
       const int i = g + lane;
       const int d = i < w1 ? 255 - (int)((a[i] >> shift) & 255u) : -1;
-      const uint32_t peers = __match_any_sync(0xffffffffu, d);
+      const uint32_t peers = same_digit_lanes(d);
       if (d >= 0 && (peers & lt) == 0u) h[d] += __popc(peers);
       __syncwarp();
     }
@@ -136,7 +153,7 @@ __device__ void radix_sort_desc(uint64_t* a, uint64_t* b, uint32_t* hist, int* s
         e = a[i];
         d = 255 - (int)((e >> shift) & 255u);
       }
-      const uint32_t peers = __match_any_sync(0xffffffffu, d);
+      const uint32_t peers = same_digit_lanes(d);
       if (d >= 0) {
         b[h[d] + __popc(peers & lt)] = e;
       }
@@ -286,7 +303,7 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
           const uint32_t key = cached ? cache[i] : score_key(srow[r.lo + i]);
           if ((key & mask) == prefix) bin = (int)((key >> shift) & 255u);
         }
-        const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+        const uint32_t peers = same_digit_lanes(bin);
         if (bin >= 0 && lane0 == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
       }
       __syncthreads();
