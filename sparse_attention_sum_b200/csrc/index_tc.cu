@@ -287,6 +287,10 @@ cudaError_t launch_index_scores_tc(const dsa_dims& d, const void* q_idx, const v
   p.n_qtiles = (p.T + p.NQ - 1) / p.NQ;
   p.n_ktiles = (p.S + kKeysPerTile - 1) / kKeysPerTile;
   const int sms = sm_count();
+  // Narrow query tiles (N <= 128: decode, one query per sequence) stream many key tiles per CTA:
+  // two CTAs per SM with two key stages each hide each other's start-up and keep four tiles
+  // in flight per SM; wide tiles keep one CTA per SM with up to six stages.
+  const int ctas_per_sm = p.N <= 128 ? 2 : 1;
   // Key-range splits per query tile: one CTA per SM, so the time is about (waves) x (tiles per
   // CTA + a fixed cost of ~3 tiles for the query load and pipeline fill).  Pick the split count
   // that minimises it; a count that leaves a nearly empty last wave loses to a finer one.
@@ -296,7 +300,7 @@ cudaError_t launch_index_scores_tc(const dsa_dims& d, const void* q_idx, const v
   for (int s2 = 1; s2 <= p.n_ktiles && s2 <= 512; ++s2) {
     const int tps = (p.n_ktiles + s2 - 1) / s2;
     const int used = (p.n_ktiles + tps - 1) / tps;           // splits that get tiles
-    const long long waves = (qt * used + sms - 1) / sms;
+    const long long waves = (qt * used + (long long)sms * ctas_per_sm - 1) / ((long long)sms * ctas_per_sm);
     const long long cost = waves * (tps + 3);
     if (best < 0 || cost < best) {
       best = cost;
@@ -316,6 +320,7 @@ cudaError_t launch_index_scores_tc(const dsa_dims& d, const void* q_idx, const v
   const size_t fixed = 1024 + (size_t)p.N * 256 + (size_t)p.N * 4 + 2 * 16 * 4 + 64 + 8 * (2 * kMaxStages + 8) + 64;
   int stages = (int)((220 * 1024 - fixed) / kTileBytes);
   if (stages > kMaxStages) stages = kMaxStages;
+  if (ctas_per_sm == 2 && stages > 2) stages = 2;
   if (stages < 2) return cudaErrorInvalidConfiguration;
   p.stages = stages;
   const size_t smem = fixed + (size_t)stages * kTileBytes;
