@@ -73,7 +73,8 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.z;
-  const int qt = blockIdx.y;
+  // later query tiles see more keys (causal): launch them first so the last wave is the cheap one
+  const int qt = (int)gridDim.y - 1 - (int)blockIdx.y;
   const int t0 = qt * p.NQ;
   const int nq_here = min(p.NQ, p.T - t0);
   const int kt_begin = blockIdx.x * p.tiles_per_split;

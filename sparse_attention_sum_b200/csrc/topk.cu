@@ -186,7 +186,8 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
   __shared__ uint32_t s_prefix, s_krem, s_bin;
   __shared__ int s_ncand;
 
-  const int b = blockIdx.y, t = blockIdx.x;
+  // later rows see more keys (causal): launch them first so the last wave is the cheap one
+  const int b = blockIdx.y, t = (int)gridDim.x - 1 - (int)blockIdx.x;
   const size_t row = (size_t)b * d.n_q + t;
   const float* srow = scores + row * d.n_kv;
   int32_t* orow = idx_out + row * k;
