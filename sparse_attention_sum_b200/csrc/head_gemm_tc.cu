@@ -13,8 +13,9 @@
 // once and reuses it for every row tile of that head.  Warp 0 streams A tiles
 // (64 columns, 16 KB) by TMA through a 4-stage ring; warp 1 issues
 // tcgen05.mma (M=128, N=NT<=256, K=16) into one of two TMEM accumulators;
-// warps 2-5 drain the other accumulator to bf16 rows in global memory, so the
-// epilogue of one tile overlaps the MMAs of the next.  Every wait is bounded.
+// warps 2-5 drain the other accumulator through swizzled shared-memory boxes
+// that TMA stores to global memory, so the epilogue of one tile overlaps the
+// MMAs of the next.  Every wait is bounded.
 #include <cuda.h>
 
 #include "dsa_common.cuh"
@@ -30,6 +31,19 @@ constexpr int kHgThreads = 192;
 constexpr int kHgStages = 4;
 constexpr int kHgABytes = 128 * 128;  // one A box: 128 rows x 64 bf16
 constexpr int kHgMaxBBytes = 128 * 1024;
+constexpr int kHgOutBox = 32 * 128;   // one output staging box: 32 rows x 64 bf16 (128-byte swizzle)
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"((uint64_t)map),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until at most N committed bulk groups of this thread still read their shared memory
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
 
 struct HgParams {
   int n_rows, H, K, N, NT;
@@ -40,7 +54,7 @@ struct HgParams {
 
 __global__ void __launch_bounds__(kHgThreads, 1)
 head_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                    HgParams p) {
+                    const __grid_constant__ CUtensorMap map_c, HgParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t a_full[kHgStages], a_empty[kHgStages], b_full, b_free, d_full[2], d_empty[2];
   __shared__ uint32_t tmem_slot;
@@ -49,6 +63,7 @@ head_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t sB = base;                          // B of the current head
   const uint32_t sA = base + kHgMaxBBytes;           // A ring
+  const uint32_t sO = sA + kHgStages * kHgABytes;    // output staging: 4 warps x 2 boxes
   const int RT = (p.n_rows + 127) / 128, NTILES = p.N / p.NT;
   const long long total = (long long)p.H * RT * NTILES;
   const long long per = (total + gridDim.x - 1) / gridDim.x;
@@ -162,10 +177,14 @@ head_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue: TMEM -> bf16 rows
+    // ------------------------------------------------------------ epilogue: TMEM -> bf16 -> TMA store
+    // Each warp converts its 32 rows, 64 columns at a time, into a 128-byte-swizzled staging box
+    // and one lane stores the box by TMA (rows past n_rows are clipped by the store).
     const int q4 = warp & 3;                          // TMEM lane quarter of this warp
     const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
+    const uint32_t stage0 = sO + (uint32_t)(q4 * 2 * kHgOutBox);
     long long nd = 0;
+    int nbox = 0;
     for (long long it = i0; it < i1; ++it, ++nd) {
       const int h = (int)(it / ((long long)RT * NTILES));
       const int rt = (int)((it / NTILES) % RT);
@@ -173,33 +192,41 @@ head_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
       const int d = (int)(nd & 1);
       if (!mbar_wait(smem_u32(&d_full[d]), (uint32_t)((nd >> 1) & 1), p.status, abort_flag)) break;
       tc_fence_after();
-      const int r = rt * 128 + q4 * 32 + lane;
-      bf16* crow = p.C + ((size_t)r * p.H + h) * p.N + nt * p.NT;
-      for (int c = 0; c < p.NT; c += 32) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + lane_addr + (uint32_t)(d * p.NT + c), v);
+      for (int c = 0; c < p.NT; c += 64, ++nbox) {
+        uint32_t v[64];
+        tmem_ld_32x32b_x32(tmem + lane_addr + (uint32_t)(d * p.NT + c), *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld_32x32b_x32(tmem + lane_addr + (uint32_t)(d * p.NT + c + 32), *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
         tmem_ld_wait();
-        if (r < p.n_rows) {
-          uint4* dst = reinterpret_cast<uint4*>(crow + c);
+        const uint32_t box = stage0 + (uint32_t)((nbox & 1) * kHgOutBox);
+        // the store issued from this buffer two boxes ago has read it
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint4 pk;
-            __nv_bfloat162 b0 = __floats2bfloat162_rn(__uint_as_float(v[8 * i]), __uint_as_float(v[8 * i + 1]));
-            __nv_bfloat162 b1 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
-            __nv_bfloat162 b3 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
-            pk.x = *reinterpret_cast<uint32_t*>(&b0);
-            pk.y = *reinterpret_cast<uint32_t*>(&b1);
-            pk.z = *reinterpret_cast<uint32_t*>(&b2);
-            pk.w = *reinterpret_cast<uint32_t*>(&b3);
-            dst[i] = pk;
+        for (int k = 0; k < 8; ++k) {                  // 16-byte chunk k of this row, swizzled by row
+          uint32_t w4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[8 * k + 2 * e]), __uint_as_float(v[8 * k + 2 * e + 1]));
+            w4[e] = *reinterpret_cast<uint32_t*>(&b2);
           }
+          const uint32_t a = box + (uint32_t)(lane * 128) + (uint32_t)(((k ^ (lane & 7)) & 7) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(w4[0]), "r"(w4[1]), "r"(w4[2]),
+                       "r"(w4[3])
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int y = rt * 128 + q4 * 32;
+          if (y < p.n_rows) tma_store_2d(&map_c, box, h * p.N + nt * p.NT + c, y);  // a partial box is clipped
+          bulk_commit();
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&d_empty[d]));
     }
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");  // stores complete before exit
   }
   tc_fence_before();
   __syncthreads();
@@ -277,16 +304,25 @@ cudaError_t launch_head_gemm_tc(int n_rows, int heads, int K, int N, const void*
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
+  // C viewed as [n_rows, H*N]; box = 64 columns x 32 rows (one epilogue warp's rows), 128-byte swizzle
+  CUtensorMap mc;
+  cuuint64_t cdims[2] = {(cuuint64_t)heads * N, (cuuint64_t)n_rows};
+  cuuint64_t cstr[1] = {(cuuint64_t)heads * N * 2};
+  cuuint32_t cbox[2] = {64u, 32u};
+  if (enc(&mc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, cdims, cstr, cbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+      CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   HgParams p{n_rows, heads, K, N, NT, b_kn, (bf16*)C, device_status_ptr()};
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long items = (long long)heads * ((n_rows + 127) / 128) * (N / NT);
   const int grid = (int)(items < sms ? items : sms);
-  const size_t smem = 1024 + kHgMaxBBytes + (size_t)kHgStages * kHgABytes;
+  const size_t smem = 1024 + kHgMaxBBytes + (size_t)kHgStages * kHgABytes + 4 * 2 * kHgOutBox;
   cudaError_t e = cudaFuncSetAttribute(head_gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  head_gemm_tc_kernel<<<grid, kHgThreads, smem, st>>>(ma, mb, p);
+  head_gemm_tc_kernel<<<grid, kHgThreads, smem, st>>>(ma, mb, mc, p);
   return cudaGetLastError();
 }
 
