@@ -18,7 +18,6 @@
 namespace dsa {
 
 constexpr int kPoolMaxC = 8;  // D_I <= 256
-constexpr int kPoolMaxSlots = 16;
 
 template <typename T>
 __global__ void pool_states_kernel(dsa_dims d, const T* __restrict__ k, const T* __restrict__ gate,

@@ -339,7 +339,7 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
   gt_base = __shfl_sync(0xffffffffu, gt_base, 0);
   eq_base = __shfl_sync(0xffffffffu, eq_base, 0);
   const uint32_t lt_mask = (1u << lane) - 1u;
-  if (!RANKED) {
+  if constexpr (!RANKED) {
     // ascending key order: key i goes to (#gt before i) + min(#eq before i, need_eq)
     for (int b0 = w0; b0 < w1; b0 += 32) {
       const int i = b0 + lane;
@@ -359,33 +359,33 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
       gt_base += __popc(m_gt);
       eq_base += __popc(m_eq);
     }
-    return;
-  }
-  for (int b0 = w0; b0 < w1; b0 += 32) {
-    const int i = b0 + lane;
-    uint32_t key = 0u;
-    if (i < w1) key = cached ? cache[i] : score_key(srow[r.lo + i]);
-    const bool is_gt = i < w1 && key > tau;
-    const bool is_eq = i < w1 && key == tau;
-    const uint32_t m_gt = __ballot_sync(0xffffffffu, is_gt);
-    const uint32_t m_eq = __ballot_sync(0xffffffffu, is_eq);
-    const uint64_t c = ((uint64_t)key << 32) | (uint32_t)(r.lo + i);
-    if (is_gt) sel[gt_base + __popc(m_gt & lt_mask)] = c;
-    if (is_eq) {
-      int rank = eq_base + __popc(m_eq & lt_mask);
-      if (rank < need_eq) sel[n_gt + rank] = c;
+  } else {
+    for (int b0 = w0; b0 < w1; b0 += 32) {
+      const int i = b0 + lane;
+      uint32_t key = 0u;
+      if (i < w1) key = cached ? cache[i] : score_key(srow[r.lo + i]);
+      const bool is_gt = i < w1 && key > tau;
+      const bool is_eq = i < w1 && key == tau;
+      const uint32_t m_gt = __ballot_sync(0xffffffffu, is_gt);
+      const uint32_t m_eq = __ballot_sync(0xffffffffu, is_eq);
+      const uint64_t c = ((uint64_t)key << 32) | (uint32_t)(r.lo + i);
+      if (is_gt) sel[gt_base + __popc(m_gt & lt_mask)] = c;
+      if (is_eq) {
+        int rank = eq_base + __popc(m_eq & lt_mask);
+        if (rank < need_eq) sel[n_gt + rank] = c;
+      }
+      gt_base += __popc(m_gt);
+      eq_base += __popc(m_eq);
     }
-    gt_base += __popc(m_gt);
-    eq_base += __popc(m_eq);
-  }
-  __syncthreads();
-  // gt keys came first in index order, then the taken tau keys in index order:
-  // the stable sort keeps every run of equal keys in ascending index order
-  radix_sort_desc<BLOCK>(sel, tmp, rhist, scan, k);
-  for (int i = threadIdx.x; i < k; i += BLOCK) {
-    const uint64_t c = sel[i];
-    orow[i] = (int32_t)(uint32_t)c;
-    if (vrow) vrow[i] = key_score((uint32_t)(c >> 32));
+    __syncthreads();
+    // gt keys came first in index order, then the taken tau keys in index order:
+    // the stable sort keeps every run of equal keys in ascending index order
+    radix_sort_desc<BLOCK>(sel, tmp, rhist, scan, k);
+    for (int i = threadIdx.x; i < k; i += BLOCK) {
+      const uint64_t c = sel[i];
+      orow[i] = (int32_t)(uint32_t)c;
+      if (vrow) vrow[i] = key_score((uint32_t)(c >> 32));
+    }
   }
 }
 
