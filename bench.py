@@ -368,13 +368,14 @@ def run_ours(a):
         line["stages_qtok_s"] = {k: round(rows / v, 1) for k, v in st.items()}
         line["fused_tensor_frac"] = round((wk["index_flop"] + wk["attend_flop"]) / step_med / 1e12
                                           / peaks["bf16_tflops"], 4)
-        traffic = profiled_traffic().get(f"attend:{wl.name}")
+        tr = profiled_traffic()
+        traffic = tr.get(f"attend:{wl.name}")
         line["roofline"] = roofline_entry("tensor", wk["attend_flop"], st["attend"], peaks, traffic)
         line["roofline"]["kernel"] = "sparse attend (dsa_sparse_attend)"
         line["roofline_stages"] = {
-            "index": roofline_entry("tensor", wk["index_flop"], st["index"], peaks),
-            "topk": roofline_entry("hbm", wk["topk_bytes"], st["topk"], peaks),
-            "attend": roofline_entry("tensor", wk["attend_flop"], st["attend"], peaks),
+            "index": roofline_entry("tensor", wk["index_flop"], st["index"], peaks, tr.get(f"index:{wl.name}")),
+            "topk": roofline_entry("hbm", wk["topk_bytes"], st["topk"], peaks, tr.get(f"topk:{wl.name}")),
+            "attend": roofline_entry("tensor", wk["attend_flop"], st["attend"], peaks, traffic),
         }
         line["e2e"] = e2e_measure(wl, a.steps, stream)
         if a.workload == "prefill":
@@ -464,7 +465,8 @@ def decode_extra(peaks, flush, stream):
            "value": round(rows / step, 1), "unit": UNIT, "ms_per_step": round(step * 1e3, 4),
            "stages_us": {k: round(v * 1e6, 1) for k, v in st.items()},
            "roofline_attend": roofline_entry("hbm", wk["attend_bytes"], st["attend"], peaks),
-           "roofline_index": roofline_entry("hbm", wk["index_bytes"], st["index"], peaks),
+           "roofline_index": roofline_entry("hbm", wk["index_bytes"], st["index"], peaks,
+                                            profiled_traffic().get("index:decode")),
            "fused_hbm_frac": round((wk["index_bytes"] + wk["topk_bytes"] + wk["attend_bytes"]) / step / 1e9
                                    / peaks["hbm_gbs"], 4)}
     del t, bufs
