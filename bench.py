@@ -377,6 +377,16 @@ def run_ours(a):
             "topk": roofline_entry("hbm", wk["topk_bytes"], st["topk"], peaks, tr.get(f"topk:{wl.name}")),
             "attend": roofline_entry("tensor", wk["attend_flop"], st["attend"], peaks, traffic),
         }
+        # IndexShare: a layer that reuses an earlier layer's selection runs only the attend.  On the
+        # 78-layer stack the pages describe, layers 0, 1 and every il % 4 == 2 compute their own (21 of 78).
+        shared = time_steps(lambda: runner.dsa_layer(dims, **args, bufs=bufs, idx_in=bufs.idx), max(3, a.steps // 2),
+                            3, flush, stream)
+        full_ms, shared_ms = statistics.median(times) * 1e3, statistics.median(shared) * 1e3
+        n_full = sum(1 for il in range(78) if il <= 1 or il % 4 == 2)
+        stack_ms = (n_full * full_ms + (78 - n_full) * shared_ms) / 78
+        line["indexshare"] = {"shared_layer_ms": round(shared_ms, 4), "full_layer_ms": round(full_ms, 4),
+                              "layers_full_of_78": n_full, "stack_avg_layer_ms": round(stack_ms, 4),
+                              "stack_avg_value": round(rows / (stack_ms / 1e3), 1), "unit": UNIT}
         line["e2e"] = e2e_measure(wl, a.steps, stream)
         if a.workload == "prefill":
             line["decode"] = decode_extra(peaks, flush, stream)
