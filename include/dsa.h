@@ -173,8 +173,9 @@ dsa_status dsa_topk_set(const dsa_dims* dims, const float* scores, const int32_t
  * Reads dims: batch, n_q, n_kv, heads, kv_heads, kd, vd, dtype.
  * q [B,T,H,kd] dtype   idx [B,T,width] int32   out [B,T,H,vd] dtype
  * lse [B,T,H] fp32 or NULL.  Softmax and accumulation are fp32.
- * bf16 with kv_heads = 1, kd in {512, 576}, vd = 512, H a multiple of 64 runs on
- * the tensor cores; other shapes run on the CUDA cores. */
+ * bf16 with kv_heads = 1 (V = the first vd columns of the K rows, same pointer and
+ * stride), kd in {512, 576}, vd = 512, H in {64, 128}, n_kv <= 65536 and width up
+ * to about 3400 runs on the tensor cores; other shapes run on the CUDA cores. */
 dsa_status dsa_sparse_attend(const dsa_dims* dims, const void* q, const void* k,
                              int64_t k_row_stride, const void* v, int64_t v_row_stride,
                              const int32_t* idx, int32_t width, float scale, void* out,

@@ -938,7 +938,8 @@ bool attend_tc_supported(const dsa_dims& d, int64_t k_stride, const void* k, con
   if ((long long)d.batch * d.n_q * d.heads < 128) return false;  // the query TMA box is 128 rows
   if (k != v || k_stride != v_stride || k_stride < d.kd || (k_stride * 2) % 16 != 0) return false;
   if (((uintptr_t)k & 15u) != 0) return false;
-  if (d.n_kv > kBitmapKeys || width > 8192) return false;  // bitmap + raw row fit in the (idle) gather stages
+  if (d.n_kv > kBitmapKeys) return false;                  // 16-bit key list
+  if (width > 8192) return false;
   if (smem_bytes(width, d.n_kv, false) > 227 * 1024) return false;
   return encode_fn() != nullptr;
 }
