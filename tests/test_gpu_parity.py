@@ -444,6 +444,45 @@ def test_full_size_layer_sampled_rows(name):
     assert torch.equal(key_order(ranked), sel)
 
 
+def test_ragged_batch_with_a_fully_padded_sequence():
+    # three causal sequences in one batch on the tensor-core path: no padding, 37 left-padded keys with a
+    # shorter cache, and one whose queries all precede its first valid key (every row selects nothing)
+    T, top_k = 300, 96
+    parts = [workloads.make("prefill", seed=21 + b, T=T) for b in range(3)]
+    wl = parts[0]
+    wl.tensors = {k: torch.cat([w.tensors[k] for w in parts], 0) for k in parts[0].tensors}
+    wl.batch, wl.top_k = 3, top_k
+    wl.tensors["kv_start"] = torch.tensor([0, 37, T + 5], dtype=torch.int32)
+    wl.tensors["kv_len"] = torch.tensor([T, T - 50, T], dtype=torch.int32)
+    t = dev(wl)
+    dims, a = layer_inputs(wl, t)
+    bufs = runner.LayerBuffers(dims, "cuda", torch.bfloat16, with_idx=True, with_lse=True)
+    runner.dsa_layer(dims, **a, bufs=bufs)
+    torch.cuda.synchronize()
+    scores = bufs.ws[: 3 * T * T * 4].view(torch.float32).view(3, T, T)
+    g_idx, g_out, g_lse = bufs.idx.cpu().numpy(), _np(bufs.out), bufs.lse.cpu().numpy()
+    K, V = kv_views(wl)
+    # the fully padded sequence: no selection, zero output, lse = -inf
+    assert np.all(g_idx[2] == O.INVALID) and np.all(g_out[2] == 0) and np.all(np.isneginf(g_lse[2]))
+    rows = [(0, 0), (0, top_k - 1), (0, top_k), (0, T - 1), (1, 0), (1, 36), (1, 37), (1, 38), (1, 37 + top_k),
+            (1, T - 51), (1, T - 50), (1, T - 1)]
+    for b, tt in rows:
+        p, ks, kl = int(wl["q_pos"][b, tt]), int(wl["kv_start"][b]), int(wl["kv_len"][b])
+        cand = O.visible_keys(p, ks, kl)
+        if len(cand) == 0:
+            assert np.all(g_idx[b, tt] == O.INVALID) and np.all(g_out[b, tt] == 0), (b, tt)
+            assert np.all(np.isneginf(g_lse[b, tt])), (b, tt)
+            continue
+        gs = scores[b, tt].cpu().numpy().astype(np.float64)[cand]
+        ref = O.index_scores_row(wl["q_idx"][b, tt], wl["k_idx"][b][cand], wl["w"][b, tt], wl.idx_scale)
+        assert np.abs(gs - ref).max() <= 2e-5 * max(1.0, np.abs(ref).max()), (b, tt)
+        assert g_idx[b, tt].tolist() == key_order(O.topk_row(cand, gs, top_k).tolist()), (b, tt)
+        check_selection_in_band(g_idx[b, tt], cand, ref, top_k, f"ragged {(b, tt)}")
+        ro, rl = O.sparse_attend_row(wl["q"][b, tt], K[b], V[b], g_idx[b, tt], wl.attn_scale)
+        assert_attend_close(g_out[b, tt], ro, torch.bfloat16, f"ragged out {(b, tt)}")
+        np.testing.assert_allclose(g_lse[b, tt], rl, atol=2e-3)
+
+
 def test_full_size_kpool_sampled_rows():
     wl = workloads.make("kpool")
     bufs = _kpool_run(wl)
