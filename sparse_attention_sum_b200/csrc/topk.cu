@@ -169,7 +169,7 @@ __device__ void radix_sort_desc(uint64_t* a, uint64_t* b, uint32_t* hist, int* s
 }
 
 template <int BLOCK, bool RANKED>
-__global__ void __launch_bounds__(BLOCK)
+__global__ void __launch_bounds__(BLOCK, BLOCK >= 1024 ? 1 : 3)
 topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restrict__ q_pos,
             const int32_t* __restrict__ kv_start, const int32_t* __restrict__ kv_len, int k,
             int cache_cap, int32_t* __restrict__ idx_out, float* __restrict__ vals_out) {
@@ -181,10 +181,12 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
   uint32_t* hist = rhist + (RANKED ? (BLOCK / 32) * 256 : 0);        // [256]
   int* scan = reinterpret_cast<int*>(hist + 256);                    // [64]
   uint32_t* hist12 = reinterpret_cast<uint32_t*>(scan + 64);         // [kHist12]
-  uint32_t* cand = hist12 + kHist12;                                 // [kCand]
-  uint32_t* cache = cand + kCand;                                    // [cache_cap]
+  uint32_t* cand = hist12 + kHist12;                                 // [kCand] candidate keys
+  uint8_t* candw = reinterpret_cast<uint8_t*>(cand + kCand);         // [kCand] their warps
+  uint32_t* cache = reinterpret_cast<uint32_t*>(candw + kCand);      // [cache_cap]
   __shared__ uint32_t s_prefix, s_krem, s_bin;
   __shared__ int s_ncand;
+  __shared__ int s_cgt[BLOCK / 32], s_ceq[BLOCK / 32];
 
   // later rows see more keys (causal): launch them first so the last wave is the cheap one
   const int b = blockIdx.y, t = (int)gridDim.x - 1 - (int)blockIdx.x;
@@ -253,23 +255,42 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
   find_crossing<BLOCK>(hist12, kHist12, (uint32_t)k, scan, &s_bin, &s_krem);
   const uint32_t b1 = s_bin, krem1 = s_krem;
   const uint32_t nb1 = hist12[b1];
+  // each warp owns a contiguous segment of the row, walked 32 keys at a time (the output order
+  // of equal keys is their index order)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int NW = BLOCK / 32;
+  const int wseg = ((n + NW - 1) / NW + 31) & ~31;
+  const int w0 = warp * wseg;
+  const int w1 = min(n, w0 + wseg);
+  const bool few = nb1 <= (uint32_t)kCand;
+  int gt12 = 0;                                       // keys of this warp whose top 12 bits exceed b1
   uint32_t prefix = 0u;
-  if (nb1 <= (uint32_t)kCand) {
-    // collect the bin's keys (any order: only their values matter here)
-    for (int base = (threadIdx.x & ~31); base < n; base += BLOCK) {
-      const int i = base + lane0;
+  if (few) {
+    // collect the bin's keys with their warp, and count the keys above the bin per warp
+    if (threadIdx.x < NW) {
+      s_cgt[threadIdx.x] = 0;
+      s_ceq[threadIdx.x] = 0;
+    }
+    for (int b0 = w0; b0 < w1; b0 += 32) {
+      const int i = b0 + lane;
       uint32_t key = 0u;
       bool in = false;
-      if (i < n) {
+      if (i < w1) {
         key = cached ? cache[i] : score_key(srow[r.lo + i]);
         in = (key >> 20) == b1;
+        gt12 += (key >> 20) > b1;
       }
       const uint32_t m = __ballot_sync(0xffffffffu, in);
       int slot = 0;
-      if (lane0 == 0 && m) slot = atomicAdd(&s_ncand, __popc(m));
+      if (lane == 0 && m) slot = atomicAdd(&s_ncand, __popc(m));
       slot = __shfl_sync(0xffffffffu, slot, 0);
-      if (in) cand[slot + __popc(m & ((1u << lane0) - 1u))] = key;
+      if (in) {
+        const int c = slot + __popc(m & ((1u << lane) - 1u));
+        cand[c] = key;
+        candw[c] = (uint8_t)warp;
+      }
     }
+    gt12 = __reduce_add_sync(0xffffffffu, gt12);
     __syncthreads();
     // bits 19..8 of the candidates
     for (int i = threadIdx.x; i < kHist12; i += BLOCK) hist12[i] = 0u;
@@ -286,6 +307,12 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
     __syncthreads();
     find_crossing<BLOCK>(hist, 256, krem2, scan, &s_bin, &s_krem);
     prefix = (b1 << 20) | (b2 << 8) | s_bin;
+    // per warp: the bin's keys above and equal to tau
+    for (int c = threadIdx.x; c < (int)nb1; c += BLOCK) {
+      if (cand[c] > prefix) atomicAdd(&s_cgt[candw[c]], 1);
+      else if (cand[c] == prefix) atomicAdd(&s_ceq[candw[c]], 1);
+    }
+    __syncthreads();
   } else {
     // a crowded bin (e.g. many equal scores): 8-bit digits over the whole row
     if (threadIdx.x == 0) {
@@ -318,21 +345,21 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
   const int need_eq = (int)s_krem;  // keys equal to tau still to take (lowest indices first)
   const int n_gt = k - need_eq;
 
-  // ---- gather: each warp owns a contiguous segment, walked 32 keys at a time,
-  // so the output order of equal keys is their index order.
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  constexpr int NW = BLOCK / 32;
-  const int wseg = ((n + NW - 1) / NW + 31) & ~31;
-  const int w0 = warp * wseg;
-  const int w1 = min(n, w0 + wseg);
+  // ---- gather: per-warp counts of keys > tau and == tau (from the collection pass, or one
+  // more pass over a crowded row), then every warp places its keys
   int c_gt = 0, c_eq = 0;
-  for (int i = w0 + lane; i < w1; i += 32) {
-    uint32_t key = cached ? cache[i] : score_key(srow[r.lo + i]);
-    c_gt += key > tau;
-    c_eq += key == tau;
+  if (few) {
+    c_gt = gt12 + s_cgt[warp];
+    c_eq = s_ceq[warp];
+  } else {
+    for (int i = w0 + lane; i < w1; i += 32) {
+      uint32_t key = cached ? cache[i] : score_key(srow[r.lo + i]);
+      c_gt += key > tau;
+      c_eq += key == tau;
+    }
+    c_gt = __reduce_add_sync(0xffffffffu, c_gt);
+    c_eq = __reduce_add_sync(0xffffffffu, c_eq);
   }
-  c_gt = __reduce_add_sync(0xffffffffu, c_gt);
-  c_eq = __reduce_add_sync(0xffffffffu, c_eq);
   int tot;
   int gt_base = block_exclusive_scan<BLOCK>(lane == 0 ? c_gt : 0, scan, tot);
   int eq_base = block_exclusive_scan<BLOCK>(lane == 0 ? c_eq : 0, scan, tot);
@@ -395,7 +422,7 @@ cudaError_t launch_topk_t(const dsa_dims& d, const float* scores, const int32_t*
                           const int32_t* kv_len, int k, int32_t* idx, float* vals, cudaStream_t st) {
   int cache_cap = d.n_kv < kTopkCacheMax ? d.n_kv : kTopkCacheMax;
   const size_t fixed = (RANKED ? (size_t)k * 16 + (size_t)(BLOCK / 32) * 256 * 4 : 0) + 256 * 4 + 64 * 4 +
-                       (size_t)(kHist12 + kCand) * 4;
+                       (size_t)(kHist12 + kCand) * 4 + kCand;
   if (fixed + (size_t)cache_cap * 4 > 220 * 1024) cache_cap = (int)((220 * 1024 - fixed) / 4);
   const size_t smem = fixed + (size_t)cache_cap * 4;
   auto kern = topk_kernel<BLOCK, RANKED>;
