@@ -502,3 +502,81 @@ def absorb_out(o_lat_rows, w_uv) -> np.ndarray:
     o = f64(o_lat_rows)
     uv = f64(w_uv)
     return np.einsum("nhl,hdl->nhd", o, uv)
+
+
+# ---------------------------------------------------------------------------
+# S9: indexer query / key preparation (RoPE, Walsh-Hadamard rotation)
+# ---------------------------------------------------------------------------
+def rope_neox(x, pos: int, n_rope: int, theta: float) -> np.ndarray:
+    """NEOX rotary embedding of the first ``n_rope`` values of ``x`` (last axis).
+
+    [ik-2063] PR #2045 "What it does": the rope part of the indexer query and
+    key gets NEOX RoPE; the K-shift commit adds that GLM-DSA has no RoPE
+    scaling (no extension, attention factor 1, frequency scale 1), so the
+    rotation is the plain one and rotations compose.  NEOX pairs value ``i``
+    with value ``i + n_rope/2`` (the halves, not neighbours) and turns pair ``i``
+    by the angle ``pos * theta**(-2i/n_rope)``.  READING: ``theta`` (the RoPE
+    base) is not on the pages; it is an argument.  Values past ``n_rope`` are
+    returned unchanged.
+    """
+    x = f64(x).copy()
+    if n_rope % 2:
+        raise ValueError("n_rope must be even")
+    half = n_rope // 2
+    for i in range(half):
+        ang = float(pos) * float(theta) ** (-2.0 * i / n_rope)
+        c, s = math.cos(ang), math.sin(ang)
+        a = x[..., i].copy()
+        b = x[..., i + half].copy()
+        x[..., i] = a * c - b * s
+        x[..., i + half] = b * c + a * s
+    return x
+
+
+def sylvester_hadamard(n: int) -> np.ndarray:
+    """The Sylvester Hadamard matrix of order ``n`` (a power of two):
+    ``H_1 = [1]``, ``H_2m = [[H_m, H_m], [H_m, -H_m]]`` ([ik-2063] K-shift commit:
+    the indexer's Hadamard input is filled with the Sylvester construction)."""
+    if n < 1 or n & (n - 1):
+        raise ValueError("Hadamard order must be a power of two")
+    h = np.ones((1, 1))
+    while h.shape[0] < n:
+        h = np.block([[h, h], [h, -h]])
+    return h
+
+
+def hadamard_rotate(x) -> np.ndarray:
+    """``H x / sqrt(D)`` along the last axis: the orthonormal Walsh-Hadamard rotation
+    ([ik-2063] decode-cache commit: indexer q and k are rotated, which leaves every
+    q.k unchanged and helps the precision of the cached keys)."""
+    x = f64(x)
+    D = x.shape[-1]
+    return x @ sylvester_hadamard(D).T / math.sqrt(D)
+
+
+def index_rotate(x, pos, n_rope: int, theta: float, ln_w=None, ln_b=None, eps: float = 1e-6,
+                 layer_norm_first: bool = False, hadamard: bool = True) -> np.ndarray:
+    """Prepare indexer queries (``[n, H_I, D]``) or keys (``[n, 1, D]``) for the score.
+
+    [ik-2063] PR #2045 "What it does": indexer_q is split into a rope part and a
+    nope part, the rope part gets NEOX RoPE, and the two are concatenated;
+    indexer_k is LayerNorm-ed (with bias) and then treated the same way.  The
+    decode-cache commit rotates both by the Walsh-Hadamard matrix before the
+    key is cached, and the K-shift commit states the cached key as
+    ``H * concat(RoPE(k_pe, pos), k_nope)``.  READING: the rope part is the first
+    ``n_rope`` values ("split rope(64)/nope(64)", and the rope part comes first
+    in the cached concat), so split and concat leave the layout unchanged; the
+    rotation is the orthonormal ``H / sqrt(D)``.  ``pos[r]`` is row r's absolute
+    position.
+    """
+    x = f64(x)
+    out = np.empty_like(x)
+    for r in range(x.shape[0]):
+        y = x[r]
+        if layer_norm_first:
+            y = layer_norm(y, ln_w, ln_b, eps)
+        y = rope_neox(y, int(pos[r]), n_rope, theta)
+        if hadamard:
+            y = hadamard_rotate(y)
+        out[r] = y
+    return out

@@ -318,6 +318,102 @@ def test_layer_norm_matches_torch_and_moments():
         O.layer_norm(x, w, b, 0.0)
 
 
+# ------------------------------------- P13 indexer query/key preparation
+def test_rope_neox_pairs_halves_with_closed_form_angles():
+    """NEOX RoPE pairs value i with value i + n_rope/2 and turns pair i by
+    pos * theta^(-2i/n_rope).  n_rope = 4, theta = 10000, pos = 3: a unit vector
+    on value 0 turns by 3 rad into values 0 and 2, one on value 1 by 3/100 rad
+    into values 1 and 3, and value 4 (past n_rope) stays put."""
+    e = np.eye(5)
+    y = O.rope_neox(e, 3, 4, 10000.0)
+    np.testing.assert_allclose(y[0], [math.cos(3), 0, math.sin(3), 0, 0], atol=1e-15)
+    np.testing.assert_allclose(y[1], [0, math.cos(0.03), 0, math.sin(0.03), 0], atol=1e-15)
+    np.testing.assert_allclose(y[2], [-math.sin(3), 0, math.cos(3), 0, 0], atol=1e-15)
+    np.testing.assert_allclose(y[3], [0, -math.sin(0.03), 0, math.cos(0.03), 0], atol=1e-15)
+    np.testing.assert_array_equal(y[4], [0, 0, 0, 0, 1])
+    np.testing.assert_array_equal(O.rope_neox(e, 0, 4, 10000.0), e)
+
+
+def test_rope_scores_depend_on_relative_position_only():
+    """<RoPE(q, m), RoPE(k, n)> = <RoPE(q, m - n), k>, and norms are kept."""
+    rng = np.random.default_rng(13)
+    q, k = rng.standard_normal(128), rng.standard_normal(128)
+    for m, n in ((5, 2), (1000, 997), (37, 40), (32767, 0)):
+        lhs = O.rope_neox(q, m, 64, 10000.0) @ O.rope_neox(k, n, 64, 10000.0)
+        rhs = O.rope_neox(q, m - n, 64, 10000.0) @ k
+        assert abs(lhs - rhs) < 1e-9
+    assert abs(np.linalg.norm(O.rope_neox(q, 777, 64, 10000.0)) - np.linalg.norm(q)) < 1e-12
+
+
+def test_sylvester_hadamard_matches_scipy_and_is_orthonormal():
+    """The Sylvester construction equals scipy's Hadamard matrix, has entries
+    (-1)^popcount(i & j), and H/sqrt(D) keeps norms and every dot product
+    (ik_llama.cpp #2045: the rotation leaves q.k unchanged)."""
+    for D in (1, 2, 4, 32, 64, 128):
+        H = O.sylvester_hadamard(D)
+        assert np.array_equal(H, scipy.linalg.hadamard(D))
+        assert np.array_equal(H @ H.T, D * np.eye(D))
+    H = O.sylvester_hadamard(128)
+    i, j = np.meshgrid(np.arange(128), np.arange(128), indexing="ij")
+    parity = np.vectorize(lambda v: bin(v).count("1") & 1)(i & j)
+    assert np.array_equal(H, 1 - 2 * parity)
+    rng = np.random.default_rng(14)
+    x, y = rng.standard_normal((2, 128))
+    hx, hy = O.hadamard_rotate(x), O.hadamard_rotate(y)
+    assert abs(hx @ hy - x @ y) < 1e-12 and abs(np.linalg.norm(hx) - np.linalg.norm(x)) < 1e-12
+    with pytest.raises(ValueError):
+        O.sylvester_hadamard(48)
+
+
+def _rot_inputs(seed=15):
+    rng = np.random.default_rng(seed)
+    xk = rng.standard_normal((3, 1, 128)) * 2 + 0.5
+    xq = rng.standard_normal((3, 4, 128))
+    ln_w = 1 + 0.1 * rng.standard_normal(128)
+    ln_b = 0.1 * rng.standard_normal(128)
+    pos = np.array([5, 100, 4000])
+    return xk, xq, ln_w, ln_b, pos
+
+
+def test_cached_key_moves_by_unrotate_rope_delta_rerotate():
+    """ik_llama.cpp #2063 (K-shift commit): the cached key is
+    H*concat(RoPE(k_pe, p), k_nope); moving it to position p + d is un-Hadamard
+    (H orthonormal and symmetric), a RoPE by d of the pe part, and re-Hadamard."""
+    xk, _, ln_w, ln_b, pos = _rot_inputs()
+    d = 37
+    cached = O.index_rotate(xk, pos, 64, 10000.0, ln_w, ln_b, 1e-6, layer_norm_first=True)
+    Hn = O.sylvester_hadamard(128) / math.sqrt(128)
+    moved = np.stack([O.rope_neox(cached[r] @ Hn, d, 64, 10000.0) @ Hn for r in range(3)])
+    direct = O.index_rotate(xk, pos + d, 64, 10000.0, ln_w, ln_b, 1e-6, layer_norm_first=True)
+    np.testing.assert_allclose(moved, direct, atol=1e-12)
+
+
+def test_key_layer_norm_comes_before_rope():
+    """Without the rotation, the nope part of a prepared key is the LayerNorm of
+    the whole input row (torch's layer_norm), untouched by RoPE; the pe part is
+    that LayerNorm turned by RoPE."""
+    xk, _, ln_w, ln_b, pos = _rot_inputs()
+    got = O.index_rotate(xk, pos, 64, 10000.0, ln_w, ln_b, 1e-6, layer_norm_first=True, hadamard=False)
+    ln = torch.nn.functional.layer_norm(torch.tensor(xk), (128,), torch.tensor(ln_w), torch.tensor(ln_b),
+                                        1e-6).numpy()
+    np.testing.assert_allclose(got[..., 64:], ln[..., 64:], atol=1e-12)
+    np.testing.assert_allclose(np.linalg.norm(got[..., :64], axis=-1), np.linalg.norm(ln[..., :64], axis=-1),
+                               atol=1e-12)
+
+
+def test_rotated_queries_and_keys_give_the_same_scores():
+    """The Hadamard rotation changes no index score (ik_llama.cpp #2045)."""
+    xk, xq, ln_w, ln_b, pos = _rot_inputs()
+    w = np.array([0.5, -1.0, 2.0, 0.25])
+    kr = O.index_rotate(xk, pos, 64, 10000.0, ln_w, ln_b, 1e-6, layer_norm_first=True)[:, 0]
+    kp = O.index_rotate(xk, pos, 64, 10000.0, ln_w, ln_b, 1e-6, layer_norm_first=True, hadamard=False)[:, 0]
+    for r in range(3):
+        qr = O.index_rotate(xq[r:r + 1], pos[r:r + 1], 64, 10000.0)[0]
+        qp = O.index_rotate(xq[r:r + 1], pos[r:r + 1], 64, 10000.0, hadamard=False)[0]
+        np.testing.assert_allclose(O.index_scores_row(qr, kr, w, 0.1), O.index_scores_row(qp, kp, w, 0.1),
+                                   atol=1e-12)
+
+
 # ------------------------------------------- planted mistakes are caught
 def _run_pins():
     failures = 0
@@ -325,7 +421,11 @@ def _run_pins():
                test_topk_matches_brute_force_with_ties, test_walsh_hadamard_rotation_leaves_scores_unchanged,
                test_expand_selection_examples, test_pooling_starts_at_first_valid_token_and_drops_partial_pool,
                lambda: test_topk_covering_all_keys_equals_dense_attention(1),
-               test_absorbed_mla_equals_literal_expand_kv):
+               test_absorbed_mla_equals_literal_expand_kv, test_rope_neox_pairs_halves_with_closed_form_angles,
+               test_rope_scores_depend_on_relative_position_only,
+               test_sylvester_hadamard_matches_scipy_and_is_orthonormal,
+               test_cached_key_moves_by_unrotate_rope_delta_rerotate, test_key_layer_norm_comes_before_rope,
+               test_rotated_queries_and_keys_give_the_same_scores):
         try:
             fn()
         except (AssertionError, ValueError, IndexError):
@@ -335,7 +435,9 @@ def _run_pins():
 
 @pytest.mark.parametrize("mutant", ["scale_outside_relu_negated", "drop_weight", "tie_largest_index",
                                     "no_dedupe", "softmax_no_max_shift_sign", "pool_from_zero",
-                                    "tail_off_by_one", "absorb_transposed"])
+                                    "tail_off_by_one", "absorb_transposed", "rope_adjacent_pairs",
+                                    "rope_frequency_exponent", "hadamard_before_rope", "layer_norm_after_rope",
+                                    "hadamard_unnormalised"])
 def test_pins_catch_planted_mistakes(monkeypatch, mutant):
     """Plant a plausible mistake in the oracle (on the CPU) and check a pin fails."""
     assert _run_pins() == 0
@@ -376,4 +478,50 @@ def test_pins_catch_planted_mistakes(monkeypatch, mutant):
             out, lse = orig(q, lat, uk, uv, row, scale)
             return out[::-1].copy(), lse[::-1].copy()
         monkeypatch.setattr(O, "mla_absorbed_row", bad2)
+    elif mutant == "rope_adjacent_pairs":
+        def gptj(x, pos, n_rope, theta):
+            x = O.f64(x).copy()
+            for i in range(n_rope // 2):
+                ang = pos * theta ** (-2.0 * i / n_rope)
+                a, b = x[..., 2 * i].copy(), x[..., 2 * i + 1].copy()
+                x[..., 2 * i] = a * math.cos(ang) - b * math.sin(ang)
+                x[..., 2 * i + 1] = b * math.cos(ang) + a * math.sin(ang)
+            return x
+        monkeypatch.setattr(O, "rope_neox", gptj)
+    elif mutant == "rope_frequency_exponent":
+        orig_rope = O.rope_neox
+        def bad_freq(x, pos, n_rope, theta):
+            x = O.f64(x).copy()
+            half = n_rope // 2
+            for i in range(half):
+                ang = pos * theta ** (-1.0 * i / n_rope)
+                a, b = x[..., i].copy(), x[..., i + half].copy()
+                x[..., i] = a * math.cos(ang) - b * math.sin(ang)
+                x[..., i + half] = b * math.cos(ang) + a * math.sin(ang)
+            return x
+        monkeypatch.setattr(O, "rope_neox", bad_freq)
+    elif mutant in ("hadamard_before_rope", "layer_norm_after_rope"):
+        def bad_rotate(x, pos, n_rope, theta, ln_w=None, ln_b=None, eps=1e-6, layer_norm_first=False,
+                       hadamard=True):
+            x = O.f64(x)
+            out = np.empty_like(x)
+            for r in range(x.shape[0]):
+                y = x[r]
+                if mutant == "hadamard_before_rope":
+                    if layer_norm_first:
+                        y = O.layer_norm(y, ln_w, ln_b, eps)
+                    if hadamard:
+                        y = O.hadamard_rotate(y)
+                    y = O.rope_neox(y, int(pos[r]), n_rope, theta)
+                else:
+                    y = O.rope_neox(y, int(pos[r]), n_rope, theta)
+                    if layer_norm_first:
+                        y = O.layer_norm(y, ln_w, ln_b, eps)
+                    if hadamard:
+                        y = O.hadamard_rotate(y)
+                out[r] = y
+            return out
+        monkeypatch.setattr(O, "index_rotate", bad_rotate)
+    elif mutant == "hadamard_unnormalised":
+        monkeypatch.setattr(O, "hadamard_rotate", lambda x: O.f64(x) @ O.sylvester_hadamard(O.f64(x).shape[-1]).T)
     assert _run_pins() > 0, f"mutant {mutant} survived every pin"
