@@ -392,6 +392,7 @@ def run_ours(a):
             line["decode"] = decode_extra(peaks, flush, stream)
             line["chunked"] = chunked_extra(peaks, flush, stream)
             line["kpool"] = kpool_extra(peaks, flush, stream)
+            line["rotate"] = rotate_extra(peaks, flush, stream)
         line["cpu_baseline"] = cpu_baseline(wl, budget_s=a.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -556,6 +557,39 @@ def kpool_extra(peaks, flush, stream):
            "roofline_absorb": roofline_entry("tensor", flop["absorb"], st["absorb_q"] + st["absorb_out"], peaks),
            "fused_tensor_frac": round(sum(flop.values()) / step / 1e12 / peaks["bf16_tflops"], 4)}
     del t, bufs
+    torch.cuda.empty_cache()
+    return res
+
+
+def rotate_extra(peaks, flush, stream):
+    """Indexer query / key preparation (dsa_index_rotate) for the prefill and decode layers.  Prefill
+    rotates 4096 tokens x 64 query heads and writes 4096 LayerNorm-ed keys; decode rotates 64 x 64 query
+    heads and appends one key per sequence at position 32767 of a 64 x 32768 key cache.  RoPE base 10000
+    (the cost does not depend on it)."""
+    import sparse_attention_sum_b200 as dsa
+    theta, res = 10000.0, {}
+    for name, n, S in (("prefill", 4096, 0), ("decode", 64, 32768)):
+        qi = {k: v.cuda() for k, v in workloads.rotate_inputs(n, 64, 128, seed=1, pos_max=S or n).items()}
+        ki = {k: v.cuda() for k, v in workloads.rotate_inputs(n, 1, 128, seed=2, pos_max=S or n, mean=0.5,
+                                                                std=2.0).items()}
+        q_out = torch.empty(n, 64, 128, dtype=torch.bfloat16, device="cuda")
+        if S:
+            cache = torch.zeros(n * S, 1, 128, dtype=torch.bfloat16, device="cuda")
+            slots = torch.arange(n, dtype=torch.int32, device="cuda") * S + (S - 1)
+            ki["pos"].fill_(S - 1)
+        else:
+            cache, slots = torch.empty(n, 1, 128, dtype=torch.bfloat16, device="cuda"), None
+        qf = lambda: dsa.index_rotate(qi["x"], q_out, 64, theta, pos=qi["pos"])
+        kf = lambda: dsa.index_rotate(ki["x"], cache, 64, theta, pos=ki["pos"], layer_norm=True, ln_w=ki["ln_w"],
+                                      ln_b=ki["ln_b"], ln_eps=1e-6, out_rows=slots)
+        tq = statistics.median(time_steps(qf, 10, 3, flush, stream))
+        tk = statistics.median(time_steps(kf, 10, 3, flush, stream))
+        q_bytes = 2 * n * 64 * 128 * 2 + 4 * n           # read and write every query value, positions
+        k_bytes = 2 * n * 128 * 2 + 4 * n * (2 if S else 1) + 2 * 128 * 4
+        res[name] = {"rows": n, "queries_us": round(tq * 1e6, 2), "keys_us": round(tk * 1e6, 2),
+                     "roofline_queries": roofline_entry("hbm", q_bytes, tq, peaks),
+                     "roofline_keys": roofline_entry("hbm", k_bytes, tk, peaks)}
+        del qi, ki, q_out, cache
     torch.cuda.empty_cache()
     return res
 

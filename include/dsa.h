@@ -247,6 +247,45 @@ dsa_status dsa_absorb_q(const dsa_dims* dims, const void* q, int32_t d, const vo
 dsa_status dsa_absorb_out(const dsa_dims* dims, const void* o_lat, int32_t L, const void* w_uv,
                           int32_t e, void* out, dsa_stream_t stream);
 
+/* S9 — indexer query / key preparation, the step that produces q_idx and the
+ * k_idx cache rows the indexer reads (ik_llama.cpp PR #2063 with the PR #2045
+ * commit messages: "What it does" splits the indexer query and key into a rope
+ * part and a nope part, gives the rope part NEOX RoPE and concatenates; the key
+ * is LayerNorm-ed with bias first; the decode-cache commit rotates both by the
+ * Walsh-Hadamard matrix and writes the keys into the indexer cache at their
+ * slot; the K-shift commit states the cached key as H * concat(RoPE(k_pe, pos),
+ * k_nope) with NEOX RoPE unscaled).  For row r < n_rows and head h < heads,
+ * with x = in[r, h, 0:dim]:
+ *   y = layer_norm ? (x - mean) / sqrt(var + ln_eps) * ln_w + ln_b : x   (biased var)
+ *   for i < n_rope/2, a = pos[r] * rope_theta^(-2i/n_rope):
+ *     y'[i]            = y[i] cos a - y[i + n_rope/2] sin a
+ *     y'[i + n_rope/2] = y[i + n_rope/2] cos a + y[i] sin a
+ *   (values from n_rope on are unchanged: the rope part is the first n_rope)
+ *   z = hadamard ? H y' / sqrt(dim) : y',   H[i][j] = (-1)^popcount(i & j)
+ *   out[dst, h, 0:dim] = z,   dst = out_rows ? out_rows[r] : r
+ * A row whose dst lies outside [0, out_capacity) is not written (a padded token
+ * can carry slot -1).  The angles are evaluated in double precision, the rest
+ * in fp32; the store rounds to out_dtype (round to nearest even for bf16).
+ * The Hadamard rotation leaves every q.k unchanged, so queries and keys must
+ * both be rotated or both not.
+ * in:  n_rows rows of heads*dim values of in_dtype, in_row_stride values apart.
+ * out: out_capacity rows of heads*dim values of out_dtype, out_row_stride apart
+ *      (a key cache [B, n_kv, dim] written at slots b*n_kv + position, say).
+ * pos [n_rows] int32 positions (may be NULL when n_rope == 0);
+ * out_rows [n_rows] int32 or NULL; ln_w, ln_b [dim] fp32 or NULL (1 and 0).
+ * Requirements (else DSA_ERR_INVALID_ARGUMENT): n_rows >= 0, heads >= 1,
+ * dim in {32, 64, 128}, n_rope even with 0 <= n_rope <= dim and (n_rope/2) a
+ * multiple of dim/32, rope_theta > 0 when n_rope > 0, ln_eps > 0 with
+ * layer_norm, strides >= heads*dim and multiples of dim/32, in and out aligned
+ * to dim/32 values, out_capacity >= n_rows when out_rows is NULL.  in and out
+ * must not overlap unless the call is exactly in place (same pointer, stride and
+ * dtype, out_rows NULL). */
+dsa_status dsa_index_rotate(int32_t n_rows, int32_t heads, int32_t dim, int32_t n_rope, float rope_theta,
+                            int32_t layer_norm, const float* ln_w, const float* ln_b, float ln_eps,
+                            int32_t hadamard, const int32_t* pos, dsa_dtype in_dtype, const void* in,
+                            int64_t in_row_stride, dsa_dtype out_dtype, void* out, int64_t out_row_stride,
+                            const int32_t* out_rows, int64_t out_capacity, dsa_stream_t stream);
+
 /* Allocation-free variant of dsa_layer_forward, for callers that cannot
  * allocate device memory where they run the layer (a serving engine that plans
  * all memory up front and forbids allocation on its decode path, code running

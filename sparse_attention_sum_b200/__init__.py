@@ -16,7 +16,7 @@ from typing import Optional
 __all__ = [
     "DsaError", "DsaLibraryError", "Dims", "lib", "lib_path", "INVALID", "F32", "BF16",
     "index_scores", "topk", "topk_set", "sparse_attend", "layer_forward", "layer_forward_static", "pool_states",
-    "expand_selection", "absorb_q", "absorb_out", "workspace_size", "get_device_status",
+    "expand_selection", "absorb_q", "absorb_out", "index_rotate", "workspace_size", "get_device_status",
     "selftest_wait_timeout", "set_kernel_policy", "OP_TOPK", "OP_LAYER_FORWARD", "STATUS",
 ]
 
@@ -87,6 +87,10 @@ _SIGS = {
                      ctypes.c_int),
     "dsa_absorb_out": ([ctypes.POINTER(Dims), _VP, ctypes.c_int32, _VP, ctypes.c_int32, _VP, _VP],
                        ctypes.c_int),
+    "dsa_index_rotate": ([ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
+                          ctypes.c_int32, _F32P, _F32P, ctypes.c_float, ctypes.c_int32, _I32P, ctypes.c_int,
+                          _VP, ctypes.c_int64, ctypes.c_int, _VP, ctypes.c_int64, _I32P, ctypes.c_int64, _VP],
+                         ctypes.c_int),
     "dsa_get_device_status": ([_VP], ctypes.c_int),
     "dsa_selftest_wait_timeout": ([ctypes.c_int64, _VP], ctypes.c_int),
 }
@@ -221,6 +225,26 @@ def absorb_q(dims: Dims, q, d: int, w_uk, L: int, q_lat, stream=None):
 def absorb_out(dims: Dims, o_lat, L: int, w_uv, e: int, out, stream=None):
     _check(lib().dsa_absorb_out(ctypes.byref(dims), _ptr(o_lat), int(L), _ptr(w_uv), int(e), _ptr(out),
                                 _stream(stream)), "dsa_absorb_out")
+
+
+def index_rotate(x, out, n_rope: int, rope_theta: float, pos=None, layer_norm: bool = False, ln_w=None,
+                 ln_b=None, ln_eps: float = 0.0, hadamard: bool = True, out_rows=None, stream=None):
+    """dsa_index_rotate: prepare indexer queries or keys.
+
+    ``x`` is ``[n_rows, heads, dim]`` and ``out`` is ``[capacity, heads, dim]``, each with its
+    last two axes contiguous (the row stride may be larger).  Row r goes to ``out[out_rows[r]]``
+    (or ``out[r]``)."""
+    for name, t in (("x", x), ("out", out)):
+        if t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+            raise ValueError(f"{name} must be [rows, heads, dim] with contiguous heads and values")
+    if out.shape[1:] != x.shape[1:]:
+        raise ValueError("x and out must have the same heads and dim")
+    n_rows, heads, dim = x.shape
+    _check(lib().dsa_index_rotate(int(n_rows), int(heads), int(dim), int(n_rope), float(rope_theta),
+                                  int(bool(layer_norm)), _ptr(ln_w), _ptr(ln_b), float(ln_eps), int(bool(hadamard)),
+                                  _ptr(pos), _dtype_code(x), _ptr(x), int(x.stride(0)), _dtype_code(out), _ptr(out),
+                                  int(out.stride(0)), _ptr(out_rows), int(out.shape[0]), _stream(stream)),
+           "dsa_index_rotate")
 
 
 def get_device_status(stream=None) -> int:

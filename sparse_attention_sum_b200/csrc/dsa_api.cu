@@ -333,6 +333,41 @@ dsa_status dsa_expand_selection(const dsa_dims* d, const int32_t* pool_idx, cons
   return ok();
 }
 
+dsa_status dsa_index_rotate(int32_t n_rows, int32_t heads, int32_t dim, int32_t n_rope, float rope_theta,
+                            int32_t layer_norm, const float* ln_w, const float* ln_b, float ln_eps,
+                            int32_t hadamard, const int32_t* pos, dsa_dtype in_dtype, const void* in,
+                            int64_t in_row_stride, dsa_dtype out_dtype, void* out, int64_t out_row_stride,
+                            const int32_t* out_rows, int64_t out_capacity, dsa_stream_t stream) {
+  REQUIRE(n_rows >= 0, "n_rows must be >= 0 (got %d)", n_rows);
+  REQUIRE(heads >= 1, "heads must be >= 1 (got %d)", heads);
+  REQUIRE(dim == 32 || dim == 64 || dim == 128, "dim must be 32, 64 or 128 (got %d)", dim);
+  const int E = dim / 32;
+  REQUIRE(n_rope >= 0 && n_rope <= dim && n_rope % 2 == 0 && (n_rope / 2) % E == 0,
+          "n_rope must be even, in [0, dim], with n_rope/2 a multiple of dim/32 (got %d)", n_rope);
+  REQUIRE(n_rope == 0 || (rope_theta > 0.f && rope_theta < INFINITY), "rope_theta must be finite and > 0");
+  REQUIRE(!layer_norm || ln_eps > 0.f, "ln_eps must be > 0 (got %g)", (double)ln_eps);
+  REQUIRE(dtype_ok(in_dtype) && dtype_ok(out_dtype), "dtypes must be DSA_F32 or DSA_BF16");
+  if (n_rows == 0) return ok();
+  REQUIRE(in && out, "in and out must be non-NULL");
+  REQUIRE(n_rope == 0 || pos, "pos must be non-NULL when n_rope > 0");
+  const int64_t row = (int64_t)heads * dim;
+  REQUIRE(in_row_stride >= row && out_row_stride >= row, "row strides must be >= heads*dim (%lld)",
+          (long long)row);
+  REQUIRE(in_row_stride % E == 0 && out_row_stride % E == 0, "row strides must be multiples of dim/32");
+  const size_t in_align = (size_t)E * (in_dtype == DSA_BF16 ? 2 : 4);
+  const size_t out_align = (size_t)E * (out_dtype == DSA_BF16 ? 2 : 4);
+  REQUIRE((uintptr_t)in % in_align == 0 && (uintptr_t)out % out_align == 0,
+          "in and out must be aligned to dim/32 values");
+  REQUIRE(out_capacity >= 0, "out_capacity must be >= 0");
+  REQUIRE(out_rows || out_capacity >= n_rows, "out_capacity must be >= n_rows when out_rows is NULL");
+  cudaError_t e = dsa::launch_index_rotate(n_rows, heads, dim, n_rope, rope_theta, layer_norm != 0, ln_w, ln_b,
+                                           ln_eps, hadamard != 0, pos, in_dtype == DSA_BF16, in, in_row_stride,
+                                           out_dtype == DSA_BF16, out, out_row_stride, out_rows, out_capacity,
+                                           (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "dsa_index_rotate launch");
+  return ok();
+}
+
 static dsa_status check_absorb(const dsa_dims* d, const void* a, int32_t K, const void* w, int32_t N,
                                void* c) {
   REQUIRE(d != nullptr, "dims is NULL");

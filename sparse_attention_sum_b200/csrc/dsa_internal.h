@@ -69,6 +69,15 @@ bool head_gemm_tc_supported(int n_rows, int heads, int K, int N, const void* A, 
 cudaError_t launch_head_gemm_tc(int n_rows, int heads, int K, int N, const void* A, const void* Bm, bool b_kn,
                                 void* C, cudaStream_t st);
 
+// Indexer query / key preparation: optional LayerNorm, NEOX RoPE of the first
+// n_rope values, optional orthonormal Walsh-Hadamard rotation, store to row
+// out_rows[r] (or r) when that row is in [0, out_cap).  dim in {32, 64, 128}.
+cudaError_t launch_index_rotate(int n_rows, int heads, int dim, int n_rope, float theta, bool layer_norm,
+                                const float* ln_w, const float* ln_b, float eps, bool hadamard,
+                                const int32_t* pos, bool in_bf16, const void* in, int64_t in_stride,
+                                bool out_bf16, void* out, int64_t out_stride, const int32_t* out_rows,
+                                int64_t out_cap, cudaStream_t st);
+
 // Bounded-wait self test.
 cudaError_t launch_wait_selftest(long long timeout_ns, cudaStream_t st);
 

@@ -1,0 +1,254 @@
+// Indexer query / key preparation ahead of the score (ik_llama.cpp PR #2063 with
+// the PR #2045 commit messages: "What it does" (split rope/nope, NEOX RoPE of the
+// rope part, concat; LayerNorm with bias on the key), the decode-cache commit
+// (Walsh-Hadamard rotation of q and k, keys written into the indexer cache at
+// their slot) and the K-shift commit (the cached key is H * concat(RoPE(k_pe,
+// pos), k_nope); NEOX RoPE without scaling)).
+//
+// One block per row (token).  Its first threads build the row's RoPE table,
+// cos and sin of pos * theta^(-2i/n_rope), in double precision, once for all
+// heads of the row.  Each warp then takes head vectors of `dim` values, up to
+// four at a time so their loads are in flight together: lane l holds values
+// l*E .. l*E+E-1 (E = dim/32) in registers, read with one vector load.
+//   LayerNorm: a warp sum for the mean, then one for the biased variance of the
+//     centred values.
+//   NEOX RoPE: value d < n_rope/2 pairs with d + n_rope/2, which lives
+//     n_rope/(2E) lanes higher; one shuffle down and one up give both partners.
+//   Walsh-Hadamard: log2(E) butterfly stages inside the lane, five over the lane
+//     bits with xor shuffles, then the 1/sqrt(dim) scale; the butterflies give
+//     y[i] = sum_j (-1)^popcount(i & j) x[j], the Sylvester matrix.
+// The row goes to out_rows[r] (its cache slot) or to r; a slot outside
+// [0, capacity) is skipped.  Each vector is read once and written once, so the
+// kernel is bound by HBM bandwidth.
+#include "dsa_common.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+
+namespace {
+
+constexpr int kRotWarps = 8;  // warps per block (fewer when a row has fewer heads)
+constexpr int kRotBatch = 4;  // head vectors per warp in flight
+
+struct RotParams {
+  const void* in;
+  void* out;
+  const int32_t* pos;
+  const int32_t* out_rows;
+  const float* ln_w;
+  const float* ln_b;
+  int64_t in_stride, out_stride, out_cap;
+  int heads, n_rope, layer_norm, hadamard;
+  float theta, eps, hscale;
+};
+
+template <int E>
+__device__ __forceinline__ void load_vals(const float* p, float (&v)[E]) {
+  if constexpr (E == 4) {
+    const float4 u = *reinterpret_cast<const float4*>(p);
+    v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+  } else if constexpr (E == 2) {
+    const float2 u = *reinterpret_cast<const float2*>(p);
+    v[0] = u.x; v[1] = u.y;
+  } else {
+    v[0] = *p;
+  }
+}
+
+template <int E>
+__device__ __forceinline__ void load_vals(const bf16* p, float (&v)[E]) {
+  if constexpr (E == 4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+  } else if constexpr (E == 2) {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+    v[0] = a.x; v[1] = a.y;
+  } else {
+    v[0] = __bfloat162float(*p);
+  }
+}
+
+template <int E>
+__device__ __forceinline__ void store_vals(float* p, const float (&v)[E]) {
+  if constexpr (E == 4) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  } else if constexpr (E == 2) {
+    *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+  } else {
+    *p = v[0];
+  }
+}
+
+template <int E>
+__device__ __forceinline__ void store_vals(bf16* p, const float (&v)[E]) {
+  if constexpr (E == 4) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
+    __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&a);
+    u.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = u;
+  } else if constexpr (E == 2) {
+    *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v[0], v[1]);
+  } else {
+    *p = __float2bfloat16_rn(v[0]);
+  }
+}
+
+template <typename Tin, typename Tout, int E>
+__global__ void __launch_bounds__(kRotWarps * 32)
+index_rotate_kernel(RotParams p) {
+  constexpr int D = 32 * E;
+  __shared__ float2 tab[D / 2];  // (cos, sin) of each RoPE pair
+  const int r = blockIdx.x;
+  const int half = p.n_rope >> 1;
+  if (half > 0) {
+    const double pos = (double)p.pos[r];
+    const double log2_theta = log2((double)p.theta);
+    for (int i = threadIdx.x; i < half; i += blockDim.x) {
+      double s, c;
+      sincos(pos * exp2(-(2.0 * i / p.n_rope) * log2_theta), &s, &c);
+      tab[i] = make_float2((float)c, (float)s);
+    }
+  }
+  __syncthreads();
+
+  const int64_t dst = p.out_rows ? (int64_t)p.out_rows[r] : (int64_t)r;
+  if (dst < 0 || dst >= p.out_cap) return;  // block-uniform; no barrier follows
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int d0 = lane * E;
+  // no __restrict__: an exactly in-place call reads and writes the same vectors
+  const Tin* src = static_cast<const Tin*>(p.in) + (int64_t)r * p.in_stride + d0;
+  Tout* dstp = static_cast<Tout*>(p.out) + dst * p.out_stride + d0;
+
+  float lw[E], lb[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    lw[e] = p.layer_norm && p.ln_w ? p.ln_w[d0 + e] : 1.f;
+    lb[e] = p.layer_norm && p.ln_b ? p.ln_b[d0 + e] : 0.f;
+  }
+  const int off = half / E;  // lane distance between the two values of a RoPE pair
+  const bool first_half = d0 < half, second_half = d0 >= half && d0 < p.n_rope;
+
+  for (int h0 = warp; h0 < p.heads; h0 += nwarps * kRotBatch) {
+    float v[kRotBatch][E];
+#pragma unroll
+    for (int u = 0; u < kRotBatch; ++u) {
+      const int h = h0 + u * nwarps;
+      if (h < p.heads) load_vals<E>(src + (int64_t)h * D, v[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < kRotBatch; ++u) {
+      const int h = h0 + u * nwarps;
+      if (h >= p.heads) break;  // warp-uniform
+      if (p.layer_norm) {
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) s += v[u][e];
+        const float mean = warp_sum(s) * (1.f / D);
+        float s2 = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          v[u][e] -= mean;
+          s2 = fmaf(v[u][e], v[u][e], s2);
+        }
+        const float inv_std = 1.f / sqrtf(warp_sum(s2) * (1.f / D) + p.eps);
+#pragma unroll
+        for (int e = 0; e < E; ++e) v[u][e] = fmaf(v[u][e] * inv_std, lw[e], lb[e]);
+      }
+      if (half > 0) {
+        float up[E], dn[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          up[e] = __shfl_down_sync(0xffffffffu, v[u][e], off);
+          dn[e] = __shfl_up_sync(0xffffffffu, v[u][e], off);
+        }
+        if (first_half) {
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const float2 cs = tab[d0 + e];
+            v[u][e] = v[u][e] * cs.x - up[e] * cs.y;
+          }
+        } else if (second_half) {
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const float2 cs = tab[d0 + e - half];
+            v[u][e] = v[u][e] * cs.x + dn[e] * cs.y;
+          }
+        }
+      }
+      if (p.hadamard) {
+#pragma unroll
+        for (int m = 1; m < E; m <<= 1) {
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            if (!(e & m)) {
+              const float a = v[u][e], b = v[u][e | m];
+              v[u][e] = a + b;
+              v[u][e | m] = a - b;
+            }
+          }
+        }
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1) {
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const float o = __shfl_xor_sync(0xffffffffu, v[u][e], m);
+            v[u][e] = (lane & m) ? o - v[u][e] : v[u][e] + o;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) v[u][e] *= p.hscale;
+      }
+      store_vals<E>(dstp + (int64_t)h * D, v[u]);
+    }
+  }
+}
+
+template <typename Tin, typename Tout>
+cudaError_t launch_rotate_t(int n_rows, int dim, const RotParams& p, cudaStream_t st) {
+  const int warps = p.heads < kRotWarps ? p.heads : kRotWarps;
+  const dim3 grid((unsigned)n_rows), block((unsigned)(32 * warps));
+  switch (dim) {
+    case 32: index_rotate_kernel<Tin, Tout, 1><<<grid, block, 0, st>>>(p); break;
+    case 64: index_rotate_kernel<Tin, Tout, 2><<<grid, block, 0, st>>>(p); break;
+    case 128: index_rotate_kernel<Tin, Tout, 4><<<grid, block, 0, st>>>(p); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_index_rotate(int n_rows, int heads, int dim, int n_rope, float theta, bool layer_norm,
+                                const float* ln_w, const float* ln_b, float eps, bool hadamard,
+                                const int32_t* pos, bool in_bf16, const void* in, int64_t in_stride,
+                                bool out_bf16, void* out, int64_t out_stride, const int32_t* out_rows,
+                                int64_t out_cap, cudaStream_t st) {
+  if (n_rows == 0) return cudaSuccess;
+  RotParams p;
+  p.in = in;
+  p.out = out;
+  p.pos = pos;
+  p.out_rows = out_rows;
+  p.ln_w = ln_w;
+  p.ln_b = ln_b;
+  p.in_stride = in_stride;
+  p.out_stride = out_stride;
+  p.out_cap = out_cap;
+  p.heads = heads;
+  p.n_rope = n_rope;
+  p.layer_norm = layer_norm ? 1 : 0;
+  p.hadamard = hadamard ? 1 : 0;
+  p.theta = theta;
+  p.eps = eps;
+  p.hscale = (float)(1.0 / sqrt((double)dim));
+  if (in_bf16)
+    return out_bf16 ? launch_rotate_t<bf16, bf16>(n_rows, dim, p, st) : launch_rotate_t<bf16, float>(n_rows, dim, p, st);
+  return out_bf16 ? launch_rotate_t<float, bf16>(n_rows, dim, p, st) : launch_rotate_t<float, float>(n_rows, dim, p, st);
+}
+
+}  // namespace dsa

@@ -104,6 +104,33 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert st == 1
 
 
+def test_index_rotate_host_validation(lib):
+    nul = None
+    a = ctypes.c_void_p(256)  # 16-byte aligned, never dereferenced: validation fails first
+    BF, F = dsa.BF16, dsa.F32
+
+    def rot(n_rows=4, heads=2, dim=128, n_rope=64, theta=10000.0, ln=0, eps=0.0, pos=a, in_dt=BF, x=a,
+            in_stride=256, out_dt=BF, out=a, out_stride=256, rows=nul, cap=4):
+        return _call(lib.dsa_index_rotate, n_rows, heads, dim, n_rope, theta, ln, nul, nul, eps, 1, pos, in_dt, x,
+                     in_stride, out_dt, out, out_stride, rows, cap, nul)
+
+    assert rot(dim=96)[0] == 1 and "dim" in rot(dim=96)[1]
+    assert rot(n_rope=62)[0] == 1                      # (n_rope/2) % (dim/32) != 0
+    assert rot(n_rope=130)[0] == 1
+    assert rot(n_rope=63, dim=32)[0] == 1              # odd
+    assert rot(theta=0.0)[0] == 1 and "rope_theta" in rot(theta=0.0)[1]
+    assert rot(ln=1, eps=0.0)[0] == 1 and "ln_eps" in rot(ln=1, eps=0.0)[1]
+    assert rot(in_stride=200)[0] == 1 and "stride" in rot(in_stride=200)[1]
+    assert rot(out_stride=258)[0] == 1                 # not a multiple of dim/32
+    assert rot(x=ctypes.c_void_p(258))[0] == 1 and "aligned" in rot(x=ctypes.c_void_p(258))[1]
+    assert rot(pos=nul)[0] == 1 and "pos" in rot(pos=nul)[1]
+    assert rot(cap=3)[0] == 1 and "out_capacity" in rot(cap=3)[1]
+    assert rot(heads=0)[0] == 1
+    assert rot(in_dt=7)[0] == 1
+    assert rot(n_rows=-1)[0] == 1
+    assert rot(n_rows=0, x=nul, out=nul)[0] == 0       # nothing to do: no launch, no pointer read
+
+
 def test_binding_raises_typed_errors(lib):
     with pytest.raises(dsa.DsaError) as ei:
         dsa._check(1, "dsa_topk")

@@ -31,7 +31,7 @@ import torch
 
 INVALID = -1
 
-__all__ = ["Workload", "make", "NAMES", "INVALID", "hot_spot_runs"]
+__all__ = ["Workload", "make", "NAMES", "INVALID", "hot_spot_runs", "rotate_inputs"]
 
 NAMES = ("tiny", "prefill", "decode", "chunked", "kpool")
 
@@ -198,3 +198,24 @@ def make(name: str, seed: Optional[int] = None, **sizes) -> Workload:
         raise KeyError(f"unknown workload {name!r}; expected one of {NAMES}")
     s = _DEFAULT_SEEDS[name] if seed is None else seed
     return _BUILDERS[name](s, **sizes)
+
+
+def rotate_inputs(n_rows: int, heads: int, dim: int = 128, seed: int = 5, pos_max: int = 32768,
+                  dtype: str = "bf16", mean: float = 0.0, std: float = 1.0) -> Dict[str, torch.Tensor]:
+    """Inputs of the indexer query / key preparation step (all on the CPU).
+
+    ``x [n_rows, heads, dim]`` ~ N(mean, std^2) (the indexer projections' output;
+    queries use 64 heads, keys one), ``pos [n_rows]`` int32 uniform in
+    ``[0, pos_max)``, and the key LayerNorm's ``ln_w = 1 + 0.1 N``,
+    ``ln_b = 0.1 N`` (fp32), drawn in that order.
+    """
+    g = torch.Generator().manual_seed(seed)
+    x = _randn(g, (n_rows, heads, dim), std)
+    if mean:
+        x.add_(mean)
+    if dtype == "bf16":
+        x = x.to(torch.bfloat16)
+    pos = torch.randint(0, pos_max, (n_rows,), generator=g, dtype=torch.int32)
+    ln_w = 1 + 0.1 * _randn(g, (dim,))
+    ln_b = 0.1 * _randn(g, (dim,))
+    return {"x": x, "pos": pos, "ln_w": ln_w, "ln_b": ln_b}
