@@ -142,3 +142,36 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(dsa, "lib_path", lambda: str(tmp_path / "libdsa.so"))
     with pytest.raises(dsa.DsaLibraryError):
         dsa.lib()
+
+
+def test_plain_c_program_links_and_calls_the_library(lib, tmp_path):
+    """include/dsa.h is plain C99 and libdsa.so links into a C program (host-only calls, no GPU)."""
+    src = tmp_path / "use_dsa.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "dsa.h"
+int main(void) {
+  dsa_dims d;
+  memset(&d, 0, sizeof d);
+  d.batch = 2; d.n_q = 3; d.n_kv = 100; d.top_k = 8;
+  printf("%s|%s|%zu|", dsa_version(), dsa_status_string(DSA_ERR_TIMEOUT),
+         dsa_workspace_size(&d, DSA_OP_LAYER_FORWARD));
+  /* host validation: a NULL dims pointer is rejected before any launch */
+  dsa_status s = dsa_index_scores(NULL, NULL, NULL, NULL, 1.0f, NULL, NULL, NULL, NULL, NULL);
+  printf("%d|%s\n", (int)s, dsa_last_error());
+  return s == DSA_ERR_INVALID_ARGUMENT ? 0 : 1;
+}
+''')
+    exe = tmp_path / "use_dsa"
+    pkg = os.path.dirname(dsa.lib_path())
+    cc = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                         str(src), "-o", str(exe), "-L", pkg, "-ldsa", f"-Wl,-rpath,{pkg}"],
+                        capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, run.stdout + run.stderr
+    version, status, ws, code, msg = run.stdout.strip().split("|")
+    assert "sm_100a" in version and status == "DSA_ERR_TIMEOUT"
+    assert int(ws) == dsa.workspace_size(dsa.Dims(batch=2, n_q=3, n_kv=100, top_k=8), dsa.OP_LAYER_FORWARD)
+    assert int(code) == 1 and "dims" in msg
