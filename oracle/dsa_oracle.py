@@ -580,3 +580,74 @@ def index_rotate(x, pos, n_rope: int, theta: float, ln_w=None, ln_b=None, eps: f
             y = hadamard_rotate(y)
         out[r] = y
     return out
+
+
+# ---------------------------------------------------------------------------
+# S2 in FP8: e4m3 indexer operands
+# ---------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def e4m3_grid() -> np.ndarray:
+    """The non-negative finite values of the e4m3 format (1 sign, 4 exponent bits
+    with bias 7, 3 mantissa bits, no infinities; the all-ones code is NaN),
+    ascending: subnormals ``m * 2**-9`` (m = 0..7), then ``2**(e-7) * (1 + m/8)``
+    for e = 1..15, m = 0..7, without e = 15, m = 7.  [ik-2063] ships the
+    indexer's tensors in F8_E4M3."""
+    vals = [m * 2.0 ** -9 for m in range(8)]
+    for e in range(1, 16):
+        for m in range(8):
+            if e == 15 and m == 7:
+                continue
+            vals.append(2.0 ** (e - 7) * (1 + m / 8))
+    return np.array(vals)
+
+
+def e4m3_round(y) -> np.ndarray:
+    """Round to the nearest e4m3 value, ties to the even code (even mantissa).
+
+    Inputs beyond the largest value's rounding range (|y| >= 464, halfway to the
+    next binade step) raise: the quantiser below scales every vector into range."""
+    y = f64(y)
+    if np.any(np.abs(y) >= 464.0):
+        raise ValueError("value outside the e4m3 range")
+    grid = e4m3_grid()
+    a = np.abs(y)
+    hi = np.clip(np.searchsorted(grid, a, side="left"), 1, grid.size - 1)
+    lo = hi - 1
+    d_lo, d_hi = a - grid[lo], grid[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))  # codes alternate even/odd along the grid
+    q = np.where(pick_hi, grid[hi], grid[lo])
+    q = np.where(a == grid[hi], grid[hi], q)
+    return np.copysign(q, y)
+
+
+def fp8_quantize(x):
+    """Quantise each vector (last axis) to e4m3 with one fp32 scale.
+
+    READING (the pages name only the F8_E4M3 format): each query-head vector and
+    each key row gets ``s = amax / 448``; the codes are ``e4m3(x * (448 / amax))``
+    with the reciprocal and the product rounded to fp32, as a kernel computes
+    them (the rounding decides the code, so it runs in the kernel's precision).
+    A zero vector has scale 1 and zero codes.  Returns (codes, scales) with
+    ``x ~= codes * scales[..., None]``.
+    """
+    x32 = np.asarray(f64(x), dtype=np.float32)
+    amax = np.abs(x32).max(axis=-1)
+    safe = np.where(amax > 0, amax, np.float32(1.0)).astype(np.float32)
+    inv = (np.float32(E4M3_MAX) / safe).astype(np.float32)
+    y = (x32 * inv[..., None]).astype(np.float32)
+    codes = e4m3_round(y.astype(np.float64))
+    scales = np.where(amax > 0, (safe / np.float32(E4M3_MAX)).astype(np.float32), np.float32(1.0))
+    return codes, scales.astype(np.float64)
+
+
+def index_scores_fp8_row(q_row, keys, w_row, scale: float) -> np.ndarray:
+    """``I[s] = sum_h w_h * relu(scale * sq_h * sk_s * (q^_h . k^_s))`` with e4m3 codes
+    q^, k^ and their scales from :func:`fp8_quantize` ([fak-sparse] §3 score with
+    FP8 operands).  The code dot products are exact in float64."""
+    qc, qs = fp8_quantize(q_row)          # [H, D], [H]
+    kc, ks = fp8_quantize(keys)           # [n, D], [n]
+    dots = qc @ kc.T                      # [H, n]
+    act = np.maximum(0.0, float(scale) * (qs[:, None] * ks[None, :]) * dots)
+    return (f64(w_row)[:, None] * act).sum(axis=0) + 0.0

@@ -1,0 +1,40 @@
+"""What e4m3 indexer operands do to the selection (CPU, oracle only).
+
+With per-vector amax scaling (the oracle's FP8 reading), the score error on the synthetic workloads is a few
+percent of the row's score scale, so an FP8 indexer cannot meet the 1e-5 tie band against the bf16 path; it
+is compared with the FP8 oracle instead (identical codes, so only accumulation order differs).  This test
+records the size of the effect: most of the f64 selection survives, and every swapped key lies close to the
+k-th score tau, as quantisation noise (not a dropped scale or a wrong sign) predicts.
+"""
+import numpy as np
+import pytest
+
+from oracle import dsa_oracle as O
+import workloads
+
+
+def _compare(wl, b, t):
+    cand = O.visible_keys(int(wl["q_pos"][b, t]), int(wl["kv_start"][b]), int(wl["kv_len"][b]))
+    keys = wl["k_idx"][b, cand]
+    s64 = O.index_scores_row(wl["q_idx"][b, t], keys, wl["w"][b, t], wl.idx_scale)
+    s8 = O.index_scores_fp8_row(wl["q_idx"][b, t], keys, wl["w"][b, t], wl.idx_scale)
+    k = min(wl.top_k, cand.size)
+    ref, got = set(O.topk_row(cand, s64, k).tolist()), set(O.topk_row(cand, s8, k).tolist())
+    tau = np.sort(s64)[::-1][k - 1]
+    scale = max(abs(tau), np.abs(s64).max())
+    where = {c: i for i, c in enumerate(cand.tolist())}
+    dist = max([abs(s64[where[c]] - tau) / scale for c in ref ^ got], default=0.0)
+    return len(ref & got) / k, dist, np.abs(s8 - s64).max() / scale
+
+
+@pytest.mark.parametrize("name,sizes,b,t", [("prefill", {"T": 2560}, 0, 2047), ("prefill", {"T": 2560}, 0, 2559),
+                                             ("decode", {"B": 2}, 1, 0)])
+def test_fp8_operands_keep_most_of_the_selection_and_swap_only_near_tau(name, sizes, b, t):
+    """Prefill recipe at 2560 tokens (top_k 2048) and decode recipe (32768 keys), smaller batches."""
+    recall, dist, err = _compare(workloads.make(name, **sizes), b, t)
+    if t == 2047:
+        assert recall == 1.0          # all 2048 visible keys are selected either way
+    else:
+        assert recall >= 0.95, recall
+    assert dist <= 0.08, dist         # swapped keys sit within a few percent of the scale from tau
+    assert 1e-3 < err < 0.1, err      # e4m3 noise: far above bf16/fp32 rounding, far below the score scale

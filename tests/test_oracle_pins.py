@@ -414,6 +414,65 @@ def test_rotated_queries_and_keys_give_the_same_scores():
                                    atol=1e-12)
 
 
+# ------------------------------------------- P14 FP8 (e4m3) indexer operands
+def test_e4m3_grid_is_the_format_and_decodes_like_torch():
+    """127 non-negative finite values: subnormal step 2^-9, smallest normal 2^-6, eight values per binade,
+    largest 448; code i decodes (torch's float8_e4m3fn) to the i-th value."""
+    g = O.e4m3_grid()
+    assert g.size == 127 and g[0] == 0 and g[1] == 2.0 ** -9 and g[8] == 2.0 ** -6 and g[-1] == 448.0
+    for e in range(1, 15):
+        binade = g[8 * e: 8 * e + 8]
+        assert np.array_equal(binade, 2.0 ** (e - 7) * (1 + np.arange(8) / 8))
+    decoded = torch.arange(127, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(decoded, g)
+
+
+def test_e4m3_rounding_ties_to_even_and_matches_torch():
+    hand = {1.0625: 1.0, 1.1875: 1.25, 2.0 ** -10: 0.0, 3 * 2.0 ** -11: 2.0 ** -9, 463.9: 448.0, -1.0625: -1.0,
+            0.3: 0.3125, 17.0: 16.0, 19.0: 20.0}
+    got = O.e4m3_round(np.array(list(hand)))
+    assert got.tolist() == list(hand.values())
+    rng = np.random.default_rng(16)
+    y = np.concatenate([rng.uniform(-463, 463, 50000), rng.uniform(-0.03, 0.03, 20000),
+                        O.e4m3_grid()[1:-1] + np.diff(O.e4m3_grid())[1:] / 2])   # exact midpoints
+    y = y.astype(np.float32).astype(np.float64)
+    ref = torch.tensor(y, dtype=torch.float32).to(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(O.e4m3_round(y), ref)
+    with pytest.raises(ValueError):
+        O.e4m3_round(np.array([464.0]))
+
+
+def test_fp8_quantization_maps_each_vector_amax_to_448_within_the_grid_error():
+    rng = np.random.default_rng(17)
+    x = rng.standard_normal((6, 5, 128)) * rng.choice([1e-3, 1.0, 50.0], (6, 5, 1))
+    x[2, 3] = 0.0
+    codes, sc = O.fp8_quantize(x)
+    amax = np.abs(x).max(axis=-1)
+    nz = amax > 0
+    assert np.array_equal(np.abs(codes).max(axis=-1)[nz], np.full(nz.sum(), 448.0))
+    assert np.all(codes[2, 3] == 0) and sc[2, 3] == 1.0
+    assert np.all(np.isin(np.abs(codes), O.e4m3_grid()))
+    # half a grid step: 2^-4 of the value in the normal range, 2^-10 * scale below it (plus fp32 inputs)
+    err = np.abs(codes * sc[..., None] - x)
+    bound = 2.0 ** -4 * np.abs(x) + 2.0 ** -10 * sc[..., None] + 1e-6 * amax[..., None]
+    assert np.all(err <= bound)
+
+
+def test_fp8_scores_equal_plain_scores_when_the_operands_are_e4m3_values_with_amax_448():
+    """Unit scales and representable operands make the quantisation exact, so the FP8 score is the plain one."""
+    rng = np.random.default_rng(18)
+    g = O.e4m3_grid()
+    q = rng.choice(g, (4, 32)) * rng.choice([-1, 1], (4, 32))
+    k = rng.choice(g, (9, 32)) * rng.choice([-1, 1], (9, 32))
+    q[:, 0] = 448.0
+    k[:, 5] = -448.0
+    w = np.array([0.5, -1.0, 2.0, 0.25])
+    assert np.array_equal(O.index_scores_fp8_row(q, k, w, 1 / 64), O.index_scores_row(q, k, w, 1 / 64))
+    # a per-vector factor of 2 changes scales only, not codes: the score doubles per factor
+    assert np.array_equal(O.index_scores_fp8_row(2 * q, k, w, 1 / 64), 2 * O.index_scores_row(q, k, w, 1 / 64))
+    assert np.array_equal(O.index_scores_fp8_row(q, 4 * k, w, 1 / 64), 4 * O.index_scores_row(q, k, w, 1 / 64))
+
+
 # ------------------------------------------- planted mistakes are caught
 def _run_pins():
     failures = 0
@@ -425,7 +484,10 @@ def _run_pins():
                test_rope_scores_depend_on_relative_position_only,
                test_sylvester_hadamard_matches_scipy_and_is_orthonormal,
                test_cached_key_moves_by_unrotate_rope_delta_rerotate, test_key_layer_norm_comes_before_rope,
-               test_rotated_queries_and_keys_give_the_same_scores):
+               test_rotated_queries_and_keys_give_the_same_scores, test_e4m3_grid_is_the_format_and_decodes_like_torch,
+               test_e4m3_rounding_ties_to_even_and_matches_torch,
+               test_fp8_quantization_maps_each_vector_amax_to_448_within_the_grid_error,
+               test_fp8_scores_equal_plain_scores_when_the_operands_are_e4m3_values_with_amax_448):
         try:
             fn()
         except (AssertionError, ValueError, IndexError):
@@ -437,7 +499,8 @@ def _run_pins():
                                     "no_dedupe", "softmax_no_max_shift_sign", "pool_from_zero",
                                     "tail_off_by_one", "absorb_transposed", "rope_adjacent_pairs",
                                     "rope_frequency_exponent", "hadamard_before_rope", "layer_norm_after_rope",
-                                    "hadamard_unnormalised"])
+                                    "hadamard_unnormalised", "e4m3_ties_away", "e4m3_two_mantissa_bits",
+                                    "fp8_key_scale_dropped"])
 def test_pins_catch_planted_mistakes(monkeypatch, mutant):
     """Plant a plausible mistake in the oracle (on the CPU) and check a pin fails."""
     assert _run_pins() == 0
@@ -524,4 +587,29 @@ def test_pins_catch_planted_mistakes(monkeypatch, mutant):
         monkeypatch.setattr(O, "index_rotate", bad_rotate)
     elif mutant == "hadamard_unnormalised":
         monkeypatch.setattr(O, "hadamard_rotate", lambda x: O.f64(x) @ O.sylvester_hadamard(O.f64(x).shape[-1]).T)
+    elif mutant == "e4m3_ties_away":
+        orig_round = O.e4m3_round
+        def away(y):
+            y = O.f64(y)
+            a = np.abs(y)
+            g = O.e4m3_grid()
+            hi = np.clip(np.searchsorted(g, a), 1, g.size - 1)
+            q = np.where(g[hi] - a <= a - g[hi - 1], g[hi], g[hi - 1])
+            return np.copysign(q, y)
+        monkeypatch.setattr(O, "e4m3_round", away)
+    elif mutant == "e4m3_two_mantissa_bits":
+        def grid2():
+            vals = [m * 2.0 ** -8 for m in range(4)]
+            for e in range(1, 16):
+                for m in range(4):
+                    vals.append(2.0 ** (e - 7) * (1 + m / 4))
+            return np.array(vals)
+        monkeypatch.setattr(O, "e4m3_grid", grid2)
+    elif mutant == "fp8_key_scale_dropped":
+        def no_kscale(q_row, keys, w_row, scale):
+            qc, qs = O.fp8_quantize(q_row)
+            kc, ks = O.fp8_quantize(keys)
+            act = np.maximum(0.0, float(scale) * qs[:, None] * (qc @ kc.T))
+            return (O.f64(w_row)[:, None] * act).sum(axis=0) + 0.0
+        monkeypatch.setattr(O, "index_scores_fp8_row", no_kscale)
     assert _run_pins() > 0, f"mutant {mutant} survived every pin"
