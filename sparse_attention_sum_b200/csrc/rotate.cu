@@ -5,11 +5,13 @@
 // their slot) and the K-shift commit (the cached key is H * concat(RoPE(k_pe,
 // pos), k_nope); NEOX RoPE without scaling)).
 //
-// One block per row (token).  Its first threads build the row's RoPE table,
-// cos and sin of pos * theta^(-2i/n_rope), in double precision, once for all
-// heads of the row.  Each warp then takes head vectors of `dim` values, up to
-// four at a time so their loads are in flight together: lane l holds values
-// l*E .. l*E+E-1 (E = dim/32) in registers, read with one vector load.
+// One block per row (token).  Each warp takes head vectors of `dim` values, up
+// to four at a time so their loads are in flight together: lane l holds values
+// l*E .. l*E+E-1 (E = dim/32) in registers, read with one vector load.  While
+// the first loads are in flight, the block builds the row's RoPE table: the
+// angle pos * f_i (f_i = theta^(-2i/n_rope), computed once on the host in
+// double) is reduced modulo 2*pi in double, so the fp32 sine and cosine see an
+// argument in [-pi, pi] whatever the position.
 //   LayerNorm: a warp sum for the mean, then one for the biased variance of the
 //     centred values.
 //   NEOX RoPE: value d < n_rope/2 pairs with d + n_rope/2, which lives
@@ -30,7 +32,11 @@ namespace {
 constexpr int kRotWarps = 8;  // warps per block (fewer when a row has fewer heads)
 constexpr int kRotBatch = 4;  // head vectors per warp in flight
 
+constexpr double kTwoPi = 6.283185307179586;      // 2*pi rounded to double
+constexpr double kInvTwoPi = 0.15915494309189535;  // 1/(2*pi) rounded to double
+
 struct RotParams {
+  double inv_freq[64];  // theta^(-2i/n_rope), i < n_rope/2
   const void* in;
   void* out;
   const int32_t* pos;
@@ -39,7 +45,7 @@ struct RotParams {
   const float* ln_b;
   int64_t in_stride, out_stride, out_cap;
   int heads, n_rope, layer_norm, hadamard;
-  float theta, eps, hscale;
+  float eps, hscale;
 };
 
 template <int E>
@@ -99,29 +105,37 @@ __device__ __forceinline__ void store_vals(bf16* p, const float (&v)[E]) {
 
 template <typename Tin, typename Tout, int E>
 __global__ void __launch_bounds__(kRotWarps * 32)
-index_rotate_kernel(RotParams p) {
+index_rotate_kernel(const __grid_constant__ RotParams p) {
   constexpr int D = 32 * E;
   __shared__ float2 tab[D / 2];  // (cos, sin) of each RoPE pair
   const int r = blockIdx.x;
   const int half = p.n_rope >> 1;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int d0 = lane * E;
+  // no __restrict__: an exactly in-place call reads and writes the same vectors
+  const Tin* src = static_cast<const Tin*>(p.in) + (int64_t)r * p.in_stride + d0;
+
+  // first batch of head vectors: loads in flight while the table is built
+  float v[kRotBatch][E];
+#pragma unroll
+  for (int u = 0; u < kRotBatch; ++u) {
+    const int h = warp + u * nwarps;
+    if (h < p.heads) load_vals<E>(src + (int64_t)h * D, v[u]);
+  }
   if (half > 0) {
     const double pos = (double)p.pos[r];
-    const double log2_theta = log2((double)p.theta);
     for (int i = threadIdx.x; i < half; i += blockDim.x) {
-      double s, c;
-      sincos(pos * exp2(-(2.0 * i / p.n_rope) * log2_theta), &s, &c);
-      tab[i] = make_float2((float)c, (float)s);
+      const double a = pos * p.inv_freq[i];
+      const double red = fma(-rint(a * kInvTwoPi), kTwoPi, a);  // a - 2*pi*k, |red| <= pi
+      float s, c;
+      sincosf((float)red, &s, &c);
+      tab[i] = make_float2(c, s);
     }
   }
   __syncthreads();
 
   const int64_t dst = p.out_rows ? (int64_t)p.out_rows[r] : (int64_t)r;
   if (dst < 0 || dst >= p.out_cap) return;  // block-uniform; no barrier follows
-
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int d0 = lane * E;
-  // no __restrict__: an exactly in-place call reads and writes the same vectors
-  const Tin* src = static_cast<const Tin*>(p.in) + (int64_t)r * p.in_stride + d0;
   Tout* dstp = static_cast<Tout*>(p.out) + dst * p.out_stride + d0;
 
   float lw[E], lb[E];
@@ -134,11 +148,12 @@ index_rotate_kernel(RotParams p) {
   const bool first_half = d0 < half, second_half = d0 >= half && d0 < p.n_rope;
 
   for (int h0 = warp; h0 < p.heads; h0 += nwarps * kRotBatch) {
-    float v[kRotBatch][E];
+    if (h0 != warp) {
 #pragma unroll
-    for (int u = 0; u < kRotBatch; ++u) {
-      const int h = h0 + u * nwarps;
-      if (h < p.heads) load_vals<E>(src + (int64_t)h * D, v[u]);
+      for (int u = 0; u < kRotBatch; ++u) {
+        const int h = h0 + u * nwarps;
+        if (h < p.heads) load_vals<E>(src + (int64_t)h * D, v[u]);
+      }
     }
 #pragma unroll
     for (int u = 0; u < kRotBatch; ++u) {
@@ -230,6 +245,7 @@ cudaError_t launch_index_rotate(int n_rows, int heads, int dim, int n_rope, floa
                                 int64_t out_cap, cudaStream_t st) {
   if (n_rows == 0) return cudaSuccess;
   RotParams p;
+  for (int i = 0; i < 64; ++i) p.inv_freq[i] = i < n_rope / 2 ? pow((double)theta, -2.0 * i / n_rope) : 0.0;
   p.in = in;
   p.out = out;
   p.pos = pos;
@@ -243,7 +259,6 @@ cudaError_t launch_index_rotate(int n_rows, int heads, int dim, int n_rope, floa
   p.n_rope = n_rope;
   p.layer_norm = layer_norm ? 1 : 0;
   p.hadamard = hadamard ? 1 : 0;
-  p.theta = theta;
   p.eps = eps;
   p.hscale = (float)(1.0 / sqrt((double)dim));
   if (in_bf16)
