@@ -2,6 +2,7 @@
 // Declarations and contracts: include/dsa.h.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <mutex>
@@ -96,7 +97,10 @@ dsa_status check_attend(const dsa_dims* d, const void* q, const void* k, int64_t
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-int g_policy = 0;  // 0: tensor-core kernels where the shape allows; 1: CUDA-core kernels only
+// 0: tensor-core kernels where the shape allows; 1: CUDA-core kernels only.  Read by every entry point,
+// possibly from several host threads while another sets it.
+std::atomic<int> g_policy{0};
+bool tc_policy() { return g_policy.load(std::memory_order_relaxed) == 0; }
 
 }  // namespace
 
@@ -177,9 +181,7 @@ const char* dsa_version(void) { return "libdsa 0.1 (sm_100a)"; }
  * the tensor-core kernels, 1 forces the CUDA-core kernels (used to compare the
  * two families on the same inputs).  Returns the previous policy. */
 int dsa_set_kernel_policy(int policy) {
-  int old = g_policy;
-  g_policy = policy == 1 ? 1 : 0;
-  return old;
+  return g_policy.exchange(policy == 1 ? 1 : 0, std::memory_order_relaxed);
 }
 
 size_t dsa_workspace_size(const dsa_dims* d, int op) {
@@ -201,7 +203,7 @@ dsa_status dsa_index_scores(const dsa_dims* d, const void* q_idx, const void* k_
   if ((s = check_visibility(q_pos, kv_start, kv_len))) return s;
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
-  if (g_policy == 0 && dsa::index_scores_tc_supported(*d)) {
+  if (tc_policy() && dsa::index_scores_tc_supported(*d)) {
     e = dsa::launch_index_scores_tc(*d, q_idx, k_idx, w, scale, q_pos, kv_start, kv_len, scores, st);
   } else {
     if (d->idx_dim > 256 || (int64_t)d->idx_heads * d->idx_dim > 16384)
@@ -250,7 +252,7 @@ dsa_status dsa_sparse_attend(const dsa_dims* d, const void* q, const void* k, in
   if (s) return s;
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
-  if (g_policy == 0 && dsa::attend_tc_supported(*d, k_row_stride, k, v, v_row_stride, width)) {
+  if (tc_policy() && dsa::attend_tc_supported(*d, k_row_stride, k, v, v_row_stride, width)) {
     e = dsa::launch_attend_tc(*d, q, k, k_row_stride, idx, width, scale, out, lse, st);
   } else {
     if (!dsa::attend_simt_supported(*d, width))
@@ -385,7 +387,7 @@ dsa_status dsa_absorb_q(const dsa_dims* d, const void* q, int32_t dq, const void
   dsa_status s = check_absorb(d, q, dq, w_uk, L, q_lat);
   if (s) return s;
   const int rows = d->batch * d->n_q;
-  cudaError_t e = g_policy == 0 && dsa::head_gemm_tc_supported(rows, d->heads, dq, L, q, w_uk, true, q_lat)
+  cudaError_t e = tc_policy() && dsa::head_gemm_tc_supported(rows, d->heads, dq, L, q, w_uk, true, q_lat)
                       ? dsa::launch_head_gemm_tc(rows, d->heads, dq, L, q, w_uk, true, q_lat, (cudaStream_t)stream)
                       : dsa::launch_head_gemm(rows, d->heads, dq, L, q, w_uk, true, q_lat, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "dsa_absorb_q launch");
@@ -397,7 +399,7 @@ dsa_status dsa_absorb_out(const dsa_dims* d, const void* o_lat, int32_t L, const
   dsa_status s = check_absorb(d, o_lat, L, w_uv, dv, out);
   if (s) return s;
   const int rows = d->batch * d->n_q;
-  cudaError_t e = g_policy == 0 && dsa::head_gemm_tc_supported(rows, d->heads, L, dv, o_lat, w_uv, false, out)
+  cudaError_t e = tc_policy() && dsa::head_gemm_tc_supported(rows, d->heads, L, dv, o_lat, w_uv, false, out)
                       ? dsa::launch_head_gemm_tc(rows, d->heads, L, dv, o_lat, w_uv, false, out, (cudaStream_t)stream)
                       : dsa::launch_head_gemm(rows, d->heads, L, dv, o_lat, w_uv, false, out, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "dsa_absorb_out launch");

@@ -175,3 +175,14 @@ int main(void) {
     assert "sm_100a" in version and status == "DSA_ERR_TIMEOUT"
     assert int(ws) == dsa.workspace_size(dsa.Dims(batch=2, n_q=3, n_kv=100, top_k=8), dsa.OP_LAYER_FORWARD)
     assert int(code) == 1 and "dims" in msg
+
+
+def test_kernel_policy_switch_returns_the_previous_setting(lib):
+    prev = dsa.set_kernel_policy(1)
+    try:
+        assert dsa.set_kernel_policy(0) == 1
+        assert dsa.set_kernel_policy(7) == 0      # anything but 1 selects the tensor-core family
+        assert dsa.set_kernel_policy(1) == 0
+        assert dsa.set_kernel_policy(1) == 1
+    finally:
+        dsa.set_kernel_policy(prev)
