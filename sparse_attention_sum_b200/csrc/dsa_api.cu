@@ -123,16 +123,17 @@ int* device_status_ptr() {
 void set_last_error(const char* msg) { g_last_error = msg; }
 
 int sm_count() {
-  static int cached[128] = {};
+  static std::atomic<int> cached[128];  // zero-initialised (static storage); several threads may fill a slot
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 128) return 148;
-  if (!cached[dev]) {
-    int n = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (!n) {
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cached[dev] = n > 0 ? n : 148;
+    if (n <= 0) n = 148;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
 }
 
 __global__ void wait_selftest_kernel(long long timeout_ns, int* status) {
