@@ -117,9 +117,15 @@ def lib():
     return _lib
 
 
-def _ptr(t) -> Optional[int]:
+def _ptr(t, dense: bool = True) -> Optional[int]:
+    """Device address of tensor ``t``.  The C ABI reads dense row-major arrays except where a row-stride
+    argument accompanies the pointer (``dense=False``: only the innermost axis must be contiguous)."""
     if t is None:
         return None
+    if dense and not t.is_contiguous():
+        raise ValueError("libdsa entry points take contiguous tensors (row-major, no gaps) for this argument")
+    if not dense and t.dim() > 0 and t.stride(-1) != 1:
+        raise ValueError("the innermost axis of a strided argument must be contiguous")
     if not t.is_cuda:
         raise ValueError("libdsa entry points take CUDA tensors")
     return t.data_ptr()
@@ -177,7 +183,7 @@ def topk_set(dims: Dims, scores, q_pos, kv_start, kv_len, k: int, idx, vals=None
 
 def sparse_attend(dims: Dims, q, k, k_row_stride: int, v, v_row_stride: int, idx, width: int,
                   scale: float, out, lse=None, stream=None):
-    _check(lib().dsa_sparse_attend(ctypes.byref(dims), _ptr(q), _ptr(k), int(k_row_stride), _ptr(v),
+    _check(lib().dsa_sparse_attend(ctypes.byref(dims), _ptr(q), _ptr(k, False), int(k_row_stride), _ptr(v, False),
                                    int(v_row_stride), _ptr(idx), int(width), scale, _ptr(out),
                                    _ptr(lse), _stream(stream)), "dsa_sparse_attend")
 
@@ -187,8 +193,8 @@ def layer_forward(dims: Dims, q_idx, k_idx, w, idx_scale: float, q_pos, kv_start
                   idx_in=None, idx_out=None, ws=None, stream=None):
     wsb = 0 if ws is None else ws.numel() * ws.element_size()
     _check(lib().dsa_layer_forward(ctypes.byref(dims), _ptr(q_idx), _ptr(k_idx), _ptr(w), idx_scale,
-                                   _ptr(q_pos), _ptr(kv_start), _ptr(kv_len), _ptr(q), _ptr(k),
-                                   int(k_row_stride), _ptr(v), int(v_row_stride), attn_scale,
+                                   _ptr(q_pos), _ptr(kv_start), _ptr(kv_len), _ptr(q), _ptr(k, False),
+                                   int(k_row_stride), _ptr(v, False), int(v_row_stride), attn_scale,
                                    _ptr(idx_in), _ptr(idx_out), _ptr(out), _ptr(lse), _ptr(ws), wsb,
                                    _stream(stream)), "dsa_layer_forward")
 
@@ -198,8 +204,8 @@ def layer_forward_static(dims: Dims, q_idx, k_idx, w, idx_scale: float, q_pos, k
                          idx_in=None, idx_out=None, stream=None):
     """dsa_layer_forward with the library's fixed scratch array (no workspace argument)."""
     _check(lib().dsa_layer_forward_static(ctypes.byref(dims), _ptr(q_idx), _ptr(k_idx), _ptr(w), idx_scale,
-                                          _ptr(q_pos), _ptr(kv_start), _ptr(kv_len), _ptr(q), _ptr(k),
-                                          int(k_row_stride), _ptr(v), int(v_row_stride), attn_scale,
+                                          _ptr(q_pos), _ptr(kv_start), _ptr(kv_len), _ptr(q), _ptr(k, False),
+                                          int(k_row_stride), _ptr(v, False), int(v_row_stride), attn_scale,
                                           _ptr(idx_in), _ptr(idx_out), _ptr(out), _ptr(lse), _stream(stream)),
            "dsa_layer_forward_static")
 
@@ -242,8 +248,9 @@ def index_rotate(x, out, n_rope: int, rope_theta: float, pos=None, layer_norm: b
     n_rows, heads, dim = x.shape
     _check(lib().dsa_index_rotate(int(n_rows), int(heads), int(dim), int(n_rope), float(rope_theta),
                                   int(bool(layer_norm)), _ptr(ln_w), _ptr(ln_b), float(ln_eps), int(bool(hadamard)),
-                                  _ptr(pos), _dtype_code(x), _ptr(x), int(x.stride(0)), _dtype_code(out), _ptr(out),
-                                  int(out.stride(0)), _ptr(out_rows), int(out.shape[0]), _stream(stream)),
+                                  _ptr(pos), _dtype_code(x), _ptr(x, False), int(x.stride(0)), _dtype_code(out),
+                                  _ptr(out, False), int(out.stride(0)), _ptr(out_rows), int(out.shape[0]),
+                                  _stream(stream)),
            "dsa_index_rotate")
 
 

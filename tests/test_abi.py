@@ -186,3 +186,14 @@ def test_kernel_policy_switch_returns_the_previous_setting(lib):
         assert dsa.set_kernel_policy(1) == 1
     finally:
         dsa.set_kernel_policy(prev)
+
+
+def test_binding_rejects_non_contiguous_dense_arguments():
+    import torch
+    with pytest.raises(ValueError, match="contiguous"):
+        dsa._ptr(torch.zeros(4, 6).t())                 # transposed view for a dense argument
+    with pytest.raises(ValueError, match="innermost"):
+        dsa._ptr(torch.zeros(4, 6)[:, ::2], dense=False)  # strided rows still need unit inner stride
+    with pytest.raises(ValueError, match="CUDA"):
+        dsa._ptr(torch.zeros(4, 6)[:, :3], dense=False)   # a row-strided view passes the layout check
+    assert dsa._ptr(None) is None
