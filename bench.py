@@ -361,6 +361,9 @@ def run_ours(a):
         "gpu_launches": 3 * a.steps,
         "clocks": clk.summary(),
     }
+    if not a.no_extras:
+        # every rank: end to end through the public API on its own replica (collective: barrier, max)
+        line["e2e"] = e2e_measure(wl, a.steps, stream, world)
     if rank == 0 and not a.no_extras:
         st = stage_times(wl, t, dims, args, bufs, 5, flush, stream)
         step_med = statistics.median(times)
@@ -377,6 +380,7 @@ def run_ours(a):
             "topk": roofline_entry("hbm", wk["topk_bytes"], st["topk"], peaks, tr.get(f"topk:{wl.name}")),
             "attend": roofline_entry("tensor", wk["attend_flop"], st["attend"], peaks, traffic),
         }
+    if rank == 0 and not a.no_extras and world == 1:
         # IndexShare: a layer that reuses an earlier layer's selection runs only the attend.  On the
         # 78-layer stack the pages describe, layers 0, 1 and every il % 4 == 2 compute their own (21 of 78).
         shared = time_steps(lambda: runner.dsa_layer(dims, **args, bufs=bufs, idx_in=bufs.idx), max(3, a.steps // 2),
@@ -387,7 +391,6 @@ def run_ours(a):
         line["indexshare"] = {"shared_layer_ms": round(shared_ms, 4), "full_layer_ms": round(full_ms, 4),
                               "layers_full_of_78": n_full, "stack_avg_layer_ms": round(stack_ms, 4),
                               "stack_avg_value": round(rows / (stack_ms / 1e3), 1), "unit": UNIT}
-        line["e2e"] = e2e_measure(wl, a.steps, stream)
         if a.workload == "prefill":
             line["decode"] = decode_extra(peaks, flush, stream)
             line["chunked"] = chunked_extra(peaks, flush, stream)
@@ -402,12 +405,14 @@ def run_ours(a):
         dist.destroy_process_group()
 
 
-def e2e_measure(wl, steps, stream):
+def e2e_measure(wl, steps, stream, world=1):
     """Same metric through the public API with host buffers.  Every step copies its inputs from
     pinned host memory to the device, runs the fused layer and reads its output back to pinned
     host memory, all inside the timed region.  Steps are pipelined the way a serving loop runs
     them: step i+1's upload (one copy stream) overlaps step i's layer (the compute stream) and
-    step i-1's download (a second copy stream); two device buffer sets alternate."""
+    step i-1's download (a second copy stream); two device buffer sets alternate.  With several
+    ranks each runs its own replica between barriers; the rate is the whole job's over the
+    slowest rank."""
     from sparse_attention_sum_b200 import runner
     host = {k: v.pin_memory() for k, v in wl.tensors.items()}
     sets = []
@@ -446,6 +451,7 @@ def e2e_measure(wl, steps, stream):
 
     run(2)
     torch.cuda.synchronize()
+    barrier(world)
     n = max(4, min(steps, 10))
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -454,8 +460,8 @@ def e2e_measure(wl, steps, stream):
     down.wait_event(computed[(n - 1) & 1])
     e1.record(down)
     e1.synchronize()
-    sec = e0.elapsed_time(e1) / 1e3 / n
-    return {"value": round(wl.batch * wl.n_q / sec, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+    sec = max_over_ranks(e0.elapsed_time(e1) / 1e3 / n, world)
+    return {"value": round(world * wl.batch * wl.n_q / sec, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": round(sec * 1e3, 3),
             "pipelined": "upload of step i+1 and download of step i-1 overlap step i's layer"}
 
