@@ -4,6 +4,9 @@ Usage: ``python -m sparse_attention_sum_b200.build [--jobs N] [--force]``.
 Each ``csrc/*.cu`` file compiles to an object under ``_build/`` and the
 objects link into ``sparse_attention_sum_b200/libdsa.so``.  A file is rebuilt
 when it or any header under ``csrc/`` or ``include/`` is newer than its object.
+Each source's compiler output (ptxas register and spill report, warnings) is
+kept in ``_build/<name>.log`` and ``_build/ptxas.log`` is their concatenation
+for the current objects.
 """
 from __future__ import annotations
 
@@ -56,11 +59,11 @@ def build(jobs: int = 8, force: bool = False, verbose: bool = False) -> str:
         objs.append(o)
         if force or not os.path.exists(o) or os.path.getmtime(o) < max(os.path.getmtime(s), hdr_mtime):
             todo.append((s, o))
-    logs = []
     if todo:
         with cf.ThreadPoolExecutor(max_workers=jobs) as ex:
             for src, rc, out in ex.map(lambda so: _compile(*so), todo):
-                logs.append(out)
+                with open(os.path.join(BUILD, os.path.basename(src)[:-3] + ".log"), "w") as f:
+                    f.write(out)
                 if rc != 0:
                     raise RuntimeError(f"nvcc failed for {os.path.basename(src)}:\n{out}")
                 if verbose:
@@ -75,8 +78,11 @@ def build(jobs: int = 8, force: bool = False, verbose: bool = False) -> str:
         if p.returncode != 0:
             raise RuntimeError(f"link failed:\n{p.stdout}{p.stderr}")
         os.replace(tmp, LIB)
-    with open(os.path.join(BUILD, "ptxas.log"), "a") as f:
-        f.write("\n".join(logs))
+    with open(os.path.join(BUILD, "ptxas.log"), "w") as f:
+        for s in srcs:
+            log = os.path.join(BUILD, os.path.basename(s)[:-3] + ".log")
+            if os.path.exists(log):
+                f.write(f"== {os.path.basename(s)}\n" + open(log).read())
     return LIB
 
 
