@@ -263,9 +263,11 @@ def roofline_entry(kind, amount, seconds, peaks, traffic=None):
     if kind == "tensor":
         achieved = amount / seconds / 1e12
         peak = peaks["bf16_tflops"]
+        sustained = peaks["bf16_tflops_sustained"]
         return {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
-                "peak_source": peaks["source"] + " (burst)"}
+                "peak_source": peaks["source"] + " (burst)",
+                "peak_sustained": sustained, "frac_sustained": round(achieved / sustained, 4)}
     achieved = amount / seconds / 1e9
     peak = peaks["hbm_gbs"]
     return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",

@@ -72,8 +72,9 @@ def test_clock_summary_reports_median_max_and_reasons():
 
 
 def test_roofline_entry_fractions():
-    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0, "source": "measured"}
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0, "bf16_tflops_sustained": 1250.0, "source": "measured"}
     r = bench.roofline_entry("tensor", 1.5e12, 2e-3, peaks)
     assert r["bound"] == "tensor" and abs(r["achieved"] - 750.0) < 1e-6 and abs(r["frac"] - 0.5) < 1e-9
+    assert r["peak_sustained"] == 1250.0 and abs(r["frac_sustained"] - 0.6) < 1e-9
     r = bench.roofline_entry("hbm", 3e9, 1e-3, peaks, traffic=123)
     assert r["unit"] == "GB/s" and abs(r["frac"] - 0.5) < 1e-9 and r["traffic"] == 123
