@@ -12,10 +12,14 @@
 // whose low 20 bits are resolved alone (12 + 8 bits).  That gives the exact
 // k-th largest key tau and how many keys equal to tau are still needed.  A
 // crowded bin (many equal scores) falls back to four 8-bit passes over the
-// row (shared atomics aggregated per warp with ballots).  Each warp
-// then walks a contiguous segment of the row 32 keys at a time; ballots and a
-// block-wide prefix sum place every key > tau and the lowest-index keys == tau,
-// which keeps the tie rule exact.  Finally the (key, index) pairs are put in
+// row (shared atomics aggregated per warp with ballots).  Each warp owns a
+// contiguous segment of the row, walked 32 keys at a time.  The pass that
+// collects the candidates also counts, per warp, the keys above the bin, and
+// tags each candidate with its warp, so the per-warp counts of keys > tau and
+// == tau come from the candidates without another pass over the row (the
+// crowded-bin path counts them in one more pass).  Ballots and a block-wide
+// prefix sum of those counts place every key > tau and the lowest-index keys
+// == tau, which keeps the tie rule exact.  Finally the (key, index) pairs are put in
 // rank order by a stable four-pass LSD radix sort on the key (descending), so
 // equal keys keep ascending index order.
 //
