@@ -6,6 +6,7 @@
  *   (2) deterministic top-k        higher score first, then smaller key index
  *   (3) sparse MLA attention       softmax(scale * q . K[i]) V[i] over the selected keys only
  *   (+) kpool variant              pooled indexer keys, pool selection expanded to tokens
+ *   (+) indexer q/k preparation    key LayerNorm, NEOX RoPE, Walsh-Hadamard rotation, cache store
  *
  * Sources: the fak note "GLM-5.2: the DSA sparse attention moves onto the pure
  * fak kernel" (score formula in section 3, the sparse attend in "What
