@@ -363,6 +363,9 @@ def test_sylvester_hadamard_matches_scipy_and_is_orthonormal():
     assert abs(hx @ hy - x @ y) < 1e-12 and abs(np.linalg.norm(hx) - np.linalg.norm(x)) < 1e-12
     with pytest.raises(ValueError):
         O.sylvester_hadamard(48)
+    # worked by hand: H_4 (1, 2, 3, 4) = (10, -2, -4, 0), and the orthonormal rotation halves it
+    assert O.hadamard_rotate(np.array([1.0, 2.0, 3.0, 4.0])).tolist() == [5.0, -1.0, -2.0, 0.0]
+    assert O.hadamard_rotate(np.array([[0.0, 0.0, 0.0, 2.0]])).tolist() == [[1.0, -1.0, -1.0, 1.0]]
 
 
 def _rot_inputs(seed=15):
