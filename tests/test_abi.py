@@ -102,6 +102,23 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert st == 2 and "bf16" in msg
     st, msg = _call(lib.dsa_selftest_wait_timeout, 5, nul)
     assert st == 1
+    # the key-ordered top-k validates like dsa_topk
+    st, msg = _call(lib.dsa_topk_set, ctypes.byref(d), p, p, p, p, 0, p, nul, nul)
+    assert st == 1 and "k must be" in msg
+    st, msg = _call(lib.dsa_topk_set, ctypes.byref(d), p, nul, p, p, 4, p, nul, nul)
+    assert st == 1 and "q_pos" in msg
+    st, msg = _call(lib.dsa_absorb_out, ctypes.byref(f32), p, 32, p, 16, p, nul)
+    assert st == 2 and "bf16" in msg
+    # the allocation-free layer: dims checked, and a layer needing more than the fixed 16 MiB refused,
+    # before any device call
+    args = (p, p, p, 1.0, p, p, p, p, p, 16, p, 16, 1.0, nul, nul, p, nul, nul)
+    st, msg = _call(lib.dsa_layer_forward_static, None, *args)
+    assert st == 1 and "dims" in msg
+    st, msg = _call(lib.dsa_layer_forward_static, ctypes.byref(dsa.Dims(batch=0, n_q=1, n_kv=1, top_k=1)), *args)
+    assert st == 1
+    big = dsa.Dims(**{**d.as_dict(), "n_q": 4096, "n_kv": 4096, "top_k": 2048})
+    st, msg = _call(lib.dsa_layer_forward_static, ctypes.byref(big), *args)
+    assert st == 3 and "16 MiB" in msg
 
 
 def test_index_rotate_host_validation(lib):
