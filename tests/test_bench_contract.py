@@ -78,3 +78,17 @@ def test_roofline_entry_fractions():
     assert r["peak_sustained"] == 1250.0 and abs(r["frac_sustained"] - 0.6) < 1e-9
     r = bench.roofline_entry("hbm", 3e9, 1e-3, peaks, traffic=123)
     assert r["unit"] == "GB/s" and abs(r["frac"] - 0.5) < 1e-9 and r["traffic"] == 123
+
+
+def test_every_profile_summary_gives_its_ncu_command():
+    """Each ncu summary names the command that made it, with the clocks left alone, and runs committed files."""
+    import glob
+    summaries = glob.glob(os.path.join(ROOT, "profiles", "*.md"))
+    assert summaries
+    for path in summaries:
+        text = open(path).read()
+        cmds = [ln for ln in text.splitlines() if ln.strip().startswith("ncu ")]
+        assert cmds, f"{path}: no ncu command"
+        for c in cmds:
+            assert "--clock-control none" in c, f"{path}: {c}"
+        assert "_work/" not in text, f"{path} refers to working files"
