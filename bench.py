@@ -360,7 +360,7 @@ def run_ours(a):
                                f"indexer {wl.idx_heads}x{wl.idx_dim}, MLA H={wl.heads} kd={wl.kd} vd={wl.vd}",
                    "l2": "flushed (256 MiB write) before every timed step",
                    "parallelism": f"replicas x{world} (one independent problem per GPU)"},
-        "gpu_launches": 3 * a.steps,
+        "gpu_launches": 3 * a.steps,   # index, top-k set, attend per fused layer step
         "clocks": clk.summary(),
     }
     if not a.no_extras:
@@ -377,6 +377,7 @@ def run_ours(a):
         traffic = tr.get(f"attend:{wl.name}")
         line["roofline"] = roofline_entry("tensor", wk["attend_flop"], st["attend"], peaks, traffic)
         line["roofline"]["kernel"] = "sparse attend (dsa_sparse_attend)"
+        line["fp8_indexer"] = fp8_indexer_extra(wl, t, dims, args, bufs, peaks, flush, stream, 5)
         line["roofline_stages"] = {
             "index": roofline_entry("tensor", wk["index_flop"], st["index"], peaks, tr.get(f"index:{wl.name}")),
             "topk": roofline_entry("hbm", wk["topk_bytes"], st["topk"], peaks, tr.get(f"topk:{wl.name}")),
@@ -388,15 +389,15 @@ def run_ours(a):
         shared = time_steps(lambda: runner.dsa_layer(dims, **args, bufs=bufs, idx_in=bufs.idx), max(3, a.steps // 2),
                             3, flush, stream)
         full_ms, shared_ms = statistics.median(times) * 1e3, statistics.median(shared) * 1e3
-        n_full = sum(1 for il in range(78) if il <= 1 or il % 4 == 2)
+        n_full = sum(1 for il in range(78) if runner.computes_own_selection(il))
         stack_ms = (n_full * full_ms + (78 - n_full) * shared_ms) / 78
         line["indexshare"] = {"shared_layer_ms": round(shared_ms, 4), "full_layer_ms": round(full_ms, 4),
                               "layers_full_of_78": n_full, "stack_avg_layer_ms": round(stack_ms, 4),
                               "stack_avg_value": round(rows / (stack_ms / 1e3), 1), "unit": UNIT}
         if a.workload == "prefill":
-            line["decode"] = decode_extra(peaks, flush, stream)
-            line["chunked"] = chunked_extra(peaks, flush, stream)
-            line["kpool"] = kpool_extra(peaks, flush, stream)
+            line["decode"] = decode_extra(peaks, flush, stream, a.cpu_seconds / 2)
+            line["chunked"] = chunked_extra(peaks, flush, stream, a.cpu_seconds / 3)
+            line["kpool"] = kpool_extra(peaks, flush, stream, a.cpu_seconds / 3)
             line["rotate"] = rotate_extra(peaks, flush, stream)
         line["cpu_baseline"] = cpu_baseline(wl, budget_s=a.cpu_seconds)
     if rank == 0:
@@ -468,7 +469,44 @@ def e2e_measure(wl, steps, stream, world=1):
             "pipelined": "upload of step i+1 and download of step i-1 overlap step i's layer"}
 
 
-def decode_extra(peaks, flush, stream):
+def fp8_indexer_extra(wl, t, dims, args, bufs, peaks, flush, stream, steps):
+    """The FP8 indexer on this workload: keys quantised once (a cache holds them as e4m3 codes), then per
+    step the queries are quantised and scored (dsa_fp8_quantize + dsa_index_scores_fp8), and the layer
+    chain runner.dsa_layer_fp8 (quantise, FP8 scores, top-k set, attend) is timed whole."""
+    import sparse_attention_sum_b200 as dsa
+    from sparse_attention_sum_b200 import runner
+    B, T, S = wl.batch, wl.n_q, wl.n_kv
+    k_codes = torch.empty(B, S, 128, dtype=torch.uint8, device="cuda")
+    k_scales = torch.empty(B, S, dtype=torch.float32, device="cuda")
+    dsa.fp8_quantize(t["k_idx"], k_codes, k_scales)
+    fp8 = runner.Fp8Buffers(dims, "cuda")
+    scores = bufs.ws[: B * T * S * 4].view(torch.float32)
+    quant = lambda: dsa.fp8_quantize(t["q_idx"], fp8.q_codes, fp8.q_scales)
+    index = lambda: dsa.index_scores_fp8(dims, fp8.q_codes, fp8.q_scales, k_codes, k_scales, args["w"],
+                                         args["idx_scale"], args["q_pos"], args["kv_start"], args["kv_len"], scores)
+    t_quant = statistics.median(time_steps(quant, max(3, steps), 2, flush, stream))
+    t_index = statistics.median(time_steps(index, max(3, steps), 2, flush, stream))
+    layer = statistics.median(time_steps(
+        lambda: runner.dsa_layer_fp8(dims, k_codes=k_codes, k_scales=k_scales, bufs=bufs, fp8=fp8, **args),
+        max(3, steps), 3, flush, stream))
+    nvis = visible_counts(wl)
+    pairs = int(nvis.sum())
+    rows = B * T
+    fp8_peaks = dict(peaks, bf16_tflops=2 * peaks["bf16_tflops"],
+                     bf16_tflops_sustained=2 * peaks["bf16_tflops_sustained"],
+                     source=peaks["source"] + " bf16 x 2 (dense e4m3 : bf16 nominal ratio)")
+    idx_bytes = B * S * (128 + 4) + rows * wl.idx_heads * (128 + 4 + 4) + 4.0 * pairs
+    res = {"layer_ms": round(layer * 1e3, 4), "value": round(rows / layer, 1), "unit": UNIT,
+           "stages_us": {"quantize_q": round(t_quant * 1e6, 2), "index_fp8": round(t_index * 1e6, 1)},
+           "roofline_index_fp8": roofline_entry("tensor", 2.0 * pairs * wl.idx_heads * wl.idx_dim, t_index,
+                                                fp8_peaks),
+           "roofline_index_fp8_hbm": roofline_entry("hbm", idx_bytes, t_index, peaks),
+           "roofline_quantize_q": roofline_entry("hbm", rows * wl.idx_heads * (256 + 128 + 4), t_quant, peaks)}
+    del k_codes, k_scales, fp8
+    return res
+
+
+def decode_extra(peaks, flush, stream, cpu_s=0.0):
     """The decode workload (64 sequences x 1 query vs 32768 cached keys) and its stages."""
     from sparse_attention_sum_b200 import runner
     wl = workloads.make("decode")
@@ -488,12 +526,15 @@ def decode_extra(peaks, flush, stream):
                                             profiled_traffic().get("index:decode")),
            "fused_hbm_frac": round((wk["index_bytes"] + wk["topk_bytes"] + wk["attend_bytes"]) / step / 1e9
                                    / peaks["hbm_gbs"], 4)}
+    res["fp8_indexer"] = fp8_indexer_extra(wl, t, dims, args, bufs, peaks, flush, stream, 10)
+    if cpu_s > 0:
+        res["cpu_baseline"] = cpu_baseline(wl, budget_s=cpu_s, whole=True)
     del t, bufs
     torch.cuda.empty_cache()
     return res
 
 
-def chunked_extra(peaks, flush, stream):
+def chunked_extra(peaks, flush, stream, cpu_s=0.0):
     """Chunked prefill: 4096 queries at positions 28672..32767 against 32768 keys (hot-spot keys)."""
     from sparse_attention_sum_b200 import runner
     wl = workloads.make("chunked")
@@ -511,12 +552,14 @@ def chunked_extra(peaks, flush, stream):
            "roofline_index": roofline_entry("tensor", wk["index_flop"], st["index"], peaks),
            "roofline_attend": roofline_entry("tensor", wk["attend_flop"], st["attend"], peaks),
            "fused_tensor_frac": round((wk["index_flop"] + wk["attend_flop"]) / step / 1e12 / peaks["bf16_tflops"], 4)}
+    if cpu_s > 0:
+        res["cpu_baseline"] = cpu_baseline(wl, budget_s=cpu_s)
     del t, bufs
     torch.cuda.empty_cache()
     return res
 
 
-def kpool_extra(peaks, flush, stream):
+def kpool_extra(peaks, flush, stream, cpu_s=0.0):
     """The kpool NoPE layer (4 sequences x 8192 tokens, left padding, kpool 4, select_k 512, H=64
     absorbed into a 512-wide latent): every call of the chain timed alone, and the whole chain."""
     import sparse_attention_sum_b200 as dsa
@@ -564,6 +607,8 @@ def kpool_extra(peaks, flush, stream):
            "roofline_attend": roofline_entry("tensor", flop["attend"], st["attend"], peaks),
            "roofline_absorb": roofline_entry("tensor", flop["absorb"], st["absorb_q"] + st["absorb_out"], peaks),
            "fused_tensor_frac": round(sum(flop.values()) / step / 1e12 / peaks["bf16_tflops"], 4)}
+    if cpu_s > 0:
+        res["cpu_baseline"] = cpu_baseline(wl, budget_s=cpu_s, row_fn=oracle_kpool_rows)
     del t, bufs
     torch.cuda.empty_cache()
     return res
@@ -612,6 +657,25 @@ def oracle_rows(wl, rows):
         O.layer_row(b, t, ts, wl.top_k, wl.idx_scale, wl.attn_scale, wl["q"], K, V)
 
 
+def oracle_kpool_rows(wl, rows, _pooled={}):
+    """The kpool layer row by row in the oracle: pooled keys of the row's sequence (once per
+    sequence), pool scores and top-k, expand_selection, then the literal expand_kv attention."""
+    from oracle import dsa_oracle as O
+    for b, t in rows:
+        f, L = int(wl["kv_start"][b]), int(wl["kv_len"][b])
+        key = (id(wl), b)
+        if key not in _pooled:
+            _pooled[key] = O.pool_states(wl["k_raw"][b], wl["gate"][b], f, L, wl.kpool, wl["ln_w"], wl["ln_b"],
+                                         wl.ln_eps)
+        pooled = _pooled[key]
+        p = int(wl["q_pos"][b, t])
+        sel, _ = O.topk_pools_row(wl["q_idx"][b, t], pooled, wl["w"][b, t], wl.idx_scale, p, f, pooled.shape[0],
+                                  wl.kpool, wl.select_k)
+        tok = O.expand_selection(sel, p, f, L, wl.kpool, pooled.shape[0], wl.out_width)
+        O.mla_masked_attention_row(wl["q_nope"][b, t], wl["latent"][b], wl["w_uk"], wl["w_uv"], tok,
+                                   wl.attn_scale)
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -623,17 +687,26 @@ def blas_threads():
     return len(os.sched_getaffinity(0))
 
 
-def cpu_baseline(wl, budget_s=15.0):
-    """Oracle query rows per second on this host, on a bounded stratified sample."""
+def cpu_baseline(wl, budget_s=15.0, whole=False, row_fn=None):
+    """Oracle query rows per second on this host: every row of the workload when ``whole`` (decode),
+    else a bounded stratified sample (first, last and top-k boundary row of every sequence, then random
+    rows until the time budget is spent)."""
     import random
+    row_fn = row_fn or oracle_rows
     T = wl.n_q
     rnd = random.Random(0)
-    order = [(b, t) for b in range(wl.batch) for t in (0, T - 1, min(T - 1, wl.top_k))]
     t0 = time.perf_counter()
+    if whole:
+        rows = [(b, t) for b in range(wl.batch) for t in range(T)]
+        row_fn(wl, rows)
+        el = time.perf_counter() - t0
+        return {"value": round(len(rows) / el, 3), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                "sample": f"all {len(rows)} query rows of {wl.name}, {el:.1f} s, f64 numpy oracle"}
+    order = [(b, t) for b in range(wl.batch) for t in (0, T - 1, min(T - 1, wl.top_k))]
     done = 0
     while time.perf_counter() - t0 < budget_s and done < 4096:
         batch = order if done == 0 else [(rnd.randrange(wl.batch), rnd.randrange(T)) for _ in range(4)]
-        oracle_rows(wl, batch)
+        row_fn(wl, batch)
         done += len(batch)
     el = time.perf_counter() - t0
     return {"value": round(done / el, 3), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",

@@ -100,6 +100,17 @@ const char* dsa_last_error(void);
 /* Library version string (static storage). */
 const char* dsa_version(void);
 
+/* Kernels launched by the most recent top-level entry point call on this host
+ * thread, comma-separated in launch order, e.g. "index_tc,topk_set,attend_tc"
+ * for a fused layer on the tensor cores; "" if that call launched nothing.
+ * Family names: index_tc / index_simt / index_tc_fp8 and fp8_quantize (S2),
+ * topk_ranked / topk_set (S3), index_topk / index_topk_fp8 (S2 + S3 fused),
+ * attend_tc / attend_simt (S4), pool_states, expand_selection, head_gemm_tc /
+ * head_gemm_simt (S8), index_rotate, wait_selftest.  Shows which kernel served a
+ * shape that more than one kernel implements (see dsa_sparse_attend).  Thread-local
+ * storage, valid until the next entry point call on the same thread. */
+const char* dsa_last_kernels(void);
+
 /* Kernel family for shapes that both the tensor-core and the CUDA-core
  * kernels implement: 0 (default) selects the tensor-core kernels, 1 the
  * CUDA-core kernels (to compare the two on the same inputs).  Process-wide;
@@ -131,6 +142,36 @@ dsa_status dsa_index_scores(const dsa_dims* dims, const void* q_idx, const void*
                             const int32_t* kv_start, const int32_t* kv_len, float* scores,
                             dsa_stream_t stream);
 
+/* S2 with FP8 operands, step 1: per-vector e4m3 quantisation.
+ * ik_llama.cpp PR #2063 (commit messages of #2045) ships the indexer tensors in
+ * F8_E4M3; the per-vector scaling is this library's reading of it.  Row r of x
+ * (dim values) gets scale s[r] = amax/448 (amax = max |x[r,:]|; 1 for a zero
+ * row) and codes[r,:] = e4m3(x[r,:] * fl(448/amax)), where fl() and the
+ * product round to fp32 and e4m3() rounds to nearest even (saturating at 448),
+ * so that x ~= codes * s.  Quantise queries as n_vectors = B*T*H_I rows of
+ * q_idx and keys as B*S rows of k_idx (once, when they enter the cache).
+ * x: n_vectors rows of dim values of in_dtype, x_row_stride values apart,
+ * aligned to 4 values.  codes: [n_vectors, dim] e4m3 bytes (dense), 4-byte
+ * aligned; scales: [n_vectors] fp32.  dim must be 128 (else DSA_ERR_UNSUPPORTED). */
+dsa_status dsa_fp8_quantize(int64_t n_vectors, int32_t dim, dsa_dtype in_dtype, const void* x,
+                            int64_t x_row_stride, void* codes, float* scales, dsa_stream_t stream);
+
+/* S2 with FP8 operands, step 2: lightning-indexer scores from e4m3 codes.
+ * I[b,t,s] = sum_h w[b,t,h] * relu(scale * sq[b,t,h] * sk[b,s] * (qc[b,t,h,:] . kc[b,s,:]))
+ * for visible s, -inf otherwise (the score of dsa_index_scores, fak note section 3,
+ * with the operands of dsa_fp8_quantize).  The code products accumulate in fp32 on
+ * the tensor cores (tcgen05 kind::f8f6f4).  A signed-zero score is written as +0.
+ * Reads dims: batch, n_q, n_kv, idx_heads, idx_dim, kpool.
+ * q_codes [B,T,H_I,128] e4m3, q_scales [B,T,H_I] fp32, k_codes [B,S,128] e4m3,
+ * k_scales [B,S] fp32, w [B,T,H_I] fp32, scores [B,T,S] fp32.  Codes 16-byte aligned.
+ * idx_dim must be 128 and idx_heads 32, 64 or 128, with batch*n_kv >= 128
+ * (else DSA_ERR_UNSUPPORTED).  The selection then runs on these scores with
+ * dsa_topk / dsa_topk_set as usual. */
+dsa_status dsa_index_scores_fp8(const dsa_dims* dims, const void* q_codes, const float* q_scales,
+                                const void* k_codes, const float* k_scales, const float* w, float scale,
+                                const int32_t* q_pos, const int32_t* kv_start, const int32_t* kv_len,
+                                float* scores, dsa_stream_t stream);
+
 /* S3 — deterministic top-k.
  * For each row (b,t): the min(k, n_visible) visible keys with the highest
  * score, ordered by higher score and then smaller key index, so ties resolve
@@ -158,6 +199,33 @@ dsa_status dsa_topk_set(const dsa_dims* dims, const float* scores, const int32_t
                         const int32_t* kv_start, const int32_t* kv_len, int32_t k, int32_t* idx,
                         float* vals, dsa_stream_t stream);
 
+/* S2 + S3 fused — the selection straight from the indexer inputs, without a
+ * score matrix in memory.  Selects exactly what dsa_index_scores followed by
+ * dsa_topk_set(k) select (the same scores, visibility and tie rule: fak note
+ * section 3, the selection is score dots plus a top-k; metrale topk_pools) and
+ * lists the keys in ascending key order, DSA_INVALID after them.  One cluster of
+ * up to 8 CTAs scores a query row on the tensor cores, keeps the scores in shared
+ * memory and selects them there (radix select over distributed shared memory), so
+ * only the index rows are written.  Meant for rows with few queries per sequence
+ * (decode): every query row reads its sequence's keys once.
+ * Reads dims: batch, n_q, n_kv, idx_heads, idx_dim, kpool (must be 0), dtype.
+ * q_idx [B,T,H_I,128] bf16, k_idx [B,S,128] bf16, w [B,T,H_I] fp32, idx [B,T,k]
+ * int32, 1 <= k <= 4096.  Requires bf16, idx_dim 128, idx_heads 32, 64 or 128
+ * and n_kv <= 131072 (else DSA_ERR_UNSUPPORTED). */
+dsa_status dsa_index_topk(const dsa_dims* dims, const void* q_idx, const void* k_idx, const float* w,
+                          float scale, const int32_t* q_pos, const int32_t* kv_start, const int32_t* kv_len,
+                          int32_t k, int32_t* idx, dsa_stream_t stream);
+
+/* S2 + S3 fused with FP8 operands: the selection dsa_index_scores_fp8 followed by
+ * dsa_topk_set(k) gives, computed as dsa_index_topk computes it (no score matrix
+ * in memory).  Arguments as in dsa_index_scores_fp8 (codes and scales of
+ * dsa_fp8_quantize, 16-byte aligned codes) plus k and idx [B,T,k] as in
+ * dsa_index_topk; the same requirements as dsa_index_topk. */
+dsa_status dsa_index_topk_fp8(const dsa_dims* dims, const void* q_codes, const float* q_scales,
+                              const void* k_codes, const float* k_scales, const float* w, float scale,
+                              const int32_t* q_pos, const int32_t* kv_start, const int32_t* kv_len,
+                              int32_t k, int32_t* idx, dsa_stream_t stream);
+
 /* S4 — sparse attention over the selected keys.
  * For every (b,t,h): U = the set of distinct entries i of idx[b,t,:] with
  * 0 <= i < S (duplicates collapse, DSA_INVALID and out-of-range entries are
@@ -175,8 +243,10 @@ dsa_status dsa_topk_set(const dsa_dims* dims, const float* scores, const int32_t
  * q [B,T,H,kd] dtype   idx [B,T,width] int32   out [B,T,H,vd] dtype
  * lse [B,T,H] fp32 or NULL.  Softmax and accumulation are fp32.
  * bf16 with kv_heads = 1 (V = the first vd columns of the K rows, same pointer and
- * stride), kd in {512, 576}, vd = 512, H in {64, 128}, n_kv <= 65536 and width up
- * to about 3400 runs on the tensor cores; other shapes run on the CUDA cores. */
+ * stride), kd in {512, 576}, vd = 512, H in {64, 128}, n_kv <= 294912 (with
+ * batch*n_kv < 2^31) and width up to about 3400 (2200 when n_kv > 65536) runs on
+ * the tensor cores; other shapes run on the CUDA cores, which dsa_last_kernels()
+ * reports as "attend_simt". */
 dsa_status dsa_sparse_attend(const dsa_dims* dims, const void* q, const void* k,
                              int64_t k_row_stride, const void* v, int64_t v_row_stride,
                              const int32_t* idx, int32_t width, float scale, void* out,
@@ -300,7 +370,9 @@ dsa_status dsa_index_rotate(int32_t n_rows, int32_t heads, int32_t dim, int32_t 
  * looks up the array's device address with that device current, so make it
  * before any stream capture.  All calls share the array and it keeps the last
  * call's contents; calls that overlap on the GPU race on it.  No part of the
- * array needs to start at zero. */
+ * array needs to start at zero.  The address is remembered with the context it
+ * was read in: after a cudaDeviceReset the next call on that device looks it up
+ * again (also outside any stream capture). */
 dsa_status dsa_layer_forward_static(const dsa_dims* dims, const void* q_idx, const void* k_idx,
                                     const float* w, float idx_scale, const int32_t* q_pos,
                                     const int32_t* kv_start, const int32_t* kv_len, const void* q,

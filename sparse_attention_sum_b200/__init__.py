@@ -15,9 +15,9 @@ from typing import Optional
 
 __all__ = [
     "DsaError", "DsaLibraryError", "Dims", "lib", "lib_path", "INVALID", "F32", "BF16",
-    "index_scores", "topk", "topk_set", "sparse_attend", "layer_forward", "layer_forward_static", "pool_states",
+    "index_scores", "index_scores_fp8", "fp8_quantize", "index_topk", "index_topk_fp8", "topk", "topk_set", "sparse_attend", "layer_forward", "layer_forward_static", "pool_states",
     "expand_selection", "absorb_q", "absorb_out", "index_rotate", "workspace_size", "get_device_status",
-    "selftest_wait_timeout", "set_kernel_policy", "OP_TOPK", "OP_LAYER_FORWARD", "STATUS",
+    "selftest_wait_timeout", "set_kernel_policy", "last_kernels", "OP_TOPK", "OP_LAYER_FORWARD", "STATUS",
 ]
 
 INVALID = -1
@@ -63,10 +63,19 @@ _SIGS = {
     "dsa_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "dsa_last_error": ([], ctypes.c_char_p),
     "dsa_version": ([], ctypes.c_char_p),
+    "dsa_last_kernels": ([], ctypes.c_char_p),
     "dsa_set_kernel_policy": ([ctypes.c_int], ctypes.c_int),
     "dsa_workspace_size": ([ctypes.POINTER(Dims), ctypes.c_int], ctypes.c_size_t),
     "dsa_index_scores": ([ctypes.POINTER(Dims), _VP, _VP, _F32P, ctypes.c_float, _I32P, _I32P,
                           _I32P, _F32P, _VP], ctypes.c_int),
+    "dsa_fp8_quantize": ([ctypes.c_int64, ctypes.c_int32, ctypes.c_int, _VP, ctypes.c_int64, _VP, _F32P, _VP],
+                         ctypes.c_int),
+    "dsa_index_scores_fp8": ([ctypes.POINTER(Dims), _VP, _F32P, _VP, _F32P, _F32P, ctypes.c_float, _I32P, _I32P,
+                              _I32P, _F32P, _VP], ctypes.c_int),
+    "dsa_index_topk": ([ctypes.POINTER(Dims), _VP, _VP, _F32P, ctypes.c_float, _I32P, _I32P, _I32P, ctypes.c_int32,
+                        _I32P, _VP], ctypes.c_int),
+    "dsa_index_topk_fp8": ([ctypes.POINTER(Dims), _VP, _F32P, _VP, _F32P, _F32P, ctypes.c_float, _I32P, _I32P,
+                            _I32P, ctypes.c_int32, _I32P, _VP], ctypes.c_int),
     "dsa_topk": ([ctypes.POINTER(Dims), _F32P, _I32P, _I32P, _I32P, ctypes.c_int32, _I32P, _F32P,
                   _VP, ctypes.c_size_t, _VP], ctypes.c_int),
     "dsa_topk_set": ([ctypes.POINTER(Dims), _F32P, _I32P, _I32P, _I32P, ctypes.c_int32, _I32P, _F32P, _VP],
@@ -152,6 +161,12 @@ def _dtype_code(t) -> int:
     raise ValueError(f"unsupported dtype {t.dtype}")
 
 
+def last_kernels() -> list:
+    """Kernel families the most recent libdsa call on this thread launched, in order."""
+    s = lib().dsa_last_kernels().decode()
+    return s.split(",") if s else []
+
+
 def set_kernel_policy(policy: int) -> int:
     return lib().dsa_set_kernel_policy(int(policy))
 
@@ -165,6 +180,41 @@ def index_scores(dims: Dims, q_idx, k_idx, w, scale: float, q_pos, kv_start, kv_
     _check(lib().dsa_index_scores(ctypes.byref(dims), _ptr(q_idx), _ptr(k_idx), _ptr(w), scale,
                                   _ptr(q_pos), _ptr(kv_start), _ptr(kv_len), _ptr(scores),
                                   _stream(stream)), "dsa_index_scores")
+
+
+def fp8_quantize(x, codes, scales, stream=None):
+    """dsa_fp8_quantize: per-vector e4m3 codes and fp32 scales of ``x [..., 128]`` (bf16 or fp32; rows may
+    be strided).  ``codes`` is a uint8 tensor ``[..., 128]``, ``scales`` fp32 ``[...]``."""
+    if x.shape[-1] != 128 or x.stride(-1) != 1:
+        raise ValueError("x must end in a contiguous axis of 128 values")
+    rows = x.reshape(-1, 128) if x.is_contiguous() else x.view(-1, 128)
+    if codes.dtype != __import__("torch").uint8 or codes.numel() != rows.shape[0] * 128:
+        raise ValueError("codes must be a uint8 tensor of x's shape")
+    if scales.numel() != rows.shape[0]:
+        raise ValueError("scales must hold one value per row of x")
+    _check(lib().dsa_fp8_quantize(int(rows.shape[0]), 128, _dtype_code(x), _ptr(rows, False), int(rows.stride(0)),
+                                  _ptr(codes), _ptr(scales), _stream(stream)), "dsa_fp8_quantize")
+
+
+def index_scores_fp8(dims: Dims, q_codes, q_scales, k_codes, k_scales, w, scale: float, q_pos, kv_start, kv_len,
+                     scores, stream=None):
+    _check(lib().dsa_index_scores_fp8(ctypes.byref(dims), _ptr(q_codes), _ptr(q_scales), _ptr(k_codes),
+                                      _ptr(k_scales), _ptr(w), scale, _ptr(q_pos), _ptr(kv_start), _ptr(kv_len),
+                                      _ptr(scores), _stream(stream)), "dsa_index_scores_fp8")
+
+
+def index_topk(dims: Dims, q_idx, k_idx, w, scale: float, q_pos, kv_start, kv_len, k: int, idx, stream=None):
+    """dsa_index_topk: the selection (ascending key order) straight from the indexer inputs."""
+    _check(lib().dsa_index_topk(ctypes.byref(dims), _ptr(q_idx), _ptr(k_idx), _ptr(w), scale, _ptr(q_pos),
+                                _ptr(kv_start), _ptr(kv_len), int(k), _ptr(idx), _stream(stream)), "dsa_index_topk")
+
+
+def index_topk_fp8(dims: Dims, q_codes, q_scales, k_codes, k_scales, w, scale: float, q_pos, kv_start, kv_len,
+                   k: int, idx, stream=None):
+    """dsa_index_topk_fp8: the FP8 selection (ascending key order) straight from the e4m3 operands."""
+    _check(lib().dsa_index_topk_fp8(ctypes.byref(dims), _ptr(q_codes), _ptr(q_scales), _ptr(k_codes),
+                                    _ptr(k_scales), _ptr(w), scale, _ptr(q_pos), _ptr(kv_start), _ptr(kv_len), int(k),
+                                    _ptr(idx), _stream(stream)), "dsa_index_topk_fp8")
 
 
 def topk(dims: Dims, scores, q_pos, kv_start, kv_len, k: int, idx, vals=None, ws=None,

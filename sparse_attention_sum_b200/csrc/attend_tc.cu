@@ -72,7 +72,8 @@ constexpr int kRopeOff = 4 * kBlockBytes;                   // 32 rope columns a
 constexpr int kStageBytes = kRopeOff + kChunk * 64;         // 36 KB
 constexpr int kQRopeBytes = 128 * 64;                       // rope query columns in smem: 8 KB
 constexpr int kXBytes = kChunk * 128 * 4;                   // exchange tile [key/4][head][4] fp32: 32 KB
-constexpr int kBitmapKeys = 65536;                          // dedupe bitmap (8 KB, aliases stage 0)
+constexpr int kNarrowKeys = 65536;                          // key lists of 16-bit entries up to here
+constexpr int kMaxKeys = kStageBytes * 8;                   // 294912: the dedupe bitmap fits one stage
 constexpr int kQCol = 128;                                  // query columns in TMEM
 constexpr int kOCol = 256;                                  // output accumulator
 constexpr int kThreads = 544;          // 17 warps
@@ -90,12 +91,16 @@ struct AttTcParams {
   int* status;
   int list_bitmap;           // 1: the dedupe bitmap fits in the key-list buffer
   int out_v8;                // 1: out is 32-byte aligned (256-bit stores)
+  int list_nbytes;           // key-list buffer size in shared memory (list_bytes)
+  int list_hi_off;           // byte offset of the high parts in the key-list buffer (S > 65536)
 };
 
-// Key-list buffer: width uint16 entries, grown to hold the dedupe bitmap of S keys when
-// `with_bitmap` (then the bitmap needs no gather stage).
-__host__ __device__ inline size_t list_bytes(int width, int S, bool with_bitmap) {
-  size_t b = (size_t)width * 2;
+// Key-list buffer: width uint16 entries (the low 16 bits of each key) and, when S > 65536, width
+// uint8 high parts after them; grown to hold the dedupe bitmap of S keys when `with_bitmap` (then
+// the bitmap needs no gather stage).
+inline size_t list_lo_bytes(int width) { return ((size_t)width * 2 + 15) & ~(size_t)15; }
+inline size_t list_bytes(int width, int S, bool with_bitmap) {
+  size_t b = list_lo_bytes(width) + (S > kNarrowKeys ? (((size_t)width + 15) & ~(size_t)15) : 0);
   const size_t bm = (size_t)((S + 31) / 32) * 4;
   if (with_bitmap && bm > b) b = bm;
   return (b + 15) & ~(size_t)15;
@@ -103,7 +108,8 @@ __host__ __device__ inline size_t list_bytes(int width, int S, bool with_bitmap)
 
 struct Smem {
   uint32_t kv, x, qrope;     // shared-window addresses
-  uint16_t* list;            // deduplicated key rows of the row being gathered (n_kv <= 65536)
+  uint16_t* list;            // deduplicated key rows of the row being gathered: low 16 bits (then
+                             // bits 16-23 of each entry when S > 65536, see put_key)
   int* wcount;               // 4 per-warp counts of the list compaction
   float* mx;                 // [2 parities][2 groups][128 rows] half-row maxima
   float* lsum;               // [2 groups][128 rows] partial row sums for the epilogue
@@ -203,6 +209,18 @@ struct RowKeys {
   int key[kListCache];
 };
 
+// The high parts sit after the low parts (list_lo_bytes(width) = p.list_hi_off bytes in).
+template <bool kWide>
+__device__ __forceinline__ void put_key(const AttTcParams& p, const Smem& sm, int pos, int key) {
+  sm.list[pos] = (uint16_t)key;
+  if (kWide) (reinterpret_cast<uint8_t*>(sm.list) + p.list_hi_off)[pos] = (uint8_t)(key >> 16);
+}
+template <bool kWide>
+__device__ __forceinline__ int get_key(const AttTcParams& p, const Smem& sm, int pos) {
+  if (!kWide) return (int)sm.list[pos];
+  return ((int)(reinterpret_cast<const uint8_t*>(sm.list) + p.list_hi_off)[pos] << 16) | (int)sm.list[pos];
+}
+
 __device__ void load_row(const AttTcParams& p, const int32_t* irow, RowKeys& rk) {
   const int tid = threadIdx.x - 5 * 32, lane = threadIdx.x & 31, w = tid >> 5;
   rk.q = (((p.width + 3) >> 2) + 31) & ~31;
@@ -249,6 +267,7 @@ __device__ bool mark_keys(const AttTcParams& p, const int32_t* irow, const RowKe
 
 // No repeated key: keep every in-range entry.  Each warp compacts its contiguous quarter of
 // the row 32 entries at a time (ballots), after a scan of the four quarters' counts.
+template <bool kWide>
 __device__ int compact_unique(const AttTcParams& p, const Smem& sm, const int32_t* irow, const RowKeys& rk) {
   const int tid = threadIdx.x - 5 * 32, lane = threadIdx.x & 31, w = tid >> 5;
   const uint32_t below = (1u << lane) - 1u;
@@ -275,7 +294,7 @@ __device__ int compact_unique(const AttTcParams& p, const Smem& sm, const int32_
       const int key = rk.key[it];
       const bool keep = key >= 0 && key < p.S;
       const uint32_t m = __ballot_sync(0xffffffffu, keep);
-      if (keep) sm.list[base + __popc(m & below)] = (uint16_t)key;
+      if (keep) put_key<kWide>(p, sm, base + __popc(m & below), key);
       base += __popc(m);
     }
   } else {
@@ -284,7 +303,7 @@ __device__ int compact_unique(const AttTcParams& p, const Smem& sm, const int32_
       const int key = e < rk.e1 ? __ldg(irow + e) : -1;
       const bool keep = key >= 0 && key < p.S;
       const uint32_t m = __ballot_sync(0xffffffffu, keep);
-      if (keep) sm.list[base + __popc(m & below)] = (uint16_t)key;
+      if (keep) put_key<kWide>(p, sm, base + __popc(m & below), key);
       base += __popc(m);
     }
   }
@@ -294,6 +313,7 @@ __device__ int compact_unique(const AttTcParams& p, const Smem& sm, const int32_
 
 // Repeated keys: order-preserving compaction by one warp, first occurrence only (not seen in
 // an earlier group of 32, lowest lane within its group).  `bitmap` must not overlap the list.
+template <bool kWide>
 __device__ int compact_first(const AttTcParams& p, const Smem& sm, const int32_t* irow, uint32_t* bitmap) {
   const int tid = threadIdx.x - 5 * 32, lane = threadIdx.x & 31;
   const int words = (p.S + 31) >> 5;
@@ -310,7 +330,7 @@ __device__ int compact_first(const AttTcParams& p, const Smem& sm, const int32_t
       __syncwarp();
       if (keep) atomicOr(&bitmap[key >> 5], 1u << (key & 31));
       const uint32_t m = __ballot_sync(0xffffffffu, keep);
-      if (keep) sm.list[n + __popc(m & ((1u << lane) - 1u))] = (uint16_t)key;
+      if (keep) put_key<kWide>(p, sm, n + __popc(m & ((1u << lane) - 1u)), key);
       n += __popc(m);
       __syncwarp();
     }
@@ -328,7 +348,8 @@ __device__ int compact_first(const AttTcParams& p, const Smem& sm, const int32_t
 // last chunks, and a row's epilogue overlaps the next row's first q.k.
 // kHalfHeads: H = 64, so the head rows 64-127 of the M = 128 tiles are padding; the warps that own
 // them skip their softmax and exchange work (separate instantiation, so H = 128 pays nothing).
-template <bool kHalfHeads>
+// kWide: S > 65536, so list entries carry an 8-bit high part (separate instantiation as well).
+template <bool kHalfHeads, bool kWide>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
                  const __grid_constant__ CUtensorMap map_rope,
@@ -345,7 +366,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   sm.kv = sm.qrope + kQRopeBytes;
   uint32_t off = sm.kv + kStages * kStageBytes - base;
   sm.list = reinterpret_cast<uint16_t*>(gb + off);
-  off += (uint32_t)list_bytes(p.width, p.S, p.list_bitmap != 0);
+  off += (uint32_t)p.list_nbytes;
   sm.mx = reinterpret_cast<float*>(gb + off);
   off += 2 * 2 * 128 * 4;
   sm.lsum = reinterpret_cast<float*>(gb + off);
@@ -458,13 +479,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       const bool dup = mark_keys(p, irow, rk, p.list_bitmap ? reinterpret_cast<uint32_t*>(sm.list) : stage_bitmap);
       int n;
       if (!dup) {
-        n = compact_unique(p, sm, irow, rk);
+        n = compact_unique<kWide>(p, sm, irow, rk);
       } else {
         if (p.list_bitmap && !wait_stage()) {
           ok = false;
           break;
         }
-        n = compact_first(p, sm, irow, stage_bitmap);
+        n = compact_first<kWide>(p, sm, irow, stage_bitmap);
       }
       fence_proxy_async_smem();                          // bitmap writes ordered before gathers into the stage
       named_sync(1, kProducerThreads);
@@ -495,7 +516,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const int li = j * kChunk + 4 * g + k;
-            rr[k] = rowbase + (int)sm.list[li < n ? li : 0];
+            rr[k] = rowbase + get_key<kWide>(p, sm, li < n ? li : 0);
           }
           if (lane < 16)
             tma_gather4(stb + w * kBlockBytes + g * 512, &map_kv, bar, (4 * (int)rank + w) * 64, rr[0], rr[1],
@@ -938,7 +959,8 @@ bool attend_tc_supported(const dsa_dims& d, int64_t k_stride, const void* k, con
   if ((long long)d.batch * d.n_q * d.heads < 128) return false;  // the query TMA box is 128 rows
   if (k != v || k_stride != v_stride || k_stride < d.kd || (k_stride * 2) % 16 != 0) return false;
   if (((uintptr_t)k & 15u) != 0) return false;
-  if (d.n_kv > kBitmapKeys) return false;                  // 16-bit key list
+  if (d.n_kv > kMaxKeys) return false;                     // the dedupe bitmap fits one gather stage
+  if ((long long)d.batch * d.n_kv > 2147483647LL) return false;  // 32-bit TMA row coordinates
   if (width > 8192) return false;
   if (smem_bytes(width, d.n_kv, false) > 227 * 1024) return false;
   return encode_fn() != nullptr;
@@ -992,9 +1014,13 @@ cudaError_t launch_attend_tc(const dsa_dims& d, const void* q, const void* k, in
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   p.list_bitmap = bitmap_in_list(width, d.n_kv) ? 1 : 0;
+  p.list_nbytes = (int)list_bytes(width, d.n_kv, p.list_bitmap != 0);
+  p.list_hi_off = (int)list_lo_bytes(width);
   p.out_v8 = ((uintptr_t)out & 31u) == 0 ? 1 : 0;
   const size_t smem = smem_bytes(width, d.n_kv, p.list_bitmap != 0);
-  auto kern = d.heads == 64 ? attend_tc_kernel<true> : attend_tc_kernel<false>;
+  const bool wide = d.n_kv > kNarrowKeys;
+  auto kern = d.heads == 64 ? (wide ? attend_tc_kernel<true, true> : attend_tc_kernel<true, false>)
+                            : (wide ? attend_tc_kernel<false, true> : attend_tc_kernel<false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   // persistent clusters: one per SM pair (or one per row when there are fewer rows)

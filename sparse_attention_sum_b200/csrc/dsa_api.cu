@@ -16,6 +16,18 @@ namespace {
 
 thread_local std::string g_last_error;
 
+// Kernel families launched by the current top-level entry point call of this host thread
+// (entry points that call other entry points record into the outer call's list).
+thread_local std::string g_kernels;
+thread_local int g_call_depth = 0;
+
+struct CallScope {
+  CallScope() {
+    if (g_call_depth++ == 0) g_kernels.clear();
+  }
+  ~CallScope() { --g_call_depth; }
+};
+
 __device__ int g_device_status;  // DSA_ERR_TIMEOUT recorded by bounded device waits
 
 dsa_status fail(dsa_status s, const char* fmt, ...) {
@@ -106,18 +118,42 @@ bool tc_policy() { return g_policy.load(std::memory_order_relaxed) == 0; }
 
 namespace dsa {
 
+void* current_context() {
+  typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+  static std::atomic<CtxGetCurrentFn> fn{nullptr};
+  CtxGetCurrentFn f = fn.load(std::memory_order_acquire);
+  if (!f) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    f = (CtxGetCurrentFn)ptr;
+    fn.store(f, std::memory_order_release);
+  }
+  CUcontext c = nullptr;
+  return f(&c) == CUDA_SUCCESS ? (void*)c : nullptr;
+}
+
 int* device_status_ptr() {
   static std::mutex mu;
+  static void* ctxs[128] = {};
   static int* ptrs[128] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  void* ctx = current_context();
   std::lock_guard<std::mutex> lock(mu);
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
-    ptrs[dev] = (int*)p;
-  }
+  if (ptrs[dev] && ctx && ctxs[dev] == ctx) return ptrs[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+  ctxs[dev] = current_context();  // the lookup binds the primary context if none was current
+  ptrs[dev] = (int*)p;
   return ptrs[dev];
+}
+
+void note_kernel(const char* name) {
+  if (!g_kernels.empty()) g_kernels += ',';
+  g_kernels += name;
 }
 
 void set_last_error(const char* msg) { g_last_error = msg; }
@@ -176,6 +212,8 @@ const char* dsa_status_string(dsa_status s) {
 
 const char* dsa_last_error(void) { return g_last_error.c_str(); }
 
+const char* dsa_last_kernels(void) { return g_kernels.c_str(); }
+
 const char* dsa_version(void) { return "libdsa 0.1 (sm_100a)"; }
 
 /* Selects which kernels serve shapes both families support: 0 (default) picks
@@ -199,12 +237,14 @@ size_t dsa_workspace_size(const dsa_dims* d, int op) {
 dsa_status dsa_index_scores(const dsa_dims* d, const void* q_idx, const void* k_idx, const float* w,
                             float scale, const int32_t* q_pos, const int32_t* kv_start,
                             const int32_t* kv_len, float* scores, dsa_stream_t stream) {
+  CallScope scope;
   dsa_status s = check_index(d, q_idx, k_idx, w, scale, scores);
   if (s) return s;
   if ((s = check_visibility(q_pos, kv_start, kv_len))) return s;
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
-  if (tc_policy() && dsa::index_scores_tc_supported(*d)) {
+  const bool tc = tc_policy() && dsa::index_scores_tc_supported(*d);
+  if (tc) {
     e = dsa::launch_index_scores_tc(*d, q_idx, k_idx, w, scale, q_pos, kv_start, kv_len, scores, st);
   } else {
     if (d->idx_dim > 256 || (int64_t)d->idx_heads * d->idx_dim > 16384)
@@ -212,6 +252,96 @@ dsa_status dsa_index_scores(const dsa_dims* d, const void* q_idx, const void* k_
     e = dsa::launch_index_scores_simt(*d, q_idx, k_idx, w, scale, q_pos, kv_start, kv_len, scores, st);
   }
   if (e != cudaSuccess) return cuda_fail(e, "dsa_index_scores launch");
+  dsa::note_kernel(tc ? "index_tc" : "index_simt");
+  return ok();
+}
+
+dsa_status dsa_fp8_quantize(int64_t n_vectors, int32_t dim, dsa_dtype in_dtype, const void* x,
+                            int64_t x_row_stride, void* codes, float* scales, dsa_stream_t stream) {
+  CallScope scope;
+  REQUIRE(n_vectors >= 0, "n_vectors must be >= 0 (got %lld)", (long long)n_vectors);
+  REQUIRE(dtype_ok(in_dtype), "in_dtype must be DSA_F32 or DSA_BF16 (got %d)", (int)in_dtype);
+  if (dim != 128) return fail(DSA_ERR_UNSUPPORTED, "dsa_fp8_quantize: dim must be 128 (got %d)", dim);
+  if (n_vectors == 0) return ok();
+  REQUIRE(x && codes && scales, "x, codes and scales must be non-NULL");
+  REQUIRE(x_row_stride >= dim, "x_row_stride (%lld) must be >= dim", (long long)x_row_stride);
+  const size_t esz = in_dtype == DSA_BF16 ? 2 : 4;
+  REQUIRE(x_row_stride % 4 == 0 && (uintptr_t)x % (4 * esz) == 0,
+          "x and its row stride must be aligned to 4 values");
+  REQUIRE((uintptr_t)codes % 4 == 0, "codes must be 4-byte aligned");
+  cudaError_t e = dsa::launch_fp8_quantize((long long)n_vectors, in_dtype == DSA_BF16, x, (long long)x_row_stride,
+                                           codes, scales, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "dsa_fp8_quantize launch");
+  dsa::note_kernel("fp8_quantize");
+  return ok();
+}
+
+dsa_status dsa_index_scores_fp8(const dsa_dims* d, const void* q_codes, const float* q_scales, const void* k_codes,
+                                const float* k_scales, const float* w, float scale, const int32_t* q_pos,
+                                const int32_t* kv_start, const int32_t* kv_len, float* scores,
+                                dsa_stream_t stream) {
+  CallScope scope;
+  dsa_status s = check_rows(d);
+  if (s) return s;
+  REQUIRE(d->idx_heads >= 1 && d->idx_dim >= 1, "idx_heads and idx_dim must be >= 1");
+  REQUIRE(q_codes && q_scales && k_codes && k_scales && w && scores,
+          "q_codes, q_scales, k_codes, k_scales, w and scores must be non-NULL");
+  REQUIRE(scale == scale, "scale must not be NaN");
+  REQUIRE(d->n_q <= 65535, "n_q must be <= 65535 for dsa_index_scores_fp8 (got %d)", d->n_q);
+  if ((s = check_visibility(q_pos, kv_start, kv_len))) return s;
+  REQUIRE(((uintptr_t)q_codes & 15u) == 0 && ((uintptr_t)k_codes & 15u) == 0, "codes must be 16-byte aligned");
+  if (!dsa::index_scores_tc_supported(*d, true))
+    return fail(DSA_ERR_UNSUPPORTED,
+                "dsa_index_scores_fp8: idx_dim 128, idx_heads in {32, 64, 128} and batch*n_kv >= 128 required");
+  cudaError_t e = dsa::launch_index_scores_tc(*d, q_codes, k_codes, w, scale, q_pos, kv_start, kv_len, scores,
+                                              (cudaStream_t)stream, q_scales, k_scales);
+  if (e != cudaSuccess) return cuda_fail(e, "dsa_index_scores_fp8 launch");
+  dsa::note_kernel("index_tc_fp8");
+  return ok();
+}
+
+dsa_status dsa_index_topk(const dsa_dims* d, const void* q_idx, const void* k_idx, const float* w, float scale,
+                          const int32_t* q_pos, const int32_t* kv_start, const int32_t* kv_len, int32_t k,
+                          int32_t* idx, dsa_stream_t stream) {
+  CallScope scope;
+  dsa_status s = check_index(d, q_idx, k_idx, w, scale, (float*)1);
+  if (s) return s;
+  if ((s = check_visibility(q_pos, kv_start, kv_len))) return s;
+  REQUIRE(idx != nullptr, "idx must be non-NULL");
+  REQUIRE(k >= 1 && k <= 4096, "k must be in [1, 4096] (got %d)", k);
+  REQUIRE(d->kpool == 0, "dsa_index_topk: kpool must be 0 (got %d)", d->kpool);
+  if (!dsa::index_topk_supported(*d, k))
+    return fail(DSA_ERR_UNSUPPORTED,
+                "dsa_index_topk: bf16, idx_dim 128, idx_heads in {32, 64, 128} and n_kv <= 131072 required");
+  cudaError_t e = dsa::launch_index_topk(*d, q_idx, k_idx, w, scale, q_pos, kv_start, kv_len, k, idx,
+                                         (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "dsa_index_topk launch");
+  dsa::note_kernel("index_topk");
+  return ok();
+}
+
+dsa_status dsa_index_topk_fp8(const dsa_dims* d, const void* q_codes, const float* q_scales, const void* k_codes,
+                              const float* k_scales, const float* w, float scale, const int32_t* q_pos,
+                              const int32_t* kv_start, const int32_t* kv_len, int32_t k, int32_t* idx,
+                              dsa_stream_t stream) {
+  CallScope scope;
+  dsa_status s = check_rows(d);
+  if (s) return s;
+  REQUIRE(d->idx_heads >= 1 && d->idx_dim >= 1, "idx_heads and idx_dim must be >= 1");
+  REQUIRE(q_codes && q_scales && k_codes && k_scales && w && idx,
+          "q_codes, q_scales, k_codes, k_scales, w and idx must be non-NULL");
+  REQUIRE(scale == scale, "scale must not be NaN");
+  REQUIRE(d->n_q <= 65535, "n_q must be <= 65535 (got %d)", d->n_q);
+  if ((s = check_visibility(q_pos, kv_start, kv_len))) return s;
+  REQUIRE(k >= 1 && k <= 4096, "k must be in [1, 4096] (got %d)", k);
+  REQUIRE(d->kpool == 0, "dsa_index_topk_fp8: kpool must be 0 (got %d)", d->kpool);
+  REQUIRE(((uintptr_t)q_codes & 15u) == 0 && ((uintptr_t)k_codes & 15u) == 0, "codes must be 16-byte aligned");
+  if (!dsa::index_topk_supported(*d, k, true))
+    return fail(DSA_ERR_UNSUPPORTED, "dsa_index_topk_fp8: idx_dim 128, idx_heads in {32, 64, 128} and n_kv <= 131072 required");
+  cudaError_t e = dsa::launch_index_topk(*d, q_codes, k_codes, w, scale, q_pos, kv_start, kv_len, k, idx,
+                                         (cudaStream_t)stream, q_scales, k_scales);
+  if (e != cudaSuccess) return cuda_fail(e, "dsa_index_topk_fp8 launch");
+  dsa::note_kernel("index_topk_fp8");
   return ok();
 }
 
@@ -222,6 +352,7 @@ dsa_status topk_checked(const dsa_dims* d, const float* scores, const int32_t* q
   if (d->batch > 65535) return fail(DSA_ERR_UNSUPPORTED, "dsa_topk: grid too large");
   cudaError_t e = dsa::launch_topk(*d, scores, q_pos, kv_start, kv_len, k, idx, vals, ranked, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "dsa_topk launch");
+  dsa::note_kernel(ranked ? "topk_ranked" : "topk_set");
   return ok();
 }
 }  // namespace
@@ -229,6 +360,7 @@ dsa_status topk_checked(const dsa_dims* d, const float* scores, const int32_t* q
 dsa_status dsa_topk(const dsa_dims* d, const float* scores, const int32_t* q_pos,
                     const int32_t* kv_start, const int32_t* kv_len, int32_t k, int32_t* idx,
                     float* vals, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  CallScope scope;
   (void)ws;
   dsa_status s = check_topk(d, scores, k, idx);
   if (s) return s;
@@ -240,6 +372,7 @@ dsa_status dsa_topk(const dsa_dims* d, const float* scores, const int32_t* q_pos
 
 dsa_status dsa_topk_set(const dsa_dims* d, const float* scores, const int32_t* q_pos, const int32_t* kv_start,
                         const int32_t* kv_len, int32_t k, int32_t* idx, float* vals, dsa_stream_t stream) {
+  CallScope scope;
   dsa_status s = check_topk(d, scores, k, idx);
   if (s) return s;
   if ((s = check_visibility(q_pos, kv_start, kv_len))) return s;
@@ -249,11 +382,13 @@ dsa_status dsa_topk_set(const dsa_dims* d, const float* scores, const int32_t* q
 dsa_status dsa_sparse_attend(const dsa_dims* d, const void* q, const void* k, int64_t k_row_stride,
                              const void* v, int64_t v_row_stride, const int32_t* idx, int32_t width,
                              float scale, void* out, float* lse, dsa_stream_t stream) {
+  CallScope scope;
   dsa_status s = check_attend(d, q, k, k_row_stride, v, v_row_stride, idx, width, out);
   if (s) return s;
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
-  if (tc_policy() && dsa::attend_tc_supported(*d, k_row_stride, k, v, v_row_stride, width)) {
+  const bool tc = tc_policy() && dsa::attend_tc_supported(*d, k_row_stride, k, v, v_row_stride, width);
+  if (tc) {
     e = dsa::launch_attend_tc(*d, q, k, k_row_stride, idx, width, scale, out, lse, st);
   } else {
     if (!dsa::attend_simt_supported(*d, width))
@@ -261,6 +396,7 @@ dsa_status dsa_sparse_attend(const dsa_dims* d, const void* q, const void* k, in
     e = dsa::launch_attend_simt(*d, q, k, k_row_stride, v, v_row_stride, idx, width, scale, out, lse, st);
   }
   if (e != cudaSuccess) return cuda_fail(e, "dsa_sparse_attend launch");
+  dsa::note_kernel(tc ? "attend_tc" : "attend_simt");
   return ok();
 }
 
@@ -270,6 +406,7 @@ dsa_status dsa_layer_forward(const dsa_dims* d, const void* q_idx, const void* k
                              int64_t k_row_stride, const void* v, int64_t v_row_stride,
                              float attn_scale, const int32_t* idx_in, int32_t* idx_out, void* out,
                              float* lse, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  CallScope scope;
   dsa_status s = check_rows(d);
   if (s) return s;
   REQUIRE(d->kpool == 0, "dsa_layer_forward: kpool must be 0 (got %d)", d->kpool);
@@ -303,6 +440,7 @@ dsa_status dsa_pool_states(const dsa_dims* d, const void* k, const void* gate, c
                            const float* ln_b, float ln_eps, const int32_t* kv_start,
                            const int32_t* kv_len, void* pooled, int32_t* n_pools,
                            dsa_stream_t stream) {
+  CallScope scope;
   REQUIRE(d != nullptr, "dims is NULL");
   REQUIRE(d->batch >= 1 && d->batch <= 65535, "batch must be in [1, 65535]");
   REQUIRE(d->kpool >= 1, "dsa_pool_states: kpool must be >= 1 (got %d)", d->kpool);
@@ -315,12 +453,14 @@ dsa_status dsa_pool_states(const dsa_dims* d, const void* k, const void* gate, c
   cudaError_t e = dsa::launch_pool_states(*d, k, gate, ln_w, ln_b, ln_eps, kv_start, kv_len, pooled,
                                           n_pools, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "dsa_pool_states launch");
+  dsa::note_kernel("pool_states");
   return ok();
 }
 
 dsa_status dsa_expand_selection(const dsa_dims* d, const int32_t* pool_idx, const int32_t* q_pos,
                                 const int32_t* kv_start, const int32_t* kv_len,
                                 const int32_t* n_pools, int32_t* tok_idx, dsa_stream_t stream) {
+  CallScope scope;
   REQUIRE(d != nullptr, "dims is NULL");
   REQUIRE(d->batch >= 1 && d->batch <= 65535, "batch must be in [1, 65535]");
   REQUIRE(d->n_q >= 1 && d->n_q <= 2147483647, "n_q must be >= 1");
@@ -333,6 +473,7 @@ dsa_status dsa_expand_selection(const dsa_dims* d, const int32_t* pool_idx, cons
   cudaError_t e = dsa::launch_expand_selection(*d, pool_idx, q_pos, kv_start, kv_len, n_pools,
                                                tok_idx, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "dsa_expand_selection launch");
+  dsa::note_kernel("expand_selection");
   return ok();
 }
 
@@ -341,6 +482,7 @@ dsa_status dsa_index_rotate(int32_t n_rows, int32_t heads, int32_t dim, int32_t 
                             int32_t hadamard, const int32_t* pos, dsa_dtype in_dtype, const void* in,
                             int64_t in_row_stride, dsa_dtype out_dtype, void* out, int64_t out_row_stride,
                             const int32_t* out_rows, int64_t out_capacity, dsa_stream_t stream) {
+  CallScope scope;
   REQUIRE(n_rows >= 0, "n_rows must be >= 0 (got %d)", n_rows);
   REQUIRE(heads >= 1, "heads must be >= 1 (got %d)", heads);
   REQUIRE(dim == 32 || dim == 64 || dim == 128, "dim must be 32, 64 or 128 (got %d)", dim);
@@ -368,6 +510,7 @@ dsa_status dsa_index_rotate(int32_t n_rows, int32_t heads, int32_t dim, int32_t 
                                            out_dtype == DSA_BF16, out, out_row_stride, out_rows, out_capacity,
                                            (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "dsa_index_rotate launch");
+  dsa::note_kernel("index_rotate");
   return ok();
 }
 
@@ -385,25 +528,29 @@ static dsa_status check_absorb(const dsa_dims* d, const void* a, int32_t K, cons
 
 dsa_status dsa_absorb_q(const dsa_dims* d, const void* q, int32_t dq, const void* w_uk, int32_t L,
                         void* q_lat, dsa_stream_t stream) {
+  CallScope scope;
   dsa_status s = check_absorb(d, q, dq, w_uk, L, q_lat);
   if (s) return s;
   const int rows = d->batch * d->n_q;
-  cudaError_t e = tc_policy() && dsa::head_gemm_tc_supported(rows, d->heads, dq, L, q, w_uk, true, q_lat)
-                      ? dsa::launch_head_gemm_tc(rows, d->heads, dq, L, q, w_uk, true, q_lat, (cudaStream_t)stream)
-                      : dsa::launch_head_gemm(rows, d->heads, dq, L, q, w_uk, true, q_lat, (cudaStream_t)stream);
+  const bool tc = tc_policy() && dsa::head_gemm_tc_supported(rows, d->heads, dq, L, q, w_uk, true, q_lat);
+  cudaError_t e = tc ? dsa::launch_head_gemm_tc(rows, d->heads, dq, L, q, w_uk, true, q_lat, (cudaStream_t)stream)
+                     : dsa::launch_head_gemm(rows, d->heads, dq, L, q, w_uk, true, q_lat, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "dsa_absorb_q launch");
+  dsa::note_kernel(tc ? "head_gemm_tc" : "head_gemm_simt");
   return ok();
 }
 
 dsa_status dsa_absorb_out(const dsa_dims* d, const void* o_lat, int32_t L, const void* w_uv,
                           int32_t dv, void* out, dsa_stream_t stream) {
+  CallScope scope;
   dsa_status s = check_absorb(d, o_lat, L, w_uv, dv, out);
   if (s) return s;
   const int rows = d->batch * d->n_q;
-  cudaError_t e = tc_policy() && dsa::head_gemm_tc_supported(rows, d->heads, L, dv, o_lat, w_uv, false, out)
-                      ? dsa::launch_head_gemm_tc(rows, d->heads, L, dv, o_lat, w_uv, false, out, (cudaStream_t)stream)
-                      : dsa::launch_head_gemm(rows, d->heads, L, dv, o_lat, w_uv, false, out, (cudaStream_t)stream);
+  const bool tc = tc_policy() && dsa::head_gemm_tc_supported(rows, d->heads, L, dv, o_lat, w_uv, false, out);
+  cudaError_t e = tc ? dsa::launch_head_gemm_tc(rows, d->heads, L, dv, o_lat, w_uv, false, out, (cudaStream_t)stream)
+                     : dsa::launch_head_gemm(rows, d->heads, L, dv, o_lat, w_uv, false, out, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "dsa_absorb_out launch");
+  dsa::note_kernel(tc ? "head_gemm_tc" : "head_gemm_simt");
   return ok();
 }
 
@@ -423,9 +570,11 @@ dsa_status dsa_get_device_status(dsa_stream_t stream) {
 }
 
 dsa_status dsa_selftest_wait_timeout(int64_t timeout_ns, dsa_stream_t stream) {
+  CallScope scope;
   REQUIRE(timeout_ns >= 1000 && timeout_ns <= 10000000000LL, "timeout_ns must be in [1e3, 1e10]");
   cudaError_t e = dsa::launch_wait_selftest((long long)timeout_ns, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "dsa_selftest_wait_timeout launch");
+  dsa::note_kernel("wait_selftest");
   return ok();
 }
 

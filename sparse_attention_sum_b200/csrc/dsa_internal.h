@@ -8,6 +8,15 @@
 
 namespace dsa {
 
+// The current driver context (CUcontext) of the calling thread, or NULL.  Device addresses
+// of __device__ variables are cached together with it: after a cudaDeviceReset the device's
+// new context holds fresh copies of those variables at other addresses.
+void* current_context();
+
+// Records that the current entry point call launched kernel family `name`
+// (returned by dsa_last_kernels).
+void note_kernel(const char* name);
+
 // Device address of the status word on the current device (bounded waits
 // record DSA_ERR_TIMEOUT there).
 int* device_status_ptr();
@@ -23,12 +32,28 @@ cudaError_t launch_index_scores_simt(const dsa_dims& d, const void* q_idx, const
                                      const float* w, float scale, const int32_t* q_pos,
                                      const int32_t* kv_start, const int32_t* kv_len, float* scores,
                                      cudaStream_t st);
-// S2 on the tensor cores (tcgen05, bf16, D_I == 128, H_I in {16,32,64,128}).
-bool index_scores_tc_supported(const dsa_dims& d);
+// S2 on the tensor cores (tcgen05, D_I == 128, H_I in {32,64,128}): bf16 operands, or e4m3
+// codes with per-vector scales (f8; q_scale/k_scale non-NULL at launch).
+bool index_scores_tc_supported(const dsa_dims& d, bool f8 = false);
 cudaError_t launch_index_scores_tc(const dsa_dims& d, const void* q_idx, const void* k_idx,
                                    const float* w, float scale, const int32_t* q_pos,
                                    const int32_t* kv_start, const int32_t* kv_len, float* scores,
-                                   cudaStream_t st);
+                                   cudaStream_t st, const float* q_scale = nullptr,
+                                   const float* k_scale = nullptr);
+
+// Per-vector e4m3 quantisation of n rows of 128 values (bf16 or fp32, row stride in elements):
+// codes [n,128] bytes, scales [n] fp32.
+cudaError_t launch_fp8_quantize(long long n, bool in_bf16, const void* x, long long x_stride, void* codes,
+                                float* scales, cudaStream_t st);
+
+// S2 + S3 fused (bf16, D_I == 128, H_I in {32,64,128}, n_kv <= 8 * 16384): one cluster per query
+// row, scores kept in shared memory; writes the selection in ascending key order (dsa_topk_set's form).
+// f8: e4m3 codes with per-vector scales (q_scale/k_scale non-NULL at launch).
+bool index_topk_supported(const dsa_dims& d, int k, bool f8 = false);
+cudaError_t launch_index_topk(const dsa_dims& d, const void* q_idx, const void* k_idx, const float* w, float scale,
+                              const int32_t* q_pos, const int32_t* kv_start, const int32_t* kv_len, int k,
+                              int32_t* idx, cudaStream_t st, const float* q_scale = nullptr,
+                              const float* k_scale = nullptr);
 
 // S3 radix select, then a rank sort (ranked) or an ascending-key-order listing of
 // the same selection (!ranked, the fused layer's set).

@@ -18,6 +18,13 @@
 // tcgen05.mma into one of two TMEM accumulators, warps 2.. run the epilogue
 // (tcgen05.ld -> relu/weight reduction -> coalesced fp32 stores).  Every
 // mbarrier wait is bounded (records DSA_ERR_TIMEOUT and aborts the CTA).
+//
+// FP8 operands (kF8): q and k arrive as e4m3 codes with one fp32 scale per
+// query-head vector and per key row (dsa_fp8_quantize).  A key row is then 128
+// bytes, one 128-byte swizzle row, and the MMA is kind::f8f6f4 with K = 32 per
+// instruction.  Since the scales are positive, relu(scale*sq*sk*dot) =
+// sk*relu(scale*sq*dot): the epilogue folds scale*sq into each accumulator
+// column and multiplies each key's sum by sk.
 #include <cuda.h>
 
 #include "dsa_common.cuh"
@@ -30,8 +37,10 @@ namespace {
 
 constexpr int kDI = 128;           // indexer head width served by this kernel
 constexpr int kKeysPerTile = 128;  // M
-constexpr int kTileBytes = kKeysPerTile * kDI * 2;  // one key stage: 32 KB
-constexpr int kMaxStages = 6;
+constexpr int kMaxStages = 8;
+// Bytes of one indexer vector and of one key stage: bf16 256 B / 32 KB, e4m3 128 B / 16 KB.
+__host__ __device__ constexpr int row_bytes(bool f8) { return f8 ? kDI : 2 * kDI; }
+__host__ __device__ constexpr int tile_bytes(bool f8) { return kKeysPerTile * row_bytes(f8); }
 
 struct IdxTcParams {
   int B, T, S, HI, NQ, N;     // N = NQ * HI
@@ -39,6 +48,8 @@ struct IdxTcParams {
   int n_qtiles, n_ktiles, tiles_per_split;
   int stages, epi_warps;
   float scale;                // applied inside relu
+  const float* q_scale;       // FP8: [B*T*H_I] per query-head vector
+  const float* k_scale;       // FP8: [B*S] per key row
   const float* w;
   const int32_t* q_pos;
   const int32_t* kv_start;
@@ -47,19 +58,24 @@ struct IdxTcParams {
   int* status;
 };
 
+template <bool kF8>
 __global__ void __launch_bounds__(320, 1)
 index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                 IdxTcParams p) {
   using namespace sm100;
+  constexpr int kTileBytes = tile_bytes(kF8);
+  constexpr uint32_t kRow = (uint32_t)row_bytes(kF8);
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* gbase = smem_raw + (base - raw);
-  // [B operand: N x 256 B][stages x 32 KB][w: NQ*HI floats][lo/hi per query][barriers]
+  // [B operand: N x kRow B][stages x kTileBytes][w: NQ*HI floats][(FP8) scale*sq: NQ*HI floats]
+  // [lo/hi per query][barriers]
   const uint32_t sB = base;
-  const uint32_t sA = sB + (uint32_t)p.N * 256u;
+  const uint32_t sA = sB + (uint32_t)p.N * kRow;
   float* w_s = reinterpret_cast<float*>(gbase + (sA - base) + (uint32_t)p.stages * kTileBytes);
-  int* lohi = reinterpret_cast<int*>(w_s + p.N);                 // [NQ][2]
+  float* ssq_s = w_s + p.N;                                       // FP8 only
+  int* lohi = reinterpret_cast<int*>(ssq_s + (kF8 ? p.N : 0));    // [NQ][2]
   uint64_t* bars = reinterpret_cast<uint64_t*>(lohi + 2 * 16 + 2); // 8-byte aligned below
   bars = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(bars) + 7) & ~uintptr_t(7));
   uint64_t* full = bars;                  // [stages]
@@ -120,7 +136,9 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
   // weights of the tile's queries (pre-multiplied by nothing: the scale stays inside relu)
   for (int i = threadIdx.x; i < p.N; i += blockDim.x) {
     const int q = i / p.HI;
-    w_s[i] = q < nq_here ? p.w[((size_t)b * p.T + t0 + q) * p.HI + (i - q * p.HI)] : 0.f;
+    const size_t col = ((size_t)b * p.T + t0 + q) * p.HI + (i - q * p.HI);
+    w_s[i] = q < nq_here ? p.w[col] : 0.f;
+    if (kF8) ssq_s[i] = q < nq_here ? p.scale * p.q_scale[col] : 0.f;
   }
   if (warp == 1 && n_compute > 0) tmem_alloc(smem_u32(tmem_slot), ncols);
   tc_fence_before();
@@ -134,9 +152,9 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
       tma_prefetch_desc(&map_q);
       tma_prefetch_desc(&map_k);
       const int qrow = (b * p.T + t0) * p.HI;
-      mbar_arrive_expect_tx(smem_u32(bfull), (uint32_t)p.N * 256u);
+      mbar_arrive_expect_tx(smem_u32(bfull), (uint32_t)p.N * kRow);
       tma_load_2d(sB, &map_q, smem_u32(bfull), 0, qrow);
-      tma_load_2d(sB + (uint32_t)p.N * 128u, &map_q, smem_u32(bfull), 64, qrow);
+      if (!kF8) tma_load_2d(sB + (uint32_t)p.N * 128u, &map_q, smem_u32(bfull), 64, qrow);
       int issued = 0;
       for (int i = 0; i < n_compute; ++i) {
         const int s = i % p.stages;
@@ -145,7 +163,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         const int krow = b * p.S + (c_begin + i) * kKeysPerTile;
         mbar_arrive_expect_tx(smem_u32(&full[s]), kTileBytes);
         tma_load_2d(dst, &map_k, smem_u32(&full[s]), 0, krow);
-        tma_load_2d(dst + kTileBytes / 2, &map_k, smem_u32(&full[s]), 64, krow);
+        if (!kF8) tma_load_2d(dst + kTileBytes / 2, &map_k, smem_u32(&full[s]), 64, krow);
         ++issued;
       }
       // on abort, let every issued copy land before the CTA exits
@@ -158,7 +176,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_compute > 0) {
-      const uint32_t idesc = idesc_bf16(128, p.N);
+      const uint32_t idesc = kF8 ? idesc_e4m3(128, p.N) : idesc_bf16(128, p.N);
       bool ok = mbar_wait(smem_u32(bfull), 0, p.status, &abort_flag);
       for (int i = 0; ok && i < n_compute; ++i) {
         const int s = i % p.stages, a = i & 1;
@@ -167,12 +185,21 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         tc_fence_after();
         const uint32_t a0 = sA + (uint32_t)s * kTileBytes;
         const uint32_t d = tmem + (uint32_t)(a * p.N);
+        if (kF8) {
+          // one 128-byte row per key: K = 32 codes (32 bytes) per instruction
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t koff = (uint32_t)(j & 3) * 32u;
-          const uint64_t ad = desc_sw128(a0 + (uint32_t)(j >> 2) * (kTileBytes / 2) + koff);
-          const uint64_t bd = desc_sw128(sB + (uint32_t)(j >> 2) * (uint32_t)p.N * 128u + koff);
-          mma_bf16_ss(d, ad, bd, idesc, j > 0 ? 1u : 0u);
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t koff = (uint32_t)j * 32u;
+            mma_f8_ss(d, desc_sw128(a0 + koff), desc_sw128(sB + koff), idesc, j > 0 ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t koff = (uint32_t)(j & 3) * 32u;
+            const uint64_t ad = desc_sw128(a0 + (uint32_t)(j >> 2) * (kTileBytes / 2) + koff);
+            const uint64_t bd = desc_sw128(sB + (uint32_t)(j >> 2) * (uint32_t)p.N * 128u + koff);
+            mma_bf16_ss(d, ad, bd, idesc, j > 0 ? 1u : 0u);
+          }
         }
         mma_commit(smem_u32(&empty[s]));
         mma_commit(smem_u32(&tfull[a]));
@@ -202,17 +229,23 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
       if (!mbar_wait(smem_u32(&tfull[a]), (ci >> 1) & 1, p.status, &abort_flag)) break;
       tc_fence_after();
       const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * p.N);
+      // FP8: this lane's key scale (keys past the sequence read a neighbour's row or nothing)
+      const float sk = kF8 && s < p.S ? p.k_scale[(size_t)b * p.S + s] : 1.f;
       for (int q = group; q < nq_here; q += ngroups) {
         float acc = 0.f;
         const float* wq = w_s + q * p.HI;
+        const float* sq = ssq_s + q * p.HI;
         for (int h0 = 0; h0 < p.HI; h0 += 32) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(trow + (uint32_t)(q * p.HI + h0), v);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            acc = fmaf(wq[h0 + j], fmaxf(p.scale * __uint_as_float(v[j]), 0.f), acc);
+          for (int j = 0; j < 32; ++j) {
+            const float sc = kF8 ? sq[h0 + j] : p.scale;
+            acc = fmaf(wq[h0 + j], fmaxf(sc * __uint_as_float(v[j]), 0.f), acc);
+          }
         }
+        if (kF8) acc *= sk;
         if (s < p.S) {
           const int lo = lohi[2 * q], hi = lohi[2 * q + 1];
           const float v = (s >= lo && s <= hi) ? (acc == 0.f ? 0.f : acc) : -INFINITY;
@@ -250,23 +283,24 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2D bf16 tensor [rows, 128] (row-major), box [64 cols, box_rows], 128-byte swizzle.
-bool make_map_bf16_128(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows) {
+// 2D tensor [rows, 128] (row-major) of bf16 (box [64 cols, box_rows]) or of e4m3 codes (box [128
+// cols, box_rows]): 128-byte box rows in the 128-byte swizzle.
+bool make_map_128(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows, bool f8) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)kDI, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)kDI * 2};
-  cuuint32_t box[2] = {64u, box_rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes(f8)};
+  cuuint32_t box[2] = {f8 ? 128u : 64u, box_rows};
   cuuint32_t estr[2] = {1u, 1u};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(m, f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr),
+             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
-bool index_scores_tc_supported(const dsa_dims& d) {
-  if (d.dtype != DSA_BF16 || d.idx_dim != kDI) return false;
+bool index_scores_tc_supported(const dsa_dims& d, bool f8) {
+  if ((!f8 && d.dtype != DSA_BF16) || d.idx_dim != kDI) return false;
   if (!(d.idx_heads == 32 || d.idx_heads == 64 || d.idx_heads == 128)) return false;
   if ((long long)d.batch * d.n_kv < 128) return false;  // the key TMA box is 128 rows
   return encode_fn() != nullptr;
@@ -275,7 +309,8 @@ bool index_scores_tc_supported(const dsa_dims& d) {
 cudaError_t launch_index_scores_tc(const dsa_dims& d, const void* q_idx, const void* k_idx,
                                    const float* w, float scale, const int32_t* q_pos,
                                    const int32_t* kv_start, const int32_t* kv_len, float* scores,
-                                   cudaStream_t st) {
+                                   cudaStream_t st, const float* q_scale, const float* k_scale) {
+  const bool f8 = q_scale != nullptr;
   IdxTcParams p{};
   p.B = d.batch;
   p.T = d.n_q;
@@ -312,29 +347,35 @@ cudaError_t launch_index_scores_tc(const dsa_dims& d, const void* q_idx, const v
   splits = (p.n_ktiles + p.tiles_per_split - 1) / p.tiles_per_split;
   p.epi_warps = p.NQ >= 2 ? 8 : 4;
   p.scale = scale;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
   p.w = w;
   p.q_pos = q_pos;
   p.kv_start = kv_start;
   p.kv_len = kv_len;
   p.scores = scores;
   p.status = device_status_ptr();
-  const size_t fixed = 1024 + (size_t)p.N * 256 + (size_t)p.N * 4 + 2 * 16 * 4 + 64 + 8 * (2 * kMaxStages + 8) + 64;
-  int stages = (int)((220 * 1024 - fixed) / kTileBytes);
-  if (stages > kMaxStages) stages = kMaxStages;
-  if (ctas_per_sm == 2 && stages > 2) stages = 2;
+  const size_t tb = (size_t)tile_bytes(f8);
+  const size_t fixed = 1024 + (size_t)p.N * row_bytes(f8) + (size_t)p.N * 4 * (f8 ? 2 : 1) + 2 * 16 * 4 + 64 +
+                       8 * (2 * kMaxStages + 8) + 64;
+  int stages = (int)((220 * 1024 - fixed) / tb);
+  if (stages > (f8 ? kMaxStages : 6)) stages = f8 ? kMaxStages : 6;
+  // two CTAs per SM: two 32 KB stages each (bf16), four 16 KB stages each (e4m3): 64 KB in flight per CTA
+  if (ctas_per_sm == 2 && stages > (f8 ? 4 : 2)) stages = f8 ? 4 : 2;
   if (stages < 2) return cudaErrorInvalidConfiguration;
   p.stages = stages;
-  const size_t smem = fixed + (size_t)stages * kTileBytes;
+  const size_t smem = fixed + (size_t)stages * tb;
 
   CUtensorMap mq, mk;
-  if (!make_map_bf16_128(&mq, q_idx, (uint64_t)d.batch * d.n_q * d.idx_heads, (uint32_t)p.N))
+  if (!make_map_128(&mq, q_idx, (uint64_t)d.batch * d.n_q * d.idx_heads, (uint32_t)p.N, f8))
     return cudaErrorInvalidValue;
-  if (!make_map_bf16_128(&mk, k_idx, (uint64_t)d.batch * d.n_kv, kKeysPerTile)) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(index_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (!make_map_128(&mk, k_idx, (uint64_t)d.batch * d.n_kv, kKeysPerTile, f8)) return cudaErrorInvalidValue;
+  auto kern = f8 ? index_tc_kernel<true> : index_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(splits, p.n_qtiles, p.B);
   const int threads = 64 + 32 * p.epi_warps;
-  index_tc_kernel<<<grid, threads, smem, st>>>(mq, mk, p);
+  kern<<<grid, threads, smem, st>>>(mq, mk, p);
   return cudaGetLastError();
 }
 

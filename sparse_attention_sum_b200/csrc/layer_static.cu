@@ -12,8 +12,11 @@
 // Every GPU that loads the library holds it until the process exits.  Its name
 // in host code is only a host-side stand-in, so the device address is fetched
 // with cudaGetSymbolAddress once per device (on the first call made with that
-// device current) and cached; that first call should therefore happen before
-// any stream capture.  All calls share the array and it keeps the last call's
+// device current) and cached together with the context it was read in; that
+// first call should therefore happen before any stream capture.  After a
+// cudaDeviceReset the device's new context has its own copy of the array, so
+// the next call looks the address up again (make that call outside a capture
+// too).  All calls share the array and it keeps the last call's
 // contents: calls whose work overlaps on the GPU (on different streams, or on
 // different host threads) race on it.  Nothing in the array has to start at
 // zero: the index-score kernel writes every score of the rows it covers and
@@ -33,6 +36,7 @@ __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 void* scratch_address(cudaError_t* err) {
   static std::mutex mu;
+  static void* ctxs[128] = {};
   static void* ptrs[128] = {};
   int dev = 0;
   *err = cudaGetDevice(&dev);
@@ -41,15 +45,15 @@ void* scratch_address(cudaError_t* err) {
     *err = cudaErrorInvalidDevice;
     return nullptr;
   }
+  void* ctx = dsa::current_context();
   std::lock_guard<std::mutex> lock(mu);
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    *err = cudaGetSymbolAddress(&p, g_static_scratch);
-    if (*err != cudaSuccess) return nullptr;
-    ptrs[dev] = p;
-  }
-  *err = cudaSuccess;
-  return ptrs[dev];
+  if (ptrs[dev] && ctx && ctxs[dev] == ctx) return ptrs[dev];
+  void* p = nullptr;
+  *err = cudaGetSymbolAddress(&p, g_static_scratch);
+  if (*err != cudaSuccess) return nullptr;
+  ctxs[dev] = dsa::current_context();  // the lookup binds the primary context if none was current
+  ptrs[dev] = p;
+  return p;
 }
 
 }  // namespace

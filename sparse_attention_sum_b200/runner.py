@@ -6,6 +6,11 @@ is one libdsa call.
   (``dsa_layer_forward``).
 * :func:`kpool_layer` -- S6-S8 with S2-S4 over pools: LayerNorm + pooling,
   pool scores, pool top-k, expand_selection, absorbed NoPE MLA attend.
+* :func:`dsa_layer_fp8` -- the layer with the FP8 indexer: quantise the queries,
+  FP8 scores against a key cache held as e4m3 codes, top-k set, sparse attend.
+* :func:`index_share_stack` -- IndexShare over a stack of layers: the layers
+  :func:`computes_own_selection` names run the whole layer, the others reuse
+  the selection of the last such layer (``idx_in``).
 """
 from __future__ import annotations
 
@@ -13,8 +18,9 @@ from typing import Dict, Optional
 
 import torch
 
-from . import (BF16, F32, OP_LAYER_FORWARD, Dims, absorb_out, absorb_q, expand_selection,
-               index_scores, layer_forward, pool_states, sparse_attend, topk, workspace_size)
+from . import (BF16, F32, OP_LAYER_FORWARD, Dims, absorb_out, absorb_q, expand_selection, fp8_quantize,
+               index_scores, index_scores_fp8, layer_forward, pool_states, sparse_attend, topk, topk_set,
+               workspace_size)
 
 
 def _code(dtype: torch.dtype) -> int:
@@ -64,6 +70,66 @@ def dsa_layer(dims: Dims, q_idx, k_idx, w, idx_scale, q_pos, kv_start, kv_len, q
                   v_row_stride, attn_scale, bufs.out, lse=bufs.lse, idx_in=idx_in, idx_out=bufs.idx,
                   ws=bufs.ws, stream=stream)
     return bufs
+
+
+class Fp8Buffers:
+    """Per-call FP8 query codes and scales of :func:`dsa_layer_fp8`."""
+
+    def __init__(self, dims: Dims, device):
+        shape = (dims.batch, dims.n_q, dims.idx_heads)
+        self.q_codes = torch.empty(*shape, dims.idx_dim, dtype=torch.uint8, device=device)
+        self.q_scales = torch.empty(*shape, dtype=torch.float32, device=device)
+
+
+def dsa_layer_fp8(dims: Dims, q_idx, k_codes, k_scales, w, idx_scale, q_pos, kv_start, kv_len, q, k, v,
+                  attn_scale, k_row_stride: int, v_row_stride: int, bufs: Optional[LayerBuffers] = None,
+                  fp8: Optional[Fp8Buffers] = None, stream=None, k_idx=None) -> LayerBuffers:
+    """The layer with the FP8 indexer, as four libdsa calls: dsa_fp8_quantize of the queries,
+    dsa_index_scores_fp8 against the key cache's e4m3 codes and scales (quantised once, when the keys
+    were written), dsa_topk_set, dsa_sparse_attend.  ``k_idx`` (the bf16 keys) is not read."""
+    if bufs is None:
+        bufs = LayerBuffers(dims, q.device, q.dtype)
+    if fp8 is None:
+        fp8 = Fp8Buffers(dims, q.device)
+    B, T, S = dims.batch, dims.n_q, dims.n_kv
+    scores = bufs.ws[: B * T * S * 4].view(torch.float32).view(B, T, S)
+    fp8_quantize(q_idx, fp8.q_codes, fp8.q_scales, stream=stream)
+    index_scores_fp8(dims, fp8.q_codes, fp8.q_scales, k_codes, k_scales, w, idx_scale, q_pos, kv_start, kv_len,
+                     scores, stream=stream)
+    topk_set(dims, scores, q_pos, kv_start, kv_len, dims.top_k, bufs.idx, stream=stream)
+    sparse_attend(dims, q, k, k_row_stride, v, v_row_stride, bufs.idx, dims.top_k, attn_scale, bufs.out,
+                  lse=bufs.lse, stream=stream)
+    return bufs
+
+
+def computes_own_selection(il: int) -> bool:
+    """IndexShare schedule (ik_llama.cpp PR #2063, IndexShare commit): layer ``il`` runs its own
+    indexer and top-k iff ``il <= 1`` or ``il % 4 == 2``; every other layer reuses the selection of
+    the most recent layer that did."""
+    return il <= 1 or il % 4 == 2
+
+
+def index_share_stack(layers, bufs=None, stream=None):
+    """Runs ``dsa_layer`` over a stack with IndexShare.
+
+    ``layers`` is a list of ``(dims, kwargs)`` pairs in layer order, ``kwargs`` as for
+    :func:`dsa_layer`; every layer's dims must have the same batch, n_q, n_kv and top_k.
+    Returns one :class:`LayerBuffers` per layer; a reusing layer's ``idx`` is the shared selection
+    tensor itself (the one it attended over).  Layer 0 must compute its own selection."""
+    out = []
+    shared = None
+    for il, (dims, kw) in enumerate(layers):
+        b = bufs[il] if bufs is not None else LayerBuffers(dims, kw["q"].device, kw["q"].dtype)
+        if computes_own_selection(il):
+            dsa_layer(dims, **kw, bufs=b, stream=stream)
+            shared = b.idx
+        else:
+            if shared is None:
+                raise ValueError("layer 0 must compute its own selection")
+            dsa_layer(dims, **kw, bufs=b, idx_in=shared, stream=stream)
+            b.idx = shared
+        out.append(b)
+    return out
 
 
 class KpoolBuffers:

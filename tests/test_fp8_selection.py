@@ -38,3 +38,19 @@ def test_fp8_operands_keep_most_of_the_selection_and_swap_only_near_tau(name, si
         assert recall >= 0.95, recall
     assert dist <= 0.08, dist         # swapped keys sit within a few percent of the scale from tau
     assert 1e-3 < err < 0.1, err      # e4m3 noise: far above bf16/fp32 rounding, far below the score scale
+
+
+def test_fp8_exact_recipe_quantises_exactly():
+    """The exact_index='fp8' inputs (integers in [-7, 7], each vector's largest magnitude 7): the oracle's
+    quantiser gives scale 1/64 and codes 64*x for every vector, and the FP8 score equals the plain score
+    exactly, so a GPU FP8 indexer can be held to the oracle bit for bit on these inputs."""
+    wl = workloads.make("prefill", T=40, exact_index="fp8")
+    for x in (wl["q_idx"].reshape(-1, 128), wl["k_idx"].reshape(-1, 128)):
+        codes, sc = O.fp8_quantize(x)
+        assert np.all(sc == 1 / 64)
+        assert np.array_equal(codes, 64 * O.f64(x))
+    for t in (0, 17, 39):
+        cand = O.visible_keys(t, 0, wl.n_kv)
+        a = O.index_scores_fp8_row(wl["q_idx"][0, t], wl["k_idx"][0][cand], wl["w"][0, t], wl.idx_scale)
+        b = O.index_scores_row(wl["q_idx"][0, t], wl["k_idx"][0][cand], wl["w"][0, t], wl.idx_scale)
+        assert np.array_equal(a, b)

@@ -14,7 +14,7 @@ import sparse_attention_sum_b200 as dsa
 from sparse_attention_sum_b200 import runner
 import workloads
 from tests.gpu_common import (ATOL, assert_attend_close, check_selection_in_band, cosine, dev, key_order,
-                              kv_views, layer_inputs, sample_rows)
+                              kv_views, layer_inputs, report, sample_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -95,6 +95,44 @@ def test_tiny_layer_covering_all_keys_is_dense_attention():
     K, V = kv_views(wl)
     dense = O.dense_causal_attend(wl["q"], K, V, wl.attn_scale, wl["q_pos"], wl["kv_start"], wl["kv_len"])
     assert_attend_close(_np(bufs.out), dense, torch.float32, "dense reduction")
+
+
+# --------------------------------- tensor-core indexer on exact (integer) scores
+@pytest.mark.parametrize("name,sizes,top_k", [("prefill", dict(T=1000), 256), ("decode", dict(B=3, S=5000), 2048),
+                                              ("chunked", dict(T=130, S=4500), 512)])
+def test_integer_indexer_on_tensor_cores_is_exact(name, sizes, top_k):
+    """The bf16 indexer at its full shape (64 heads x 128) on integer inputs (q_I, k_I in [-4, 4],
+    w in {1/2, 1, 2, 4}, scale 1/8): every score is a multiple of 1/16 below 2^17, so the tcgen05
+    kernel's TMEM accumulation, relu*w epilogue, signed-zero rule and skipped tiles must give the
+    oracle's scores exactly, and the selection must be the oracle's bit for bit (with many genuine
+    ties for the index tie-break).  Prefill runs 8 query tiles x 8 key tiles with ragged tails,
+    decode the narrow two-CTA-per-SM configuration with key-range splits, chunked a causal offset
+    with hot spots."""
+    wl = workloads.make(name, exact_index=True, **sizes)
+    wl.top_k = top_k
+    t = dev(wl)
+    dims, a = layer_inputs(wl, t)
+    B, T, S = wl.batch, wl.n_q, wl.n_kv
+    scores = torch.empty(B, T, S, dtype=torch.float32, device="cuda")
+    dsa.index_scores(dims, a["q_idx"], a["k_idx"], a["w"], a["idx_scale"], a["q_pos"], a["kv_start"],
+                     a["kv_len"], scores)
+    assert dsa.last_kernels() == ["index_tc"]
+    idx = torch.empty(B, T, top_k, dtype=torch.int32, device="cuda")
+    dsa.topk(dims, scores, a["q_pos"], a["kv_start"], a["kv_len"], top_k, idx)
+    fused = runner.dsa_layer(dims, **a)
+    assert dsa.last_kernels() == ["index_tc", "topk_set", "attend_tc"]
+    torch.cuda.synchronize()
+    ref = O.index_scores(wl["q_idx"], wl["k_idx"], wl["w"], wl.idx_scale, wl["q_pos"], wl["kv_start"],
+                         wl["kv_len"])
+    got = scores.cpu().numpy().astype(np.float64)
+    assert np.array_equal(got, ref)
+    assert not np.any(np.signbit(got[got == 0]))                  # zero scores are +0
+    ref_idx = O.topk(ref, top_k, wl["q_pos"], wl["kv_start"], wl["kv_len"])
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    assert torch.equal(fused.idx, key_order(torch.tensor(ref_idx, dtype=torch.int32, device="cuda")))
+    n_ties = int(sum(np.sum(ref[b, tt] == ref[b, tt, ref_idx[b, tt, -1]]) > 1
+                     for b in range(B) for tt in range(T) if ref_idx[b, tt, -1] >= 0))
+    report(f"exact indexer {name}", rows=B * T, rows_with_tie_at_kth=n_ties)
 
 
 # --------------------------------------------------------- top-k edge cases
@@ -242,7 +280,7 @@ def test_small_bf16_layer_against_oracle(name, sizes):
     fused = runner.dsa_layer(dims, **a)
     torch.cuda.synchronize()
     assert torch.equal(fused.idx, key_order(idx))
-    assert_attend_close(_np(fused.out), _np(out), torch.bfloat16, f"{name} fused vs composition")
+    assert_attend_close(_np(fused.out), _np(out), torch.bfloat16, f"{name} fused vs composition", gpu_pair=True)
 
 
 @pytest.mark.parametrize("name,sizes,top_k", [("prefill", dict(T=300), 96), ("decode", dict(B=2, S=5000), 2048)])
@@ -328,8 +366,65 @@ def test_tensor_core_kernels_match_cuda_core_kernels(name, sizes, top_k):
         outs.append((o, l))
     dsa.set_kernel_policy(0)
     torch.cuda.synchronize()
-    assert_attend_close(_np(outs[1][0]), _np(outs[0][0]), torch.bfloat16, "tc vs simt attend")
+    assert_attend_close(_np(outs[1][0]), _np(outs[0][0]), torch.bfloat16, "tc vs simt attend", gpu_pair=True)
     assert (outs[1][1] - outs[0][1]).abs().max().item() <= 2e-3
+
+
+# ------------------------------------------------- caches past 16-bit key indices
+def test_long_cache_layer_stays_on_tensor_cores():
+    """A 70000-key cache (past 65536, where a key index needs more than 16 bits): the fused layer
+    still runs index_tc, topk_set and attend_tc, and every row matches the oracle."""
+    S = 70000
+    wl = workloads.make("decode", B=3, S=S)
+    t = dev(wl)
+    dims, a = layer_inputs(wl, t)
+    bufs = runner.LayerBuffers(dims, "cuda", torch.bfloat16, with_idx=True, with_lse=True)
+    runner.dsa_layer(dims, **a, bufs=bufs)
+    assert dsa.last_kernels() == ["index_tc", "topk_set", "attend_tc"]
+    torch.cuda.synchronize()
+    scores = bufs.ws[: 3 * S * 4].view(torch.float32).view(3, 1, S)
+    g_idx, g_out, g_lse = bufs.idx.cpu().numpy(), _np(bufs.out), bufs.lse.cpu().numpy()
+    assert int((bufs.idx > 65535).sum()) > 1000          # the selection reaches past 16 bits
+    K, V = kv_views(wl)
+    for b in range(3):
+        cand = O.visible_keys(S - 1, 0, S)
+        ref = O.index_scores_row(wl["q_idx"][b, 0], wl["k_idx"][b], wl["w"][b, 0], wl.idx_scale)
+        gs = scores[b, 0].cpu().numpy().astype(np.float64)
+        assert np.abs(gs - ref).max() <= 2e-5 * max(1.0, np.abs(ref).max())
+        assert g_idx[b, 0].tolist() == key_order(O.topk_row(cand, gs, wl.top_k).tolist())
+        check_selection_in_band(g_idx[b, 0], cand, ref, wl.top_k, f"long cache row {b}")
+        ro, rl = O.sparse_attend_row(wl["q"][b, 0], K[b], V[b], g_idx[b, 0], wl.attn_scale)
+        assert_attend_close(g_out[b, 0], ro, torch.bfloat16, f"long cache out {b}")
+        np.testing.assert_allclose(g_lse[b, 0], rl, atol=2e-3)
+
+
+@pytest.mark.parametrize("H,kd", [(128, 576), (64, 512)])
+def test_long_cache_attend_set_semantics(H, kd):
+    """dsa_sparse_attend on the tensor cores over a 70000-row latent with index rows that mix keys
+    above and below 65536, duplicates (the first-occurrence compaction), INVALID and out-of-range
+    entries, against the oracle's set-semantics attention."""
+    rng = np.random.default_rng(H)
+    B, T, S, W = 1, 130 if H == 64 else 6, 70000, 2048
+    q = torch.tensor(rng.standard_normal((B, T, H, kd)), dtype=torch.bfloat16)
+    lat = torch.tensor(rng.standard_normal((B, S, kd)) * 0.5, dtype=torch.bfloat16)
+    idx = rng.integers(0, S, size=(B, T, W)).astype(np.int32)
+    idx[0, 0, ::5] = O.INVALID
+    idx[0, 1, 1024:] = idx[0, 1, :1024]                   # duplicates
+    idx[0, 2, ::9] = S + 5                                # out of range
+    idx[0, 3, :] = np.arange(65536 - 1024, 65536 + 1024)  # straddles the 16-bit boundary
+    d = dsa.Dims(batch=B, n_q=T, n_kv=S, heads=H, kv_heads=1, kd=kd, vd=512, top_k=W, dtype=dsa.BF16)
+    out = torch.empty(B, T, H, 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, T, H, dtype=torch.float32, device="cuda")
+    ld = lat.cuda()
+    dsa.sparse_attend(d, q.cuda(), ld, kd, ld, kd, torch.tensor(idx).cuda(), W, 0.07, out, lse)
+    assert dsa.last_kernels() == ["attend_tc"]
+    torch.cuda.synchronize()
+    K, V = lat.unsqueeze(2), lat[..., :512].unsqueeze(2)
+    rows = range(T) if T <= 8 else list(range(6)) + [64, 100, T - 1]
+    for tt in rows:
+        ro, rl = O.sparse_attend_row(q[0, tt], K[0], V[0], idx[0, tt], 0.07)
+        assert_attend_close(_np(out[0, tt]), ro, torch.bfloat16, f"wide attend H{H} row {tt}")
+        np.testing.assert_allclose(lse[0, tt].cpu().numpy(), rl, atol=2e-3)
 
 
 # ------------------------------------------------------------- kpool (small)
@@ -358,6 +453,7 @@ def _kpool_check(wl, bufs, rows):
     out = _np(bufs.out)
     q_lat = _np(bufs.q_lat)
     refpool = {}
+    worst = (1.0, 0.0)
     for b in range(B):
         f, L = int(wl["kv_start"][b]), int(wl["kv_len"][b])
         assert npools[b] == O.n_pools_of(f, L, kp)
@@ -383,9 +479,12 @@ def _kpool_check(wl, bufs, rows):
         # absorbed attention over the GPU's token rows vs the literal expand_kv form
         ro, _ = O.mla_masked_attention_row(wl["q_nope"][b, tt], wl["latent"][b], wl["w_uk"], wl["w_uv"],
                                            tok_idx[b, tt], wl.attn_scale)
-        assert_attend_close(out[b, tt], ro, torch.bfloat16, f"kpool out {(b, tt)}")
+        c, r = assert_attend_close(out[b, tt], ro, torch.bfloat16, f"kpool out {(b, tt)}")
+        worst = (min(worst[0], c), max(worst[1], r))
         np.testing.assert_allclose(q_lat[b, tt], O.absorb_q(wl["q_nope"][b, tt][None], wl["w_uk"])[0],
                                    atol=3e-2, rtol=1e-2)
+    report(f"kpool T={wl.n_q}", rows=len(rows), worst_cosine=f"{worst[0]:.7f}",
+           worst_maxabs_over_rms=f"{worst[1]:.4f}")
 
 
 def test_kpool_small_against_oracle():
@@ -411,25 +510,35 @@ def _full_layer(name):
 
 @pytest.mark.parametrize("name", ["prefill", "decode", "chunked"])
 def test_full_size_layer_sampled_rows(name):
+    """The workloads bench.py times, in its launch configuration: 256 sampled query rows (every
+    row of decode's 64) against the oracle element by element, structure on every row."""
     wl, t, dims, bufs = _full_layer(name)
     B, T, S = wl.batch, wl.n_q, wl.n_kv
     scores = bufs.ws[: B * T * S * 4].view(torch.float32).view(B, T, S)
     g_idx = bufs.idx.cpu().numpy()
+    g_out = bufs.out.cpu()
+    g_lse = bufs.lse.cpu().numpy()
     K, V = kv_views(wl)
-    rows = sample_rows(wl, 12)
+    rows = [(b, tt) for b in range(B) for tt in range(T)] if B * T <= 256 else sample_rows(wl, 256)
     diffs = 0
+    worst_cos, worst_rel, worst_idx = 1.0, 0.0, 0.0
     for b, tt in rows:
         p, ks, kl = int(wl["q_pos"][b, tt]), int(wl["kv_start"][b]), int(wl["kv_len"][b])
         cand = O.visible_keys(p, ks, kl)
         ref = O.index_scores_row(wl["q_idx"][b, tt], wl["k_idx"][b][cand], wl["w"][b, tt], wl.idx_scale)
         gs = scores[b, tt].cpu().numpy().astype(np.float64)[cand]
-        assert np.abs(gs - ref).max() <= 2e-5 * max(1.0, np.abs(ref).max())
+        err = np.abs(gs - ref).max() / max(1.0, np.abs(ref).max())
+        assert err <= 2e-5, (b, tt, err)
+        worst_idx = max(worst_idx, err)
         assert g_idx[b, tt].tolist() == key_order(O.topk_row(cand, gs, wl.top_k).tolist())
         diffs += check_selection_in_band(g_idx[b, tt], cand, ref, wl.top_k, f"{name} {(b, tt)}") > 0
         ro, rl = O.sparse_attend_row(wl["q"][b, tt], K[b], V[b], g_idx[b, tt], wl.attn_scale)
-        assert_attend_close(_np(bufs.out[b, tt]), ro, torch.bfloat16, f"{name} out {(b, tt)}")
-        np.testing.assert_allclose(bufs.lse[b, tt].cpu().numpy(), rl, atol=2e-3)
+        c, r = assert_attend_close(_np(g_out[b, tt]), ro, torch.bfloat16, f"{name} out {(b, tt)}")
+        worst_cos, worst_rel = min(worst_cos, c), max(worst_rel, r)
+        np.testing.assert_allclose(g_lse[b, tt], rl, atol=2e-3)
     assert diffs <= max(1, len(rows) // 4)
+    report(f"full {name}", rows=len(rows), index_err_over_scale=f"{worst_idx:.2e}", rows_in_tie_band=diffs,
+           worst_cosine=f"{worst_cos:.7f}", worst_maxabs_over_rms=f"{worst_rel:.4f}")
     # every row: count, visibility, ascending key order, and the same set dsa_topk ranks
     sel = bufs.idx
     qp = t["q_pos"].view(B, T, 1).long()
@@ -486,7 +595,7 @@ def test_ragged_batch_with_a_fully_padded_sequence():
 def test_full_size_kpool_sampled_rows():
     wl = workloads.make("kpool")
     bufs = _kpool_run(wl)
-    rows = sample_rows(wl, 8, extra=[(3, 1028), (3, 1029), (1, 20)])
+    rows = sample_rows(wl, 256, extra=[(3, 1028), (3, 1029), (1, 20)])
     _kpool_check(wl, bufs, rows)
 
 
@@ -518,15 +627,83 @@ def test_multi_sequence_batch_equals_sequences_alone():
         assert torch.equal(alone.out[0], whole.out[b])
 
 
-def test_index_reuse_skips_selection():
-    wl = workloads.make("prefill", T=300)
-    wl.top_k = 64
+def test_index_share_attends_over_a_foreign_selection():
+    """IndexShare (ik_llama.cpp PR #2063): idx_in is another layer's selection.  Here it is the
+    oracle's top-k over a different seed's indexer inputs, with INVALID padding, repeated keys,
+    out-of-range entries and an empty row planted in it; the fused layer must skip S2/S3 (its own
+    indexer inputs are never read, idx_out is never written) and attend over that selection as a
+    set, equal to the oracle's attention row by row."""
+    T, top_k = 300, 96
+    wl = workloads.make("prefill", T=T)
+    other = workloads.make("prefill", seed=77, T=T)
+    wl.top_k = top_k
+    ref_scores = O.index_scores(other["q_idx"], other["k_idx"], other["w"], other.idx_scale, other["q_pos"],
+                                other["kv_start"], other["kv_len"])
+    sel = O.topk(ref_scores, top_k, other["q_pos"], other["kv_start"], other["kv_len"]).astype(np.int32)
+    sel[0, 120:130, 80:] = O.INVALID                          # padding inside a full row
+    sel[0, 130:140, 48:] = sel[0, 130:140, :48]               # every key twice
+    sel[0, 140:150, ::7] = T + 13                             # out of range
+    sel[0, 150] = O.INVALID                                   # empty row
+    sel[0, 151, :] = sel[0, 151, 0]                           # one key, repeated
     t = dev(wl)
     dims, a = layer_inputs(wl, t)
-    first = runner.dsa_layer(dims, **a)
-    again = runner.dsa_layer(dims, **a, idx_in=first.idx.clone(), bufs=runner.LayerBuffers(dims, "cuda", torch.bfloat16))
+    a["q_idx"] = torch.full_like(a["q_idx"], float("nan"))   # must not be read
+    idx_in = torch.tensor(sel).cuda()
+    bufs = runner.LayerBuffers(dims, "cuda", torch.bfloat16, with_idx=True, with_lse=True)
+    bufs.idx.fill_(12345)
+    runner.dsa_layer(dims, **a, bufs=bufs, idx_in=idx_in)
+    assert dsa.last_kernels() == ["attend_tc"]
     torch.cuda.synchronize()
-    assert torch.equal(first.out, again.out)
+    assert bool((bufs.idx == 12345).all())
+    K, V = kv_views(wl)
+    g_out, g_lse = _np(bufs.out), bufs.lse.cpu().numpy()
+    worst = (1.0, 0.0)
+    for tt in range(T):
+        ro, rl = O.sparse_attend_row(wl["q"][0, tt], K[0], V[0], sel[0, tt], wl.attn_scale)
+        if tt == 150:
+            assert np.all(g_out[0, tt] == 0) and np.all(np.isneginf(g_lse[0, tt]))
+            continue
+        c, r = assert_attend_close(g_out[0, tt], ro, torch.bfloat16, f"foreign selection row {tt}")
+        worst = (min(worst[0], c), max(worst[1], r))
+        np.testing.assert_allclose(g_lse[0, tt], rl, atol=2e-3)
+    report("index share, foreign selection", rows=T, worst_cosine=f"{worst[0]:.7f}",
+           worst_maxabs_over_rms=f"{worst[1]:.4f}")
+    # the same rows through dsa_sparse_attend: identical bits
+    again = torch.empty_like(bufs.out)
+    dsa.sparse_attend(dims, a["q"], a["k"], a["k_row_stride"], a["v"], a["v_row_stride"], idx_in, top_k,
+                      a["attn_scale"], again)
+    torch.cuda.synchronize()
+    assert torch.equal(again, bufs.out)
+
+
+def test_index_share_stack_follows_the_layer_schedule():
+    """A 7-layer stack under IndexShare: layers 0, 1, 2 and 6 run their own indexer and top-k (il <= 1
+    or il % 4 == 2), layers 3-5 reuse layer 2's selection.  Each layer has its own inputs; every
+    layer's output equals the oracle's attention over the selection that layer used, and each
+    computing layer's selection is its own indexer's (within the tie band of the oracle scores)."""
+    T, top_k = 200, 64
+    layers, wls = [], []
+    for il in range(7):
+        wl = workloads.make("prefill", seed=100 + il, T=T)
+        wl.top_k = top_k
+        t = dev(wl)
+        dims, a = layer_inputs(wl, t)
+        layers.append((dims, a))
+        wls.append(wl)
+    outs = runner.index_share_stack(layers)
+    torch.cuda.synchronize()
+    assert [runner.computes_own_selection(il) for il in range(7)] == [True, True, True, False, False, False, True]
+    assert outs[3].idx is outs[2].idx and outs[5].idx is outs[2].idx and outs[6].idx is not outs[2].idx
+    for il, (wl, b) in enumerate(zip(wls, outs)):
+        g_idx, g_out = b.idx.cpu().numpy(), _np(b.out)
+        K, V = kv_views(wl)
+        for tt in (0, 63, 64, 117, T - 1):
+            if runner.computes_own_selection(il):
+                cand = O.visible_keys(tt, 0, T)
+                ref = O.index_scores_row(wl["q_idx"][0, tt], wl["k_idx"][0][cand], wl["w"][0, tt], wl.idx_scale)
+                check_selection_in_band(g_idx[0, tt], cand, ref, top_k, f"layer {il} row {tt}")
+            ro, _ = O.sparse_attend_row(wl["q"][0, tt], K[0], V[0], g_idx[0, tt], wl.attn_scale)
+            assert_attend_close(g_out[0, tt], ro, torch.bfloat16, f"layer {il} row {tt}")
 
 
 def test_bounded_wait_expires_and_reports_timeout():
@@ -536,3 +713,60 @@ def test_bounded_wait_expires_and_reports_timeout():
     assert dsa.get_device_status() == 0       # cleared
     x = torch.ones(4, device="cuda") * 2
     assert x.sum().item() == 8
+
+
+# ------------------------------------------- fused indexer -> top-k (no score matrix)
+@pytest.mark.parametrize("name,sizes,top_k", [("decode", dict(B=5, S=32768), 2048), ("decode", dict(B=3, S=5000), 2048),
+                                              ("decode", dict(B=2, S=70000), 2048), ("prefill", dict(T=300), 96),
+                                              ("chunked", dict(T=40, S=4500), 512)])
+def test_fused_index_topk_equals_scores_then_topk_set(name, sizes, top_k):
+    """dsa_index_topk (one cluster per query row: scores in shared memory, radix select across the
+    cluster) selects exactly what dsa_index_scores + dsa_topk_set select, listed the same way, and
+    writes nothing but the index rows.  Cases: decode rows of 32768 keys (two CTAs per row), short
+    caches (one CTA), 70000 keys (eight CTAs), causal prefill rows with fewer visible keys than k,
+    and a chunked offset with hot spots."""
+    wl = workloads.make(name, **sizes)
+    wl.top_k = top_k
+    t = dev(wl)
+    dims, a = layer_inputs(wl, t)
+    B, T, S = wl.batch, wl.n_q, wl.n_kv
+    fused = torch.full((B, T, top_k), 12345, dtype=torch.int32, device="cuda")
+    dsa.index_topk(dims, a["q_idx"], a["k_idx"], a["w"], a["idx_scale"], a["q_pos"], a["kv_start"], a["kv_len"],
+                   top_k, fused)
+    assert dsa.last_kernels() == ["index_topk"]
+    scores = torch.empty(B, T, S, dtype=torch.float32, device="cuda")
+    dsa.index_scores(dims, a["q_idx"], a["k_idx"], a["w"], a["idx_scale"], a["q_pos"], a["kv_start"], a["kv_len"],
+                     scores)
+    ref = torch.empty_like(fused)
+    dsa.topk_set(dims, scores, a["q_pos"], a["kv_start"], a["kv_len"], top_k, ref)
+    torch.cuda.synchronize()
+    if T == 1:
+        # one query per row: the same tcgen05 tile shape as the standalone indexer, identical scores
+        assert torch.equal(fused, ref)
+    else:
+        # several queries per tile in the standalone indexer: compare each row against the oracle
+        g = fused.cpu().numpy()
+        for b, tt in sample_rows(wl, 24):
+            cand = O.visible_keys(int(wl["q_pos"][b, tt]), int(wl["kv_start"][b]), int(wl["kv_len"][b]))
+            r = O.index_scores_row(wl["q_idx"][b, tt], wl["k_idx"][b][cand], wl["w"][b, tt], wl.idx_scale)
+            check_selection_in_band(g[b, tt], cand, r, top_k, f"fused {name} {(b, tt)}")
+            assert g[b, tt].tolist() == key_order(g[b, tt].tolist())
+        n_same = int((fused == ref).all(-1).sum())
+        report(f"fused index_topk {name}", rows=B * T, rows_equal_to_unfused=n_same)
+
+
+def test_fused_index_topk_is_exact_on_integer_scores():
+    """Integer indexer inputs (exact scores, many ties at the k-th score) at decode and prefill shapes:
+    the fused selection equals the oracle's top-k set bit for bit."""
+    for name, sizes, top_k in (("decode", dict(B=4, S=20000), 2048), ("prefill", dict(T=400), 128)):
+        wl = workloads.make(name, exact_index=True, **sizes)
+        t = dev(wl)
+        dims, a = layer_inputs(wl, t)
+        got = torch.empty(wl.batch, wl.n_q, top_k, dtype=torch.int32, device="cuda")
+        dsa.index_topk(dims, a["q_idx"], a["k_idx"], a["w"], a["idx_scale"], a["q_pos"], a["kv_start"],
+                       a["kv_len"], top_k, got)
+        torch.cuda.synchronize()
+        ref = O.index_scores(wl["q_idx"], wl["k_idx"], wl["w"], wl.idx_scale, wl["q_pos"], wl["kv_start"],
+                             wl["kv_len"])
+        want = O.topk(ref, top_k, wl["q_pos"], wl["kv_start"], wl["kv_len"])
+        assert torch.equal(got.cpu(), key_order(torch.tensor(want, dtype=torch.int32))), name

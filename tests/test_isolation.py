@@ -59,10 +59,14 @@ def test_bench_reaches_the_oracle_only_from_its_cpu_arms():
                 users.add(fn.name)
     top = {n.module for n in tree.body if isinstance(n, ast.ImportFrom) and n.module}
     assert not any(m.startswith("oracle") for m in top), "bench.py imports the oracle at module level"
-    assert users == {"oracle_rows"}, users
-    callers = set()
+    assert users == {"oracle_rows", "oracle_kpool_rows"}, users
+    # the oracle row functions are called only by the CPU arms, or handed to cpu_baseline as its row_fn
+    allowed = {"cpu_baseline", "run_reference"}
     for fn in [n for n in ast.walk(tree) if isinstance(n, ast.FunctionDef)]:
+        as_row_fn = set()
         for node in ast.walk(fn):
-            if isinstance(node, ast.Call) and getattr(node.func, "id", None) == "oracle_rows":
-                callers.add(fn.name)
-    assert callers <= {"cpu_baseline", "run_reference"}, callers
+            if isinstance(node, ast.Call) and getattr(node.func, "id", None) == "cpu_baseline":
+                as_row_fn |= {id(k.value) for k in node.keywords if k.arg == "row_fn"}
+        for node in ast.walk(fn):
+            if isinstance(node, ast.Name) and node.id in users and fn.name not in users:
+                assert fn.name in allowed or id(node) in as_row_fn, f"{fn.name} reaches {node.id}"

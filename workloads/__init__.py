@@ -117,16 +117,41 @@ def _tiny(seed: int) -> Workload:
     return wl
 
 
-def _mla_common(name, seed, B, T, S, q_pos, latent_std, hot_spots=False) -> Workload:
+def _int_vectors(g: torch.Generator, shape, fp8: bool) -> torch.Tensor:
+    """Integer indexer vectors: uniform in [-4, 4]; with ``fp8``, uniform in [-7, 7] with one entry
+    of every vector (last axis) set to 7, so that every vector's largest magnitude is exactly 7."""
+    if not fp8:
+        return torch.randint(-4, 5, shape, generator=g)
+    x = torch.randint(-7, 8, shape, generator=g)
+    pos = torch.randint(0, shape[-1], shape[:-1], generator=g)
+    x.scatter_(-1, pos.unsqueeze(-1), 7)
+    return x
+
+
+def _mla_common(name, seed, B, T, S, q_pos, latent_std, hot_spots=False, exact_index=False) -> Workload:
+    """The bf16 MLA workloads.  ``exact_index`` swaps the indexer inputs for the
+    integer recipe of the tiny workload (q_I, k_I integers in [-4, 4], w in
+    {1/2, 1, 2, 4}, indexer scale 1/8) at the same shapes: every score is then a
+    multiple of 1/16 below 2^17, exact in fp32 whatever the summation order.
+    ``exact_index="fp8"`` draws q_I, k_I in [-7, 7] with each vector's largest
+    magnitude exactly 7 (no hot spots): scores stay multiples of 1/16 below 2^19,
+    and a per-vector e4m3 quantisation with scale amax/448 is then exact (scale
+    1/64, codes 64*x)."""
     g = torch.Generator().manual_seed(seed)
     HI, DI, H, KD, VD = 64, 128, 128, 576, 512
     wl = Workload(name, seed, "bf16", B, T, S, HI, DI, 2048, H, 1, KD, VD,
-                  idx_scale=1.0 / math.sqrt(128.0), attn_scale=1.0 / math.sqrt(192.0))
+                  idx_scale=1.0 / 8.0 if exact_index else 1.0 / math.sqrt(128.0),
+                  attn_scale=1.0 / math.sqrt(192.0))
     ts = wl.tensors
-    ts["q_idx"] = _randn_bf16(g, (B, T, HI, DI))
+    if exact_index:
+        ts["q_idx"] = _int_vectors(g, (B, T, HI, DI), exact_index == "fp8").to(torch.bfloat16)
+    else:
+        ts["q_idx"] = _randn_bf16(g, (B, T, HI, DI))
+    if exact_index == "fp8" and hot_spots:
+        raise ValueError("exact_index='fp8' needs every key's largest magnitude to stay 7 (no hot spots)")
     k_idx = torch.empty(B, S, DI, dtype=torch.bfloat16)
     for b in range(B):
-        kb = _randn(g, (S, DI))
+        kb = _int_vectors(g, (S, DI), exact_index == "fp8").to(torch.float32) if exact_index else _randn(g, (S, DI))
         if hot_spots:
             # 10% of the keys (51 runs of 64) get +3 on every indexer-key channel.
             starts = hot_spot_runs(g, S, max(1, (S // 10) // 64), 64)
@@ -134,7 +159,10 @@ def _mla_common(name, seed, B, T, S, q_pos, latent_std, hot_spots=False) -> Work
                 kb[s0:s0 + 64] += 3.0
         k_idx[b] = kb.to(torch.bfloat16)
     ts["k_idx"] = k_idx
-    ts["w"] = _randn(g, (B, T, HI), std=1.0 / 8.0)
+    if exact_index:
+        ts["w"] = torch.tensor([0.5, 1.0, 2.0, 4.0])[torch.randint(0, 4, (B, T, HI), generator=g)]
+    else:
+        ts["w"] = _randn(g, (B, T, HI), std=1.0 / 8.0)
     ts["q"] = _randn_bf16(g, (B * T, H, KD)).view(B, T, H, KD)
     ts["latent"] = _randn_bf16(g, (B * S, KD), std=latent_std).view(B, S, KD)
     ts["q_pos"] = q_pos.to(torch.int32)
@@ -143,19 +171,20 @@ def _mla_common(name, seed, B, T, S, q_pos, latent_std, hot_spots=False) -> Work
     return wl
 
 
-def _prefill(seed: int, T: int = 4096) -> Workload:
+def _prefill(seed: int, T: int = 4096, exact_index: bool = False) -> Workload:
     q_pos = torch.arange(T).view(1, T)
-    return _mla_common("prefill", seed, 1, T, T, q_pos, latent_std=0.5)
+    return _mla_common("prefill", seed, 1, T, T, q_pos, latent_std=0.5, exact_index=exact_index)
 
 
-def _decode(seed: int, B: int = 64, S: int = 32768) -> Workload:
+def _decode(seed: int, B: int = 64, S: int = 32768, exact_index: bool = False) -> Workload:
     q_pos = torch.full((B, 1), S - 1)
-    return _mla_common("decode", seed, B, 1, S, q_pos, latent_std=0.5)
+    return _mla_common("decode", seed, B, 1, S, q_pos, latent_std=0.5, exact_index=exact_index)
 
 
-def _chunked(seed: int, T: int = 4096, S: int = 32768) -> Workload:
+def _chunked(seed: int, T: int = 4096, S: int = 32768, exact_index: bool = False) -> Workload:
     q_pos = (S - T + torch.arange(T)).view(1, T)
-    return _mla_common("chunked", seed, 1, T, S, q_pos, latent_std=1.0, hot_spots=True)
+    return _mla_common("chunked", seed, 1, T, S, q_pos, latent_std=1.0, hot_spots=True,
+                       exact_index=exact_index)
 
 
 def _kpool(seed: int, T: int = 8192, pads=(0, 17, 513, 1029)) -> Workload:
@@ -192,7 +221,9 @@ def make(name: str, seed: Optional[int] = None, **sizes) -> Workload:
     """Build workload ``name`` (one of :data:`NAMES`).
 
     ``sizes`` overrides the sequence/batch sizes (``T``, ``S``, ``B``, ``pads``)
-    for scaled-down parity cases; the distributions stay the same.
+    for scaled-down parity cases; the distributions stay the same.  The bf16 MLA
+    workloads also take ``exact_index=True`` (integer indexer inputs, see
+    ``_mla_common``).
     """
     if name not in _BUILDERS:
         raise KeyError(f"unknown workload {name!r}; expected one of {NAMES}")
