@@ -506,6 +506,44 @@ def fp8_indexer_extra(wl, t, dims, args, bufs, peaks, flush, stream, steps):
     return res
 
 
+def fused_select_extra(wl, t, dims, args, bufs, peaks, flush, stream, steps):
+    """The selection without a score matrix (dsa_index_topk, and dsa_index_topk_fp8 on a key cache held as
+    e4m3 codes), alone and followed by the sparse attend, against the two-kernel selection."""
+    import sparse_attention_sum_b200 as dsa
+    from sparse_attention_sum_b200 import runner
+    B, T, S = wl.batch, wl.n_q, wl.n_kv
+    rows = B * T
+    a = args
+    k_codes = torch.empty(B, S, 128, dtype=torch.uint8, device="cuda")
+    k_scales = torch.empty(B, S, dtype=torch.float32, device="cuda")
+    dsa.fp8_quantize(t["k_idx"], k_codes, k_scales)
+    fp8 = runner.Fp8Buffers(dims, "cuda")
+    sel = lambda: dsa.index_topk(dims, a["q_idx"], a["k_idx"], a["w"], a["idx_scale"], a["q_pos"], a["kv_start"],
+                                 a["kv_len"], wl.top_k, bufs.idx)
+
+    def sel8():
+        dsa.fp8_quantize(t["q_idx"], fp8.q_codes, fp8.q_scales)
+        dsa.index_topk_fp8(dims, fp8.q_codes, fp8.q_scales, k_codes, k_scales, a["w"], a["idx_scale"], a["q_pos"],
+                           a["kv_start"], a["kv_len"], wl.top_k, bufs.idx)
+    att = lambda: dsa.sparse_attend(dims, a["q"], a["k"], a["k_row_stride"], a["v"], a["v_row_stride"], bufs.idx,
+                                    wl.top_k, a["attn_scale"], bufs.out)
+    med = lambda f: statistics.median(time_steps(f, max(3, steps), 3, flush, stream))
+    t_sel, t_sel8 = med(sel), med(sel8)
+    t_layer = med(lambda: (sel(), att()))
+    t_layer8 = med(lambda: (sel8(), att()))
+    nvis = int(visible_counts(wl).sum())
+    sel_bytes = B * S * 256 + rows * wl.idx_heads * (256 + 4) + 4.0 * rows * wl.top_k
+    sel8_bytes = B * S * (128 + 4) + rows * wl.idx_heads * (256 + 128 + 4 + 4 + 4) + 4.0 * rows * wl.top_k
+    res = {"select_us": round(t_sel * 1e6, 1), "select_fp8_us": round(t_sel8 * 1e6, 1),
+           "layer_ms": round(t_layer * 1e3, 4), "layer_value": round(rows / t_layer, 1),
+           "layer_fp8_ms": round(t_layer8 * 1e3, 4), "layer_fp8_value": round(rows / t_layer8, 1), "unit": UNIT,
+           "roofline_select": roofline_entry("hbm", sel_bytes, t_sel, peaks),
+           "roofline_select_fp8": roofline_entry("hbm", sel8_bytes, t_sel8, peaks),
+           "index_flop": 2.0 * nvis * wl.idx_heads * wl.idx_dim}
+    del k_codes, k_scales, fp8
+    return res
+
+
 def decode_extra(peaks, flush, stream, cpu_s=0.0):
     """The decode workload (64 sequences x 1 query vs 32768 cached keys) and its stages."""
     from sparse_attention_sum_b200 import runner
@@ -527,6 +565,7 @@ def decode_extra(peaks, flush, stream, cpu_s=0.0):
            "fused_hbm_frac": round((wk["index_bytes"] + wk["topk_bytes"] + wk["attend_bytes"]) / step / 1e9
                                    / peaks["hbm_gbs"], 4)}
     res["fp8_indexer"] = fp8_indexer_extra(wl, t, dims, args, bufs, peaks, flush, stream, 10)
+    res["fused_select"] = fused_select_extra(wl, t, dims, args, bufs, peaks, flush, stream, 10)
     if cpu_s > 0:
         res["cpu_baseline"] = cpu_baseline(wl, budget_s=cpu_s, whole=True)
     del t, bufs

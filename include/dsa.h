@@ -260,8 +260,12 @@ dsa_status dsa_sparse_attend(const dsa_dims* dims, const void* q, const void* k,
  * selection is written to idx_out [B,T,top_k] when idx_out != NULL, or kept in
  * the workspace.  The selection is the set dsa_topk(top_k) picks (same
  * scores, same tie rule) listed in ascending key order, DSA_INVALID after it:
- * the attention reads it as a set, so no rank sort is spent on it.  All other
- * arguments are as in the three calls above.
+ * the attention reads it as a set, so no rank sort is spent on it.  With one
+ * query per sequence (n_q = 1, decode) and a shape dsa_index_topk takes, the
+ * selection comes from dsa_index_topk (the same keys; the scores stay on chip
+ * and the workspace's score region is not written); otherwise from
+ * dsa_index_scores into the workspace and dsa_topk_set.  All other arguments are
+ * as in the three calls above.
  * Reads dims: every field of the three calls; kpool must be 0. */
 dsa_status dsa_layer_forward(const dsa_dims* dims, const void* q_idx, const void* k_idx,
                              const float* w, float idx_scale, const int32_t* q_pos,

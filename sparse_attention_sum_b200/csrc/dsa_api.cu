@@ -426,10 +426,16 @@ dsa_status dsa_layer_forward(const dsa_dims* d, const void* q_idx, const void* k
     float* scores = (float*)ws;
     int32_t* idx_ws = (int32_t*)((char*)ws + align256(rows * d->n_kv * sizeof(float)));
     int32_t* idx = idx_out ? idx_out : idx_ws;
-    if ((s = dsa_index_scores(d, q_idx, k_idx, w, idx_scale, q_pos, kv_start, kv_len, scores, stream)))
-      return s;
-    // the attention reads the selection as a set: same keys as dsa_topk, listed in key order
-    if ((s = dsa_topk_set(d, scores, q_pos, kv_start, kv_len, d->top_k, idx, nullptr, stream))) return s;
+    if (tc_policy() && d->n_q == 1 && dsa::index_topk_supported(*d, d->top_k)) {
+      // one query per sequence (decode): the fused selection keeps each row's scores on chip
+      if ((s = dsa_index_topk(d, q_idx, k_idx, w, idx_scale, q_pos, kv_start, kv_len, d->top_k, idx, stream)))
+        return s;
+    } else {
+      if ((s = dsa_index_scores(d, q_idx, k_idx, w, idx_scale, q_pos, kv_start, kv_len, scores, stream)))
+        return s;
+      // the attention reads the selection as a set: same keys as dsa_topk, listed in key order
+      if ((s = dsa_topk_set(d, scores, q_pos, kv_start, kv_len, d->top_k, idx, nullptr, stream))) return s;
+    }
     sel = idx;
   }
   return dsa_sparse_attend(d, q, k, k_row_stride, v, v_row_stride, sel, d->top_k, attn_scale, out,

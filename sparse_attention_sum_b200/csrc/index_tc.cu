@@ -24,12 +24,21 @@
 // bytes, one 128-byte swizzle row, and the MMA is kind::f8f6f4 with K = 32 per
 // instruction.  Since the scales are positive, relu(scale*sq*sk*dot) =
 // sk*relu(scale*sq*dot): the epilogue folds scale*sq into each accumulator
-// column and multiplies each key's sum by sk.
+// column and multiplies each key's sum by sk.  The producer warp brings each
+// tile's 128 key scales into a shared-memory ring of stages + 2 slots (4-byte
+// cp.async completing on the slot's own barrier, which the epilogue waits on),
+// so no epilogue waits on a global load.  A slot is refilled only after the
+// epilogue has finished the tile that used it: the producer runs at most
+// `stages` tiles ahead of the MMA, and the MMA at most two ahead of the epilogue.
+//
+// The head reduction (index_epilogue.cuh) folds w_h * |scale| (* sq_h) into one
+// weight per accumulator column, computed once per CTA.
 #include <cuda.h>
 
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
 #include "dsa_sm100.cuh"
+#include "index_epilogue.cuh"
 
 namespace dsa {
 
@@ -69,13 +78,14 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* gbase = smem_raw + (base - raw);
-  // [B operand: N x kRow B][stages x kTileBytes][w: NQ*HI floats][(FP8) scale*sq: NQ*HI floats]
+  // [B operand: N x kRow B][stages x kTileBytes][wsc: NQ*HI floats][(FP8) key scales: (stages+2) x 128]
   // [lo/hi per query][barriers]
   const uint32_t sB = base;
   const uint32_t sA = sB + (uint32_t)p.N * kRow;
-  float* w_s = reinterpret_cast<float*>(gbase + (sA - base) + (uint32_t)p.stages * kTileBytes);
-  float* ssq_s = w_s + p.N;                                       // FP8 only
-  int* lohi = reinterpret_cast<int*>(ssq_s + (kF8 ? p.N : 0));    // [NQ][2]
+  const int sk_slots = p.stages + 2;
+  float* wsc_s = reinterpret_cast<float*>(gbase + (sA - base) + (uint32_t)p.stages * kTileBytes);
+  float* sk_s = wsc_s + p.N;                                      // FP8 only
+  int* lohi = reinterpret_cast<int*>(sk_s + (kF8 ? sk_slots * kKeysPerTile : 0));  // [NQ][2]
   uint64_t* bars = reinterpret_cast<uint64_t*>(lohi + 2 * 16 + 2); // 8-byte aligned below
   bars = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(bars) + 7) & ~uintptr_t(7));
   uint64_t* full = bars;                  // [stages]
@@ -84,7 +94,8 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
   uint64_t* tempty = tfull + 2;           // [2]
   uint64_t* bfull = tempty + 2;           // [1]
   uint64_t* drain = bfull + 1;            // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* skfull = drain + 1;           // [stages + 2] (FP8)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(skfull + kMaxStages + 2);
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -125,6 +136,8 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
+    if (kF8)
+      for (int s = 0; s < sk_slots; ++s) mbar_init(smem_u32(&skfull[s]), 32);  // one cp.async arrival per lane
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&tfull[a]), 1);
       mbar_init(smem_u32(&tempty[a]), p.epi_warps);
@@ -133,12 +146,12 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     mbar_init(smem_u32(drain), 1);
     fence_barrier_init();
   }
-  // weights of the tile's queries (pre-multiplied by nothing: the scale stays inside relu)
+  // folded weight of each accumulator column: w * |scale| (* sq with FP8 operands)
+  const float ascale = fabsf(p.scale);
   for (int i = threadIdx.x; i < p.N; i += blockDim.x) {
     const int q = i / p.HI;
     const size_t col = ((size_t)b * p.T + t0 + q) * p.HI + (i - q * p.HI);
-    w_s[i] = q < nq_here ? p.w[col] : 0.f;
-    if (kF8) ssq_s[i] = q < nq_here ? p.scale * p.q_scale[col] : 0.f;
+    wsc_s[i] = q < nq_here ? (kF8 ? p.w[col] * ascale * p.q_scale[col] : p.w[col] * ascale) : 0.f;
   }
   if (warp == 1 && n_compute > 0) tmem_alloc(smem_u32(tmem_slot), ncols);
   tc_fence_before();
@@ -148,26 +161,44 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && n_compute > 0) {
-      tma_prefetch_desc(&map_q);
-      tma_prefetch_desc(&map_k);
-      const int qrow = (b * p.T + t0) * p.HI;
-      mbar_arrive_expect_tx(smem_u32(bfull), (uint32_t)p.N * kRow);
-      tma_load_2d(sB, &map_q, smem_u32(bfull), 0, qrow);
-      if (!kF8) tma_load_2d(sB + (uint32_t)p.N * 128u, &map_q, smem_u32(bfull), 64, qrow);
+    if (n_compute > 0) {
+      if (lane == 0) {
+        tma_prefetch_desc(&map_q);
+        tma_prefetch_desc(&map_k);
+        const int qrow = (b * p.T + t0) * p.HI;
+        mbar_arrive_expect_tx(smem_u32(bfull), (uint32_t)p.N * kRow);
+        tma_load_2d(sB, &map_q, smem_u32(bfull), 0, qrow);
+        if (!kF8) tma_load_2d(sB + (uint32_t)p.N * 128u, &map_q, smem_u32(bfull), 64, qrow);
+      }
       int issued = 0;
       for (int i = 0; i < n_compute; ++i) {
         const int s = i % p.stages;
-        if (!mbar_wait(smem_u32(&empty[s]), ((i / p.stages) & 1) ^ 1, p.status, &abort_flag)) break;
-        const uint32_t dst = sA + (uint32_t)s * kTileBytes;
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(smem_u32(&empty[s]), ((i / p.stages) & 1) ^ 1, p.status, &abort_flag);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         const int krow = b * p.S + (c_begin + i) * kKeysPerTile;
-        mbar_arrive_expect_tx(smem_u32(&full[s]), kTileBytes);
-        tma_load_2d(dst, &map_k, smem_u32(&full[s]), 0, krow);
-        if (!kF8) tma_load_2d(dst + kTileBytes / 2, &map_k, smem_u32(&full[s]), 64, krow);
+        if (lane == 0) {
+          const uint32_t dst = sA + (uint32_t)s * kTileBytes;
+          mbar_arrive_expect_tx(smem_u32(&full[s]), kTileBytes);
+          tma_load_2d(dst, &map_k, smem_u32(&full[s]), 0, krow);
+          if (!kF8) tma_load_2d(dst + kTileBytes / 2, &map_k, smem_u32(&full[s]), 64, krow);
+        }
+        if (kF8) {
+          // the tile's 128 key scales, four per lane (keys past the sequence read its last scale)
+          const int key0 = (c_begin + i) * kKeysPerTile + 4 * lane;
+          const int slot = i % sk_slots;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int key = min(key0 + e, p.S - 1);
+            cp_async_4(smem_u32(sk_s + slot * kKeysPerTile + 4 * lane + e), p.k_scale + (size_t)b * p.S + key);
+          }
+          cp_async_mbar_arrive(smem_u32(&skfull[slot]));
+        }
         ++issued;
       }
+      if (kF8) cp_async_wait_all();
       // on abort, let every issued copy land before the CTA exits
-      if (abort_flag) {
+      if (lane == 0 && abort_flag) {
         mbar_wait(smem_u32(bfull), 0, nullptr, nullptr);
         for (int i = max(0, issued - p.stages); i < issued; ++i)
           mbar_wait(smem_u32(&full[i % p.stages]), (i / p.stages) & 1, nullptr, nullptr);
@@ -215,6 +246,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     const int group = ew >> 2;                     // 0 or 1 (two warps per quarter when 8 warps)
     const int ngroups = p.epi_warps >> 2;
     const int key_in_tile = quarter * 32 + lane;
+    const bool neg = p.scale < 0.f;               // relu(scale * x) = |scale| * relu(-x)
     int ci = 0;  // compute-tile ordinal
     for (int kt = kt_begin; kt < kt_end; ++kt) {
       const int s = kt * kKeysPerTile + key_in_tile;
@@ -229,21 +261,21 @@ index_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
       if (!mbar_wait(smem_u32(&tfull[a]), (ci >> 1) & 1, p.status, &abort_flag)) break;
       tc_fence_after();
       const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * p.N);
-      // FP8: this lane's key scale (keys past the sequence read a neighbour's row or nothing)
-      const float sk = kF8 && s < p.S ? p.k_scale[(size_t)b * p.S + s] : 1.f;
+      // FP8: this lane's key scale, brought in with the tile
+      float sk = 1.f;
+      if (kF8) {
+        const int slot = ci % sk_slots;
+        if (!mbar_wait(smem_u32(&skfull[slot]), (uint32_t)((ci / sk_slots) & 1), p.status, &abort_flag)) break;
+        sk = sk_s[slot * kKeysPerTile + key_in_tile];
+      }
       for (int q = group; q < nq_here; q += ngroups) {
         float acc = 0.f;
-        const float* wq = w_s + q * p.HI;
-        const float* sq = ssq_s + q * p.HI;
+        const float* wq = wsc_s + q * p.HI;
         for (int h0 = 0; h0 < p.HI; h0 += 32) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(trow + (uint32_t)(q * p.HI + h0), v);
           tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float sc = kF8 ? sq[h0 + j] : p.scale;
-            acc = fmaf(wq[h0 + j], fmaxf(sc * __uint_as_float(v[j]), 0.f), acc);
-          }
+          acc += neg ? head_sum32<true>(v, wq + h0) : head_sum32<false>(v, wq + h0);
         }
         if (kF8) acc *= sk;
         if (s < p.S) {
@@ -356,8 +388,9 @@ cudaError_t launch_index_scores_tc(const dsa_dims& d, const void* q_idx, const v
   p.scores = scores;
   p.status = device_status_ptr();
   const size_t tb = (size_t)tile_bytes(f8);
-  const size_t fixed = 1024 + (size_t)p.N * row_bytes(f8) + (size_t)p.N * 4 * (f8 ? 2 : 1) + 2 * 16 * 4 + 64 +
-                       8 * (2 * kMaxStages + 8) + 64;
+  const size_t fixed = 1024 + (size_t)p.N * row_bytes(f8) + (size_t)p.N * 4 +
+                       (f8 ? (kMaxStages + 2) * kKeysPerTile * 4 : 0) + 2 * 16 * 4 + 64 +
+                       8 * (2 * kMaxStages + 8 + kMaxStages + 2) + 64;
   int stages = (int)((220 * 1024 - fixed) / tb);
   if (stages > (f8 ? kMaxStages : 6)) stages = f8 ? kMaxStages : 6;
   // two CTAs per SM: two 32 KB stages each (bf16), four 16 KB stages each (e4m3): 64 KB in flight per CTA

@@ -26,7 +26,9 @@
 //
 // FP8 operands (kF8): the e4m3 codes and per-vector scales of dsa_fp8_quantize, scored as the FP8
 // indexer does (kind::f8f6f4, K = 32 per instruction, one 128-byte row per key; the epilogue folds
-// scale * sq into each head column and multiplies a key's sum by its scale sk).
+// w * |scale| * sq into each head column and multiplies a key's sum by its scale sk, which the
+// producer warp brings into a shared-memory ring with cp.async as in the FP8 indexer).  The head
+// reduction is index_epilogue.cuh's, so the scores are the standalone indexer's bit for bit.
 //
 // Warp roles while scoring: warp 0 issues the TMA loads (the query's H_I x 128 block once, then a
 // ring of 128-key stages), warp 1 issues the MMAs into two TMEM accumulators, warps 2-5 run the
@@ -38,6 +40,7 @@
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
 #include "dsa_sm100.cuh"
+#include "index_epilogue.cuh"
 
 namespace dsa {
 
@@ -103,15 +106,17 @@ index_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* gbase = smem_raw + (base - raw);
-  // [q block: HI x kRow][stages x kTileBytes][keys: chunk x 4 B][hist: 4 x 256][w: HI][(FP8) scale*sq: HI]
-  // [misc][barriers]
+  // [q block: HI x kRow][stages x kTileBytes][keys: chunk x 4 B][hist: 4 x 256][wsc: HI]
+  // [(FP8) key scales: (stages+2) x 128][misc][barriers]
   const uint32_t sB = base;
   const uint32_t sA = sB + (uint32_t)p.HI * kRow;
+  const int sk_slots = p.stages + 2;
   uint32_t* keys = reinterpret_cast<uint32_t*>(gbase + (sA - base) + (uint32_t)p.stages * kTileBytes);
   uint32_t* hist = keys + p.chunk;                        // [kLevels][256]
-  float* w_s = reinterpret_cast<float*>(hist + kLevels * 256);
-  float* ssq_s = w_s + p.HI;                               // FP8 only
-  int* misc = reinterpret_cast<int*>(ssq_s + p.HI);        // [0] bin, [1] remaining, [2..3] gt/eq counts,
+  float* wsc_s = reinterpret_cast<float*>(hist + kLevels * 256);
+  float* sk_s = wsc_s + p.HI;                              // FP8 only
+  int* misc = reinterpret_cast<int*>(sk_s + (kF8 ? sk_slots * kKeysPerTile : 0));  // [0] bin, [1] remaining,
+                                                           // [2..3] gt/eq counts,
                                                            // [4..4+kWarps) warp scans, [16..] warp eq scans
   uint64_t* bars = reinterpret_cast<uint64_t*>(misc + 32);
   uint64_t* full = bars;
@@ -120,7 +125,8 @@ index_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
   uint64_t* tempty = tfull + 2;
   uint64_t* bfull = tempty + 2;
   uint64_t* drain = bfull + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* skfull = drain + 1;                            // [stages + 2] (FP8)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(skfull + kMaxStages + 2);
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -138,9 +144,10 @@ index_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
   const uint32_t ncols = p.HI * 2 <= 64 ? 64 : (p.HI * 2 <= 128 ? 128 : 256);
 
   for (int i = threadIdx.x; i < kLevels * 256; i += kThreads) hist[i] = 0u;
+  const float ascale = fabsf(p.scale);
   for (int i = threadIdx.x; i < p.HI; i += kThreads) {
-    w_s[i] = p.w[row * p.HI + i];
-    ssq_s[i] = kF8 ? p.scale * p.q_scale[row * p.HI + i] : p.scale;
+    const long long col = row * p.HI + i;
+    wsc_s[i] = kF8 ? p.w[col] * ascale * p.q_scale[col] : p.w[col] * ascale;
   }
   if (threadIdx.x == 0) {
     abort_flag = 0;
@@ -152,6 +159,8 @@ index_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
       mbar_init(smem_u32(&tfull[a]), 1);
       mbar_init(smem_u32(&tempty[a]), 4);
     }
+    if (kF8)
+      for (int s = 0; s < sk_slots; ++s) mbar_init(smem_u32(&skfull[s]), 32);  // one cp.async arrival per lane
     mbar_init(smem_u32(bfull), 1);
     mbar_init(smem_u32(drain), 1);
     fence_barrier_init();
@@ -164,24 +173,42 @@ index_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
 
   // ---------------------------------------------------------------- scoring
   if (warp == 0) {
-    if (lane == 0 && n_tiles > 0) {
-      tma_prefetch_desc(&map_q);
-      tma_prefetch_desc(&map_k);
-      mbar_arrive_expect_tx(smem_u32(bfull), (uint32_t)p.HI * kRow);
-      tma_load_2d(sB, &map_q, smem_u32(bfull), 0, (int)(row * p.HI));
-      if (!kF8) tma_load_2d(sB + (uint32_t)p.HI * 128u, &map_q, smem_u32(bfull), 64, (int)(row * p.HI));
+    if (n_tiles > 0) {
+      if (lane == 0) {
+        tma_prefetch_desc(&map_q);
+        tma_prefetch_desc(&map_k);
+        mbar_arrive_expect_tx(smem_u32(bfull), (uint32_t)p.HI * kRow);
+        tma_load_2d(sB, &map_q, smem_u32(bfull), 0, (int)(row * p.HI));
+        if (!kF8) tma_load_2d(sB + (uint32_t)p.HI * 128u, &map_q, smem_u32(bfull), 64, (int)(row * p.HI));
+      }
       int issued = 0;
       for (int i = 0; i < n_tiles; ++i) {
         const int s = i % p.stages;
-        if (!mbar_wait(smem_u32(&empty[s]), ((i / p.stages) & 1) ^ 1, p.status, &abort_flag)) break;
-        const uint32_t dst = sA + (uint32_t)s * kTileBytes;
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(smem_u32(&empty[s]), ((i / p.stages) & 1) ^ 1, p.status, &abort_flag);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         const int krow = b * p.S + (t_begin + i) * kKeysPerTile;
-        mbar_arrive_expect_tx(smem_u32(&full[s]), kTileBytes);
-        tma_load_2d(dst, &map_k, smem_u32(&full[s]), 0, krow);
-        if (!kF8) tma_load_2d(dst + kTileBytes / 2, &map_k, smem_u32(&full[s]), 64, krow);
+        if (lane == 0) {
+          const uint32_t dst = sA + (uint32_t)s * kTileBytes;
+          mbar_arrive_expect_tx(smem_u32(&full[s]), kTileBytes);
+          tma_load_2d(dst, &map_k, smem_u32(&full[s]), 0, krow);
+          if (!kF8) tma_load_2d(dst + kTileBytes / 2, &map_k, smem_u32(&full[s]), 64, krow);
+        }
+        if (kF8) {
+          // the tile's 128 key scales, four per lane (keys past the sequence read its last scale)
+          const int key0 = (t_begin + i) * kKeysPerTile + 4 * lane;
+          const int slot = i % sk_slots;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int key = min(key0 + e, p.S - 1);
+            cp_async_4(smem_u32(sk_s + slot * kKeysPerTile + 4 * lane + e), p.k_scale + (size_t)b * p.S + key);
+          }
+          cp_async_mbar_arrive(smem_u32(&skfull[slot]));
+        }
         ++issued;
       }
-      if (abort_flag) {  // let every issued copy land before the shared memory is reused or freed
+      if (kF8) cp_async_wait_all();
+      if (lane == 0 && abort_flag) {  // let every issued copy land before the shared memory is reused or freed
         mbar_wait(smem_u32(bfull), 0, nullptr, nullptr);
         for (int i = max(0, issued - p.stages); i < issued; ++i)
           mbar_wait(smem_u32(&full[i % p.stages]), (i / p.stages) & 1, nullptr, nullptr);
@@ -222,20 +249,25 @@ index_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
   } else {
     // epilogue: lane quarter (warp & 3) of each tile, one key per thread
     const int quarter = warp & 3;
+    const bool neg = p.scale < 0.f;                      // relu(scale * x) = |scale| * relu(-x)
     for (int i = 0; i < n_tiles; ++i) {
       const int a = i & 1;
       if (!mbar_wait(smem_u32(&tfull[a]), (i >> 1) & 1, p.status, &abort_flag)) break;
       tc_fence_after();
       const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * p.HI);
       const int s = (t_begin + i) * kKeysPerTile + quarter * 32 + lane;
-      const float sk = kF8 && s <= l1 && s >= l0 ? p.k_scale[(size_t)b * p.S + s] : 1.f;
+      float sk = 1.f;
+      if (kF8) {
+        const int slot = i % sk_slots;
+        if (!mbar_wait(smem_u32(&skfull[slot]), (uint32_t)((i / sk_slots) & 1), p.status, &abort_flag)) break;
+        sk = sk_s[slot * kKeysPerTile + quarter * 32 + lane];
+      }
       float acc = 0.f;
       for (int h0 = 0; h0 < p.HI; h0 += 32) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(trow + (uint32_t)h0, v);
         tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) acc = fmaf(w_s[h0 + j], fmaxf(ssq_s[h0 + j] * __uint_as_float(v[j]), 0.f), acc);
+        acc += neg ? head_sum32<true>(v, wsc_s + h0) : head_sum32<false>(v, wsc_s + h0);
       }
       if (kF8) acc *= sk;
       tc_fence_before();
@@ -409,7 +441,8 @@ int cluster_for(int S) {
 
 size_t fused_smem(int HI, int stages, int chunk, bool f8) {
   return 1024 + (size_t)HI * row_bytes(f8) + (size_t)stages * tile_bytes(f8) + (size_t)chunk * 4 +
-         kLevels * 256 * 4 + (size_t)HI * 8 + 32 * 4 + 8 * (2 * kMaxStages + 6) + 16;
+         kLevels * 256 * 4 + (size_t)HI * 4 + (f8 ? (size_t)(stages + 2) * kKeysPerTile * 4 : 0) + 32 * 4 +
+         8 * (2 * kMaxStages + 6 + kMaxStages + 2) + 16;
 }
 
 }  // namespace

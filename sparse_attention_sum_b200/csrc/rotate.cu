@@ -22,6 +22,16 @@
 // The row goes to out_rows[r] (its cache slot) or to r; a slot outside
 // [0, capacity) is skipped.  Each vector is read once and written once, so the
 // kernel is bound by HBM bandwidth.
+//
+// dim = 128 with n_rope in {0, 64, 128} (the indexer's shape) takes a second
+// kernel, index_rotate128_kernel, that spends fewer shuffles per vector: four
+// lanes share a vector, lane t of the four holding values 32t .. 32t+31, so
+// five of the seven Walsh-Hadamard stages run inside the lane and two cross
+// lanes (xor 1 and 2), the RoPE partner of a value sits in lane t^1 (n_rope 64)
+// or t^2 (n_rope 128) at the same register, and a LayerNorm sum takes two
+// shuffles.  A block of 128 threads takes 32 consecutive head vectors, whatever
+// rows they belong to, so the key step (one head per row) fills the GPU as
+// well as the query step; the RoPE table holds the block's rows.
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
 
@@ -223,8 +233,128 @@ index_rotate_kernel(const __grid_constant__ RotParams p) {
   }
 }
 
+constexpr int k128Vectors = 32;               // head vectors per block of the dim-128 kernel
+constexpr int k128Threads = 4 * k128Vectors;  // four lanes per vector
+
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(k128Threads)
+index_rotate128_kernel(const __grid_constant__ RotParams p, long long n_vec) {
+  // (cos, sin) per (row of the block, angle); rows spanned by 32 vectors <= 32
+  __shared__ float2 tab[k128Vectors][64];
+  __shared__ float lnw[128], lnb[128];
+  const int lane = threadIdx.x & 31;
+  const int t = lane & 3;                                   // quarter of the vector this lane holds
+  const long long v0 = (long long)blockIdx.x * k128Vectors;
+  const long long v = v0 + (threadIdx.x >> 2);
+  const bool live = v < n_vec;
+  const long long r = live ? v / p.heads : 0;
+  const int h = live ? (int)(v - r * p.heads) : 0;
+  const long long r0 = v0 / p.heads;                        // first row of the block
+  const int half = p.n_rope >> 1;
+
+  float x[32];
+  if (live) {
+    const Tin* src = static_cast<const Tin*>(p.in) + r * p.in_stride + (long long)h * 128 + 32 * t;
+#pragma unroll
+    for (int e = 0; e < 32; e += 4) load_vals<4>(src + e, *reinterpret_cast<float(*)[4]>(&x[e]));
+  } else {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) x[e] = 0.f;
+  }
+  // the RoPE table of the block's rows (loads in flight meanwhile)
+  if (half > 0) {
+    const long long last = min(n_vec, v0 + k128Vectors) - 1;
+    const int n_rows = (int)(last / p.heads - r0) + 1;
+    for (int i = threadIdx.x; i < n_rows * half; i += k128Threads) {
+      const int rr = i / half, a = i - rr * half;
+      const double ang = (double)p.pos[r0 + rr] * p.inv_freq[a];
+      const double red = fma(-rint(ang * kInvTwoPi), kTwoPi, ang);  // |red| <= pi
+      float sn, cs;
+      sincosf((float)red, &sn, &cs);
+      tab[rr][a] = make_float2(cs, sn);
+    }
+  }
+  if (p.layer_norm) {
+    lnw[threadIdx.x] = p.ln_w ? p.ln_w[threadIdx.x] : 1.f;
+    lnb[threadIdx.x] = p.ln_b ? p.ln_b[threadIdx.x] : 0.f;
+  }
+  __syncthreads();
+
+  if (p.layer_norm) {
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) s += x[e];
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    const float mean = s * (1.f / 128.f);
+    float s2 = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      x[e] -= mean;
+      s2 = fmaf(x[e], x[e], s2);
+    }
+    s2 += __shfl_xor_sync(0xffffffffu, s2, 1);
+    s2 += __shfl_xor_sync(0xffffffffu, s2, 2);
+    const float inv_std = 1.f / sqrtf(s2 * (1.f / 128.f) + p.eps);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) x[e] = fmaf(x[e] * inv_std, lnw[32 * t + e], lnb[32 * t + e]);
+  }
+  if (half > 0) {
+    // NEOX pairs (i, i + half): half = 32 pairs lanes t^1 among t < 2; half = 64 pairs t^2
+    const int m = half >> 5;
+    const bool in_rope = 32 * t < p.n_rope;
+    const bool first = (t & m) == 0;
+    const int a0 = half == 32 ? 0 : 32 * (t & 1);            // angle index of register e is a0 + e
+    const float2* tr = tab[(int)(r - r0)];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const float o = __shfl_xor_sync(0xffffffffu, x[e], m);
+      const float2 cs = tr[a0 + e];
+      if (in_rope) x[e] = first ? x[e] * cs.x - o * cs.y : x[e] * cs.x + o * cs.y;
+    }
+  }
+  if (p.hadamard) {
+    // bits 0-4 of the value index inside the lane, bits 5-6 across the four lanes
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        if (!(e & m)) {
+          const float a = x[e], b = x[e | m];
+          x[e] = a + b;
+          x[e | m] = a - b;
+        }
+      }
+    }
+#pragma unroll
+    for (int m = 1; m < 4; m <<= 1) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float o = __shfl_xor_sync(0xffffffffu, x[e], m);
+        x[e] = (t & m) ? o - x[e] : x[e] + o;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 32; ++e) x[e] *= p.hscale;
+  }
+  if (!live) return;
+  const long long dst = p.out_rows ? (long long)p.out_rows[r] : r;
+  if (dst < 0 || dst >= p.out_cap) return;
+  Tout* dstp = static_cast<Tout*>(p.out) + dst * p.out_stride + (long long)h * 128 + 32 * t;
+#pragma unroll
+  for (int e = 0; e < 32; e += 4) store_vals<4>(dstp + e, *reinterpret_cast<const float(*)[4]>(&x[e]));
+}
+
 template <typename Tin, typename Tout>
 cudaError_t launch_rotate_t(int n_rows, int dim, const RotParams& p, cudaStream_t st) {
+  if (dim == 128 && (p.n_rope == 0 || p.n_rope == 64 || p.n_rope == 128)) {
+    const long long n_vec = (long long)n_rows * p.heads;
+    const long long blocks = (n_vec + k128Vectors - 1) / k128Vectors;
+    if (blocks < 2147483647LL) {
+      index_rotate128_kernel<Tin, Tout><<<(unsigned)blocks, k128Threads, 0, st>>>(p, n_vec);
+      return cudaGetLastError();
+    }
+  }
   const int warps = p.heads < kRotWarps ? p.heads : kRotWarps;
   const dim3 grid((unsigned)n_rows), block((unsigned)(32 * warps));
   switch (dim) {

@@ -19,8 +19,8 @@ from typing import Dict, Optional
 import torch
 
 from . import (BF16, F32, OP_LAYER_FORWARD, Dims, absorb_out, absorb_q, expand_selection, fp8_quantize,
-               index_scores, index_scores_fp8, layer_forward, pool_states, sparse_attend, topk, topk_set,
-               workspace_size)
+               index_scores, index_scores_fp8, index_topk_fp8, layer_forward, pool_states, sparse_attend, topk,
+               topk_set, workspace_size)
 
 
 def _code(dtype: torch.dtype) -> int:
@@ -84,9 +84,10 @@ class Fp8Buffers:
 def dsa_layer_fp8(dims: Dims, q_idx, k_codes, k_scales, w, idx_scale, q_pos, kv_start, kv_len, q, k, v,
                   attn_scale, k_row_stride: int, v_row_stride: int, bufs: Optional[LayerBuffers] = None,
                   fp8: Optional[Fp8Buffers] = None, stream=None, k_idx=None) -> LayerBuffers:
-    """The layer with the FP8 indexer, as four libdsa calls: dsa_fp8_quantize of the queries,
+    """The layer with the FP8 indexer as libdsa calls: dsa_fp8_quantize of the queries, then
     dsa_index_scores_fp8 against the key cache's e4m3 codes and scales (quantised once, when the keys
-    were written), dsa_topk_set, dsa_sparse_attend.  ``k_idx`` (the bf16 keys) is not read."""
+    were written) and dsa_topk_set, or dsa_index_topk_fp8 when there is one query per sequence, then
+    dsa_sparse_attend.  ``k_idx`` (the bf16 keys) is not read."""
     if bufs is None:
         bufs = LayerBuffers(dims, q.device, q.dtype)
     if fp8 is None:
@@ -94,9 +95,14 @@ def dsa_layer_fp8(dims: Dims, q_idx, k_codes, k_scales, w, idx_scale, q_pos, kv_
     B, T, S = dims.batch, dims.n_q, dims.n_kv
     scores = bufs.ws[: B * T * S * 4].view(torch.float32).view(B, T, S)
     fp8_quantize(q_idx, fp8.q_codes, fp8.q_scales, stream=stream)
-    index_scores_fp8(dims, fp8.q_codes, fp8.q_scales, k_codes, k_scales, w, idx_scale, q_pos, kv_start, kv_len,
-                     scores, stream=stream)
-    topk_set(dims, scores, q_pos, kv_start, kv_len, dims.top_k, bufs.idx, stream=stream)
+    if dims.n_q == 1:
+        # one query per sequence: the fused selection (same keys, no score matrix)
+        index_topk_fp8(dims, fp8.q_codes, fp8.q_scales, k_codes, k_scales, w, idx_scale, q_pos, kv_start, kv_len,
+                       dims.top_k, bufs.idx, stream=stream)
+    else:
+        index_scores_fp8(dims, fp8.q_codes, fp8.q_scales, k_codes, k_scales, w, idx_scale, q_pos, kv_start, kv_len,
+                         scores, stream=stream)
+        topk_set(dims, scores, q_pos, kv_start, kv_len, dims.top_k, bufs.idx, stream=stream)
     sparse_attend(dims, q, k, k_row_stride, v, v_row_stride, bufs.idx, dims.top_k, attn_scale, bufs.out,
                   lse=bufs.lse, stream=stream)
     return bufs
