@@ -299,26 +299,53 @@ def profiled_traffic():
 
 
 def profile_once(a):
-    """One call of each stage entry point (three launches), for a profiler to capture."""
+    """One call of each entry point of the chosen path, no timing (for a profiler to capture).
+    --what layer: dsa_index_scores, dsa_topk_set, dsa_sparse_attend; fused: dsa_index_topk; fp8:
+    dsa_fp8_quantize of the queries, dsa_index_scores_fp8, dsa_index_topk_fp8 (keys quantised first);
+    rotate: dsa_index_rotate of T tokens x 64 query heads, then of T keys."""
     import sparse_attention_sum_b200 as dsa
     from sparse_attention_sum_b200 import runner
     torch.cuda.set_device(0)
     dsa.lib()
-    sizes = {k: v for k, v in (("T", a.T), ("S", a.S)) if v}
-    wl = workloads.make(a.workload, **sizes)
-    t = device_inputs(wl)
-    dims, args = layer_args(wl, t)
-    bufs = runner.LayerBuffers(dims, "cuda", torch.bfloat16, with_idx=True)
-    B, T, S = wl.batch, wl.n_q, wl.n_kv
-    scores = bufs.ws[: B * T * S * 4].view(torch.float32)
-    dsa.index_scores(dims, args["q_idx"], args["k_idx"], args["w"], args["idx_scale"], args["q_pos"],
-                     args["kv_start"], args["kv_len"], scores)
-    dsa.topk_set(dims, scores, args["q_pos"], args["kv_start"], args["kv_len"], wl.top_k, bufs.idx)
-    dsa.sparse_attend(dims, args["q"], args["k"], args["k_row_stride"], args["v"], args["v_row_stride"],
-                      bufs.idx, wl.top_k, args["attn_scale"], bufs.out)
+    if a.what == "rotate":
+        n = a.T or 4096
+        qi = {k: v.cuda() for k, v in workloads.rotate_inputs(n, 64, 128, seed=1, pos_max=n).items()}
+        ki = {k: v.cuda() for k, v in workloads.rotate_inputs(n, 1, 128, seed=2, pos_max=n, mean=0.5, std=2.0).items()}
+        q_out = torch.empty(n, 64, 128, dtype=torch.bfloat16, device="cuda")
+        k_out = torch.empty(n, 1, 128, dtype=torch.bfloat16, device="cuda")
+        dsa.index_rotate(qi["x"], q_out, 64, 10000.0, pos=qi["pos"])
+        dsa.index_rotate(ki["x"], k_out, 64, 10000.0, pos=ki["pos"], layer_norm=True, ln_w=ki["ln_w"], ln_b=ki["ln_b"],
+                         ln_eps=1e-6)
+        name = f"rotate T={n}"
+    else:
+        sizes = {k: v for k, v in (("T", a.T), ("S", a.S), ("B", a.B)) if v}
+        wl = workloads.make(a.workload, **sizes)
+        t = device_inputs(wl)
+        dims, args = layer_args(wl, t)
+        bufs = runner.LayerBuffers(dims, "cuda", torch.bfloat16, with_idx=True)
+        B, T, S = wl.batch, wl.n_q, wl.n_kv
+        scores = bufs.ws[: B * T * S * 4].view(torch.float32)
+        ia = (args["q_pos"], args["kv_start"], args["kv_len"])
+        if a.what == "layer":
+            dsa.index_scores(dims, args["q_idx"], args["k_idx"], args["w"], args["idx_scale"], *ia, scores)
+            dsa.topk_set(dims, scores, *ia, wl.top_k, bufs.idx)
+            dsa.sparse_attend(dims, args["q"], args["k"], args["k_row_stride"], args["v"], args["v_row_stride"],
+                              bufs.idx, wl.top_k, args["attn_scale"], bufs.out)
+        elif a.what == "fused":
+            dsa.index_topk(dims, args["q_idx"], args["k_idx"], args["w"], args["idx_scale"], *ia, wl.top_k, bufs.idx)
+        elif a.what == "fp8":
+            kc = torch.empty(B, S, 128, dtype=torch.uint8, device="cuda")
+            ks = torch.empty(B, S, dtype=torch.float32, device="cuda")
+            dsa.fp8_quantize(t["k_idx"], kc, ks)
+            f8 = runner.Fp8Buffers(dims, "cuda")
+            dsa.fp8_quantize(t["q_idx"], f8.q_codes, f8.q_scales)
+            dsa.index_scores_fp8(dims, f8.q_codes, f8.q_scales, kc, ks, args["w"], args["idx_scale"], *ia, scores)
+            dsa.index_topk_fp8(dims, f8.q_codes, f8.q_scales, kc, ks, args["w"], args["idx_scale"], *ia, wl.top_k,
+                               bufs.idx)
+        name = wl.name
     torch.cuda.synchronize()
     status = dsa.get_device_status()
-    print(json.dumps({"profile_once": wl.name, "device_status": status,
+    print(json.dumps({"profile_once": name, "what": a.what, "device_status": status,
                       "device_bytes": torch.cuda.max_memory_allocated()}), flush=True)
     if status != 0:
         sys.exit(1)
@@ -798,6 +825,9 @@ def main(argv=None):
                     help="one call of each stage entry point, no timing (for an ncu capture)")
     ap.add_argument("--T", type=int, default=0, help="--profile-once: queries per sequence (smaller capture)")
     ap.add_argument("--S", type=int, default=0, help="--profile-once: keys per sequence (smaller capture)")
+    ap.add_argument("--B", type=int, default=0, help="--profile-once: sequences (decode; smaller capture)")
+    ap.add_argument("--what", choices=["layer", "fused", "fp8", "rotate"], default="layer",
+                    help="--profile-once: which path to run once")
     a = ap.parse_args(argv)
     a.warmup = max(3, a.warmup)  # at least three untimed warm-up steps
     if a.impl == "reference":

@@ -247,9 +247,10 @@ index_rotate128_kernel(const __grid_constant__ RotParams p, long long n_vec) {
   const long long v0 = (long long)blockIdx.x * k128Vectors;
   const long long v = v0 + (threadIdx.x >> 2);
   const bool live = v < n_vec;
-  const long long r = live ? v / p.heads : 0;
-  const int h = live ? (int)(v - r * p.heads) : 0;
   const long long r0 = v0 / p.heads;                        // first row of the block
+  // lanes past the last vector take the block's first row (table index 0) and store nothing
+  const long long r = live ? v / p.heads : r0;
+  const int h = live ? (int)(v - r * p.heads) : 0;
   const int half = p.n_rope >> 1;
 
   float x[32];
