@@ -586,7 +586,8 @@ def decode_extra(peaks, flush, stream, cpu_s=0.0):
     res = {"workload": f"decode: B={wl.batch} T=1 S={wl.n_kv} top_k={wl.top_k}",
            "value": round(rows / step, 1), "unit": UNIT, "ms_per_step": round(step * 1e3, 4),
            "stages_us": {k: round(v * 1e6, 1) for k, v in st.items()},
-           "roofline_attend": roofline_entry("hbm", wk["attend_bytes"], st["attend"], peaks),
+           "roofline_attend": roofline_entry("hbm", wk["attend_bytes"], st["attend"], peaks,
+                                             profiled_traffic().get("attend:decode")),
            "roofline_index": roofline_entry("hbm", wk["index_bytes"], st["index"], peaks,
                                             profiled_traffic().get("index:decode")),
            "fused_hbm_frac": round((wk["index_bytes"] + wk["topk_bytes"] + wk["attend_bytes"]) / step / 1e9

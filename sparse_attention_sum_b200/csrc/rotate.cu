@@ -23,15 +23,14 @@
 // [0, capacity) is skipped.  Each vector is read once and written once, so the
 // kernel is bound by HBM bandwidth.
 //
-// dim = 128 with n_rope in {0, 64, 128} (the indexer's shape) takes a second
-// kernel, index_rotate128_kernel, that spends fewer shuffles per vector: four
+// dim = 128 with n_rope in {0, 64, 128} (the indexer's shape), 16-byte aligned
+// rows, takes a second kernel, index_rotate128_kernel, that spends fewer shuffles per vector: four
 // lanes share a vector, lane t of the four holding values 32t .. 32t+31, so
 // five of the seven Walsh-Hadamard stages run inside the lane and two cross
 // lanes (xor 1 and 2), the RoPE partner of a value sits in lane t^1 (n_rope 64)
 // or t^2 (n_rope 128) at the same register, and a LayerNorm sum takes two
-// shuffles.  A block of 128 threads takes 32 consecutive head vectors, whatever
-// rows they belong to, so the key step (one head per row) fills the GPU as
-// well as the query step; the RoPE table holds the block's rows.
+// shuffles.  A block of 128 threads takes 32 consecutive head vectors of one row
+// (rows of 32, 64, ... heads: the query step); the RoPE table holds that row.
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
 
@@ -236,11 +235,54 @@ index_rotate_kernel(const __grid_constant__ RotParams p) {
 constexpr int k128Vectors = 32;               // head vectors per block of the dim-128 kernel
 constexpr int k128Threads = 4 * k128Vectors;  // four lanes per vector
 
+// 32 consecutive values of a lane: 16-byte loads and stores.
+__device__ __forceinline__ void load32(const bf16* p, float (&x)[32]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 u = reinterpret_cast<const uint4*>(p)[i];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+      x[8 * i + 2 * j] = f.x;
+      x[8 * i + 2 * j + 1] = f.y;
+    }
+  }
+}
+__device__ __forceinline__ void load32(const float* p, float (&x)[32]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 u = reinterpret_cast<const float4*>(p)[i];
+    x[4 * i] = u.x;
+    x[4 * i + 1] = u.y;
+    x[4 * i + 2] = u.z;
+    x[4 * i + 3] = u.w;
+  }
+}
+__device__ __forceinline__ void store32(bf16* p, const float (&x)[32]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      __nv_bfloat162 b = __floats2bfloat162_rn(x[8 * i + 2 * j], x[8 * i + 2 * j + 1]);
+      w[j] = *reinterpret_cast<uint32_t*>(&b);
+    }
+    reinterpret_cast<uint4*>(p)[i] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+__device__ __forceinline__ void store32(float* p, const float (&x)[32]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    reinterpret_cast<float4*>(p)[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+}
+
 template <typename Tin, typename Tout>
-__global__ void __launch_bounds__(k128Threads)
+__global__ void __launch_bounds__(k128Threads, 6)
 index_rotate128_kernel(const __grid_constant__ RotParams p, long long n_vec) {
-  // (cos, sin) per (row of the block, angle); rows spanned by 32 vectors <= 32
-  __shared__ float2 tab[k128Vectors][64];
+  // (cos, sin) per (row of the block, angle): one row when heads is a multiple of 32, up to 32
+  // rows for other head counts
+  __shared__ __align__(16) float2 tab[k128Vectors][64];
   __shared__ float lnw[128], lnb[128];
   const int lane = threadIdx.x & 31;
   const int t = lane & 3;                                   // quarter of the vector this lane holds
@@ -255,9 +297,7 @@ index_rotate128_kernel(const __grid_constant__ RotParams p, long long n_vec) {
 
   float x[32];
   if (live) {
-    const Tin* src = static_cast<const Tin*>(p.in) + r * p.in_stride + (long long)h * 128 + 32 * t;
-#pragma unroll
-    for (int e = 0; e < 32; e += 4) load_vals<4>(src + e, *reinterpret_cast<float(*)[4]>(&x[e]));
+    load32(static_cast<const Tin*>(p.in) + r * p.in_stride + (long long)h * 128 + 32 * t, x);
   } else {
 #pragma unroll
     for (int e = 0; e < 32; ++e) x[e] = 0.f;
@@ -301,21 +341,27 @@ index_rotate128_kernel(const __grid_constant__ RotParams p, long long n_vec) {
     for (int e = 0; e < 32; ++e) x[e] = fmaf(x[e] * inv_std, lnw[32 * t + e], lnb[32 * t + e]);
   }
   if (half > 0) {
-    // NEOX pairs (i, i + half): half = 32 pairs lanes t^1 among t < 2; half = 64 pairs t^2
+    // NEOX pairs (i, i + half): half = 32 pairs lanes t^1 among t < 2; half = 64 pairs t^2.
+    // first half: x cos - o sin; second half: x cos + o sin (the sign goes onto sin's bits)
     const int m = half >> 5;
     const bool in_rope = 32 * t < p.n_rope;
-    const bool first = (t & m) == 0;
+    const uint32_t neg = (t & m) == 0 ? 0x80000000u : 0u;
     const int a0 = half == 32 ? 0 : 32 * (t & 1);            // angle index of register e is a0 + e
-    const float2* tr = tab[(int)(r - r0)];
+    const float4* tr = reinterpret_cast<const float4*>(&tab[(int)(r - r0)][a0]);
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const float o = __shfl_xor_sync(0xffffffffu, x[e], m);
-      const float2 cs = tr[a0 + e];
-      if (in_rope) x[e] = first ? x[e] * cs.x - o * cs.y : x[e] * cs.x + o * cs.y;
+    for (int e = 0; e < 32; e += 2) {
+      const float4 cs = tr[e >> 1];                           // (cos, sin) of angles a0+e, a0+e+1
+      const float o0 = __shfl_xor_sync(0xffffffffu, x[e], m);
+      const float o1 = __shfl_xor_sync(0xffffffffu, x[e + 1], m);
+      if (in_rope) {
+        x[e] = fmaf(o0, __uint_as_float(__float_as_uint(cs.y) ^ neg), x[e] * cs.x);
+        x[e + 1] = fmaf(o1, __uint_as_float(__float_as_uint(cs.w) ^ neg), x[e + 1] * cs.z);
+      }
     }
   }
   if (p.hadamard) {
-    // bits 0-4 of the value index inside the lane, bits 5-6 across the four lanes
+    // bits 0-4 of the value index inside the lane, bits 5-6 across the four lanes:
+    // x' = x + o on the lower lane of a pair, o - x on the upper one
 #pragma unroll
     for (int m = 1; m < 32; m <<= 1) {
 #pragma unroll
@@ -329,10 +375,11 @@ index_rotate128_kernel(const __grid_constant__ RotParams p, long long n_vec) {
     }
 #pragma unroll
     for (int m = 1; m < 4; m <<= 1) {
+      const float sg = (t & m) ? -1.f : 1.f;
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
         const float o = __shfl_xor_sync(0xffffffffu, x[e], m);
-        x[e] = (t & m) ? o - x[e] : x[e] + o;
+        x[e] = fmaf(x[e], sg, o);
       }
     }
 #pragma unroll
@@ -341,14 +388,18 @@ index_rotate128_kernel(const __grid_constant__ RotParams p, long long n_vec) {
   if (!live) return;
   const long long dst = p.out_rows ? (long long)p.out_rows[r] : r;
   if (dst < 0 || dst >= p.out_cap) return;
-  Tout* dstp = static_cast<Tout*>(p.out) + dst * p.out_stride + (long long)h * 128 + 32 * t;
-#pragma unroll
-  for (int e = 0; e < 32; e += 4) store_vals<4>(dstp + e, *reinterpret_cast<const float(*)[4]>(&x[e]));
+  store32(static_cast<Tout*>(p.out) + dst * p.out_stride + (long long)h * 128 + 32 * t, x);
 }
 
 template <typename Tin, typename Tout>
 cudaError_t launch_rotate_t(int n_rows, int dim, const RotParams& p, cudaStream_t st) {
-  if (dim == 128 && (p.n_rope == 0 || p.n_rope == 64 || p.n_rope == 128)) {
+  // the dim-128 kernel moves 16 bytes per access: rows and bases must allow it
+  const auto al16 = [](const void* q) { return ((uintptr_t)q & 15u) == 0; };
+  const bool aligned = al16(p.in) && al16(p.out) && p.in_stride % (16 / (int)sizeof(Tin)) == 0 &&
+                       p.out_stride % (16 / (int)sizeof(Tout)) == 0;
+  // one-head rows (keys) stay on the general kernel: there a block's 32 vectors span 32 rows, and
+  // building 32 rows of angles per block costs more than the shuffles it saves
+  if (dim == 128 && aligned && p.heads % k128Vectors == 0 && (p.n_rope == 0 || p.n_rope == 64 || p.n_rope == 128)) {
     const long long n_vec = (long long)n_rows * p.heads;
     const long long blocks = (n_vec + k128Vectors - 1) / k128Vectors;
     if (blocks < 2147483647LL) {

@@ -65,6 +65,10 @@ CASES = [
     ("dim 64 rope only", 20, 17, 64, "f32", torch.bfloat16, 64, False, False),
     ("dim 128 n_rope 8", 70, 1, 128, "bf16", torch.bfloat16, 8, True, False),
     ("dim 128 all rope", 19, 12, 128, "f32", torch.float32, 128, True, True),
+    # rows of whole 32-head blocks take the four-lanes-per-vector kernel: every n_rope it serves
+    ("32 heads all rope f32", 33, 32, 128, "f32", torch.float32, 128, True, True),
+    ("64 heads no rope", 21, 64, 128, "bf16", torch.bfloat16, 0, False, True),
+    ("96 heads rope only", 9, 96, 128, "bf16", torch.float32, 64, True, False),
 ]
 
 
@@ -91,6 +95,20 @@ def test_strided_rows_in_and_out():
     _rotate(inp, out, 64, False, True, x=xin)
     _assert_close(out, _oracle(inp, slice(None), 64, False, True), torch.bfloat16)
     assert (big[:, :128] == 7.0).all() and (big[:, 128 + heads * dim:] == 7.0).all()
+
+
+def test_rows_aligned_to_eight_bytes_only():
+    """A row stride of 132 values (4-value aligned, not 8): the dim-128 kernel's 16-byte accesses
+    cannot serve it, so the general kernel runs; both layouts give the oracle's values."""
+    n_rows, heads, dim = 37, 1, 128
+    inp = workloads.rotate_inputs(n_rows, heads, dim, seed=29, mean=0.5, std=2.0)
+    wide = torch.zeros(n_rows, 132, dtype=torch.bfloat16)
+    wide[:, 4:132] = inp["x"].reshape(n_rows, -1)
+    xin = wide.cuda()[:, 4:132].unflatten(1, (heads, dim))
+    out = torch.empty(n_rows, heads, dim, dtype=torch.bfloat16, device="cuda")
+    _rotate(inp, out, 64, True, True, x=xin)
+    assert dsa.last_kernels() == ["index_rotate"]
+    _assert_close(out, _oracle(inp, slice(None), 64, True, True), torch.bfloat16)
 
 
 def test_in_place():
