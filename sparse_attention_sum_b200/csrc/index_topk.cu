@@ -13,13 +13,14 @@
 // 128 in two 64-wide swizzled blocks, TMEM accumulators, the relu*w reduction per lane), and keeps
 // each score as an order-preserving 32-bit key in shared memory.  The epilogue also counts the
 // top 8 bits of every key (the first histogram of the selection).  Then the cluster selects:
-//   1. four rounds of 8 bits: each CTA histograms its keys that match the prefix found so far,
-//      every CTA reads all C histograms through distributed shared memory and walks the same bins
-//      from the top, so all agree on the next 8 bits of the k-th largest key tau and on how many
-//      keys equal to tau still have to be taken;
-//   2. each CTA counts its keys above and equal to tau; through distributed shared memory every CTA
-//      learns the counts of the lower ranks, so it knows how many of its tau keys to take (ties go to
-//      the smaller index, and lower ranks hold smaller indices) and where its keys start in the row;
+//   1. four rounds of 8 bits: each CTA histograms its keys that match the prefix found so far and
+//      stores the histogram into every CTA of the cluster (distributed shared memory; the freed key
+//      stages hold the copies), so every CTA walks the same summed bins from the top, locally, and
+//      all agree on the next 8 bits of the k-th largest key tau and on how many keys equal to tau
+//      still have to be taken;
+//   2. each CTA counts its keys above and equal to tau and stores the counts into every CTA, so each
+//      knows the counts of the lower ranks: how many of its tau keys to take (ties go to the smaller
+//      index, and lower ranks hold smaller indices) and where its keys start in the row;
 //   3. each warp lists its contiguous segment of keys in order (ballots), at offsets from a scan of
 //      the warps' counts.
 // A row with at most k visible keys lists them all.  Nothing is written but the index rows.
@@ -43,6 +44,17 @@
 #include "index_epilogue.cuh"
 
 namespace dsa {
+
+#ifdef DSA_TRACE
+// Optional per-tile timeline of CTA 0 (build with -DDSA_TRACE): g_fused_trace[event][tile] = %globaltimer.
+__device__ unsigned long long g_fused_trace[8][256];
+#define FTRACE(ev, i)                                                                       \
+  do {                                                                                      \
+    if (blockIdx.x == 0 && (i) < 256) g_fused_trace[ev][(i)] = sm100::globaltimer();        \
+  } while (0)
+#else
+#define FTRACE(ev, i) ((void)0)
+#endif
 
 namespace {
 
@@ -88,12 +100,11 @@ __device__ __forceinline__ uint32_t cluster_size() {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// 32-bit load from the shared memory of CTA `rank` of the cluster at the same offset as `local`.
-__device__ __forceinline__ uint32_t ld_cluster(const void* local, uint32_t rank) {
-  uint32_t remote, v;
+// 32-bit store into the shared memory of CTA `rank` of the cluster at the same offset as `local`.
+__device__ __forceinline__ void st_cluster(void* local, uint32_t rank, uint32_t v) {
+  uint32_t remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
-  return v;
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(remote), "r"(v) : "memory");
 }
 
 template <bool kF8>
@@ -115,10 +126,10 @@ index_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
   uint32_t* hist = keys + p.chunk;                        // [kLevels][256]
   float* wsc_s = reinterpret_cast<float*>(hist + kLevels * 256);
   float* sk_s = wsc_s + p.HI;                              // FP8 only
-  int* misc = reinterpret_cast<int*>(sk_s + (kF8 ? sk_slots * kKeysPerTile : 0));  // [0] bin, [1] remaining,
-                                                           // [2..3] gt/eq counts,
-                                                           // [4..4+kWarps) warp scans, [16..] warp eq scans
-  uint64_t* bars = reinterpret_cast<uint64_t*>(misc + 32);
+  // misc: [0] bin, [1] remaining, [4..4+kWarps) warp gt counts, [16..16+kWarps) warp eq counts,
+  // [32..32+2C) every rank's (gt, eq) totals, pushed by the ranks
+  int* misc = reinterpret_cast<int*>(sk_s + (kF8 ? sk_slots * kKeysPerTile : 0));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(misc + 48);
   uint64_t* full = bars;
   uint64_t* empty = full + kMaxStages;
   uint64_t* tfull = empty + kMaxStages;
@@ -189,6 +200,7 @@ index_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         const int krow = b * p.S + (t_begin + i) * kKeysPerTile;
         if (lane == 0) {
+          FTRACE(0, i);
           const uint32_t dst = sA + (uint32_t)s * kTileBytes;
           mbar_arrive_expect_tx(smem_u32(&full[s]), kTileBytes);
           tma_load_2d(dst, &map_k, smem_u32(&full[s]), 0, krow);
@@ -222,6 +234,7 @@ index_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         const int s = i % p.stages, a = i & 1;
         if (!mbar_wait(smem_u32(&tempty[a]), ((i >> 1) & 1) ^ 1, p.status, &abort_flag)) break;
         if (!mbar_wait(smem_u32(&full[s]), (i / p.stages) & 1, p.status, &abort_flag)) break;
+        FTRACE(1, i);
         tc_fence_after();
         const uint32_t a0 = sA + (uint32_t)s * kTileBytes;
         const uint32_t d = tmem + (uint32_t)(a * p.HI);
@@ -242,6 +255,7 @@ index_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         }
         mma_commit(smem_u32(&empty[s]));
         mma_commit(smem_u32(&tfull[a]));
+        FTRACE(2, i);
       }
       mma_commit(smem_u32(drain));
       mbar_wait(smem_u32(drain), 0, nullptr, nullptr);
@@ -253,6 +267,7 @@ index_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     for (int i = 0; i < n_tiles; ++i) {
       const int a = i & 1;
       if (!mbar_wait(smem_u32(&tfull[a]), (i >> 1) & 1, p.status, &abort_flag)) break;
+      if (quarter == 0 && lane == 0) FTRACE(3, i);
       tc_fence_after();
       const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * p.HI);
       const int s = (t_begin + i) * kKeysPerTile + quarter * 32 + lane;
@@ -270,6 +285,7 @@ index_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         acc += neg ? head_sum32<true>(v, wsc_s + h0) : head_sum32<false>(v, wsc_s + h0);
       }
       if (kF8) acc *= sk;
+      if (quarter == 0 && lane == 0) FTRACE(4, i);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tempty[a]));
@@ -278,12 +294,15 @@ index_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         keys[s - l0] = key;
         atomicAdd(&hist[key >> 24], 1u);
       }
+      __syncwarp();
+      if (quarter == 0 && lane == 0) FTRACE(5, i);
     }
   }
   tc_fence_before();
   __syncthreads();
 
   // ---------------------------------------------------------------- selection
+  if (threadIdx.x == 0) FTRACE(6, 0);
   int32_t* orow = p.idx + row * p.k;
   if (n_vis <= p.k) {
     // every visible key: this CTA's keys sit at positions l0 - vis.lo .. in the ascending list
@@ -291,18 +310,43 @@ index_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     if (rank == C - 1)
       for (int i = n_vis + threadIdx.x; i < p.k; i += kThreads) orow[i] = DSA_INVALID;
   } else {
+    // After scoring, the key stages are free.  Every CTA pushes each round's histogram and its final
+    // counts into every CTA of the cluster (remote stores into the stage area), so the walks read
+    // only local shared memory.  A cluster barrier first makes sure no CTA is still scoring into
+    // its stages.
+    uint32_t* hall = reinterpret_cast<uint32_t*>(gbase + (sA - base));  // [kLevels][C][256]
+    int* call = misc + 32;                                              // [C][2]: each rank's gt, eq
+    cluster_sync();
+    if (threadIdx.x == 0) FTRACE(7, 0);
     uint32_t prefix = 0u, mask = 0u;
     int remaining = p.k;                                 // keys still to take at and below the prefix
     for (int lev = 0; lev < kLevels; ++lev) {
       const int shift = 24 - 8 * lev;
       uint32_t* h = hist + lev * 256;
       if (lev > 0) {
-        for (int i = threadIdx.x; i < n_local; i += kThreads) {
-          const uint32_t key = keys[i];
-          if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
+        // four keys per thread in flight
+        for (int i0 = threadIdx.x; i0 < n_local; i0 += 4 * kThreads) {
+          uint32_t k4[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u * kThreads;
+            k4[u] = i < n_local ? keys[i] : 0u;
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u * kThreads;
+            if (i < n_local && (k4[u] & mask) == prefix) atomicAdd(&h[(k4[u] >> shift) & 255u], 1u);
+          }
         }
+        __syncthreads();                                 // this round's local histogram is complete
       }
-      cluster_sync();                                    // every CTA's histogram of this round is complete
+      for (int bin = threadIdx.x; bin < 256; bin += kThreads) {
+        const uint32_t v = h[bin];
+        uint32_t* dst = hall + (lev * C + rank) * 256 + bin;
+        for (uint32_t r = 0; r < C; ++r) st_cluster(dst, r, v);
+      }
+      if (threadIdx.x == 0) FTRACE(7, 3 * lev + 1);
+      cluster_sync();                                    // every CTA holds every CTA's histogram
       if (warp == 0) {
         // bins from the top: lane l holds bins 255-8l .. 248-8l, summed over the cluster
         uint32_t c[8], tot = 0;
@@ -310,7 +354,7 @@ index_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         for (int j = 0; j < 8; ++j) {
           const int bin = 255 - 8 * lane - j;
           uint32_t v = 0;
-          for (uint32_t r = 0; r < C; ++r) v += ld_cluster(&h[bin], r);
+          for (uint32_t r = 0; r < C; ++r) v += hall[(lev * C + r) * 256 + bin];
           c[j] = v;
           tot += v;
         }
@@ -335,6 +379,7 @@ index_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         }
       }
       __syncthreads();
+      if (threadIdx.x == 0) FTRACE(7, 3 * lev + 2);
       prefix |= (uint32_t)misc[0] << shift;
       mask |= 255u << shift;
       remaining = misc[1];
@@ -342,37 +387,39 @@ index_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     }
     const uint32_t tau = prefix;                         // the k-th largest key
     const int need_eq = remaining;                       // keys equal to tau to take (>= 1)
-    // per-warp counts over contiguous segments, in key order
+    // per-warp counts over contiguous segments, in key order, 64 keys per step
     const int seg = (n_local + kWarps - 1) / kWarps;
     const int e0 = min(n_local, warp * seg), e1 = min(n_local, e0 + seg);
     int gt = 0, eq = 0;
-    for (int i0 = e0; i0 < e1; i0 += 32) {
-      const int i = i0 + lane;
-      const uint32_t key = i < e1 ? keys[i] : 0u;
-      gt += __popc(__ballot_sync(0xffffffffu, i < e1 && key > tau));
-      eq += __popc(__ballot_sync(0xffffffffu, i < e1 && key == tau));
+    for (int i0 = e0; i0 < e1; i0 += 64) {
+      const int ia = i0 + lane, ib = i0 + 32 + lane;
+      const uint32_t ka = ia < e1 ? keys[ia] : 0u, kb = ib < e1 ? keys[ib] : 0u;
+      gt += __popc(__ballot_sync(0xffffffffu, ia < e1 && ka > tau)) + __popc(__ballot_sync(0xffffffffu, ib < e1 && kb > tau));
+      eq += __popc(__ballot_sync(0xffffffffu, ia < e1 && ka == tau)) + __popc(__ballot_sync(0xffffffffu, ib < e1 && kb == tau));
     }
     if (lane == 0) {
       misc[4 + warp] = gt;
       misc[16 + warp] = eq;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int g = 0, e = 0;
-      for (int k = 0; k < kWarps; ++k) {
-        g += misc[4 + k];
-        e += misc[16 + k];
-      }
-      misc[2] = g;
-      misc[3] = e;
+    int g_all = 0, e_all = 0;
+    for (int k = 0; k < kWarps; ++k) {
+      g_all += misc[4 + k];
+      e_all += misc[16 + k];
     }
-    cluster_sync();                                      // every CTA's totals are published
+    if (threadIdx.x < C) {                               // push (gt, eq) to rank threadIdx.x
+      st_cluster(&call[2 * rank], threadIdx.x, (uint32_t)g_all);
+      st_cluster(&call[2 * rank + 1], threadIdx.x, (uint32_t)e_all);
+    }
+    if (threadIdx.x == 0) FTRACE(7, 12);
+    cluster_sync();                                      // every CTA holds every CTA's totals
+    if (threadIdx.x == 0) FTRACE(7, 13);
     int gt_before = 0, eq_before = 0;
     for (uint32_t r = 0; r < rank; ++r) {
-      gt_before += (int)ld_cluster(&misc[2], r);
-      eq_before += (int)ld_cluster(&misc[3], r);
+      gt_before += call[2 * r];
+      eq_before += call[2 * r + 1];
     }
-    const int take = max(0, min(need_eq - eq_before, misc[3]));      // this CTA's tau keys to take
+    const int take = max(0, min(need_eq - eq_before, e_all));        // this CTA's tau keys to take
     int out = gt_before + min(eq_before, need_eq);                   // where this CTA's keys start
     int eq_rank = 0;                                                 // tau keys before this warp's segment
     for (int k = 0; k < warp; ++k) {
@@ -381,21 +428,27 @@ index_topk_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     }
     out += min(eq_rank, take);
     const uint32_t below = (1u << lane) - 1u;
-    for (int i0 = e0; i0 < e1; i0 += 32) {
-      const int i = i0 + lane;
-      const uint32_t key = i < e1 ? keys[i] : 0u;
-      const bool is_gt = i < e1 && key > tau;
-      const bool is_eq = i < e1 && key == tau;
-      const uint32_t m_eq = __ballot_sync(0xffffffffu, is_eq);
-      const int my_eq = eq_rank + __popc(m_eq & below);
-      const bool sel = is_gt || (is_eq && my_eq < take);
-      const uint32_t m_sel = __ballot_sync(0xffffffffu, sel);
-      const int pos = out + __popc(m_sel & below);
-      if (sel && pos < p.k) orow[pos] = l0 + i;        // always true unless an expired wait left keys unscored
-      out += __popc(m_sel);
-      eq_rank += __popc(m_eq);
+    for (int i0 = e0; i0 < e1; i0 += 64) {
+      const int ib = i0 + 32 + lane;
+      const uint32_t kb = ib < e1 ? keys[ib] : 0u;       // the second half's keys load with the first's
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int i = i0 + 32 * half + lane;
+        const uint32_t key = half ? kb : (i < e1 ? keys[i] : 0u);
+        const bool is_gt = i < e1 && key > tau;
+        const bool is_eq = i < e1 && key == tau;
+        const uint32_t m_eq = __ballot_sync(0xffffffffu, is_eq);
+        const int my_eq = eq_rank + __popc(m_eq & below);
+        const bool sel = is_gt || (is_eq && my_eq < take);
+        const uint32_t m_sel = __ballot_sync(0xffffffffu, sel);
+        const int pos = out + __popc(m_sel & below);
+        if (sel && pos < p.k) orow[pos] = l0 + i;      // always true unless an expired wait left keys unscored
+        out += __popc(m_sel);
+        eq_rank += __popc(m_eq);
+      }
     }
   }
+  if (threadIdx.x == 0) FTRACE(6, 1);
   cluster_sync();  // no CTA leaves while a peer may still read its shared memory
   if (warp == 1) {
     tc_fence_after();
@@ -441,7 +494,7 @@ int cluster_for(int S) {
 
 size_t fused_smem(int HI, int stages, int chunk, bool f8) {
   return 1024 + (size_t)HI * row_bytes(f8) + (size_t)stages * tile_bytes(f8) + (size_t)chunk * 4 +
-         kLevels * 256 * 4 + (size_t)HI * 4 + (f8 ? (size_t)(stages + 2) * kKeysPerTile * 4 : 0) + 32 * 4 +
+         kLevels * 256 * 4 + (size_t)HI * 4 + (f8 ? (size_t)(stages + 2) * kKeysPerTile * 4 : 0) + 48 * 4 +
          8 * (2 * kMaxStages + 6 + kMaxStages + 2) + 16;
 }
 
@@ -511,3 +564,9 @@ cudaError_t launch_index_topk(const dsa_dims& d, const void* q_idx, const void* 
 }
 
 }  // namespace dsa
+
+#ifdef DSA_TRACE
+extern "C" int dsa_fused_trace_read(unsigned long long* host) {
+  return (int)cudaMemcpyFromSymbol(host, dsa::g_fused_trace, sizeof(dsa::g_fused_trace));
+}
+#endif
