@@ -215,6 +215,35 @@ def test_pool_gate_softmax_is_per_channel_over_slots():
     assert pooled[1, 1] == pytest.approx(kn[4:8, 1].mean(), abs=1e-14)
 
 
+def test_pool_topk_matches_brute_force_over_fully_visible_pools():
+    """topk_pools_row against brute force on tiny inputs: every pool is scored from the pooled keys one
+    (query head, pool) dot at a time, a pool is a candidate only when all its kpool tokens lie between
+    the first valid token and the query (the pages' 'valid only if all kpool slots are valid'), and the
+    candidates are ranked by a full sort on (score descending, pool id ascending).  Integer operands
+    give many exact ties."""
+    rng = np.random.default_rng(11)
+    kp, n_pools, H, D = 4, 9, 2, 3
+    pooled = rng.integers(-2, 3, size=(n_pools, D)).astype(float)
+    q = rng.integers(-2, 3, size=(H, D)).astype(float)
+    w = np.array([1.0, 0.5])
+    for f in (0, 3):
+        for q_pos in range(f - 1, f + n_pools * kp + 2):
+            for sel_k in (1, 3, 12):
+                got, _ = O.topk_pools_row(q, pooled, w, 0.5, q_pos, f, n_pools, kp, sel_k)
+                cands = []
+                for pid in range(n_pools):
+                    last_token = f + pid * kp + kp - 1
+                    if q_pos >= f and last_token <= q_pos:
+                        score = 0.0
+                        for h in range(H):
+                            dot = sum(q[h, d] * pooled[pid, d] for d in range(D))
+                            score += w[h] * max(0.0, 0.5 * dot)
+                        cands.append((-score, pid))
+                want = [pid for _, pid in sorted(cands)[:sel_k]]
+                want += [O.INVALID] * (sel_k - len(want))
+                assert got.tolist() == want, (f, q_pos, sel_k)
+
+
 # -------------------------------------------------------- P8 expand cases
 def test_expand_selection_examples():
     g = _golden("hand_kpool.json")
@@ -490,7 +519,8 @@ def _run_pins():
                test_rotated_queries_and_keys_give_the_same_scores, test_e4m3_grid_is_the_format_and_decodes_like_torch,
                test_e4m3_rounding_ties_to_even_and_matches_torch,
                test_fp8_quantization_maps_each_vector_amax_to_448_within_the_grid_error,
-               test_fp8_scores_equal_plain_scores_when_the_operands_are_e4m3_values_with_amax_448):
+               test_fp8_scores_equal_plain_scores_when_the_operands_are_e4m3_values_with_amax_448,
+               test_pool_topk_matches_brute_force_over_fully_visible_pools):
         try:
             fn()
         except (AssertionError, ValueError, IndexError):
@@ -503,7 +533,7 @@ def _run_pins():
                                     "tail_off_by_one", "absorb_transposed", "rope_adjacent_pairs",
                                     "rope_frequency_exponent", "hadamard_before_rope", "layer_norm_after_rope",
                                     "hadamard_unnormalised", "e4m3_ties_away", "e4m3_two_mantissa_bits",
-                                    "fp8_key_scale_dropped"])
+                                    "fp8_key_scale_dropped", "pool_visible_at_first_token"])
 def test_pins_catch_planted_mistakes(monkeypatch, mutant):
     """Plant a plausible mistake in the oracle (on the CPU) and check a pin fails."""
     assert _run_pins() == 0
@@ -615,4 +645,12 @@ def test_pins_catch_planted_mistakes(monkeypatch, mutant):
             act = np.maximum(0.0, float(scale) * qs[:, None] * (qc @ kc.T))
             return (O.f64(w_row)[:, None] * act).sum(axis=0) + 0.0
         monkeypatch.setattr(O, "index_scores_fp8_row", no_kscale)
+    elif mutant == "pool_visible_at_first_token":
+        # a pool counted visible once its first token is, instead of all of its tokens
+        def early(q_pos, kv_start, n_pools, kpool):
+            f = int(kv_start)
+            if q_pos < f:
+                return np.zeros(0, dtype=np.int64)
+            return np.arange(0, min((int(q_pos) - f) // kpool + 1, int(n_pools)), dtype=np.int64)
+        monkeypatch.setattr(O, "visible_pools", early)
     assert _run_pins() > 0, f"mutant {mutant} survived every pin"
