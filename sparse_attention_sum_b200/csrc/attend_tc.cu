@@ -26,16 +26,19 @@
 // value-side query blocks 128-255 as the A operand of q.k (two bf16 per
 // column), O 256-511.  The 32 rope columns of each CTA use a 64-byte-swizzled
 // shared-memory operand.
-// The bf16 probabilities overwrite the first 32 columns of their score buffer
-// and feed P.V straight from tensor memory.  Every tcgen05.mma here costs about
+// The bf16 probabilities go to the first 16 KB of the chunk's exchange tile (its
+// fp32 partial scores are consumed by then), as a 128-byte-swizzled K-major
+// operand of P.V: a score buffer is free again as soon as it has been read, so
+// the q.k two chunks ahead never waits for P.V, and the exchange tile returns
+// to the peer once P.V has read it.  Every tcgen05.mma here costs about
 // 100 cycles whatever its N up to 128, so q.k uses N = 64 keys per instruction
 // and P.V N = 256 value columns.  The running maximum only moves (and O is
 // rescaled in TMEM) when it grows by more than 2^8.
 //
-// Warp roles per CTA: warps 0-3 and 13-16 load the query columns into TMEM, then
-// run the softmax and the epilogue (one head row per thread, TMEM lanes 0-127;
-// the two groups take the two halves of every chunk's keys and of O); warps
-// 9-12 read the same score rows and push them to the peer (buffer reuse is
+// Warp roles per CTA: warps 0-3 and 13-16 run the softmax and the epilogue (one
+// head row per thread, TMEM lanes 0-127; the two groups take the two halves of
+// every chunk's keys and of O); warps 9-12 load the query columns into TMEM,
+// read the same score rows and push them to the peer (buffer reuse is
 // acknowledged by the peer); warp 4 issues tcgen05.mma from a polling scheduler
 // (and loads the CTA's rope query columns by TMA); warps 5-8 stage and
 // deduplicate the index row, then each issues the gathers of one value block
@@ -114,7 +117,7 @@ struct Smem {
   float* mx;                 // [2 parities][2 groups][128 rows] half-row maxima
   float* lsum;               // [2 groups][128 rows] partial row sums for the epilogue
   uint64_t *qfull, *qrope_full, *list_ready, *list_taken, *kv_full, *kv_empty, *s_full, *s_read, *p_full, *o_done,
-      *o_free, *xfull, *xfree, *xread, *mxready, *lready, *drain;
+      *o_free, *xfull, *xfree, *mxready, *lready, *drain;
   uint32_t* tmem_slot;
   int* n_list;               // [2]: list length of the published row, by row parity
   int* dup_flag;
@@ -137,6 +140,10 @@ __device__ __forceinline__ uint32_t map_peer(uint32_t addr, uint32_t peer) {
 __device__ __forceinline__ void st_async_v4(uint32_t addr, const uint32_t* v, uint32_t remote_bar) {
   asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
                "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(remote_bar)
+               : "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t* v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
                : "memory");
 }
 __device__ __forceinline__ void st_global_v8(void* ptr, const uint32_t* v) {
@@ -384,8 +391,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   sm.o_done = sm.p_full + 2;
   sm.xfull = sm.o_done + 2;
   sm.xfree = sm.xfull + 2;
-  sm.xread = sm.xfree + 2;
-  sm.mxready = sm.xread + 2;
+  sm.mxready = sm.xfree + 2;
   sm.o_free = sm.mxready + 2;
   sm.lready = sm.o_free + 1;
   sm.drain = sm.lready + 1;
@@ -419,13 +425,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&sm.s_full[s]), 1);
-      mbar_init(smem_u32(&sm.s_read[s]), 4);      // exchange warps have read the score buffer
-      mbar_init(smem_u32(&sm.p_full[s]), 8);      // both softmax groups
+      mbar_init(smem_u32(&sm.s_read[s]), 12);     // the 4 exchange and 8 softmax warps have read the score buffer
+      mbar_init(smem_u32(&sm.p_full[s]), 8);      // both softmax groups wrote their P columns
       mbar_init(smem_u32(&sm.mxready[s]), 8);
       mbar_init(smem_u32(&sm.o_done[s]), 1);
       mbar_init(smem_u32(&sm.xfull[s]), 1);       // armed by our softmax; completed by the peer's st.async bytes
       mbar_init(smem_u32(&sm.xfree[s]), 4);       // one arrival per peer exchange warp
-      mbar_init(smem_u32(&sm.xread[s]), 8);       // one arrival per local softmax warp
     }
     mbar_init(smem_u32(sm.drain), 1);
     fence_barrier_init();
@@ -575,13 +580,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           }
         }
 #endif
-        // q.k of chunk gq: at a row start its query is loaded; its stage is loaded; P.V of chunk
-        // gq-2 (same score buffer) is done
+        // q.k of chunk gq: at a row start its query is loaded; its stage is loaded; the scores of
+        // chunk gq-2 (same score buffer) have been read
         if (qn > 0 &&
             (qj > 0 || (mbar_test_wait(smem_u32(sm.qfull), qi & 1) &&
                         (!rope || mbar_test_wait(smem_u32(sm.qrope_full), qi & 1)))) &&
             mbar_test_wait(smem_u32(&sm.kv_full[gq % kStages]), (uint32_t)((gq / kStages) & 1)) &&
-            mbar_test_wait(smem_u32(&sm.o_done[gq & 1]), (uint32_t)(((gq >> 1) & 1) ^ 1))) {
+            mbar_test_wait(smem_u32(&sm.s_read[gq & 1]), (uint32_t)(((gq >> 1) & 1) ^ 1))) {
           tc_fence_after();
           const uint32_t st = sm.kv + (gq % kStages) * kStageBytes;
           const uint32_t d = tmem + (gq & 1) * kChunk;
@@ -608,15 +613,16 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           }
           progressed = true;
         }
-        // P.V of chunk gp: its P is in TMEM; at a row start the previous row's O has been read
+        // P.V of chunk gp: its P is in the exchange tile; at a row start the previous row's O has been read
         if (gp < gq && (pj > 0 || p_ne == 0 || mbar_test_wait(smem_u32(sm.o_free), (p_ne - 1) & 1)) &&
             mbar_test_wait(smem_u32(&sm.p_full[gp & 1]), (uint32_t)((gp >> 1) & 1))) {
           tc_fence_after();
           const uint32_t st = sm.kv + (gp % kStages) * kStageBytes;
+          const uint32_t pt = sm.x + (uint32_t)(gp & 1) * kXBytes;   // P: 128 head rows x 64 keys, 128 B each
 #pragma unroll
           for (int k = 0; k < kChunk / 16; ++k) {
             const uint64_t bd = desc_sw128(st + k * 2048, 1024, kBlockBytes);
-            mma_bf16_ts(tmem + kOCol, tmem + (gp & 1) * kChunk + k * 8, bd, id_pv, (pj | k) ? 1u : 0u);
+            mma_bf16_ss(tmem + kOCol, desc_sw128(pt + k * 32), bd, id_pv, (pj | k) ? 1u : 0u);
           }
           mma_commit(smem_u32(&sm.kv_empty[gp % kStages]));
           mma_commit(smem_u32(&sm.o_done[gp & 1]));
@@ -691,8 +697,16 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       }
     };
     if (my_rows > 0) load_q(0);
-    long long gc = 0;
+    long long gc = 0, pend = -1;   // pend: the chunk whose exchange tile still has to go back to the peer
     bool ok = true;
+    // P.V of chunk c has read its P (the first half of our exchange tile c & 1): the peer may refill the tile
+    auto give_back = [&](long long c) {
+      if (!mbar_wait(smem_u32(&sm.o_done[c & 1]), (uint32_t)((c >> 1) & 1), p.status, abort_flag)) return false;
+      if (q4 == 1 && lane == 0) TRACE(14, c);
+      __syncwarp();
+      if (lane == 0) arrive_remote_relaxed(map_peer(smem_u32(&sm.xfree[c & 1]), peer));
+      return true;
+    };
     for (int i = 0; ok && i < my_rows; ++i) {
       if (!(ok = mbar_wait(smem_u32(sm.list_ready), i & 1, p.status, abort_flag))) break;
       const int n = sm.n_list[i & 1];
@@ -728,23 +742,20 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           if (lane == 0) mbar_arrive(smem_u32(&sm.s_read[sb]));
         }
         if (q4 == 1 && lane == 0) TRACE(4, gc);
-        if (j + 1 == nch) break;                     // the last chunk's buffer is released below
-        // once our softmax has read our buffer sb of chunk gc, the peer may refill it
-        if (!(ok = mbar_wait(smem_u32(&sm.xread[sb]), use, p.status, abort_flag))) break;
-        __syncwarp();
-        if (lane == 0) arrive_remote_relaxed(map_peer(smem_u32(&sm.xfree[sb]), peer));
+        if (j + 1 == nch) break;                     // the row's last chunk continues below
+        // the previous chunk's tile goes back after this chunk's push, which therefore never waits for a P.V
+        if (pend >= 0 && !(ok = give_back(pend))) break;
+        pend = gc;
       }
       if (ok && nch > 0) {
-        // the row's last q.k is complete (its scores were just read): load the next row's query,
-        // then release the last chunk's exchange buffer
+        // the row's last q.k is complete (its scores were just read): load the next row's query first
         if (i + 1 < my_rows) load_q(i + 1);
-        const int sb = (int)(gc & 1);
-        if (!(ok = mbar_wait(smem_u32(&sm.xread[sb]), (uint32_t)((gc >> 1) & 1), p.status, abort_flag))) break;
-        __syncwarp();
-        if (lane == 0) arrive_remote_relaxed(map_peer(smem_u32(&sm.xfree[sb]), peer));
+        if (pend >= 0 && !(ok = give_back(pend))) break;
+        pend = gc;
         ++gc;
       }
     }
+    if (ok && pend >= 0) give_back(pend);
   } else if (warp < 4 || warp >= 13) {
     // ---------------------------------------------------------------- softmax + epilogue
     // Group g (warps 0-3 or 13-16) takes keys 32g..32g+31 of every chunk and O columns 128g..128g+127.
@@ -829,7 +840,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         if (!act) {
           // head rows >= H (H = 64): keep every barrier's count, compute nothing
           __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&sm.xread[sb]));
+          if (lane == 0) mbar_arrive(smem_u32(&sm.s_read[sb]));
           if (lane == 0) mbar_arrive(smem_u32(&sm.mxready[sb]));
           if (!(ok = mbar_wait(smem_u32(&sm.mxready[sb]), use, p.status, abort_flag))) break;
           if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[sb]));
@@ -839,6 +850,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk + 32 * g, v);
         tmem_ld_wait();
+        // the score buffer may be refilled by the q.k two chunks ahead
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.s_read[sb]));
         if (lead) TRACE(5, gc);
         if (!(ok = wait_cluster(smem_u32(&sm.xfull[sb]), use, p.status, abort_flag))) break;
         if (lead) {
@@ -859,10 +874,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             mx = fmaxf(mx, x);
           }
         }
-        // our buffer sb is read (values are in registers); the exchange warps tell the peer
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&sm.xread[sb]));
-        // row maximum over both halves of the chunk
+        // row maximum over both halves of the chunk (once both groups pass this barrier, every
+        // fp32 value of exchange tile sb has been read, and P may overwrite its first half)
         float* mxb = sm.mx + sb * 256;
         mxb[g * 128 + r] = mx;
         __syncwarp();
@@ -899,11 +912,14 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           pk[c / 2] = pack_bf16(p0, p1);
         }
         if (lead) TRACE(10, gc);
-        // P (keys 32g..32g+31) overwrites columns 16g..16g+15 of the score buffer once the exchange warps have read it
-        if (!(ok = mbar_wait(smem_u32(&sm.s_read[sb]), use, p.status, abort_flag))) break;
-        tmem_st_32x32b_x16(tmem + lane_addr + sb * kChunk + 16 * g, pk);
-        tmem_st_wait();
-        tc_fence_before();
+        // P of keys 32g..32g+31: 16-byte chunks 4g..4g+3 of row r of the 128-byte-swizzled K-major
+        // tile at the start of exchange tile sb (chunk c of row r sits at position c ^ (r & 7))
+        {
+          const uint32_t prow = sm.x + (uint32_t)sb * kXBytes + (uint32_t)r * 128u;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) st_shared_v4(prow + ((uint32_t)((4 * g + k) ^ (r & 7)) << 4), &pk[4 * k]);
+        }
+        fence_proxy_async_smem();                   // visible to the tensor core's operand reads
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[sb]));
         if (lead) TRACE(7, gc);
