@@ -41,9 +41,12 @@
 // read the same score rows and push them to the peer (buffer reuse is
 // acknowledged by the peer); warp 4 issues tcgen05.mma from a polling scheduler
 // (and loads the CTA's rope query columns by TMA); warps 5-8 stage and
-// deduplicate the index row, then each issues the gathers of one value block
-// and a quarter of the rope block (TMA runs them off the load/store pipe that
-// the softmax and exchange warps use).  Every mbarrier wait is bounded.
+// deduplicate the index row, then issue the TMA gathers of value blocks 0-2
+// (TMA runs them off the load/store pipe that the softmax and exchange warps
+// use, but each gather costs its issuing warp about 60 ns); warps 17-19 issue
+// those of value block 3 and the rope columns, so that seven warps share the 80
+// gathers of a chunk.
+// Every mbarrier wait is bounded.
 #include <cuda.h>
 
 #include "dsa_common.cuh"
@@ -79,8 +82,9 @@ constexpr int kNarrowKeys = 65536;                          // key lists of 16-b
 constexpr int kMaxKeys = kStageBytes * 8;                   // 294912: the dedupe bitmap fits one stage
 constexpr int kQCol = 128;                                  // query columns in TMEM
 constexpr int kOCol = 256;                                  // output accumulator
-constexpr int kThreads = 544;          // 17 warps
-constexpr int kProducerThreads = 128;  // warps 5-8
+constexpr int kThreads = 640;          // 20 warps (registers are granted per 4 warps: 17 cost as much)
+constexpr int kProducerThreads = 128;  // warps 5-8: key lists and TMA gathers of value blocks 0-2
+constexpr int kCopyWarps = 3;          // warps 17-19: TMA gathers of value block 3 and the rope columns
 
 struct AttTcParams {
   int B, T, S, H, kd, width;
@@ -117,7 +121,7 @@ struct Smem {
   float* mx;                 // [2 parities][2 groups][128 rows] half-row maxima
   float* lsum;               // [2 groups][128 rows] partial row sums for the epilogue
   uint64_t *qfull, *qrope_full, *list_ready, *list_taken, *kv_full, *kv_empty, *s_full, *s_read, *p_full, *o_done,
-      *o_free, *xfull, *xfree, *mxready, *lready, *drain;
+      *o_free, *xfull, *xfree, *mxready, *lready, *drain, *list_free;
   uint32_t* tmem_slot;
   int* n_list;               // [2]: list length of the published row, by row parity
   int* dup_flag;
@@ -359,8 +363,7 @@ __device__ int compact_first(const AttTcParams& p, const Smem& sm, const int32_t
 template <bool kHalfHeads, bool kWide>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
-                 const __grid_constant__ CUtensorMap map_rope,
-                 AttTcParams p) {
+                 const __grid_constant__ CUtensorMap map_rope, AttTcParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ int s_misc[5];
   __shared__ int s_wcount[4];
@@ -395,7 +398,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   sm.o_free = sm.mxready + 2;
   sm.lready = sm.o_free + 1;
   sm.drain = sm.lready + 1;
-  sm.tmem_slot = reinterpret_cast<uint32_t*>(sm.drain + 1);
+  sm.list_free = sm.drain + 1;
+  sm.tmem_slot = reinterpret_cast<uint32_t*>(sm.list_free + 1);
   sm.n_list = &s_misc[0];                        // [0], [1]
   sm.dup_flag = &s_misc[2];
   sm.abort_flag = &s_misc[3];
@@ -420,7 +424,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     mbar_init(smem_u32(sm.o_free), 8);           // per non-empty row: the epilogue has read O
     mbar_init(smem_u32(sm.lready), 8);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&sm.kv_full[s]), 1);     // one expect-tx arrival; the gathers complete the bytes
+      // one expect-tx arrival per gathering warp set (warps 5-8, then each of warps 17-19); the
+      // TMA gathers complete the bytes
+      mbar_init(smem_u32(&sm.kv_full[s]), 1 + kCopyWarps);
       mbar_init(smem_u32(&sm.kv_empty[s]), 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -433,6 +439,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       mbar_init(smem_u32(&sm.xfree[s]), 4);       // one arrival per peer exchange warp
     }
     mbar_init(smem_u32(sm.drain), 1);
+    mbar_init(smem_u32(sm.list_free), kCopyWarps);  // per row: warps 17-19 are done with its list
     fence_barrier_init();
     for (int s = 0; s < 2; ++s) mbar_arrive_expect_tx(smem_u32(&sm.xfull[s]), 64u * p.H * 4u);  // first use of each buffer
   }
@@ -447,12 +454,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
   if (warp >= 5 && warp <= 8) {
     // ---------------------------------------------------------------- lists + gathers
-    const int w = warp - 5;                              // 0..3: value block w; rope rows 16w..16w+15
-    const uint32_t stage_bytes = rope ? kStageBytes : 4 * kBlockBytes;
-    if (lane == 0) {
-      tma_prefetch_desc(&map_kv);
-      if (rope) tma_prefetch_desc(&map_rope);
-    }
+    const int w = warp - 5;                              // 0..3: gathers 12w..12w+11 of each chunk
+    if (lane == 0) tma_prefetch_desc(&map_kv);
     long long gc = 0;                                    // global chunk counter
     bool ok = true;
     for (int i = 0; i < my_rows; ++i) {
@@ -460,10 +463,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       const int32_t* irow = p.idx + row * p.width;
       RowKeys rk;
       load_row(p, irow, rk);                             // in flight while the waits below run
-      // every consumer has read the previous row's length before this row's is published
+      // every consumer has read the previous row's length before this row's is published, and the
+      // copy warps have issued the previous row's copies (they read its list)
       const int s0 = (int)(gc % kStages);
       bool got = true;
-      if (w == 0 && lane == 0) got = i == 0 || mbar_wait(smem_u32(sm.list_taken), (i - 1) & 1, p.status, abort_flag);
+      if (w == 0 && lane == 0)
+        got = i == 0 || (mbar_wait(smem_u32(sm.list_taken), (i - 1) & 1, p.status, abort_flag) &&
+                         mbar_wait(smem_u32(sm.list_free), (i - 1) & 1, p.status, abort_flag));
       if (named_any(1, kProducerThreads, !got)) {
         ok = false;
         break;
@@ -507,27 +513,25 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           break;
         if (w == 0 && lane == 0) {
           TRACE(0, gc);
-          mbar_arrive_expect_tx(smem_u32(&sm.kv_full[s]), stage_bytes);
+          mbar_arrive_expect_tx(smem_u32(&sm.kv_full[s]), 3 * kBlockBytes);
         }
         const uint32_t stb = sm.kv + s * kStageBytes;
         const uint32_t bar = smem_u32(&sm.kv_full[s]);
         // TMA tile::gather4: four selected rows per instruction, written in the swizzled operand
         // layout.  Rows past the list repeat the list's first key (their scores are masked, P = 0).
-        // Lanes 0-15 gather 64 value columns of keys 4*lane..4*lane+3 into block w; lanes 16-19
-        // gather the 32 rope columns of keys 4*(4w+lane-16).. into the 64-byte swizzled rope block.
-        const int g = lane < 16 ? lane : 4 * w + (lane - 16);
-        if (lane < 16 || (rope && lane < 20)) {
+        // Gather o = 12w + lane (lane < 12) brings the 64 columns of value block o / 16 of keys
+        // 4g..4g+3, g = o % 16 (a gather costs its warp about 60 ns to issue, so the 48 gathers of
+        // a chunk are spread over the four warps; block 3 and the rope columns are the copy warps').
+        if (lane < 12) {
+          const int o = 12 * w + lane, b = o >> 4, g = o & 15;
           int rr[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const int li = j * kChunk + 4 * g + k;
             rr[k] = rowbase + get_key<kWide>(p, sm, li < n ? li : 0);
           }
-          if (lane < 16)
-            tma_gather4(stb + w * kBlockBytes + g * 512, &map_kv, bar, (4 * (int)rank + w) * 64, rr[0], rr[1],
-                        rr[2], rr[3]);
-          else
-            tma_gather4(stb + kRopeOff + g * 256, &map_rope, bar, rope_col, rr[0], rr[1], rr[2], rr[3]);
+          tma_gather4(stb + b * kBlockBytes + g * 512, &map_kv, bar, (4 * (int)rank + b) * 64, rr[0], rr[1], rr[2],
+                      rr[3]);
         }
         if (w == 0 && lane == 0) TRACE(11, gc);
       }
@@ -756,6 +760,56 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       }
     }
     if (ok && pend >= 0) give_back(pend);
+  } else if (warp >= 17) {
+    // ---------------------------------------------------------------- more TMA gathers
+    // Gather o = 11 (warp - 17) + lane of the 16 of value block 3 (o < 16: keys 4o..4o+3, latent
+    // columns (4 rank + 3) * 64 ..) and, when kd = 576, the 16 of the CTA's 32 rope columns (o - 16:
+    // keys 4(o-16).., 64-byte swizzled rope block).  Each warp arms the stage's barrier with its
+    // own bytes.
+    const int cw = warp - 17;
+    const int nops = rope ? 32 : 16;
+    const int o = 11 * cw + lane;
+    const bool mine = lane < 11 && o < nops;
+    uint32_t bytes = 0;                               // this warp's bytes per chunk
+    for (int k = 11 * cw; k < 11 * cw + 11 && k < nops; ++k) bytes += k < 16 ? 512u : 256u;
+    if (lane == 0) {
+      tma_prefetch_desc(&map_kv);
+      if (rope) tma_prefetch_desc(&map_rope);
+    }
+    long long gc = 0;
+    bool ok = true;
+    for (int i = 0; ok && i < my_rows; ++i) {
+      const size_t row = row_of(i);
+      if (!(ok = mbar_wait(smem_u32(sm.list_ready), i & 1, p.status, abort_flag))) break;
+      const int n = sm.n_list[i & 1];
+      const int nch = (n + kChunk - 1) / kChunk;
+      const int rowbase = (int)(row / p.T) * p.S;
+      for (int j = 0; j < nch; ++j, ++gc) {
+        const int s = (int)(gc % kStages);
+        if (!(ok = mbar_wait(smem_u32(&sm.kv_empty[s]), (uint32_t)(((gc / kStages) & 1) ^ 1), p.status, abort_flag)))
+          break;
+        const uint32_t stb = sm.kv + s * kStageBytes;
+        const uint32_t bar = smem_u32(&sm.kv_full[s]);
+        if (lane == 0) mbar_arrive_expect_tx(bar, bytes);
+        if (mine) {
+          const int g = o & 15;
+          int rr[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int li = j * kChunk + 4 * g + k;
+            rr[k] = rowbase + get_key<kWide>(p, sm, li < n ? li : 0);
+          }
+          if (o < 16)
+            tma_gather4(stb + 3 * kBlockBytes + g * 512, &map_kv, bar, (4 * (int)rank + 3) * 64, rr[0], rr[1], rr[2],
+                        rr[3]);
+          else
+            tma_gather4(stb + kRopeOff + g * 256, &map_rope, bar, rope_col, rr[0], rr[1], rr[2], rr[3]);
+        }
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(sm.list_free));   // this row's list may be rewritten
+    }
   } else if (warp < 4 || warp >= 13) {
     // ---------------------------------------------------------------- softmax + epilogue
     // Group g (warps 0-3 or 13-16) takes keys 32g..32g+31 of every chunk and O columns 128g..128g+127.
@@ -1013,7 +1067,7 @@ cudaError_t launch_attend_tc(const dsa_dims& d, const void* q, const void* k, in
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   // latent viewed as [B*S rows, kd cols] with the caller's row stride; box = 64 cols x 1 row (gather4)
-  CUtensorMap mkv;
+  CUtensorMap mkv, mrope;
   cuuint64_t kdims[2] = {(cuuint64_t)d.kd, (cuuint64_t)d.batch * d.n_kv};
   cuuint64_t kstrides[1] = {(cuuint64_t)k_stride * 2};
   cuuint32_t kbox[2] = {64u, 1u};
@@ -1023,7 +1077,6 @@ cudaError_t launch_attend_tc(const dsa_dims& d, const void* q, const void* k, in
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   // the same rows, 32 rope columns per box with the 64-byte swizzle of the rope operand
-  CUtensorMap mrope;
   cuuint32_t rbox[2] = {32u, 1u};
   if (enc(&mrope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(k), kdims, kstrides, rbox, estr,
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
