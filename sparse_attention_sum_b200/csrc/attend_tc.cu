@@ -121,7 +121,7 @@ struct Smem {
   float* mx;                 // [2 parities][2 groups][128 rows] half-row maxima
   float* lsum;               // [2 groups][128 rows] partial row sums for the epilogue
   uint64_t *qfull, *qrope_full, *list_ready, *list_taken, *kv_full, *kv_empty, *s_full, *s_read, *p_full, *o_done,
-      *o_free, *xfull, *xfree, *mxready, *lready, *drain, *list_free;
+      *o_free, *xfull, *xfree, *xread1, *mxready, *lready, *drain, *list_free;
   uint32_t* tmem_slot;
   int* n_list;               // [2]: list length of the published row, by row parity
   int* dup_flag;
@@ -392,9 +392,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   sm.s_read = sm.s_full + 2;
   sm.p_full = sm.s_read + 2;
   sm.o_done = sm.p_full + 2;
-  sm.xfull = sm.o_done + 2;
-  sm.xfree = sm.xfull + 2;
-  sm.mxready = sm.xfree + 2;
+  sm.xfull = sm.o_done + 2;                      // [buffer][half]
+  sm.xfree = sm.xfull + 4;                       // [buffer][half]
+  sm.xread1 = sm.xfree + 4;
+  sm.mxready = sm.xread1 + 2;
   sm.o_free = sm.mxready + 2;
   sm.lready = sm.o_free + 1;
   sm.drain = sm.lready + 1;
@@ -435,13 +436,16 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       mbar_init(smem_u32(&sm.p_full[s]), 8);      // both softmax groups wrote their P columns
       mbar_init(smem_u32(&sm.mxready[s]), 8);
       mbar_init(smem_u32(&sm.o_done[s]), 1);
-      mbar_init(smem_u32(&sm.xfull[s]), 1);       // armed by our softmax; completed by the peer's st.async bytes
-      mbar_init(smem_u32(&sm.xfree[s]), 4);       // one arrival per peer exchange warp
+      for (int h = 0; h < 2; ++h) {
+        mbar_init(smem_u32(&sm.xfull[2 * s + h]), 1);  // armed by our softmax; completed by the peer's st.async bytes
+        mbar_init(smem_u32(&sm.xfree[2 * s + h]), 4);  // one arrival per peer exchange warp
+      }
+      mbar_init(smem_u32(&sm.xread1[s]), 4);      // the group-1 softmax warps have read half 1
     }
     mbar_init(smem_u32(sm.drain), 1);
     mbar_init(smem_u32(sm.list_free), kCopyWarps);  // per row: warps 17-19 are done with its list
     fence_barrier_init();
-    for (int s = 0; s < 2; ++s) mbar_arrive_expect_tx(smem_u32(&sm.xfull[s]), 64u * p.H * 4u);  // first use of each buffer
+    for (int s = 0; s < 4; ++s) mbar_arrive_expect_tx(smem_u32(&sm.xfull[s]), 32u * p.H * 4u);  // first use of each half
   }
   if (warp == 4) tmem_alloc(smem_u32(sm.tmem_slot), 512);
   tc_fence_before();
@@ -703,12 +707,17 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     if (my_rows > 0) load_q(0);
     long long gc = 0, pend = -1;   // pend: the chunk whose exchange tile still has to go back to the peer
     bool ok = true;
-    // P.V of chunk c has read its P (the first half of our exchange tile c & 1): the peer may refill the tile
+    // Exchange tile c & 1 goes back to the peer in two halves: half 1 (keys 32-63) once our group-1
+    // softmax warps have read it, half 0 (keys 0-31, overwritten by P) once P.V of chunk c has read P.
     auto give_back = [&](long long c) {
-      if (!mbar_wait(smem_u32(&sm.o_done[c & 1]), (uint32_t)((c >> 1) & 1), p.status, abort_flag)) return false;
+      const uint32_t ph = (uint32_t)((c >> 1) & 1);
+      if (!mbar_wait(smem_u32(&sm.xread1[c & 1]), ph, p.status, abort_flag)) return false;
+      __syncwarp();
+      if (lane == 0) arrive_remote_relaxed(map_peer(smem_u32(&sm.xfree[2 * (c & 1) + 1]), peer));
+      if (!mbar_wait(smem_u32(&sm.o_done[c & 1]), ph, p.status, abort_flag)) return false;
       if (q4 == 1 && lane == 0) TRACE(14, c);
       __syncwarp();
-      if (lane == 0) arrive_remote_relaxed(map_peer(smem_u32(&sm.xfree[c & 1]), peer));
+      if (lane == 0) arrive_remote_relaxed(map_peer(smem_u32(&sm.xfree[2 * (c & 1)]), peer));
       return true;
     };
     for (int i = 0; ok && i < my_rows; ++i) {
@@ -732,14 +741,19 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&sm.s_read[sb]));
           if (q4 == 1 && lane == 0) TRACE(3, gc);
-          // the peer has read its buffer sb from chunk gc-2
-          if (!(ok = wait_cluster(smem_u32(&sm.xfree[sb]), use ^ 1u, p.status, abort_flag))) break;
-          const uint32_t dst = dst0 + (uint32_t)sb * kXBytes;
           // [key/4][head][4 keys]: each store writes 4 keys of head r, the warp 512 contiguous
-          // bytes; each store completes its bytes on the peer's barrier (no round trip here)
-          const uint32_t xbar = map_peer(smem_u32(&sm.xfull[sb]), peer);
+          // bytes; each store completes its bytes on the peer's barrier of that half (no round trip
+          // here).  Half 1 first: the peer returns it as soon as its softmax has read it, half 0
+          // only after its P.V (P overwrites half 0).
+          const uint32_t dst = dst0 + (uint32_t)sb * kXBytes;
+          if (!(ok = wait_cluster(smem_u32(&sm.xfree[2 * sb + 1]), use ^ 1u, p.status, abort_flag))) break;
+          const uint32_t xbar1 = map_peer(smem_u32(&sm.xfull[2 * sb + 1]), peer);
 #pragma unroll
-          for (int c = 0; c < kChunk; c += 4) st_async_v4(dst + c * 512, &v[c], xbar);
+          for (int c = 32; c < kChunk; c += 4) st_async_v4(dst + c * 512, &v[c], xbar1);
+          if (!(ok = wait_cluster(smem_u32(&sm.xfree[2 * sb]), use ^ 1u, p.status, abort_flag))) break;
+          const uint32_t xbar0 = map_peer(smem_u32(&sm.xfull[2 * sb]), peer);
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) st_async_v4(dst + c * 512, &v[c], xbar0);
         } else {
           // head rows >= H: nothing to read or send
           __syncwarp();
@@ -895,6 +909,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           // head rows >= H (H = 64): keep every barrier's count, compute nothing
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&sm.s_read[sb]));
+          if (lane == 0 && g == 1) mbar_arrive(smem_u32(&sm.xread1[sb]));
           if (lane == 0) mbar_arrive(smem_u32(&sm.mxready[sb]));
           if (!(ok = mbar_wait(smem_u32(&sm.mxready[sb]), use, p.status, abort_flag))) break;
           if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[sb]));
@@ -909,10 +924,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.s_read[sb]));
         if (lead) TRACE(5, gc);
-        if (!(ok = wait_cluster(smem_u32(&sm.xfull[sb]), use, p.status, abort_flag))) break;
-        if (lead) {
-          TRACE(6, gc);
-          mbar_arrive_expect_tx(smem_u32(&sm.xfull[sb]), 64u * p.H * 4u);  // arm the next use (H rows)
+        // our half g of exchange tile sb (keys 32g..32g+31 of the peer's partial scores)
+        if (!(ok = wait_cluster(smem_u32(&sm.xfull[2 * sb + g]), use, p.status, abort_flag))) break;
+        if (q4 == 0 && lane == 0) {
+          if (g == 0) TRACE(6, gc);
+          mbar_arrive_expect_tx(smem_u32(&sm.xfull[2 * sb + g]), 32u * p.H * 4u);  // arm the next use (H rows)
         }
         const float4* xr = xcol + sb * (kXBytes / 16) + 8 * g * 128;
         const int valid = n - j * kChunk - 32 * g;
@@ -927,6 +943,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             v[c + k] = __float_as_uint(x);
             mx = fmaxf(mx, x);
           }
+        }
+        if (g == 1) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&sm.xread1[sb]));   // half 1 may go back to the peer
         }
         // row maximum over both halves of the chunk (once both groups pass this barrier, every
         // fp32 value of exchange tile sb has been read, and P may overwrite its first half)
@@ -1014,7 +1034,7 @@ EncodeTiledFn encode_fn() {
 
 size_t smem_bytes(int width, int S, bool with_bitmap) {
   return 1024 + 2 * (size_t)kXBytes + kQRopeBytes + (size_t)kStages * kStageBytes + list_bytes(width, S, with_bitmap) +
-         2 * 2 * 128 * 4 + 2 * 128 * 4 + 8 * 40 + 16;
+         2 * 2 * 128 * 4 + 2 * 128 * 4 + 8 * 48 + 16;
 }
 
 bool bitmap_in_list(int width, int S) { return smem_bytes(width, S, true) <= 227 * 1024; }
