@@ -77,7 +77,9 @@ constexpr int kBlockBytes = kChunk * 128;                   // one 64-col block 
 constexpr int kRopeOff = 4 * kBlockBytes;                   // 32 rope columns after the 4 value blocks
 constexpr int kStageBytes = kRopeOff + kChunk * 64;         // 36 KB
 constexpr int kQRopeBytes = 128 * 64;                       // rope query columns in smem: 8 KB
-constexpr int kXBytes = kChunk * 128 * 4;                   // exchange tile [key/4][head][4] fp32: 32 KB
+// exchange tile, fp32 [key half][head quarter][key/4 within the half][32 heads][4 keys]: 32 KB; the P rows
+// of a head quarter (128-byte rows at the start of the tile) cover exactly that quarter's half-0 scores
+constexpr int kXBytes = kChunk * 128 * 4;
 constexpr int kNarrowKeys = 65536;                          // key lists of 16-bit entries up to here
 constexpr int kMaxKeys = kStageBytes * 8;                   // 294912: the dedupe bitmap fits one stage
 constexpr int kQCol = 128;                                  // query columns in TMEM
@@ -395,8 +397,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   sm.xfull = sm.o_done + 2;                      // [buffer][half]
   sm.xfree = sm.xfull + 4;                       // [buffer][half]
   sm.xread1 = sm.xfree + 4;
-  sm.mxready = sm.xread1 + 2;
-  sm.o_free = sm.mxready + 2;
+  sm.mxready = sm.xread1 + 2;                    // [buffer][head quarter]
+  sm.o_free = sm.mxready + 8;
   sm.lready = sm.o_free + 1;
   sm.drain = sm.lready + 1;
   sm.list_free = sm.drain + 1;
@@ -432,15 +434,17 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&sm.s_full[s]), 1);
-      mbar_init(smem_u32(&sm.s_read[s]), 12);     // the 4 exchange and 8 softmax warps have read the score buffer
-      mbar_init(smem_u32(&sm.p_full[s]), 8);      // both softmax groups wrote their P columns
-      mbar_init(smem_u32(&sm.mxready[s]), 8);
+      // softmax warps that own real head rows: all 8, or those of the first two quarters when H = 64
+      const uint32_t n_sm = kHalfHeads ? 4u : 8u;
+      mbar_init(smem_u32(&sm.s_read[s]), 4 + n_sm);  // the exchange and softmax warps have read the score buffer
+      mbar_init(smem_u32(&sm.p_full[s]), n_sm);   // both softmax groups wrote their P columns
+      for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&sm.mxready[4 * s + q]), 2);  // the quarter's two softmax warps
       mbar_init(smem_u32(&sm.o_done[s]), 1);
       for (int h = 0; h < 2; ++h) {
         mbar_init(smem_u32(&sm.xfull[2 * s + h]), 1);  // armed by our softmax; completed by the peer's st.async bytes
         mbar_init(smem_u32(&sm.xfree[2 * s + h]), 4);  // one arrival per peer exchange warp
       }
-      mbar_init(smem_u32(&sm.xread1[s]), 4);      // the group-1 softmax warps have read half 1
+      mbar_init(smem_u32(&sm.xread1[s]), n_sm / 2);  // the group-1 softmax warps have read half 1
     }
     mbar_init(smem_u32(sm.drain), 1);
     mbar_init(smem_u32(sm.list_free), kCopyWarps);  // per row: warps 17-19 are done with its list
@@ -667,7 +671,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
-    const uint32_t dst0 = map_peer(sm.x + (uint32_t)r * 16, peer);  // head r's 16 bytes of each [key/4][head][4] row
+    const uint32_t dst0 = map_peer(sm.x + (uint32_t)(q4 * 4096 + lane * 16), peer);  // head r's 16 bytes of each key/4 row
     const bool real = r < p.H;
     const bool act = !kHalfHeads || q4 < 2;        // warp-uniform: this warp's head rows exist
     // Query of row i into TMEM: the CTA's 256 value-side columns of head r as bf16 pairs in
@@ -741,7 +745,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&sm.s_read[sb]));
           if (q4 == 1 && lane == 0) TRACE(3, gc);
-          // [key/4][head][4 keys]: each store writes 4 keys of head r, the warp 512 contiguous
+          // each store writes 4 keys of head r, the warp 512 contiguous
           // bytes; each store completes its bytes on the peer's barrier of that half (no round trip
           // here).  Half 1 first: the peer returns it as soon as its softmax has read it, half 0
           // only after its P.V (P overwrites half 0).
@@ -749,11 +753,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           if (!(ok = wait_cluster(smem_u32(&sm.xfree[2 * sb + 1]), use ^ 1u, p.status, abort_flag))) break;
           const uint32_t xbar1 = map_peer(smem_u32(&sm.xfull[2 * sb + 1]), peer);
 #pragma unroll
-          for (int c = 32; c < kChunk; c += 4) st_async_v4(dst + c * 512, &v[c], xbar1);
+          for (int c = 32; c < kChunk; c += 4) st_async_v4(dst + 16384 + (c - 32) * 128, &v[c], xbar1);
           if (!(ok = wait_cluster(smem_u32(&sm.xfree[2 * sb]), use ^ 1u, p.status, abort_flag))) break;
           const uint32_t xbar0 = map_peer(smem_u32(&sm.xfull[2 * sb]), peer);
 #pragma unroll
-          for (int c = 0; c < 32; c += 4) st_async_v4(dst + c * 512, &v[c], xbar0);
+          for (int c = 0; c < 32; c += 4) st_async_v4(dst + c * 128, &v[c], xbar0);
         } else {
           // head rows >= H: nothing to read or send
           __syncwarp();
@@ -834,7 +838,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const bool lead = g == 0 && q4 == 0 && lane == 0;
     const bool real = r < p.H;
     const bool act = !kHalfHeads || q4 < 2;         // warp-uniform: this warp's head rows exist
-    const float4* xcol = reinterpret_cast<const float4*>(gb + (sm.x - base)) + r;  // head r of [key/4][head][4]
+    // head r's 4-key groups in the exchange tile: quarter q4, lane
+    const float4* xcol = reinterpret_cast<const float4*>(gb + (sm.x - base)) + q4 * 256 + lane;
     long long gc = 0;
     bool ok = true;
     // the epilogue of a row runs after the next row's query load, so it overlaps that row's first q.k
@@ -900,21 +905,22 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         }
         continue;
       }
+      if (!act) {
+        // head rows >= H (H = 64): no per-chunk work and no per-chunk barrier (nothing would keep
+        // these warps from running chunks ahead); only the row's epilogue barriers count them
+        gc += nch;
+        pending = true;
+        p_row = row;
+        p_last = gc - 1;
+        p_mref = 0.f;
+        p_lsum = 0.f;
+        continue;
+      }
       float m_ref = -INFINITY, l_sum = 0.f;
       for (int j = 0; ok && j < nch; ++j, ++gc) {
         const int sb = (int)(gc & 1);
         const uint32_t use = (uint32_t)((gc >> 1) & 1);
         if (!(ok = mbar_wait(smem_u32(&sm.s_full[sb]), use, p.status, abort_flag))) break;
-        if (!act) {
-          // head rows >= H (H = 64): keep every barrier's count, compute nothing
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&sm.s_read[sb]));
-          if (lane == 0 && g == 1) mbar_arrive(smem_u32(&sm.xread1[sb]));
-          if (lane == 0) mbar_arrive(smem_u32(&sm.mxready[sb]));
-          if (!(ok = mbar_wait(smem_u32(&sm.mxready[sb]), use, p.status, abort_flag))) break;
-          if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[sb]));
-          continue;
-        }
         tc_fence_after();
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + lane_addr + sb * kChunk + 32 * g, v);
@@ -930,12 +936,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           if (g == 0) TRACE(6, gc);
           mbar_arrive_expect_tx(smem_u32(&sm.xfull[2 * sb + g]), 32u * p.H * 4u);  // arm the next use (H rows)
         }
-        const float4* xr = xcol + sb * (kXBytes / 16) + 8 * g * 128;
+        const float4* xr = xcol + sb * (kXBytes / 16) + g * 1024;
         const int valid = n - j * kChunk - 32 * g;
         float mx = -INFINITY;
 #pragma unroll
         for (int c = 0; c < 32; c += 4) {
-          const float4 x4 = xr[(c / 4) * 128];
+          const float4 x4 = xr[(c / 4) * 32];
           const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
@@ -948,13 +954,14 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&sm.xread1[sb]));   // half 1 may go back to the peer
         }
-        // row maximum over both halves of the chunk (once both groups pass this barrier, every
-        // fp32 value of exchange tile sb has been read, and P may overwrite its first half)
+        // row maximum over both halves of the chunk, agreed by the two warps of this head quarter;
+        // once both pass this barrier the quarter's half-0 scores have been read, and its P rows,
+        // which occupy exactly those bytes, may be written
         float* mxb = sm.mx + sb * 256;
         mxb[g * 128 + r] = mx;
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&sm.mxready[sb]));
-        if (!(ok = mbar_wait(smem_u32(&sm.mxready[sb]), use, p.status, abort_flag))) break;
+        if (lane == 0) mbar_arrive(smem_u32(&sm.mxready[4 * sb + q4]));
+        if (!(ok = mbar_wait(smem_u32(&sm.mxready[4 * sb + q4]), use, p.status, abort_flag))) break;
         mx = fmaxf(mx, mxb[(1 - g) * 128 + r]);
         if (lead) TRACE(9, gc);
         // move the reference maximum only when it grows by more than 2^8 (both groups agree)
@@ -993,6 +1000,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 #pragma unroll
           for (int k = 0; k < 4; ++k) st_shared_v4(prow + ((uint32_t)((4 * g + k) ^ (r & 7)) << 4), &pk[4 * k]);
         }
+        if (lead) TRACE(15, gc);
         fence_proxy_async_smem();                   // visible to the tensor core's operand reads
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[sb]));
