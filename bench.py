@@ -649,8 +649,8 @@ def kpool_extra(peaks, flush, stream, cpu_s=0.0):
                                                t["kv_start"], t["kv_len"], bufs.pooled, bufs.n_pools),
         "index": lambda: dsa.index_scores(di, t["q_idx"], bufs.pooled, t["w"], wl.idx_scale, t["q_pos"],
                                           t["kv_start"], t["kv_len"], bufs.pool_scores),
-        "topk": lambda: dsa.topk(di, bufs.pool_scores, t["q_pos"], t["kv_start"], t["kv_len"], di.top_k,
-                                 bufs.pool_idx),
+        "topk": lambda: dsa.topk_set(di, bufs.pool_scores, t["q_pos"], t["kv_start"], t["kv_len"], di.top_k,
+                                     bufs.pool_idx),
         "expand": lambda: dsa.expand_selection(dp, bufs.pool_idx, t["q_pos"], t["kv_start"], t["kv_len"],
                                                bufs.n_pools, bufs.tok_idx),
         "absorb_q": lambda: dsa.absorb_q(da, t["q_nope"], dq, t["w_uk"], L, bufs.q_lat),
@@ -659,6 +659,12 @@ def kpool_extra(peaks, flush, stream, cpu_s=0.0):
         "absorb_out": lambda: dsa.absorb_out(da, bufs.o_lat, L, t["w_uv"], dv, bufs.out),
     }
     st = {k: statistics.median(time_steps(f, 3, 1, flush, stream)) for k, f in calls.items()}
+    # the ranked selection of the same pools (dsa_topk), which the layer does not need
+    ranked = torch.empty_like(bufs.pool_idx)
+    topk_ranked = statistics.median(time_steps(
+        lambda: dsa.topk(di, bufs.pool_scores, t["q_pos"], t["kv_start"], t["kv_len"], di.top_k, ranked),
+        3, 1, flush, stream))
+    del ranked
     index_pairs = int(torch.isfinite(bufs.pool_scores).sum())
     attend_pairs = int((bufs.tok_idx >= 0).sum())
     valid_rows = int((t["q_pos"] >= t["kv_start"].view(-1, 1)).sum())
@@ -670,6 +676,7 @@ def kpool_extra(peaks, flush, stream, cpu_s=0.0):
                        f"select_k={wl.select_k} width={wl.out_width}, NoPE MLA H={H} latent {L}",
            "value": round(B * T / step, 1), "value_valid_rows": round(valid_rows / step, 1), "unit": UNIT,
            "ms_per_step": round(step * 1e3, 3), "stages_us": {k: round(v * 1e6, 1) for k, v in st.items()},
+           "topk_ranked_us": round(topk_ranked * 1e6, 1),
            "roofline_index": roofline_entry("tensor", flop["index"], st["index"], peaks),
            "roofline_attend": roofline_entry("tensor", flop["attend"], st["attend"], peaks),
            "roofline_absorb": roofline_entry("tensor", flop["absorb"], st["absorb_q"] + st["absorb_out"], peaks),

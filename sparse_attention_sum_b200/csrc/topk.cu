@@ -11,8 +11,9 @@
 // keys of the bin that holds the k-th largest become a small candidate set
 // whose low 20 bits are resolved alone (12 + 8 bits).  That gives the exact
 // k-th largest key tau and how many keys equal to tau are still needed.  A
-// crowded bin (many equal scores) falls back to four 8-bit passes over the
-// row (shared atomics aggregated per warp with ballots).  Each warp owns a
+// crowded bin (more keys than the candidate buffer holds, e.g. near-equal
+// scores) resolves the same two digits with one filtered pass over the row
+// each instead.  Each warp owns a
 // contiguous segment of the row, walked 32 keys at a time.  The pass that
 // collects the candidates also counts, per warp, the keys above the bin, and
 // tags each candidate with its warp, so the per-warp counts of keys > tau and
@@ -188,7 +189,7 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
   uint32_t* cand = hist12 + kHist12;                                 // [kCand] candidate keys
   uint8_t* candw = reinterpret_cast<uint8_t*>(cand + kCand);         // [kCand] their warps
   uint32_t* cache = reinterpret_cast<uint32_t*>(candw + kCand);      // [cache_cap]
-  __shared__ uint32_t s_prefix, s_krem, s_bin;
+  __shared__ uint32_t s_krem, s_bin;
   __shared__ int s_ncand;
   __shared__ int s_cgt[BLOCK / 32], s_ceq[BLOCK / 32];
 
@@ -318,32 +319,27 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
     }
     __syncthreads();
   } else {
-    // a crowded bin (e.g. many equal scores): 8-bit digits over the whole row
-    if (threadIdx.x == 0) {
-      s_prefix = 0u;
-      s_krem = (uint32_t)k;
+    // a crowded bin (more than kCand keys share the top 12 bits, e.g. near-equal scores): bits 19..8 of
+    // the bin's keys, then bits 7..0 of the keys under that 24-bit prefix, each one filtered pass over
+    // the row with plain shared atomics (the same digits the candidate path resolves)
+    for (int i = threadIdx.x; i < kHist12; i += BLOCK) hist12[i] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += BLOCK) {
+      const uint32_t key = cached ? cache[i] : score_key(srow[r.lo + i]);
+      if ((key >> 20) == b1) atomicAdd(&hist12[(key >> 8) & 4095u], 1u);
     }
     __syncthreads();
-    uint32_t mask = 0u;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = threadIdx.x; i < 256; i += BLOCK) hist[i] = 0u;
-      __syncthreads();
-      for (int base = (threadIdx.x & ~31); base < n; base += BLOCK) {
-        const int i = base + lane0;
-        int bin = -1;
-        if (i < n) {
-          const uint32_t key = cached ? cache[i] : score_key(srow[r.lo + i]);
-          if ((key & mask) == prefix) bin = (int)((key >> shift) & 255u);
-        }
-        const uint32_t peers = same_digit_lanes(bin);
-        if (bin >= 0 && lane0 == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
-      }
-      __syncthreads();
-      const uint32_t krem = s_krem;
-      find_crossing<BLOCK>(hist, 256, krem, scan, &s_bin, &s_krem);
-      prefix |= s_bin << shift;
-      mask |= 255u << shift;
+    find_crossing<BLOCK>(hist12, kHist12, krem1, scan, &s_bin, &s_krem);
+    const uint32_t p24 = (b1 << 12) | s_bin, krem2 = s_krem;
+    for (int i = threadIdx.x; i < 256; i += BLOCK) hist[i] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += BLOCK) {
+      const uint32_t key = cached ? cache[i] : score_key(srow[r.lo + i]);
+      if ((key >> 8) == p24) atomicAdd(&hist[key & 255u], 1u);
     }
+    __syncthreads();
+    find_crossing<BLOCK>(hist, 256, krem2, scan, &s_bin, &s_krem);
+    prefix = (p24 << 8) | s_bin;
   }
   const uint32_t tau = prefix;
   const int need_eq = (int)s_krem;  // keys equal to tau still to take (lowest indices first)

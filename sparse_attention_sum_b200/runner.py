@@ -5,7 +5,7 @@ is one libdsa call.
 * :func:`dsa_layer`   -- S1-S5: indexer scores, top-k, sparse MLA attend
   (``dsa_layer_forward``).
 * :func:`kpool_layer` -- S6-S8 with S2-S4 over pools: LayerNorm + pooling,
-  pool scores, pool top-k, expand_selection, absorbed NoPE MLA attend.
+  pool scores, pool top-k (as a set, in pool order), expand_selection, absorbed NoPE MLA attend.
 * :func:`dsa_layer_fp8` -- the layer with the FP8 indexer: quantise the queries,
   FP8 scores against a key cache held as e4m3 codes, top-k set, sparse attend.
 * :func:`index_share_stack` -- IndexShare over a stack of layers: the layers
@@ -177,7 +177,9 @@ def kpool_layer(dims: Dict[str, Dims], q_idx, k_raw, gate, ln_w, ln_b, ln_eps, w
                 stream=stream)
     index_scores(di, q_idx, bufs.pooled, w, idx_scale, q_pos, kv_start, kv_len, bufs.pool_scores,
                  stream=stream)
-    topk(di, bufs.pool_scores, q_pos, kv_start, kv_len, di.top_k, bufs.pool_idx, stream=stream)
+    # the attention reads the expanded tokens as a set, so the pools are selected as one (key order, as the
+    # token layer lists its selection); dsa_topk ranks the same pools
+    topk_set(di, bufs.pool_scores, q_pos, kv_start, kv_len, di.top_k, bufs.pool_idx, stream=stream)
     expand_selection(dp, bufs.pool_idx, q_pos, kv_start, kv_len, bufs.n_pools, bufs.tok_idx,
                      stream=stream)
     L = da.kd

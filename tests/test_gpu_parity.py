@@ -474,7 +474,8 @@ def _kpool_check(wl, bufs, rows):
             if cand.size else np.zeros(0)
         if cand.size:
             assert np.abs(pool_scores[b, tt, cand] - ref_sc).max() <= 2e-5 * max(1, np.abs(ref_sc).max())
-        assert pool_idx[b, tt].tolist() == O.topk_row(cand, pool_scores[b, tt, cand], wl.select_k).tolist()
+        # the layer selects its pools as a set, listed in pool order (dsa_topk_set)
+        assert pool_idx[b, tt].tolist() == key_order(O.topk_row(cand, pool_scores[b, tt, cand], wl.select_k).tolist())
         check_selection_in_band(pool_idx[b, tt], cand, ref_sc, wl.select_k, f"kpool pools {(b, tt)}")
         want_tok = O.expand_selection(pool_idx[b, tt], p, f, L, kp, npools[b], wl.out_width)
         assert tok_idx[b, tt].tolist() == want_tok.tolist()
