@@ -59,6 +59,8 @@ namespace dsa {
 // Optional per-chunk timeline of the first cluster (build with -DDSA_TRACE):
 // g_attend_trace[cta rank][event][chunk] = %globaltimer.
 __device__ unsigned long long g_attend_trace[2][16][512];
+// g_attend_span[cta][0] = entry, [1] = exit (%globaltimer), every CTA
+__device__ unsigned long long g_attend_span[1024][2];
 #define TRACE(ev, j)                                                                             \
   do {                                                                                           \
     if (blockIdx.x < 2 && (j) < 512) g_attend_trace[blockIdx.x & 1][ev][(j)] = sm100::globaltimer(); \
@@ -368,6 +370,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                  const __grid_constant__ CUtensorMap map_rope, AttTcParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ int s_misc[5];
+#ifdef DSA_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < 1024) g_attend_span[blockIdx.x][0] = sm100::globaltimer();
+#endif
   __shared__ int s_wcount[4];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -1017,6 +1022,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // no remote access to a CTA that has exited
+#ifdef DSA_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < 1024) g_attend_span[blockIdx.x][1] = sm100::globaltimer();
+#endif
   if (warp == 4) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -1135,6 +1143,9 @@ cudaError_t launch_attend_tc(const dsa_dims& d, const void* q, const void* k, in
 #ifdef DSA_TRACE
 extern "C" int dsa_trace_read(unsigned long long* host) {
   return (int)cudaMemcpyFromSymbol(host, dsa::g_attend_trace, sizeof(dsa::g_attend_trace));
+}
+extern "C" int dsa_trace_span(unsigned long long* host) {
+  return (int)cudaMemcpyFromSymbol(host, dsa::g_attend_span, sizeof(dsa::g_attend_span));
 }
 extern "C" int dsa_trace_clear() {
   static unsigned long long zero[2 * 16 * 512];

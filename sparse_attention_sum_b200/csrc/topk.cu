@@ -7,14 +7,15 @@
 //
 // One block per row.  Scores become order-preserving uint32 keys (signed
 // zeros merged) and are cached in shared memory when the visible range fits.
-// One pass counts the top 12 bits of every key (plain shared atomics); the
+// One pass (16-byte loads) counts the top 12 bits of every key (plain shared atomics); the
 // keys of the bin that holds the k-th largest become a small candidate set
 // whose low 20 bits are resolved alone (12 + 8 bits).  That gives the exact
 // k-th largest key tau and how many keys equal to tau are still needed.  A
 // crowded bin (more keys than the candidate buffer holds, e.g. near-equal
 // scores) resolves the same two digits with one filtered pass over the row
 // each instead.  Each warp owns a
-// contiguous segment of the row, walked 32 keys at a time.  The pass that
+// contiguous segment of the row, walked 128 keys at a time (four per lane, their
+// loads and ballots independent).  The pass that
 // collects the candidates also counts, per warp, the keys above the bin, and
 // tags each candidate with its warp, so the per-warp counts of keys > tau and
 // == tau come from the candidates without another pass over the row (the
@@ -32,6 +33,21 @@
 #include "dsa_internal.h"
 
 namespace dsa {
+
+#ifdef DSA_TRACE
+// Optional phase timeline of a few rows (build with -DDSA_TRACE): g_topk_trace[row][phase] = %globaltimer.
+__device__ unsigned long long g_topk_trace[8][8];
+#define TOPK_TRACE(ph)                                                                         \
+  do {                                                                                         \
+    if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.x < 8) {                               \
+      unsigned long long t_;                                                                   \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                   \
+      g_topk_trace[blockIdx.x][ph] = t_;                                                       \
+    }                                                                                          \
+  } while (0)
+#else
+#define TOPK_TRACE(ph) ((void)0)
+#endif
 
 constexpr int kTopkCacheMax = 40960;  // keys cached in shared memory (160 KB)
 constexpr int kHist12 = 4096;         // first-pass histogram: the top 12 bits of a key
@@ -234,33 +250,63 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
   // ---- threshold: tau = the k-th largest key.  One pass over the row (filling the cache)
   // counts the top 12 bits; the keys of the bin holding the k-th largest then become a small
   // candidate set, and the low 20 bits are resolved over it alone (12 + 8 bits).
-  const int lane0 = threadIdx.x & 31;
+  TOPK_TRACE(0);
   for (int i = threadIdx.x; i < kHist12; i += BLOCK) hist12[i] = 0u;
   if (threadIdx.x == 0) s_ncand = 0;
   __syncthreads();
-  constexpr int kU = 8;                 // independent loads in flight per thread
-  for (int base = (threadIdx.x & ~31); base < n; base += BLOCK * kU) {
-    float v[kU];
+  {
+    // the row as 16-byte vectors (eight in flight per thread) between a scalar head and tail
+    auto one = [&](int i) {
+      const uint32_t key = score_key(__ldg(srow + r.lo + i));
+      if (cached) cache[i] = key;
+      atomicAdd(&hist12[key >> 20], 1u);
+    };
+    const int head = min(n, (int)(((16u - ((uint32_t)(uintptr_t)(srow + r.lo) & 15u)) & 15u) >> 2));
+    const int nv = (n - head) >> 2;
+    const float4* s4 = reinterpret_cast<const float4*>(srow + r.lo + head);
+    if ((int)threadIdx.x < head) one(threadIdx.x);
+    constexpr int kV = BLOCK >= 1024 ? 8 : 4;   // 16-byte loads in flight per thread (rows of n_kv <= 8192 take 512)
+    for (int base = threadIdx.x; base < nv; base += BLOCK * kV) {
+      float4 v[kV];
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int i = base + u * BLOCK + lane0;
-      v[u] = i < n ? __ldg(srow + r.lo + i) : 0.f;
-    }
+      for (int u = 0; u < kV; ++u) {
+        const int j = base + u * BLOCK;
+        v[u] = j < nv ? __ldg(s4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int i = base + u * BLOCK + lane0;
-      if (i < n) {
-        const uint32_t key = score_key(v[u]);
-        if (cached) cache[i] = key;
-        atomicAdd(&hist12[key >> 20], 1u);
+      for (int u = 0; u < kV; ++u) {
+        const int j = base + u * BLOCK;
+        if (j < nv) {
+          const int i = head + 4 * j;
+          const uint32_t k0 = score_key(v[u].x), k1 = score_key(v[u].y), k2 = score_key(v[u].z),
+                         k3 = score_key(v[u].w);
+          if (cached) {
+            if (head == 0) {
+              *reinterpret_cast<uint4*>(cache + i) = make_uint4(k0, k1, k2, k3);
+            } else {
+              cache[i] = k0;
+              cache[i + 1] = k1;
+              cache[i + 2] = k2;
+              cache[i + 3] = k3;
+            }
+          }
+          atomicAdd(&hist12[k0 >> 20], 1u);
+          atomicAdd(&hist12[k1 >> 20], 1u);
+          atomicAdd(&hist12[k2 >> 20], 1u);
+          atomicAdd(&hist12[k3 >> 20], 1u);
+        }
       }
     }
+    const int t0 = head + 4 * nv;
+    if ((int)threadIdx.x < n - t0) one(t0 + threadIdx.x);
   }
   __syncthreads();
+  TOPK_TRACE(1);
   find_crossing<BLOCK>(hist12, kHist12, (uint32_t)k, scan, &s_bin, &s_krem);
   const uint32_t b1 = s_bin, krem1 = s_krem;
+  TOPK_TRACE(2);
   const uint32_t nb1 = hist12[b1];
-  // each warp owns a contiguous segment of the row, walked 32 keys at a time (the output order
+  // each warp owns a contiguous segment of the row, walked 128 keys at a time (the output order
   // of equal keys is their index order)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   constexpr int NW = BLOCK / 32;
@@ -276,27 +322,40 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
       s_cgt[threadIdx.x] = 0;
       s_ceq[threadIdx.x] = 0;
     }
-    for (int b0 = w0; b0 < w1; b0 += 32) {
-      const int i = b0 + lane;
-      uint32_t key = 0u;
-      bool in = false;
-      if (i < w1) {
-        key = cached ? cache[i] : score_key(srow[r.lo + i]);
-        in = (key >> 20) == b1;
-        gt12 += (key >> 20) > b1;
+    // four keys per lane per step (independent loads and ballots); the order of the candidates
+    // does not matter, each carries its warp
+    for (int b0 = w0; b0 < w1; b0 += 128) {
+      uint32_t key[4], m[4];
+      bool in[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = b0 + 32 * q + lane;
+        key[q] = i < w1 ? (cached ? cache[i] : score_key(srow[r.lo + i])) : 0u;
+        in[q] = i < w1 && (key[q] >> 20) == b1;
+        gt12 += (i < w1 && (key[q] >> 20) > b1) ? 1 : 0;
       }
-      const uint32_t m = __ballot_sync(0xffffffffu, in);
-      int slot = 0;
-      if (lane == 0 && m) slot = atomicAdd(&s_ncand, __popc(m));
-      slot = __shfl_sync(0xffffffffu, slot, 0);
-      if (in) {
-        const int c = slot + __popc(m & ((1u << lane) - 1u));
-        cand[c] = key;
-        candw[c] = (uint8_t)warp;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) m[q] = __ballot_sync(0xffffffffu, in[q]);
+      const int tot = __popc(m[0]) + __popc(m[1]) + __popc(m[2]) + __popc(m[3]);
+      if (tot) {
+        int slot = 0;
+        if (lane == 0) slot = atomicAdd(&s_ncand, tot);
+        slot = __shfl_sync(0xffffffffu, slot, 0);
+        const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (in[q]) {
+            const int c = slot + __popc(m[q] & lt);
+            cand[c] = key[q];
+            candw[c] = (uint8_t)warp;
+          }
+          slot += __popc(m[q]);
+        }
       }
     }
     gt12 = __reduce_add_sync(0xffffffffu, gt12);
     __syncthreads();
+    TOPK_TRACE(3);
     // bits 19..8 of the candidates
     for (int i = threadIdx.x; i < kHist12; i += BLOCK) hist12[i] = 0u;
     __syncthreads();
@@ -341,6 +400,11 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
     find_crossing<BLOCK>(hist, 256, krem2, scan, &s_bin, &s_krem);
     prefix = (p24 << 8) | s_bin;
   }
+  TOPK_TRACE(4);
+#ifdef DSA_TRACE
+  if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.x < 8)
+    g_topk_trace[blockIdx.x][7] = ((unsigned long long)few << 32) | nb1;
+#endif
   const uint32_t tau = prefix;
   const int need_eq = (int)s_krem;  // keys equal to tau still to take (lowest indices first)
   const int n_gt = k - need_eq;
@@ -360,6 +424,7 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
     c_gt = __reduce_add_sync(0xffffffffu, c_gt);
     c_eq = __reduce_add_sync(0xffffffffu, c_eq);
   }
+  TOPK_TRACE(5);
   int tot;
   int gt_base = block_exclusive_scan<BLOCK>(lane == 0 ? c_gt : 0, scan, tot);
   int eq_base = block_exclusive_scan<BLOCK>(lane == 0 ? c_eq : 0, scan, tot);
@@ -367,25 +432,37 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
   eq_base = __shfl_sync(0xffffffffu, eq_base, 0);
   const uint32_t lt_mask = (1u << lane) - 1u;
   if constexpr (!RANKED) {
-    // ascending key order: key i goes to (#gt before i) + min(#eq before i, need_eq)
-    for (int b0 = w0; b0 < w1; b0 += 32) {
-      const int i = b0 + lane;
-      uint32_t key = 0u;
-      if (i < w1) key = cached ? cache[i] : score_key(srow[r.lo + i]);
-      const bool is_gt = i < w1 && key > tau;
-      const bool is_eq = i < w1 && key == tau;
-      const uint32_t m_gt = __ballot_sync(0xffffffffu, is_gt);
-      const uint32_t m_eq = __ballot_sync(0xffffffffu, is_eq);
-      const int gt_before = gt_base + __popc(m_gt & lt_mask);
-      const int eq_before = eq_base + __popc(m_eq & lt_mask);
-      if (is_gt || (is_eq && eq_before < need_eq)) {
-        const int pos = gt_before + min(eq_before, need_eq);
-        orow[pos] = r.lo + i;
-        if (vrow) vrow[pos] = key_score(key);
+    // ascending key order: key i goes to (#gt before i) + min(#eq before i, need_eq); four keys
+    // per lane per step, their loads and ballots independent
+    for (int b0 = w0; b0 < w1; b0 += 128) {
+      uint32_t key[4], m_gt[4], m_eq[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = b0 + 32 * q + lane;
+        key[q] = i < w1 ? (cached ? cache[i] : score_key(srow[r.lo + i])) : 0u;
       }
-      gt_base += __popc(m_gt);
-      eq_base += __popc(m_eq);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = b0 + 32 * q + lane;
+        m_gt[q] = __ballot_sync(0xffffffffu, i < w1 && key[q] > tau);
+        m_eq[q] = __ballot_sync(0xffffffffu, i < w1 && key[q] == tau);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = b0 + 32 * q + lane;
+        const bool is_gt = (m_gt[q] >> lane) & 1u, is_eq = (m_eq[q] >> lane) & 1u;
+        const int gt_before = gt_base + __popc(m_gt[q] & lt_mask);
+        const int eq_before = eq_base + __popc(m_eq[q] & lt_mask);
+        if (is_gt || (is_eq && eq_before < need_eq)) {
+          const int pos = gt_before + min(eq_before, need_eq);
+          orow[pos] = r.lo + i;
+          if (vrow) vrow[pos] = key_score(key[q]);
+        }
+        gt_base += __popc(m_gt[q]);
+        eq_base += __popc(m_eq[q]);
+      }
     }
+    TOPK_TRACE(6);
   } else {
     for (int b0 = w0; b0 < w1; b0 += 32) {
       const int i = b0 + lane;
@@ -444,3 +521,9 @@ cudaError_t launch_topk(const dsa_dims& d, const float* scores, const int32_t* q
 }
 
 }  // namespace dsa
+
+#ifdef DSA_TRACE
+extern "C" int dsa_topk_trace_read(unsigned long long* host) {
+  return (int)cudaMemcpyFromSymbol(host, dsa::g_topk_trace, sizeof(dsa::g_topk_trace));
+}
+#endif
