@@ -20,7 +20,11 @@
 // and summed (fp32 addition is commutative, so both CTAs see bit-identical
 // scores and take identical online-softmax decisions).  The exchange uses
 // st.async, which completes the peer's barrier by byte count, so the sender
-// never waits for a round trip.
+// never waits for a round trip.  A tile travels in two 16 KB halves (keys 0-31
+// and 32-63), each with its own barriers, laid out by head quarter
+// ([half][quarter][key/4][32 heads][4 keys] fp32): the first half also holds the
+// chunk's P (below) and returns to the peer after P.V, the second returns as
+// soon as the softmax has read it.
 //
 // Tensor memory (512 columns): score buffers 0-63 and 64-127, the CTA's four
 // value-side query blocks 128-255 as the A operand of q.k (two bf16 per
@@ -37,7 +41,10 @@
 //
 // Warp roles per CTA: warps 0-3 and 13-16 run the softmax and the epilogue (one
 // head row per thread, TMEM lanes 0-127; the two groups take the two halves of
-// every chunk's keys and of O); warps 9-12 load the query columns into TMEM,
+// every chunk's keys and of O, and the two warps of a head quarter agree on its
+// row maxima through their own barrier, after which the quarter's P rows
+// overwrite exactly its consumed half-0 scores; with H = 64 the warps of the two
+// padding quarters take part in no per-chunk barrier); warps 9-12 load the query columns into TMEM,
 // read the same score rows and push them to the peer (buffer reuse is
 // acknowledged by the peer); warp 4 issues tcgen05.mma from a polling scheduler
 // (and loads the CTA's rope query columns by TMA); warps 5-8 stage and
