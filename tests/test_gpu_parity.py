@@ -404,9 +404,11 @@ def test_long_cache_layer_stays_on_tensor_cores():
 def test_long_cache_attend_set_semantics(H, kd):
     """dsa_sparse_attend on the tensor cores over a 70000-row latent with index rows that mix keys
     above and below 65536, duplicates (the first-occurrence compaction), INVALID and out-of-range
-    entries, against the oracle's set-semantics attention."""
+    entries, against the oracle's set-semantics attention; rows 100 and T-1 run as a cluster's second
+    or third row."""
     rng = np.random.default_rng(H)
-    B, T, S, W = 1, 130 if H == 64 else 6, 70000, 2048
+    # more rows than the kernel's 74 persistent clusters, so clusters run a second and a third row
+    B, T, S, W = 1, 130 if H == 64 else 150, 70000, 2048
     q = torch.tensor(rng.standard_normal((B, T, H, kd)), dtype=torch.bfloat16)
     lat = torch.tensor(rng.standard_normal((B, S, kd)) * 0.5, dtype=torch.bfloat16)
     idx = rng.integers(0, S, size=(B, T, W)).astype(np.int32)
