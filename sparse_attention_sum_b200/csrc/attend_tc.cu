@@ -478,11 +478,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     if (lane == 0) tma_prefetch_desc(&map_kv);
     long long gc = 0;                                    // global chunk counter
     bool ok = true;
+    // a row's index entries are read into registers while the previous row's gathers are issued
+    RowKeys rk;
+    if (my_rows > 0) load_row(p, p.idx + row_of(0) * p.width, rk);
     for (int i = 0; i < my_rows; ++i) {
       const size_t row = row_of(i);
       const int32_t* irow = p.idx + row * p.width;
-      RowKeys rk;
-      load_row(p, irow, rk);                             // in flight while the waits below run
       // every consumer has read the previous row's length before this row's is published, and the
       // copy warps have issued the previous row's copies (they read its list)
       const int s0 = (int)(gc % kStages);
@@ -522,11 +523,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       named_sync(1, kProducerThreads);
       if (w == 0 && lane == 0) {
         sm.n_list[i & 1] = n;
-        TRACE(8, 1);
+        if (i < 100) TRACE(8, 402 + i);
         mbar_arrive(smem_u32(sm.list_ready));
       }
       const int nch = (n + kChunk - 1) / kChunk;
       const int rowbase = (int)(row / p.T) * p.S;        // latent row of key 0 of this query's sequence
+      if (i + 1 < my_rows) load_row(p, p.idx + row_of(i + 1) * p.width, rk);  // the next row's entries
       for (int j = 0; j < nch; ++j, ++gc) {
         const int s = (int)(gc % kStages);
         if (!(ok = mbar_wait(smem_u32(&sm.kv_empty[s]), (uint32_t)(((gc / kStages) & 1) ^ 1), p.status, abort_flag)))
@@ -691,27 +693,32 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     // q.k of earlier rows is complete (these warps have read all their scores).
     auto load_q = [&](int i) {
       const size_t qrow = row_of(i);
+      if (warp == 9 && lane == 0 && i < 200) TRACE(8, 2 + 2 * i);
       if (warp == 9 && lane == 0 && rope) {
         mbar_arrive_expect_tx(smem_u32(sm.qrope_full), kQRopeBytes);
         tma_load_2d(sm.qrope, &map_q, smem_u32(sm.qrope_full), rope_col, (int)(qrow * p.H));
       }
       const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (qrow * p.H + (real ? r : 0)) * p.kd + rank * 256);
+      // two batches of sixteen 16-byte loads (64 columns each): the rows' lines are in L2 (prefetched
+      // during the previous row), so each batch costs one L2 round trip
 #pragma unroll 1
-      for (int c0 = 0; act && c0 < 128; c0 += 32) {      // 32 columns = 64 bf16 = 8 x 16 bytes
-        uint32_t qv[32];
+      for (int c0 = 0; act && c0 < 128; c0 += 64) {      // 64 columns = 128 bf16 = 16 x 16 bytes
+        uint32_t qv[64];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < 16; ++k) {
           const uint4 u = real ? qsrc[c0 / 4 + k] : make_uint4(0, 0, 0, 0);
           qv[4 * k] = u.x;
           qv[4 * k + 1] = u.y;
           qv[4 * k + 2] = u.z;
           qv[4 * k + 3] = u.w;
         }
-        tmem_st_32x32b_x32(tmem + lane_addr + kQCol + c0, qv);
+        tmem_st_32x32b_x32(tmem + lane_addr + kQCol + c0, *reinterpret_cast<const uint32_t(*)[32]>(&qv[0]));
+        tmem_st_32x32b_x32(tmem + lane_addr + kQCol + c0 + 32, *reinterpret_cast<const uint32_t(*)[32]>(&qv[32]));
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
+      if (warp == 9 && lane == 0 && i < 200) TRACE(8, 3 + 2 * i);
       if (lane == 0) mbar_arrive(smem_u32(sm.qfull));
       // the following row's query lines are pulled into L2 meanwhile
       if (i + 1 < my_rows && real) {
