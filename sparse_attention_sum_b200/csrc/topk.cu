@@ -432,6 +432,32 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
   eq_base = __shfl_sync(0xffffffffu, eq_base, 0);
   const uint32_t lt_mask = (1u << lane) - 1u;
   if constexpr (!RANKED) {
+    if (c_eq == 0) {
+      // no key of this warp equals tau (the usual case): a key is taken iff it is above tau, after
+      // every taken key of the earlier warps; one ballot per four keys
+      int base = gt_base + min(eq_base, need_eq);
+      for (int b0 = w0; b0 < w1; b0 += 128) {
+        uint32_t key[4], m[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int i = b0 + 32 * q + lane;
+          key[q] = i < w1 ? (cached ? cache[i] : score_key(srow[r.lo + i])) : 0u;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) m[q] = __ballot_sync(0xffffffffu, b0 + 32 * q + lane < w1 && key[q] > tau);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if ((m[q] >> lane) & 1u) {
+            const int pos = base + __popc(m[q] & lt_mask);
+            orow[pos] = r.lo + b0 + 32 * q + lane;
+            if (vrow) vrow[pos] = key_score(key[q]);
+          }
+          base += __popc(m[q]);
+        }
+      }
+      TOPK_TRACE(6);
+      return;
+    }
     // ascending key order: key i goes to (#gt before i) + min(#eq before i, need_eq); four keys
     // per lane per step, their loads and ballots independent
     for (int b0 = w0; b0 < w1; b0 += 128) {
