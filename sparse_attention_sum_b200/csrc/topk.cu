@@ -5,7 +5,8 @@
 // glm5next_dsa_ref topk_pools; ik_llama.cpp #2045 ggml_top_k(min(top_k,
 // n_tokens))).
 //
-// One block per row.  Scores become order-preserving uint32 keys (signed
+// One block per row: 1024 threads for rows of more than 8192 keys, 512 up to 8192, and 256 (six
+// blocks per SM, so that short rows overlap) up to 4096.  Scores become order-preserving uint32 keys (signed
 // zeros merged) and are cached in shared memory when the visible range fits.
 // One pass (16-byte loads) counts the top 12 bits of every key (plain shared atomics); the
 // keys of the bin that holds the k-th largest become a small candidate set
@@ -51,7 +52,7 @@ __device__ unsigned long long g_topk_trace[8][8];
 
 constexpr int kTopkCacheMax = 40960;  // keys cached in shared memory (160 KB)
 constexpr int kHist12 = 4096;         // first-pass histogram: the top 12 bits of a key
-constexpr int kCand = 4096;           // keys of the threshold's 12-bit bin resolved on their own
+constexpr int kCand = 4096;           // keys of the threshold's 12-bit bin resolved on their own (at most)
 
 // Block-wide exclusive scan of one int per thread; returns the block total.
 template <int BLOCK>
@@ -101,27 +102,53 @@ __device__ __forceinline__ uint32_t same_digit_lanes(int d) {
 template <int BLOCK>
 __device__ void find_crossing(const uint32_t* hist, int nbins, uint32_t kneed, int* scan, uint32_t* s_bin,
                               uint32_t* s_krem) {
-  const int per = nbins >= BLOCK ? nbins / BLOCK : 1;    // digits per thread (<= 8)
+  const int per = nbins >= BLOCK ? nbins / BLOCK : 1;    // digits per thread (<= 8 from 512 threads up)
   const int owners = nbins / per;
-  uint32_t cnt[8];
-  uint32_t lsum = 0;
-#pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    cnt[u] = (u < per && (int)threadIdx.x < owners) ? hist[nbins - 1 - (per * (int)threadIdx.x + u)] : 0u;
-    lsum += cnt[u];
-  }
-  int total;
-  const uint32_t excl = (uint32_t)block_exclusive_scan<BLOCK>((int)lsum, scan, total);
-  if ((int)threadIdx.x < owners && excl < kneed && excl + lsum >= kneed) {
-    uint32_t c = excl;
+  const int top = nbins - 1 - per * (int)threadIdx.x;   // this thread's digits: top, top - 1, ..., top - per + 1
+  const bool own = (int)threadIdx.x < owners;
+  if constexpr (BLOCK >= 512) {
+    // at most eight digits: held in registers between the scan and the walk
+    uint32_t cnt[8];
+    uint32_t lsum = 0;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      if (u < per && c + cnt[u] >= kneed) {
-        *s_bin = (uint32_t)(nbins - 1 - (per * (int)threadIdx.x + u));
-        *s_krem = kneed - c;
-        break;
+      cnt[u] = (u < per && own) ? hist[top - u] : 0u;
+      lsum += cnt[u];
+    }
+    int total;
+    const uint32_t excl = (uint32_t)block_exclusive_scan<BLOCK>((int)lsum, scan, total);
+    if (own && excl < kneed && excl + lsum >= kneed) {
+      uint32_t c = excl;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (u < per && c + cnt[u] >= kneed) {
+          *s_bin = (uint32_t)(top - u);
+          *s_krem = kneed - c;
+          break;
+        }
+        c += cnt[u];
       }
-      c += cnt[u];
+    }
+  } else {
+    // more digits per thread: summed first, walked again by the one thread holding the crossing
+    uint32_t lsum = 0;
+    if (own) {
+#pragma unroll 8
+      for (int u = 0; u < per; ++u) lsum += hist[top - u];
+    }
+    int total;
+    const uint32_t excl = (uint32_t)block_exclusive_scan<BLOCK>((int)lsum, scan, total);
+    if (own && excl < kneed && excl + lsum >= kneed) {
+      uint32_t c = excl;
+      for (int u = 0; u < per; ++u) {
+        const uint32_t cnt = hist[top - u];
+        if (c + cnt >= kneed) {
+          *s_bin = (uint32_t)(top - u);
+          *s_krem = kneed - c;
+          break;
+        }
+        c += cnt;
+      }
     }
   }
   __syncthreads();
@@ -190,11 +217,12 @@ __device__ void radix_sort_desc(uint64_t* a, uint64_t* b, uint32_t* hist, int* s
 }
 
 template <int BLOCK, bool RANKED>
-__global__ void __launch_bounds__(BLOCK, BLOCK >= 1024 ? 1 : 3)
+__global__ void __launch_bounds__(BLOCK, BLOCK >= 1024 ? 1 : (BLOCK >= 512 ? 3 : 6))
 topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restrict__ q_pos,
             const int32_t* __restrict__ kv_start, const int32_t* __restrict__ kv_len, int k,
-            int cache_cap, int32_t* __restrict__ idx_out, float* __restrict__ vals_out) {
+            int cache_cap, int cand_cap_arg, int32_t* __restrict__ idx_out, float* __restrict__ vals_out) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int cand_cap = BLOCK >= 512 ? kCand : cand_cap_arg;         // a compile-time size from 512 threads up
   const int ksel = RANKED ? k : 0;                                   // the unranked variant keeps no pairs
   uint64_t* sel = reinterpret_cast<uint64_t*>(smem_raw);            // [k]   selected (key, index)
   uint64_t* tmp = sel + ksel;                                        // [k]   sort ping-pong
@@ -202,9 +230,9 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
   uint32_t* hist = rhist + (RANKED ? (BLOCK / 32) * 256 : 0);        // [256]
   int* scan = reinterpret_cast<int*>(hist + 256);                    // [64]
   uint32_t* hist12 = reinterpret_cast<uint32_t*>(scan + 64);         // [kHist12]
-  uint32_t* cand = hist12 + kHist12;                                 // [kCand] candidate keys
-  uint8_t* candw = reinterpret_cast<uint8_t*>(cand + kCand);         // [kCand] their warps
-  uint32_t* cache = reinterpret_cast<uint32_t*>(candw + kCand);      // [cache_cap]
+  uint32_t* cand = hist12 + kHist12;                                 // [cand_cap] candidate keys
+  uint8_t* candw = reinterpret_cast<uint8_t*>(cand + cand_cap);      // [cand_cap] their warps
+  uint32_t* cache = reinterpret_cast<uint32_t*>(candw + cand_cap);   // [cache_cap] (cand_cap % 16 == 0)
   __shared__ uint32_t s_krem, s_bin;
   __shared__ int s_ncand;
   __shared__ int s_cgt[BLOCK / 32], s_ceq[BLOCK / 32];
@@ -313,7 +341,7 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
   const int wseg = ((n + NW - 1) / NW + 31) & ~31;
   const int w0 = warp * wseg;
   const int w1 = min(n, w0 + wseg);
-  const bool few = nb1 <= (uint32_t)kCand;
+  const bool few = nb1 <= (uint32_t)cand_cap;
   int gt12 = 0;                                       // keys of this warp whose top 12 bits exceed b1
   uint32_t prefix = 0u;
   if (few) {
@@ -378,7 +406,7 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
     }
     __syncthreads();
   } else {
-    // a crowded bin (more than kCand keys share the top 12 bits, e.g. near-equal scores): bits 19..8 of
+    // a crowded bin (more than cand_cap keys share the top 12 bits, e.g. near-equal scores): bits 19..8 of
     // the bin's keys, then bits 7..0 of the keys under that 24-bit prefix, each one filtered pass over
     // the row with plain shared atomics (the same digits the candidate path resolves)
     for (int i = threadIdx.x; i < kHist12; i += BLOCK) hist12[i] = 0u;
@@ -524,14 +552,19 @@ template <int BLOCK, bool RANKED>
 cudaError_t launch_topk_t(const dsa_dims& d, const float* scores, const int32_t* q_pos, const int32_t* kv_start,
                           const int32_t* kv_len, int k, int32_t* idx, float* vals, cudaStream_t st) {
   int cache_cap = d.n_kv < kTopkCacheMax ? d.n_kv : kTopkCacheMax;
+  // short rows (256-thread blocks, six per SM) keep a candidate buffer of half a row, at least 1024 keys:
+  // a threshold bin holding more takes the crowded-bin passes instead (the same result)
+  int cand_cap = kCand;
+  if (BLOCK <= 256) cand_cap = std::min(kCand, std::max(1024, ((d.n_kv / 2) + 15) & ~15));
   const size_t fixed = (RANKED ? (size_t)k * 16 + (size_t)(BLOCK / 32) * 256 * 4 : 0) + 256 * 4 + 64 * 4 +
-                       (size_t)(kHist12 + kCand) * 4 + kCand;
+                       (size_t)(kHist12 + cand_cap) * 4 + cand_cap;
   if (fixed + (size_t)cache_cap * 4 > 220 * 1024) cache_cap = (int)((220 * 1024 - fixed) / 4);
   const size_t smem = fixed + (size_t)cache_cap * 4;
   auto kern = topk_kernel<BLOCK, RANKED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(d.n_q, d.batch), BLOCK, smem, st>>>(d, scores, q_pos, kv_start, kv_len, k, cache_cap, idx, vals);
+  kern<<<dim3(d.n_q, d.batch), BLOCK, smem, st>>>(d, scores, q_pos, kv_start, kv_len, k, cache_cap, cand_cap, idx,
+                                                  vals);
   return cudaGetLastError();
 }
 }  // namespace
@@ -542,8 +575,11 @@ cudaError_t launch_topk(const dsa_dims& d, const float* scores, const int32_t* q
   if (d.n_kv > 8192)
     return ranked ? launch_topk_t<1024, true>(d, scores, q_pos, kv_start, kv_len, k, idx, vals, st)
                   : launch_topk_t<1024, false>(d, scores, q_pos, kv_start, kv_len, k, idx, vals, st);
-  return ranked ? launch_topk_t<512, true>(d, scores, q_pos, kv_start, kv_len, k, idx, vals, st)
-                : launch_topk_t<512, false>(d, scores, q_pos, kv_start, kv_len, k, idx, vals, st);
+  if (d.n_kv > 4096)
+    return ranked ? launch_topk_t<512, true>(d, scores, q_pos, kv_start, kv_len, k, idx, vals, st)
+                  : launch_topk_t<512, false>(d, scores, q_pos, kv_start, kv_len, k, idx, vals, st);
+  return ranked ? launch_topk_t<256, true>(d, scores, q_pos, kv_start, kv_len, k, idx, vals, st)
+                : launch_topk_t<256, false>(d, scores, q_pos, kv_start, kv_len, k, idx, vals, st);
 }
 
 }  // namespace dsa
