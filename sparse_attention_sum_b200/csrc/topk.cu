@@ -106,15 +106,27 @@ __device__ void find_crossing(const uint32_t* hist, int nbins, uint32_t kneed, i
   const int owners = nbins / per;
   const int top = nbins - 1 - per * (int)threadIdx.x;   // this thread's digits: top, top - 1, ..., top - per + 1
   const bool own = (int)threadIdx.x < owners;
+  const bool vec = (per & 3) == 0;                       // whole aligned groups of four: 16-byte loads
+  const uint4* h4 = reinterpret_cast<const uint4*>(hist);
   if constexpr (BLOCK >= 512) {
     // at most eight digits: held in registers between the scan and the walk
     uint32_t cnt[8];
+    if (vec) {
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        const uint4 v = (own && 4 * g < per) ? h4[(top - 3 - 4 * g) >> 2] : make_uint4(0u, 0u, 0u, 0u);
+        cnt[4 * g] = v.w;                                // digit top - 4g
+        cnt[4 * g + 1] = v.z;
+        cnt[4 * g + 2] = v.y;
+        cnt[4 * g + 3] = v.x;
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) cnt[u] = (u < per && own) ? hist[top - u] : 0u;
+    }
     uint32_t lsum = 0;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      cnt[u] = (u < per && own) ? hist[top - u] : 0u;
-      lsum += cnt[u];
-    }
+    for (int u = 0; u < 8; ++u) lsum += cnt[u];
     int total;
     const uint32_t excl = (uint32_t)block_exclusive_scan<BLOCK>((int)lsum, scan, total);
     if (own && excl < kneed && excl + lsum >= kneed) {
@@ -133,8 +145,14 @@ __device__ void find_crossing(const uint32_t* hist, int nbins, uint32_t kneed, i
     // more digits per thread: summed first, walked again by the one thread holding the crossing
     uint32_t lsum = 0;
     if (own) {
-#pragma unroll 8
-      for (int u = 0; u < per; ++u) lsum += hist[top - u];
+      if (vec) {
+        for (int g = 0; g < per; g += 4) {
+          const uint4 v = h4[(top - 3 - g) >> 2];
+          lsum += (v.x + v.y) + (v.z + v.w);
+        }
+      } else {
+        for (int u = 0; u < per; ++u) lsum += hist[top - u];
+      }
     }
     int total;
     const uint32_t excl = (uint32_t)block_exclusive_scan<BLOCK>((int)lsum, scan, total);
@@ -152,6 +170,13 @@ __device__ void find_crossing(const uint32_t* hist, int nbins, uint32_t kneed, i
     }
   }
   __syncthreads();
+}
+
+// Zeroes the 4096-bin histogram (16-byte aligned) with 16-byte stores.
+template <int BLOCK>
+__device__ __forceinline__ void clear_hist12(uint32_t* hist12) {
+  uint4* h4 = reinterpret_cast<uint4*>(hist12);
+  for (int i = threadIdx.x; i < kHist12 / 4; i += BLOCK) h4[i] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 // Stable LSD radix sort of m (key, index) pairs by key, descending: four 8-bit
@@ -279,7 +304,7 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
   // counts the top 12 bits; the keys of the bin holding the k-th largest then become a small
   // candidate set, and the low 20 bits are resolved over it alone (12 + 8 bits).
   TOPK_TRACE(0);
-  for (int i = threadIdx.x; i < kHist12; i += BLOCK) hist12[i] = 0u;
+  clear_hist12<BLOCK>(hist12);
   if (threadIdx.x == 0) s_ncand = 0;
   __syncthreads();
   {
@@ -385,7 +410,7 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
     __syncthreads();
     TOPK_TRACE(3);
     // bits 19..8 of the candidates
-    for (int i = threadIdx.x; i < kHist12; i += BLOCK) hist12[i] = 0u;
+    clear_hist12<BLOCK>(hist12);
     __syncthreads();
     for (int c = threadIdx.x; c < (int)nb1; c += BLOCK) atomicAdd(&hist12[(cand[c] >> 8) & 4095u], 1u);
     __syncthreads();
@@ -409,7 +434,7 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
     // a crowded bin (more than cand_cap keys share the top 12 bits, e.g. near-equal scores): bits 19..8 of
     // the bin's keys, then bits 7..0 of the keys under that 24-bit prefix, each one filtered pass over
     // the row with plain shared atomics (the same digits the candidate path resolves)
-    for (int i = threadIdx.x; i < kHist12; i += BLOCK) hist12[i] = 0u;
+    clear_hist12<BLOCK>(hist12);
     __syncthreads();
     for (int i = threadIdx.x; i < n; i += BLOCK) {
       const uint32_t key = cached ? cache[i] : score_key(srow[r.lo + i]);
