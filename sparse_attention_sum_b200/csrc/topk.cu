@@ -54,9 +54,12 @@ constexpr int kTopkCacheMax = 40960;  // keys cached in shared memory (160 KB)
 constexpr int kHist12 = 4096;         // first-pass histogram: the top 12 bits of a key
 constexpr int kCand = 4096;           // keys of the threshold's 12-bit bin resolved on their own (at most)
 
-// Block-wide exclusive scan of one int per thread; returns the block total.
+// Block-wide exclusive scan of one int per thread; returns the block total.  One barrier: every
+// warp scans the (at most 32) warp totals itself.  The caller reaches a barrier before `scratch`
+// (>= BLOCK/32 ints) is written again.
 template <int BLOCK>
-__device__ __forceinline__ int block_exclusive_scan(int v, int* scratch /*>= BLOCK/32 + 1*/, int& total) {
+__device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int& total) {
+  constexpr int NW = BLOCK / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int x = v;
 #pragma unroll
@@ -66,19 +69,15 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch /*>= BLO
   }
   if (lane == 31) scratch[warp] = x;
   __syncthreads();
-  if (warp == 0) {
-    int s = lane < BLOCK / 32 ? scratch[lane] : 0;
+  const int w = lane < NW ? scratch[lane] : 0;
+  int s = w;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xffffffffu, s, o);
-      if (lane >= o) s += y;
-    }
-    if (lane < BLOCK / 32) scratch[lane] = s;  // inclusive warp totals
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, s, o);
+    if (lane >= o) s += y;
   }
-  __syncthreads();
-  int warp_base = warp > 0 ? scratch[warp - 1] : 0;
-  total = scratch[BLOCK / 32 - 1];
-  __syncthreads();
+  total = __shfl_sync(0xffffffffu, s, NW - 1);
+  const int warp_base = __shfl_sync(0xffffffffu, s - w, warp);
   return warp_base + x - v;
 }
 
@@ -478,11 +477,27 @@ topk_kernel(dsa_dims d, const float* __restrict__ scores, const int32_t* __restr
     c_eq = __reduce_add_sync(0xffffffffu, c_eq);
   }
   TOPK_TRACE(5);
-  int tot;
-  int gt_base = block_exclusive_scan<BLOCK>(lane == 0 ? c_gt : 0, scan, tot);
-  int eq_base = block_exclusive_scan<BLOCK>(lane == 0 ? c_eq : 0, scan, tot);
-  gt_base = __shfl_sync(0xffffffffu, gt_base, 0);
-  eq_base = __shfl_sync(0xffffffffu, eq_base, 0);
+  // the warps' counts, scanned by every warp itself (one barrier): keys of earlier warps above / equal to tau
+  if (lane == 0) {
+    scan[warp] = c_gt;
+    scan[32 + warp] = c_eq;
+  }
+  __syncthreads();
+  int gt_base, eq_base;
+  {
+    const int g = lane < NW ? scan[lane] : 0, e = lane < NW ? scan[32 + lane] : 0;
+    int sg = g, se = e;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int yg = __shfl_up_sync(0xffffffffu, sg, o), ye = __shfl_up_sync(0xffffffffu, se, o);
+      if (lane >= o) {
+        sg += yg;
+        se += ye;
+      }
+    }
+    gt_base = __shfl_sync(0xffffffffu, sg - g, warp);
+    eq_base = __shfl_sync(0xffffffffu, se - e, warp);
+  }
   const uint32_t lt_mask = (1u << lane) - 1u;
   if constexpr (!RANKED) {
     if (c_eq == 0) {
