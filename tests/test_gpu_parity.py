@@ -186,6 +186,28 @@ def test_topk_bit_exact_with_heavy_ties(S, k):
     _topk_case(scores, q_pos, kv_start, kv_len, k)
 
 
+def test_topk_long_rows_with_adversarial_structure():
+    # rows of 32768 keys (the 1024-thread kernel) built against estimates of the threshold from a
+    # regular subset of the row: row 0 puts the top k at positions 0 and 1 mod 32 (a comb), row 1 makes
+    # every key at 16 mod 32 large, row 2 is plain normal data, row 3 has 3000 keys tied at the k-th
+    # largest value; each set of rows is also seen from an unaligned first visible key.  All exact
+    # against the oracle.
+    rng = np.random.default_rng(7)
+    S, k, T = 32768, 2048, 4
+    scores = rng.standard_normal((1, T, S)).astype(np.float32)
+    pos = np.arange(S)
+    comb = (pos % 32 == 0) | (pos % 32 == 1)
+    scores[0, 0, comb] = 10.0 + rng.random(int(comb.sum())).astype(np.float32)
+    strided = pos % 32 == 16
+    scores[0, 1, strided] = 10.0 + rng.random(int(strided.sum())).astype(np.float32)
+    kth = np.sort(scores[0, 3])[::-1][k - 1]
+    tie = rng.choice(S, 3000, replace=False)
+    scores[0, 3, tie] = kth
+    q_pos = [[S - 1] * T]
+    for start in (0, 5, 3):
+        _topk_case(scores, q_pos, [start], [S], k)
+
+
 def test_topk_distinct_and_padded_rows():
     rng = np.random.default_rng(0)
     S = 9000
